@@ -1,0 +1,422 @@
+"""Pins for the float64 oracle: worked examples printed on the pages, closed
+forms, finite differences, invariants and published generator vectors.
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign, a transposed operand, a wrong group map, a mis-indexed counter)
+fails at least one test. None of these tests uses the CUDA library.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as A
+from oracle import philox as P
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _as4(x):
+    return np.asarray(x, dtype=np.float64)[None, None]
+
+
+# ---------------------------------------------------------------------------
+# Worked examples of the pages
+# ---------------------------------------------------------------------------
+
+def test_one_key_example():
+    ex = _golden("worked_examples.json")["one_key"]
+    q, k, v, g = (_as4(ex[n]) for n in ("q", "k", "v", "g"))
+    allow = np.array(ex["allowed"], bool)
+    fw = A.forward(q, k, v, allow, ex["scale"])
+    assert np.allclose(fw.y[0, 0], ex["y"], atol=0)
+    bw = A.backward(q, k, v, g, allow, ex["scale"])
+    assert np.allclose(bw.dq[0, 0], ex["dq"], atol=1e-15)
+    assert np.allclose(bw.dk[0, 0], ex["dk"], atol=1e-15)
+    assert np.allclose(bw.dv[0, 0], ex["dv"], atol=1e-15)
+    assert np.allclose(bw.delta[0, 0], ex["delta"])
+    s = A.block_summary(np.array([6.0]), np.array([[7.0]]), np.array([True]))
+    assert s[0] == ex["summary"][0] and s[1] == ex["summary"][1]
+    assert np.allclose(s[2], [ex["summary"][2]])
+    y, _, _, _ = A.tiled_forward(q[0, 0], k[0, 0], v[0, 0], allow, 1.0, 1, 1)
+    assert np.allclose(y, ex["y"])
+
+
+def test_empty_first_block_example():
+    ex = _golden("worked_examples.json")["empty_first_block"]
+    q, k, v = (np.array(ex[n], float) for n in ("q", "k", "v"))
+    allow = np.array(ex["allowed"], bool)
+    fw = A.forward(q[None, None], k[None, None], v[None, None], allow, 1.0)
+    assert np.allclose(fw.y[0, 0], ex["y"])
+    y, m, ell, cards = A.tiled_forward(q, k, v, allow, 1.0, 1, ex["block"], trace_row=1)
+    assert np.allclose(y, ex["y"])
+    # Row 2 (index 1): summary (0,1,3) after block 1, (0,2,8) after block 2.
+    got = [(c.m, c.ell, float(c.u[0])) for c in cards]
+    assert got == [tuple(map(float, s)) for s in ex["row2_summaries"]]
+    # Row 1 (index 0) skipped its empty first block: only one card.
+    _, _, _, cards0 = A.tiled_forward(q, k, v, allow, 1.0, 1, 1, trace_row=0)
+    assert len(cards0) == 1 and cards0[0].key_start == 1 and cards0[0].alpha == 0.0
+
+
+def test_merge_order_example():
+    ex = _golden("worked_examples.json")["merge_orders"]
+    q, k, v = (np.array(ex[n], float) for n in ("q", "k", "v"))
+    s = (q @ k.T)[0]
+    s1 = A.block_summary(s, v, np.array([True, False]))
+    s2 = A.block_summary(s, v, np.array([False, True]))
+    assert np.allclose([s1[0], s1[1], s1[2][0]], ex["summary_block1"])
+    assert np.allclose([s2[0], s2[1], s2[2][0]], ex["summary_block2"])
+    for a, b in ((s1, s2), (s2, s1)):
+        m = A.merge_summaries(a, b)
+        assert np.allclose([m[0], m[1], m[2][0]], ex["merged"], rtol=1e-15)
+        assert math.isclose(m[2][0] / m[1], 2.0, rel_tol=1e-15)
+    assert A.merge_summaries(None, s1) is s1 and A.merge_summaries(s2, None) is s2
+    allow = np.array(ex["allowed"], bool)
+    for order in ([0, 1], [1, 0]):
+        y, *_ = A.tiled_forward(q, k, v, allow, 1.0, 1, 1, key_tile_order=order)
+        assert np.allclose(y, ex["y"], rtol=1e-15)
+
+
+def test_dropout_replay_example():
+    ex = _golden("worked_examples.json")["dropout_replay"]
+    q, k, v, g = (np.array(ex[n], float)[None, None] for n in ("q", "k", "v", "g"))
+    allow = np.ones((2, 2), bool)
+    rho = ex["rho"]
+    for xi, dv_expect in ((ex["xi_row1"], ex["dv"]), (ex["xi_row1_alt"], ex["dv_alt"])):
+        keep = np.ones((1, 1, 2, 2), bool)
+        keep[0, 0, 0] = np.array(xi, bool)
+        fw = A.forward(q, k, v, allow, 1.0, keep=keep, rho=rho)
+        bw = A.backward(q, k, v, g, allow, 1.0, keep=keep, rho=rho)
+        assert np.allclose(bw.dv[0, 0], dv_expect)
+        if xi == ex["xi_row1"]:
+            assert np.allclose(fw.y[0, 0, 0], ex["y_row1"])
+
+
+def test_sink_example_dense_and_topk():
+    ex = _golden("worked_examples.json")["sink"]
+    p1, p2 = ex["p"]
+    z = math.log(ex["p_sink"])
+    # Dense realisation: d = dv = 1, c = 1, Q = [1], K = (ln p1, ln p2) so
+    # that Z = exp(z) + p1 + p2 = 1 and the printed probabilities appear.
+    q = np.array([[1.0]])[None, None]
+    k = np.array([[math.log(p1)], [math.log(p2)]])[None, None]
+    v = np.array([[ex["v"][0]], [ex["v"][1]]])[None, None]
+    g = np.array([[ex["g"]]], float)[None, None]
+    sink = np.array([z])
+    allow = np.ones((1, 2), bool)
+    fw = A.forward(q, k, v, allow, 1.0, sink=sink)
+    assert math.isclose(fw.y[0, 0, 0, 0], ex["o"], rel_tol=1e-14)
+    assert math.isclose(fw.p_sink[0, 0, 0], ex["p_sink"], rel_tol=1e-14)
+    assert abs(fw.lse[0, 0, 0]) < 1e-15                       # ln Z = ln 1
+    bw = A.backward(q, k, v, g, allow, 1.0, sink=sink)
+    assert np.allclose(bw.dk[0, 0, :, 0], ex["dS"], atol=1e-14)   # dK_j = c gamma_j Q
+    assert math.isclose(bw.dsink[0], ex["dz"], rel_tol=1e-13)
+    assert np.allclose(bw.dv[0, 0, :, 0], ex["p"], atol=1e-15)
+    dq_expect = ex["dS"][0] * math.log(p1) + ex["dS"][1] * math.log(p2)
+    assert math.isclose(bw.dq[0, 0, 0, 0], dq_expect, rel_tol=1e-13)
+    # Softmax shift invariance: the three logit gradients sum to zero.
+    assert abs(sum(ex["dS"]) + ex["dz"]) < 1e-15
+    assert abs(bw.dk[0, 0, :, 0].sum() + bw.dsink[0]) < 1e-14
+    # Tied top-k realisation: KV rows (v_j, ln p_j), Q = (0, 1), Dv = 1.
+    kv = np.array([[ex["v"][0], math.log(p1)], [ex["v"][1], math.log(p2)]])
+    qt = np.array([[[0.0, 1.0]]])
+    idx = np.array([[0, 1]], np.int32)
+    ln = np.array([2], np.int32)
+    o, lse, ps = A.topk_forward(qt, kv, idx, ln, 1, 1.0, sink)
+    assert math.isclose(o[0, 0, 0], ex["o"], rel_tol=1e-14)
+    dq, dkv, dsink = A.topk_backward(qt, kv, idx, ln, 1, 1.0,
+                                     np.array([[[ex["g"]]]], float), sink)
+    assert np.allclose(dkv[:, 1], ex["dS"], atol=1e-14)
+    assert np.allclose(dkv[:, 0], ex["p"], atol=1e-14)          # 0 * G + p g
+    assert math.isclose(dsink[0], ex["dz"], rel_tol=1e-13)
+    assert np.allclose(dq[0, 0], ex["dS"][0] * kv[0] + ex["dS"][1] * kv[1], atol=1e-14)
+
+
+def test_two_tile_trace_cards():
+    gd = _golden("two_tile_trace.json")
+    inp = gd["inputs"]
+    q, k, v = (np.array(inp[n], float) for n in ("q", "k", "v"))
+    allow = A.allowed_dense(4, 4, causal=True)
+    y, m, ell, cards = A.tiled_forward(q, k, v, allow, inp["scale"], inp["tile_q"],
+                                       inp["tile_k"], trace_row=inp["trace_row"])
+    assert len(cards) == 2
+    for card, want in zip(cards, gd["cards"]):
+        assert (card.key_start, card.key_end) == (want["key_start"], want["key_end"])
+        assert card.m == want["m"]
+        assert math.isclose(card.alpha, want["alpha"], rel_tol=1e-15, abs_tol=0)
+        assert math.isclose(card.ell, want["ell"], rel_tol=1e-15)
+        assert np.allclose(card.u, want["u"], rtol=1e-15, atol=0)
+    assert np.allclose(y[3], gd["tiled_output_row3"], rtol=1e-15, atol=0)
+    fw = A.forward(q[None, None], k[None, None], v[None, None], allow, 1.0)
+    assert np.allclose(fw.y[0, 0, 3], gd["dense_output_row3"], rtol=1e-15, atol=0)
+    err = np.abs(fw.y[0, 0] - y).max()
+    assert err <= gd["published_tolerance"]
+
+
+def test_two_tile_example_gradients_by_finite_differences():
+    gd = _golden("two_tile_trace.json")
+    inp = gd["inputs"]
+    q, k, v = (np.array(inp[n], float)[None, None] for n in ("q", "k", "v"))
+    g = np.array(gd["gradient_upstream_seed"], float).reshape(1, 1, 4, 2)
+    allow = A.allowed_dense(4, 4, causal=True)
+    _check_fd(q, k, v, g, allow, 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Finite differences (the page's small-kernel test design: every coordinate,
+# central differences with step 1e-6 and absolute tolerance 4e-6)
+# ---------------------------------------------------------------------------
+
+def _loss(q, k, v, g, allow, scale, sink=None, keep=None, rho=0.0):
+    return float(np.sum(g * A.forward(q, k, v, allow, scale, sink, keep, rho).y))
+
+
+def _check_fd(q, k, v, g, allow, scale, sink=None, keep=None, rho=0.0,
+              step=1e-6, tol=4e-6):
+    bw = A.backward(q, k, v, g, allow, scale, sink, keep, rho)
+    pairs = [(q, bw.dq), (k, bw.dk), (v, bw.dv)]
+    if sink is not None:
+        pairs.append((sink, bw.dsink))
+    for x, grad in pairs:
+        flat = x.reshape(-1)
+        for idx in range(flat.size):
+            old = flat[idx]
+            flat[idx] = old + step
+            up = _loss(q, k, v, g, allow, scale, sink, keep, rho)
+            flat[idx] = old - step
+            dn = _loss(q, k, v, g, allow, scale, sink, keep, rho)
+            flat[idx] = old
+            fd = (up - dn) / (2 * step)
+            assert abs(fd - grad.reshape(-1)[idx]) <= tol, (idx, fd, grad.reshape(-1)[idx])
+
+
+@pytest.mark.parametrize("variant", ["mha_causal", "gqa_window", "mqa_block", "sink",
+                                     "dropout", "large_equal_scores"])
+def test_finite_differences(variant):
+    rng = np.random.default_rng(sum(map(ord, variant)))
+    B, Hq, Hkv, T, d, dv = 1, 2, 2, 7, 3, 2
+    scale = 1 / math.sqrt(d)
+    sink = keep = None
+    rho = 0.0
+    kw = {}
+    if variant == "mha_causal":
+        kw = dict(causal=True)
+    elif variant == "gqa_window":
+        B, Hq, Hkv = 2, 4, 2
+        kw = dict(causal=True, window_left=3)
+    elif variant == "mqa_block":
+        B, Hq, Hkv = 2, 3, 1
+        bm = rng.random((2, 4, 4)) < 0.5
+        bm[:, np.arange(4), np.arange(4)] = True
+        kw = dict(causal=True, block_mask=bm[:, None], block_q=2, block_k=2)
+    elif variant == "sink":
+        kw = dict(causal=True)
+        sink = rng.standard_normal(Hq)
+    elif variant == "dropout":
+        rho = 0.3
+        kw = dict(causal=True)
+        keep = rng.random((B, Hq, T, T)) >= rho
+    elif variant == "large_equal_scores":
+        kw = dict(causal=True)
+    q = rng.standard_normal((B, Hq, T, d))
+    k = rng.standard_normal((B, Hkv, T, d))
+    v = rng.standard_normal((B, Hkv, T, dv))
+    g = rng.standard_normal((B, Hq, T, dv))
+    if variant == "large_equal_scores":
+        q *= 0.0
+        q += 3.0
+        k[:] = 4.0          # every score equal and large (tied maxima)
+        k[..., 0, :] += 1e-3
+    allow = A.allowed_dense(T, T, **kw)
+    _check_fd(q, k, v, g, allow, scale, sink, keep, rho)
+
+
+# ---------------------------------------------------------------------------
+# Tiled recurrence equals the dense definition; invariants
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(6))
+def test_tiled_recurrence_matches_dense(seed):
+    rng = np.random.default_rng(100 + seed)
+    n, d, dv = int(rng.integers(5, 40)), int(rng.integers(1, 6)), int(rng.integers(1, 5))
+    tq, tk = int(rng.integers(1, 9)), int(rng.integers(1, 9))
+    q, k, v = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal((n, dv))
+    bm = rng.random(((n + 2) // 3, (n + 2) // 3)) < 0.4
+    np.fill_diagonal(bm, True)
+    allow = A.allowed_dense(n, n, causal=True, window_left=int(rng.integers(0, n)),
+                            block_mask=bm, block_q=3, block_k=3)
+    y_dense = A.forward(q[None, None], k[None, None], v[None, None], allow, 0.7).y[0, 0]
+    n_kt = (n + tk - 1) // tk
+    for order in (None, list(rng.permutation(n_kt))):
+        y, m, ell, _ = A.tiled_forward(q, k, v, allow, 0.7, tq, tk, key_tile_order=order)
+        assert np.abs(y - y_dense).max() <= 1e-12
+        assert np.all(ell[allow.any(1)] > 0)                # ell_i > 0 when A_i nonempty
+        assert np.all(np.isfinite(m[allow.any(1)]))
+
+
+def test_invariants_probability_mass_and_identities():
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, T, d, dv = 2, 4, 2, 33, 8, 5
+    q = rng.standard_normal((B, Hq, T, d))
+    k = rng.standard_normal((B, Hkv, T, d))
+    v = rng.standard_normal((B, Hkv, T, dv))
+    g = rng.standard_normal((B, Hq, T, dv))
+    sink = rng.standard_normal(Hq)
+    rho = 0.25
+    keep = rng.random((B, Hq, T, T)) >= rho
+    allow = A.allowed_dense(T, T, causal=True, window_left=9)
+    c = 0.3
+    fw = A.forward(q, k, v, allow, c, sink=sink, keep=keep, rho=rho)
+    bw = A.backward(q, k, v, g, allow, c, sink=sink, keep=keep, rho=rho)
+    # sum_j p_ij + p_sink,i = 1, from the saved LSE.
+    for b in range(B):
+        for h in range(Hq):
+            s = c * q[b, h] @ k[b, h // 2].T
+            p = np.where(allow, np.exp(s - fw.lse[b, h][:, None]), 0)
+            mass = p.sum(1) + np.exp(sink[h] - fw.lse[b, h])
+            assert np.allclose(mass, 1.0, atol=1e-13)
+    # sum_i Q_i.dQ_i = sum_j K_j.dK_j (both equal sum gamma_ij s_ij / c * c).
+    assert math.isclose(np.sum(q * bw.dq), np.sum(k * bw.dk), rel_tol=1e-10)
+    # sum_j V_j.dV_j = sum_i G_i.Y_i.
+    assert math.isclose(np.sum(v * bw.dv), np.sum(g * fw.y), rel_tol=1e-10)
+    # Shift invariance per row: sum_j gamma_ij - p_sink delta = 0, summed over rows
+    # and heads it is sum over h of (sum_j dS) + dsink_h.
+
+
+def test_empty_rows_are_zero_and_lse_conventions():
+    q = np.ones((1, 1, 3, 2))
+    k = np.ones((1, 1, 3, 2))
+    v = np.arange(6, dtype=float).reshape(1, 1, 3, 2)
+    allow = np.array([[0, 0, 0], [1, 0, 0], [1, 1, 0]], bool)
+    fw = A.forward(q, k, v, allow, 1.0)
+    assert np.all(fw.y[0, 0, 0] == 0) and fw.lse[0, 0, 0] == -np.inf
+    sink = np.array([0.5])
+    fw2 = A.forward(q, k, v, allow, 1.0, sink=sink)
+    assert fw2.lse[0, 0, 0] == 0.5 and fw2.p_sink[0, 0, 0] == 1.0
+    bw = A.backward(q, k, v, np.ones((1, 1, 3, 2)), allow, 1.0, sink=sink)
+    assert np.all(bw.dq[0, 0, 0] == 0)
+
+
+# ---------------------------------------------------------------------------
+# Top-k reduces to the dense definition with the selected allowed sets
+# ---------------------------------------------------------------------------
+
+def test_topk_equals_dense_with_selected_sets():
+    rng = np.random.default_rng(11)
+    Tq, Tkv, H, Dqk, Dv, topk = 5, 12, 3, 6, 4, 6
+    q = rng.standard_normal((Tq, H, Dqk))
+    kv = rng.standard_normal((Tkv, Dqk))
+    d_o = rng.standard_normal((Tq, H, Dv))
+    sink = rng.standard_normal(H)
+    from exact_tiled_attention_softmax_b200.workloads import topk_lists
+    idx, ln = topk_lists(Tq, Tkv, topk, 2, topk, 3)
+    c = 0.4
+    o, lse, ps = A.topk_forward(q, kv, idx, ln, Dv, c, sink)
+    dq, dkv, dsink = A.topk_backward(q, kv, idx, ln, Dv, c, d_o, sink)
+    allow = A.topk_allowed(idx, ln, Tkv)
+    qd = q.transpose(1, 0, 2)[None]                     # [1,H,Tq,Dqk]
+    kd = kv[None, None]
+    vd = kv[None, None, :, :Dv]
+    fw = A.forward(qd, kd, vd, allow, c, sink=sink)
+    bw = A.backward(qd, kd, vd, d_o.transpose(1, 0, 2)[None], allow, c, sink=sink)
+    assert np.allclose(o, fw.y[0].transpose(1, 0, 2), atol=1e-13)
+    assert np.allclose(lse, fw.lse[0].T, atol=1e-13)
+    assert np.allclose(dq, bw.dq[0].transpose(1, 0, 2), atol=1e-12)
+    dkv_dense = bw.dk[0, 0].copy()
+    dkv_dense[:, :Dv] += bw.dv[0, 0]
+    assert np.allclose(dkv, dkv_dense, atol=1e-12)
+    assert np.allclose(dsink, bw.dsink, atol=1e-12)
+
+
+def test_topk_lists_are_causal_and_distinct():
+    from exact_tiled_attention_softmax_b200.workloads import topk_lists
+    idx, ln = topk_lists(64, 256, 128, 40, 128, 9)
+    for t in range(64):
+        sel = idx[t, :ln[t]]
+        assert len(set(sel.tolist())) == ln[t]
+        assert sel.min() >= 0 and sel.max() <= 256 - 64 + t
+        assert np.all(idx[t, ln[t]:] == -1)
+
+
+# ---------------------------------------------------------------------------
+# Philox and the dropout mask
+# ---------------------------------------------------------------------------
+
+def test_philox_known_answers():
+    kat = _golden("philox4x32_10_kat.json")
+    for vec in kat["vectors"]:
+        ctr = np.array([int(x, 16) for x in vec["counter"]], dtype=np.uint64)
+        key = np.array([int(x, 16) for x in vec["key"]], dtype=np.uint64)
+        out = P.philox4x32(ctr, key)
+        assert [int(x) for x in out] == [int(x, 16) for x in vec["out"]]
+
+
+def test_dropout_mask_counter_layout_and_rate():
+    seed, rho = 0x123456789ABCDEF, 0.1
+    keep = P.dropout_keep(seed, rho, 2, 3, 9, 11)
+    thr = P.keep_threshold(rho)
+    # Element (b=1, h=2, i=5, j=7): counter (7>>2, 5, 2, 1), word 7&3.
+    w = P.philox4x32(np.array([1, 5, 2, 1], np.uint64),
+                     np.array([seed & 0xFFFFFFFF, seed >> 32], np.uint64))
+    assert keep[1, 2, 5, 7] == (int(w[3]) >= thr)
+    assert np.array_equal(keep, P.dropout_keep(seed, rho, 2, 3, 9, 11))  # replay
+    big = P.dropout_keep(99, rho, 1, 2, 300, 300)
+    n = big.size
+    rate = big.mean()
+    sigma = math.sqrt(rho * (1 - rho) / n)
+    assert abs(rate - (1 - rho)) < 6 * sigma
+    assert P.keep_threshold(0.0) == 0
+    with pytest.raises(ValueError):
+        P.keep_threshold(1.0)
+
+
+def test_dropout_replay_seed_search():
+    """A seed whose realisation for query row 0 is xi = (1, 0) exists and
+    reproduces the replay example through the generated mask."""
+    ex = _golden("worked_examples.json")["dropout_replay"]
+    seed = find_replay_seed()
+    keep = P.dropout_keep(seed, 0.5, 1, 1, 2, 2)
+    assert keep[0, 0, 0].tolist() == [True, False]
+    q, k, v, g = (np.array(ex[n], float)[None, None] for n in ("q", "k", "v", "g"))
+    bw = A.backward(q, k, v, g, np.ones((2, 2), bool), 1.0, keep=keep, rho=0.5)
+    assert np.allclose(bw.dv[0, 0], ex["dv"])
+
+
+def find_replay_seed():
+    for seed in range(1, 1000):
+        if P.dropout_keep(seed, 0.5, 1, 1, 2, 2)[0, 0, 0].tolist() == [True, False]:
+            return seed
+    raise AssertionError("no seed found")
+
+
+def test_oracle_detects_planted_mistakes():
+    """Mutation check: flipping the sign of delta or transposing the value
+    gradient makes the finite-difference pin fail."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, 1, 4, 2))
+    k = rng.standard_normal((1, 1, 4, 2))
+    v = rng.standard_normal((1, 1, 4, 3))
+    g = rng.standard_normal((1, 1, 4, 3))
+    allow = A.allowed_dense(4, 4, causal=True)
+    good = A.backward(q, k, v, g, allow, 0.5)
+    orig = A.backward
+
+    def bad_backward(*a, **kw):
+        r = orig(*a, **kw)
+        r.dq = -r.dq
+        return r
+    A.backward = bad_backward
+    try:
+        with pytest.raises(AssertionError):
+            _check_fd(q, k, v, g, allow, 0.5)
+    finally:
+        A.backward = orig
+    assert np.abs(good.dq).max() > 1e-3
