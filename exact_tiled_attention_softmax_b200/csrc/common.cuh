@@ -1,0 +1,136 @@
+// Shared device-side definitions: parameter blocks, the allowed-set predicate,
+// the Philox4x32-10 dropout generator and dtype-generic loads/stores.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/attn.h"
+
+namespace attn {
+
+// Byte offsets inside every workspace.
+constexpr size_t kStatusBytes = 256;  // status word lives at offset 0
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Allowed-set descriptor as the kernels see it.
+struct MaskP {
+  uint32_t flags;
+  int64_t window;  // W: j > i - W
+  const uint8_t* bm;
+  int32_t bq, bk;
+  int64_t bm_sb, bm_sh, bm_sq;
+  const float* sink;  // [Hq] or null
+  int dropout;        // 0/1
+  uint32_t keep_thr;  // keep iff philox word >= keep_thr
+  float inv_keep;     // 1 / (1 - rho)
+  uint32_t seed_lo, seed_hi;
+};
+
+// Dense problem: all strides in elements for (b, h, t); innermost stride 1.
+struct DenseP {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t sq[3], sk[3], sv[3];
+  int B, Hq, Hkv, T, d, dv;
+  float scale;
+  MaskP m;
+};
+
+// Shared-KV top-k problem.
+struct TopkP {
+  const void* q;   // [Tq, H, Dqk]
+  const void* kv;  // [Tkv, Dqk]; V = first Dv columns
+  int64_t sq_t, sq_h, skv;
+  const int32_t* idx;
+  int64_t idx_stride;
+  int32_t topk_max;
+  const int32_t* len;  // may be null
+  int Tq, Tkv, H, Dqk, Dv;
+  float scale;
+  const float* sink;
+};
+
+__device__ __forceinline__ float ld(const float* p) { return *p; }
+__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void st(float* p, float x) { *p = x; }
+__device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+
+// The allowed-set predicate A_i (flags intersect).
+__device__ __forceinline__ bool allowed(const MaskP& m, int b, int h, int64_t i, int64_t j) {
+  if ((m.flags & ATTN_MASK_CAUSAL) && j > i) return false;
+  if ((m.flags & ATTN_MASK_WINDOW) && j <= i - m.window) return false;
+  if (m.flags & ATTN_MASK_BLOCK) {
+    const uint8_t* row = m.bm + b * m.bm_sb + h * m.bm_sh + (i / m.bq) * m.bm_sq;
+    if (!row[j / m.bk]) return false;
+  }
+  return true;
+}
+
+// Key range [lo, hi] that can hold allowed keys for query row i.
+__device__ __forceinline__ void key_range(const MaskP& m, int64_t i, int64_t n_k,
+                                          int64_t& lo, int64_t& hi) {
+  lo = 0;
+  hi = n_k - 1;
+  if (m.flags & ATTN_MASK_CAUSAL) hi = i < hi ? i : hi;
+  if (m.flags & ATTN_MASK_WINDOW) {
+    int64_t w = i - m.window + 1;
+    lo = w > 0 ? w : 0;
+  }
+}
+
+// Query range [lo, hi] that can hold key j in its allowed set.
+__device__ __forceinline__ void query_range(const MaskP& m, int64_t j, int64_t n_q,
+                                            int64_t& lo, int64_t& hi) {
+  lo = 0;
+  hi = n_q - 1;
+  if (m.flags & ATTN_MASK_CAUSAL) lo = j;
+  if (m.flags & ATTN_MASK_WINDOW) {
+    int64_t w = j + m.window - 1;
+    hi = w < hi ? w : hi;
+  }
+}
+
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel Random
+// Numbers: As Easy as 1, 2, 3", SC'11): two 32x32->64 multiplies per round
+// by fixed odd constants, word exchange, key folded into the high halves,
+// key advanced by the Weyl increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint32_t uint4_word(const uint4& w, int idx) {
+  return idx == 0 ? w.x : idx == 1 ? w.y : idx == 2 ? w.z : w.w;
+}
+
+// Keep decision xi for pair (b, h, i, j): counter (j>>2, i, h, b).
+__device__ __forceinline__ bool dropout_keep(const MaskP& m, int b, int h, int64_t i, int64_t j) {
+  uint4 w = philox4x32_10(make_uint4((uint32_t)(j >> 2), (uint32_t)i, (uint32_t)h, (uint32_t)b),
+                          m.seed_lo, m.seed_hi);
+  return uint4_word(w, (int)(j & 3)) >= m.keep_thr;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+}  // namespace attn

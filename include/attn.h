@@ -1,0 +1,178 @@
+/*
+ * attn.h -- C ABI of the exact tiled masked softmax attention library.
+ *
+ * The library computes, on one NVIDIA B200 (sm_100a), exact masked softmax
+ * attention with a per-row running summary (m, l, z) carried across key
+ * tiles, and its reverse pass, which recomputes the scores tile by tile from
+ * the saved log-sum-exp instead of storing the probability grid.
+ *
+ * Definitions
+ *   Forward ("Tiled attention and its recomputed reverse pass are exact",
+ *   alphabetamath.cc, proof steps 1.1-2.1; "Accumulate attention without
+ *   keeping the full grid", intale.github.io, section "Rescale earlier mass
+ *   before adding a new tile"): for query row i with allowed key set A_i,
+ *       s_ij = c <Q_i, K_j>,   p_ij = exp(s_ij) / (exp(z_h) + sum_{l in A_i} exp(s_il)),
+ *       Y_i  = sum_{j in A_i} p~_ij V_j,  LSE_i = ln(exp(z_h) + sum_{l in A_i} exp(s_il)).
+ *   z_h is the optional per-head sink logit ("DeepSeek Sparse Attention
+ *   Forward and Backward", icavan.github.io, section 2.2; absent = -inf), and
+ *   p~_ij = p_ij xi_ij / (1 - rho) the optional inverted dropout ("A
+ *   different dropout mask changes the reverse result", alphabetamath.cc).
+ *   Reverse (same proof, steps 4.1-6.1; DSA note, sections 3.1-3.5):
+ *       delta_i = <G_i, Y_i>,  gamma_ij = p_ij (xi_ij/(1-rho) <G_i, V_j> - delta_i),
+ *       dQ_i = c sum_j gamma_ij K_j,  dK_j = c sum_i gamma_ij Q_i,
+ *       dV_j = sum_i p~_ij G_i,       dz_h = -sum_{b,i} exp(z_h - LSE_i) delta_i.
+ *   Query head h reads K/V head h / (Hq / Hkv); shared K/V heads sum the
+ *   pullbacks of every query head that reads them.
+ *
+ * Memory and ownership
+ *   Every tensor pointer is a DEVICE pointer owned by the caller. The library
+ *   allocates no device memory; scratch space is the caller's workspace,
+ *   sized by attn_fwd_workspace_size / attn_bwd_workspace_size. All work is
+ *   enqueued asynchronously on the caller's stream (a cudaStream_t passed as
+ *   void*; NULL = the legacy default stream). Outputs are overwritten, never
+ *   accumulated into. The library may cache host-side state per device
+ *   (TMA descriptors, kernel attributes).
+ *
+ * Errors
+ *   Every call returns an attn_status synchronously. Argument problems are
+ *   found on the host before any launch (ATTN_ERR_INVALID_ARG: shape, stride,
+ *   dtype, alignment, Hq % Hkv != 0, a dropout rate outside [0,1), ...).
+ *   Conditions only the device can see (a top-k index outside [0, Tkv), a
+ *   fixed-point overflow, a pipeline wait that ran out) are written to a
+ *   status word at the start of the workspace; read it with attn_get_status
+ *   after the stream has reached the call. No call traps the GPU, and on any
+ *   error the outputs' contents are unspecified.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_VERSION 100 /* major * 100 + minor */
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* bad shape, stride, dtype, alignment, pointer */
+  ATTN_ERR_UNSUPPORTED = 2, /* a valid request with no kernel for it */
+  ATTN_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
+  ATTN_ERR_DEVICE = 5       /* the device recorded an error (attn_get_status) */
+} attn_status;
+
+/* Device-side error bits reported through attn_get_status. */
+#define ATTN_DEVERR_TOPK_INDEX 0x1u  /* a listed index outside [0, Tkv) was skipped */
+#define ATTN_DEVERR_OVERFLOW 0x2u    /* a fixed-point dKV contribution saturated */
+#define ATTN_DEVERR_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
+
+typedef enum attn_dtype { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+
+/* A strided tensor view. Strides count elements, not bytes; the innermost
+ * dimension must have stride 1. Unused trailing entries are ignored. */
+typedef struct attn_tensor {
+  void* data;
+  int32_t dtype; /* attn_dtype */
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} attn_tensor;
+
+/* Allowed-set flags. A_i is the intersection of every enabled set. */
+#define ATTN_MASK_CAUSAL 0x1u /* j <= i */
+#define ATTN_MASK_WINDOW 0x2u /* j >  i - window_left */
+#define ATTN_MASK_BLOCK 0x4u  /* block_mask[i / block_q][j / block_k] != 0 */
+#define ATTN_MASK_TOPK 0x8u   /* j listed in topk_idxs[t][0 : topk_length[t]] */
+
+/* The allowed-set descriptor ("Tiled attention and its recomputed reverse
+ * pass are exact": the fixed allowed sets A_i; causal, windowed and packed
+ * intervals from "Accumulate attention without keeping the full grid",
+ * section "Change attention evaluation inside the existing model"; the
+ * shared-KV index lists of the DSA note, section 1). Pointers are device
+ * pointers. */
+typedef struct attn_mask {
+  uint32_t flags;
+  int64_t window_left; /* W >= 1 with ATTN_MASK_WINDOW */
+  /* ATTN_MASK_BLOCK: uint8 grid, element (b, h, r, c) at
+   * block_mask[b*bm_stride_b + h*bm_stride_h + r*bm_stride_q + c]; a zero
+   * stride broadcasts. Rows ceil(Tq/block_q), columns ceil(Tk/block_k). */
+  const uint8_t* block_mask;
+  int32_t block_q, block_k;
+  int64_t bm_stride_b, bm_stride_h, bm_stride_q;
+  /* ATTN_MASK_TOPK: int32 [Tq, topk_stride]; entries at positions >=
+   * topk_length[t] (or >= topk_max when topk_length is NULL) are ignored.
+   * Each listed position counts once. */
+  const int32_t* topk_idxs;
+  int64_t topk_stride;
+  int32_t topk_max;
+  const int32_t* topk_length;
+  /* Optional per-query-head sink logit z_h, fp32 [Hq]; NULL = no sink. */
+  const float* sink;
+  /* Optional inverted dropout: rate in [0, 1), 0 = off. The keep decision for
+   * pair (b, h, i, j) is word (j & 3) of Philox4x32-10 at counter
+   * (j >> 2, i, h, b) and key (seed low 32 bits, seed high 32 bits), kept iff
+   * that word >= floor(rate * 2^32). Both passes evaluate it; no mask is
+   * stored. */
+  float dropout_p;
+  uint64_t dropout_seed;
+} attn_mask;
+
+/* Layouts
+ *   Dense:  q [B,Hq,T,d], k [B,Hkv,T,d], v [B,Hkv,T,dv], o [B,Hq,T,dv],
+ *           lse fp32 [B,Hq,T]. Any stride order (BHSD, BSHD, ...).
+ *   Top-k (ATTN_MASK_TOPK, shared KV): q [Tq,H,Dqk], k = KV [Tkv,Dqk],
+ *           v = the view KV[:, :Dv] (same data pointer and row stride as k),
+ *           o [Tq,H,Dv], lse fp32 [Tq,H]. dk receives dKV [Tkv,Dqk]; dv is NULL.
+ *           Query token t sits at causal position Tkv - Tq + t; the lists
+ *           must respect causality themselves.
+ *   dtype: all of q, k, v, o (and do, dq, dk, dv) share one dtype, ATTN_F32
+ *   or ATTN_BF16. Accumulation is fp32 in every path.
+ */
+
+/* Workspace bytes attn_fwd needs for these shapes and mask (>= 256). */
+size_t attn_fwd_workspace_size(const attn_tensor* q, const attn_tensor* k,
+                               const attn_tensor* v, const attn_mask* mask);
+
+/* Workspace bytes attn_bwd needs for these shapes and mask (>= 256). */
+size_t attn_bwd_workspace_size(const attn_tensor* q, const attn_tensor* k,
+                               const attn_tensor* v, const attn_mask* mask);
+
+/* Forward pass: writes o = Y and lse (natural log, sink-inclusive: DSA note,
+ * section 7.1). Rows whose allowed set is empty get Y = 0 and LSE = -inf
+ * (or z_h with a sink). scale is c. */
+attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k,
+                     const attn_tensor* v, const attn_mask* mask, float scale,
+                     attn_tensor* o, attn_tensor* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Reverse pass for upstream gradient do_ (= G): recomputes the scores from
+ * q, k and the saved lse, forms delta from o and do_, and writes dq, dk, dv
+ * (top-k: dk = dKV, dv = NULL) and, when mask->sink is set and dsink is not
+ * NULL, dsink fp32 [Hq]. dk, dv, dKV and dsink are deterministic (bitwise
+ * identical across runs); dq is not guaranteed to be. */
+attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k,
+                     const attn_tensor* v, const attn_tensor* o,
+                     const attn_tensor* do_, const attn_tensor* lse,
+                     const attn_mask* mask, float scale, attn_tensor* dq,
+                     attn_tensor* dk, attn_tensor* dv, float* dsink,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word at the
+ * start of `workspace`. *device_bits receives the ATTN_DEVERR_* bits (0 when
+ * clean). Returns ATTN_ERR_DEVICE when any bit was set. */
+attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits);
+
+/* Static, human-readable text for a status code. */
+const char* attn_status_string(attn_status status);
+
+/* ATTN_VERSION of the built library. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+that include/attn.h declares, and rejects bad arguments before any launch.
+No test here runs a kernel, so the file needs no GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import exact_tiled_attention_softmax_b200 as eta
+    if not os.path.exists(eta.library_path()):
+        from exact_tiled_attention_softmax_b200 import build
+        build.build()
+    return eta.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_fwd_workspace_size", "attn_bwd_workspace_size",
+            "attn_get_status", "attn_status_string", "attn_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    text = open(HEADER).read()
+    ver = int(re.search(r"#define ATTN_VERSION (\d+)", text).group(1))
+    assert lib.attn_version() == ver
+    for code in range(6):
+        assert lib.attn_status_string(code)
+    assert b"unknown" in lib.attn_status_string(99)
+
+
+def _t(shape, dtype=1, data=0x1000, stride=None):
+    import exact_tiled_attention_softmax_b200 as eta
+    c = eta.AttnTensorC()
+    c.data = data
+    c.dtype = dtype
+    c.ndim = len(shape)
+    st = [1] * len(shape)
+    for i in range(len(shape) - 2, -1, -1):
+        st[i] = st[i + 1] * shape[i + 1]
+    for i, n in enumerate(shape):
+        c.shape[i] = n
+        c.stride[i] = (stride or st)[i]
+    return c
+
+
+def _call_fwd(lib, q, k, v, o, lse, mask=None, ws=0x100000, ws_bytes=1 << 20, scale=0.1):
+    return lib.attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
+                        ctypes.byref(mask) if mask else None, ctypes.c_float(scale),
+                        ctypes.byref(o), ctypes.byref(lse), ws, ws_bytes, None)
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    import exact_tiled_attention_softmax_b200 as eta
+    q, k, v = _t([1, 4, 64, 128]), _t([1, 2, 64, 128]), _t([1, 2, 64, 128])
+    o, lse = _t([1, 4, 64, 128]), _t([1, 4, 64], dtype=0)
+    # Hq not a multiple of Hkv
+    assert _call_fwd(lib, q, _t([1, 3, 64, 128]), _t([1, 3, 64, 128]), o, lse) == eta.ATTN_ERR_INVALID_ARG
+    # key length differs from query length
+    assert _call_fwd(lib, q, _t([1, 2, 65, 128]), v, o, lse) == eta.ATTN_ERR_INVALID_ARG
+    # inner stride not 1
+    assert _call_fwd(lib, _t([1, 4, 64, 128], stride=[64 * 256, 64 * 256, 256, 2]), k, v, o,
+                     lse) == eta.ATTN_ERR_INVALID_ARG
+    # mixed dtypes
+    assert _call_fwd(lib, q, _t([1, 2, 64, 128], dtype=0), v, o, lse) == eta.ATTN_ERR_INVALID_ARG
+    # lse must be fp32
+    assert _call_fwd(lib, q, k, v, o, _t([1, 4, 64], dtype=1)) == eta.ATTN_ERR_INVALID_ARG
+    # head width beyond the kernels
+    big = _t([1, 4, 64, 640])
+    assert _call_fwd(lib, big, _t([1, 2, 64, 640]), v, o, lse) == eta.ATTN_ERR_UNSUPPORTED
+    # dropout rate outside [0, 1)
+    m = eta.AllowedSet(causal=True, dropout_p=1.0).to_c()
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # window without a width
+    m = eta.AttnMaskC()
+    m.flags = eta.ATTN_MASK_WINDOW
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # unknown flag bits
+    m.flags = 0x100
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # workspace missing or too small
+    assert _call_fwd(lib, q, k, v, o, lse, ws=0) == eta.ATTN_ERR_WORKSPACE
+    assert _call_fwd(lib, q, k, v, o, lse, ws_bytes=16) == eta.ATTN_ERR_WORKSPACE
+    assert _call_fwd(lib, q, k, v, o, lse, ws=0x100010) == eta.ATTN_ERR_WORKSPACE
+    # non-finite scale
+    assert _call_fwd(lib, q, k, v, o, lse, scale=float("nan")) == eta.ATTN_ERR_INVALID_ARG
+
+
+def test_topk_arguments_rejected_on_host(lib):
+    import exact_tiled_attention_softmax_b200 as eta
+    q = _t([16, 4, 64])
+    kv = _t([32, 64])
+    v_ok = _t([32, 48], stride=[64, 1])
+    v_bad = _t([32, 48], data=0x2000, stride=[64, 1])
+    o, lse = _t([16, 4, 48]), _t([16, 4], dtype=0)
+    m = eta.AttnMaskC()
+    m.flags = eta.ATTN_MASK_TOPK
+    m.topk_idxs = 0x3000
+    m.topk_max = 8
+    m.topk_stride = 8
+    # V must be a view of the same KV rows
+    assert _call_fwd(lib, q, kv, v_bad, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # causal flag is carried by the lists themselves
+    m.flags = eta.ATTN_MASK_TOPK | eta.ATTN_MASK_CAUSAL
+    assert _call_fwd(lib, q, kv, v_ok, o, lse, mask=m) == eta.ATTN_ERR_UNSUPPORTED
+    m.flags = eta.ATTN_MASK_TOPK
+    m.topk_stride = 4
+    assert _call_fwd(lib, q, kv, v_ok, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # Dv larger than Dqk
+    assert _call_fwd(lib, q, kv, _t([32, 80], stride=[64, 1]), _t([16, 4, 80]), lse,
+                     mask=m) == eta.ATTN_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_cover_scratch(lib):
+    import exact_tiled_attention_softmax_b200 as eta
+    q, k, v = _t([2, 8, 256, 64]), _t([2, 4, 256, 64]), _t([2, 4, 256, 64])
+    f = lib.attn_fwd_workspace_size(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), None)
+    b = lib.attn_bwd_workspace_size(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), None)
+    rows = 2 * 8 * 256
+    assert f >= 256 and f % 256 == 0
+    assert b >= 256 + rows * 4 + rows * 64 * 4
+    m = eta.AttnMaskC()
+    m.flags = eta.ATTN_MASK_TOPK
+    m.topk_idxs = 0x3000
+    m.topk_max = m.topk_stride = 8
+    qt, kv, vt = _t([16, 4, 64]), _t([32, 64]), _t([32, 48], stride=[64, 1])
+    bt = lib.attn_bwd_workspace_size(ctypes.byref(qt), ctypes.byref(kv), ctypes.byref(vt), ctypes.byref(m))
+    assert bt >= 256 + 16 * 4 * 4 + 32 * 64 * 8
