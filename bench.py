@@ -1,0 +1,304 @@
+"""Throughput of exact tiled masked softmax attention, forward + reverse, on B200.
+
+Default workload (causal_8k): B=1, H=32, T=8192, d=dv=128, bf16, causal.
+One step = attn_fwd + attn_bwd over one batch already resident in HBM.
+value = algorithmic TFLOP/s over all ranks: allowed pairs x (2d + 2dv + 6d + 4dv)
+(= 1792 flops per pair at d = dv = 128), divided by the max over ranks of the
+summed CUDA-event step times. L2 is flushed (a 256 MB write) before every
+step, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the float64 CPU oracle on a sample
+
+Multi-GPU runs are independent replicas (the dense path has no exchange
+step): each rank runs the same workload; torch.distributed is used only for
+the barrier and the max-over-ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_softmax_b200 import workloads as W  # noqa: E402
+
+METRIC = "attention fwd+bwd TFLOP/s (bf16) and % of B200 dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def allowed_pairs(case: W.DenseCase) -> int:
+    """Sum over (b, h, i) of |A_i| for the causal / window workloads."""
+    T = case.T
+    if case.block_size:
+        raise ValueError("block-mask workloads need the mask to count pairs")
+    i = np.arange(T, dtype=np.int64)
+    lo = np.zeros(T, np.int64) if not case.window_left else np.maximum(0, i - case.window_left + 1)
+    hi = i if case.causal else np.full(T, T - 1, np.int64)
+    return int(case.B * case.Hq * np.sum(hi - lo + 1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        rows = [[c.strip() for c in ln.split(",")] for ln in getattr(self, "lines", [])]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(case: W.DenseCase, budget_s: float = 12.0):
+    """The float64 oracle, as it stands, on a bounded sample of the workload:
+    whole (b, h) slices of the same shape, one after another, until the time
+    budget is spent; scaled to TFLOP/s by the algorithmic flops of the slices
+    it finished."""
+    import oracle
+    rng = np.random.default_rng(case.seed)
+    T, d = case.T, case.d
+    allow = oracle.allowed_dense(T, T, causal=case.causal, window_left=case.window_left)
+    per_head_pairs = int(allow.sum())
+    q = W.round_to_bf16(rng.standard_normal((1, 1, T, d), dtype=np.float32)).astype(np.float64)
+    k = W.round_to_bf16(rng.standard_normal((1, 1, T, d), dtype=np.float32)).astype(np.float64)
+    v = W.round_to_bf16(rng.standard_normal((1, 1, T, d), dtype=np.float32)).astype(np.float64)
+    g = W.round_to_bf16(rng.standard_normal((1, 1, T, d), dtype=np.float32)).astype(np.float64)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        fw = oracle.forward(q, k, v, allow, case.scale)
+        oracle.backward(q, k, v, g, allow, case.scale, y=fw.y)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    flops = done * per_head_pairs * case.flops_per_pair
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{done} (b,h) slice(s) of B=1 H=1 T={T} d={d} causal fwd+bwd in float64 NumPy, "
+                      f"{el:.1f} s; oracle BLAS threads = all host cores"}
+
+
+def run_reference(args, case, rank, world):
+    """--impl reference: the oracle is the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    vals = []
+    for _ in range(max(args.warmup, 0)):
+        cpu_baseline(case, budget_s=1.0)
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(case, budget_s=max(2.0, 60.0 / max(args.steps, 1)))["value"])
+    v = statistics.median(vals)
+    cb = cpu_baseline(case, budget_s=1.0)
+    cb["value"] = v
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case.name, "B": case.B, "H": case.Hq, "T": case.T, "d": case.d,
+                       "mask": "causal"},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="causal_8k", choices=["causal_8k", "causal_2k"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    case = W.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, case, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import exact_tiled_attention_softmax_b200 as eta
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    eta.load_library()
+
+    q, k, v, g = W.dense_inputs(case)
+    tq, tk, tv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v, g))
+    allowed = eta.AllowedSet(causal=case.causal, window_left=case.window_left)
+    scale = case.scale
+    o = torch.empty_like(tq)
+    lse = torch.empty(tq.shape[:-1], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+    ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
+        eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    n_ev = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for s in range(n_ev):
+            flush.fill_(s & 0xFF)
+            e0, e1, e2 = ev[s]
+            e0.record(stream)
+            eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
+            e1.record(stream)
+            eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_fwd = [a.elapsed_time(b) for a, b, _ in ev]
+    t_bwd = [b.elapsed_time(c) for _, b, c in ev]
+    total_ms = sum(f + b for f, b in zip(t_fwd, t_bwd))
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / n_ev
+    pairs = allowed_pairs(case)
+    flops_step = pairs * case.flops_per_pair
+    value = world * flops_step * n_ev / (total_ms / 1e3) / 1e12
+
+    # End to end through the public API: pinned host inputs in, results out.
+    hq, hk, hv, hg = (x.to("cpu").pin_memory() for x in (tq, tk, tv, tg))
+    hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (dq, dk, dv))
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
+    d2h = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
+    e2e_ms = []
+    for s in range(n_ev + 2):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.fill_(s & 0xFF)
+        a0.record(stream)
+        tq.copy_(hq, non_blocking=True)
+        tk.copy_(hk, non_blocking=True)
+        tv.copy_(hv, non_blocking=True)
+        tg.copy_(hg, non_blocking=True)
+        step()
+        hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True)
+        hdv.copy_(dv, non_blocking=True)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        if s >= 2:
+            e2e_ms.append(a0.elapsed_time(a1))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        tt = torch.tensor([e2e_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_total = float(tt.item())
+    e2e_value = world * flops_step * len(e2e_ms) / (e2e_total / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    bwd_ms = statistics.mean(t_bwd)
+    bwd_flops = pairs * (6 * case.d + 4 * case.dv)
+    achieved = bwd_flops / (bwd_ms / 1e3) / 1e12
+    fwd_ms = statistics.mean(t_fwd)
+    fwd_achieved = pairs * (2 * case.d + 2 * case.dv) / (fwd_ms / 1e3) / 1e12
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": case.name, "B": case.B, "H": case.Hq, "T": case.T, "d": case.d,
+                       "dv": case.dv, "mask": "causal", "allowed_pairs": pairs,
+                       "flops_per_pair": case.flops_per_pair, "l2": "flushed (256 MB write) before every step",
+                       "parallelism": f"replicas x{world}"},
+            "pct_of_peak": {"measured_bf16_burst": 100 * value / world / peak,
+                            "nvidia_dense_bf16_spec_2250": 100 * value / world / 2250.0},
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_achieved, "bwd_tflops": achieved,
+            "roofline": {"bound": "tensor", "kernel": "attn_bwd (prepare + bwd_kernel + dq_finish)",
+                         "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                         "traffic": None, "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(W.DenseCase(
+                "causal_8k_slice", 1, 1, 1, case.T, case.d, case.dv, "bf16", case.scale, causal=True,
+                seed=case.seed))
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

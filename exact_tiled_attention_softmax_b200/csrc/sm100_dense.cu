@@ -1,26 +1,1063 @@
-// Placeholder: the tensor-core path is not wired in yet.
+// Tensor-core path for dense bf16 attention with d = dv = 128 on sm_100a.
+//
+// Forward: one CTA per (128-row query tile, query head, batch row). A TMA
+// producer warp streams 128-key K/V tiles through a two-stage ring; one
+// thread issues tcgen05 MMAs (S = Q K^T into a double-buffered TMEM tile,
+// O += P V into a TMEM accumulator); a 128-thread softmax warpgroup owns one
+// row per thread (TMEM lane = row) and applies the running-summary update of
+// "Accumulate attention without keeping the full grid", section "Rescale
+// earlier mass before adding a new tile": tile maximum, new maximum, the
+// rescale factor alpha, shifted exponentials and the running sum, with empty
+// tiles skipped without touching the state ("Tiled attention and its
+// recomputed reverse pass are exact", proof step 1.1). The maximum is only
+// moved when it grows by more than 2^8 (in base-2 units); the output stays
+// exact because every stored term shares the same reference maximum.
+//
+// Reverse: one CTA per (128-key tile, K/V head, batch row) walks every query
+// head of its group and every 64-row query tile that can see its keys. Per
+// step it recomputes S^T = K Q^T and dP^T = V dO^T, forms
+// P = exp(S - LSE) and gamma = P (dP - delta) in registers (DSA note,
+// sections 3.3-3.4; exactness proof, step 4.1), and accumulates
+// dV += P~^T dO and dK += gamma^T Q in TMEM for the whole CTA (a fixed order,
+// hence deterministic), while dQ^T = K^T gamma^T goes to an fp32 buffer by
+// bulk reduce-add.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
 #include "sm100_dense.h"
+#include "sm100_ptx.cuh"
 
 namespace attn {
 
-size_t sm100_fwd_workspace_bytes(int, int, int, const attn_mask*) { return 0; }
-size_t sm100_bwd_extra_workspace_bytes(int, int, int, int, const attn_mask*) { return 0; }
-bool sm100_dense_supported(const DenseP&, const attn_tensor*, const attn_tensor*, const attn_tensor*,
-                           const attn_tensor*) {
-  return false;
+using namespace sm100;
+
+namespace {
+
+constexpr int kD = 128;          // head width handled here (d = dv)
+constexpr int kBN = 128;         // keys per tile
+constexpr int kBM = 128;         // forward query rows per CTA
+constexpr int kBMb = 64;         // reverse query rows per step
+constexpr int kStages = 2;       // K/V ring depth (forward), Q/dO ring depth (reverse)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // move the running max only past 2^8
+
+enum : uint8_t { kEmpty = 0, kFull = 1, kPartial = 2 };
+
+// ------------------------------------------------------------------ masks
+
+// Is every (i, j) of the rectangle [r0, r1] x [c0, c1] inside the
+// causal/window band, and is any? Row i allows [max(c0, i-W+1), min(c1, i)],
+// so some row qualifies iff i can be chosen with c0 <= i (causal) and
+// i <= c1 + W - 1 (window).
+__device__ __forceinline__ void band_test(const MaskP& m, int64_t r0, int64_t r1, int64_t c0, int64_t c1, bool& any,
+                                          bool& all) {
+  const bool causal = m.flags & ATTN_MASK_CAUSAL, window = m.flags & ATTN_MASK_WINDOW;
+  all = true;
+  if (causal && c1 > r0) all = false;
+  if (window && c0 < r1 - m.window + 1) all = false;
+  int64_t lo = r0, hi = r1;
+  if (causal && c0 > lo) lo = c0;
+  if (window && c1 + m.window - 1 < hi) hi = c1 + m.window - 1;
+  any = c0 <= c1 && lo <= hi;
 }
-bool sm100_dense_bwd_supported(const DenseP&, const attn_tensor*, const attn_tensor*, const attn_tensor*,
-                               const attn_tensor*) {
-  return false;
+
+// Class of the (64-row query slice qs, 128-key tile kt) pair.
+__device__ uint8_t tile_class(const MaskP& m, int T, int b, int h, int qs, int kt) {
+  const int64_t r0 = (int64_t)qs * kBMb, r1 = (r0 + kBMb < T ? r0 + kBMb : T) - 1;
+  const int64_t c0 = (int64_t)kt * kBN, c1e = c0 + kBN - 1, c1 = (c1e < T ? c1e : T - 1);
+  if (r0 > r1 || c0 > c1) return kEmpty;
+  bool any = false, all = c1e <= T - 1;
+  if (!(m.flags & ATTN_MASK_BLOCK)) {
+    bool a, f;
+    band_test(m, r0, r1, c0, c1, a, f);
+    any = a;
+    all = all && f;
+  } else {
+    const uint8_t* base = m.bm + b * m.bm_sb + h * m.bm_sh;
+    for (int64_t rb = r0 / m.bq; rb <= r1 / m.bq; ++rb) {
+      const int64_t rr0 = rb * m.bq > r0 ? rb * m.bq : r0;
+      const int64_t rr1 = rb * m.bq + m.bq - 1 < r1 ? rb * m.bq + m.bq - 1 : r1;
+      for (int64_t cb = c0 / m.bk; cb <= c1 / m.bk; ++cb) {
+        const int64_t cc0 = cb * m.bk > c0 ? cb * m.bk : c0;
+        const int64_t cc1 = cb * m.bk + m.bk - 1 < c1 ? cb * m.bk + m.bk - 1 : c1;
+        bool a, f;
+        band_test(m, rr0, rr1, cc0, cc1, a, f);
+        if (base[rb * m.bm_sq + cb]) {
+          any = any || a;
+          all = all && f;
+        } else {
+          all = false;
+        }
+      }
+    }
+  }
+  return any ? (all ? kFull : kPartial) : kEmpty;
 }
-cudaError_t sm100_dense_fwd(const DenseP&, void*, const int64_t[3], float*, const int64_t[3], void*, uint32_t*,
-                            cudaStream_t) {
-  return cudaErrorNotSupported;
+
+struct ClassTable {
+  const uint8_t* cls;  // null: compute analytically
+  int nb, nh;          // slices along batch and head (1 = broadcast)
+  int nqs, nkt;
+};
+
+__device__ __forceinline__ uint8_t lookup_class(const ClassTable& ct, const MaskP& m, int T, int b, int h, int qs,
+                                                int kt) {
+  if (!ct.cls) return tile_class(m, T, b, h, qs, kt);
+  const int sb = ct.nb > 1 ? b : 0, sh = ct.nh > 1 ? h : 0;
+  return ct.cls[(((int64_t)sb * ct.nh + sh) * ct.nqs + qs) * ct.nkt + kt];
 }
-cudaError_t sm100_dense_bwd(const DenseP&, const void*, const int64_t[3], const void*, const int64_t[3],
-                            const float*, const int64_t[3], float*, float*, void*, const int64_t[3], void*,
-                            const int64_t[3], void*, const int64_t[3], void*, uint32_t*, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+__global__ void classify_kernel(MaskP m, int T, int B, int Hq, ClassTable ct, uint8_t* out) {
+  const int64_t n = (int64_t)ct.nb * ct.nh * ct.nqs * ct.nkt;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int kt = (int)(e % ct.nkt);
+    const int qs = (int)((e / ct.nkt) % ct.nqs);
+    const int sh = (int)((e / ((int64_t)ct.nkt * ct.nqs)) % ct.nh);
+    const int sb = (int)(e / ((int64_t)ct.nkt * ct.nqs * ct.nh));
+    out[e] = tile_class(m, T, sb, sh, qs, kt);
+  }
+  (void)B;
+  (void)Hq;
+}
+
+// Forward tile class for a 128-row query tile: merge its two 64-row slices.
+__device__ __forceinline__ uint8_t fwd_class(const ClassTable& ct, const MaskP& m, int T, int b, int h, int qt,
+                                             int kt) {
+  const uint8_t a = lookup_class(ct, m, T, b, h, 2 * qt, kt);
+  const uint8_t c = (2 * qt + 1) * kBMb < T ? lookup_class(ct, m, T, b, h, 2 * qt + 1, kt) : a;
+  if (a == kEmpty && c == kEmpty) return kEmpty;
+  if (a == kFull && c == kFull) return kFull;
+  return kPartial;
+}
+
+// ------------------------------------------------------------- forward
+
+struct FwdArgs {
+  MaskP m;
+  ClassTable ct;
+  int B, Hq, Hkv, T;
+  float scale_log2;  // c * log2(e)
+  __nv_bfloat16* o;
+  int64_t so[3];
+  float* lse;
+  int64_t sl[3];
+  uint32_t* status;
+};
+
+// Shared-memory map of the forward kernel (offsets from a 1024-aligned base).
+constexpr uint32_t kTileBytes = kBN * kD * 2;  // 32 KB: 128 rows x 128 bf16
+constexpr uint32_t kFwdQ = 0;
+constexpr uint32_t kFwdK = kFwdQ + kTileBytes;
+constexpr uint32_t kFwdV = kFwdK + kStages * kTileBytes;
+constexpr uint32_t kFwdP = kFwdV + kStages * kTileBytes;
+constexpr uint32_t kFwdCtl = kFwdP + kTileBytes;
+constexpr uint32_t kFwdSmem = kFwdCtl + 1024 + 1024;  // control block + alignment slack
+
+struct FwdCtl {
+  uint64_t q_full;
+  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, o_done;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+// Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
+__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int& lo, int& hi) {
+  const int nkt = (T + kBN - 1) / kBN;
+  lo = 0;
+  hi = nkt - 1;
+  if (m.flags & ATTN_MASK_CAUSAL) {
+    const int last = (q0 + kBM - 1 < T - 1 ? q0 + kBM - 1 : T - 1) / kBN;
+    hi = last < hi ? last : hi;
+  }
+  if (m.flags & ATTN_MASK_WINDOW) {
+    const int64_t first = (int64_t)q0 - m.window + 1;
+    lo = first > 0 ? (int)(first / kBN) : 0;
+  }
+}
+
+__global__ void __launch_bounds__(256, 1)
+fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+           const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  FwdCtl* ctl = reinterpret_cast<FwdCtl*>(smem + kFwdCtl);
+  volatile uint32_t* abort_flag = &ctl->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqt = (a.T + kBM - 1) / kBM;
+  const int bh = blockIdx.x % (a.B * a.Hq);
+  const int qt = nqt - 1 - (int)(blockIdx.x / (a.B * a.Hq));  // longest query tiles first
+  const int h = bh % a.Hq, b = bh / a.Hq;
+  const int kvh = h / (a.Hq / a.Hkv);
+  const int q0 = qt * kBM;
+  int kt_lo, kt_hi;
+  fwd_key_tiles(a.m, a.T, q0, kt_lo, kt_hi);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&ctl->q_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl->k_full[s]), 1);
+      mbar_init(smem_u32(&ctl->v_full[s]), 1);
+      mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&ctl->s_full[s]), 1);
+      mbar_init(smem_u32(&ctl->s_empty[s]), 128);
+    }
+    mbar_init(smem_u32(&ctl->p_full), 128);
+    mbar_init(smem_u32(&ctl->o_done), 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 256;  // S buffers at columns 0 and 128, O at 256
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    const uint32_t qf = smem_u32(&ctl->q_full);
+    mbar_expect_tx(qf, kTileBytes);
+    tma_load_4d(sbase + kFwdQ, &tq, qf, 0, q0, h, b);
+    tma_load_4d(sbase + kFwdQ + kTileBytes / 2, &tq, qf, 64, q0, h, b);
+    int n = 0;
+    for (int kt = kt_lo; kt <= kt_hi; ++kt) {
+      if (fwd_class(a.ct, a.m, a.T, b, h, qt, kt) == kEmpty) continue;
+      const int s = n % kStages;
+      if (!wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, a.status)) break;
+      const uint32_t kf = smem_u32(&ctl->k_full[s]), vf = smem_u32(&ctl->v_full[s]);
+      const uint32_t kd = sbase + kFwdK + s * kTileBytes, vd = sbase + kFwdV + s * kTileBytes;
+      mbar_expect_tx(kf, kTileBytes);
+      tma_load_4d(kd, &tk, kf, 0, kt * kBN, kvh, b);
+      tma_load_4d(kd + kTileBytes / 2, &tk, kf, 64, kt * kBN, kvh, b);
+      mbar_expect_tx(vf, kTileBytes);
+      tma_load_4d(vd, &tv, vf, 0, kt * kBN, kvh, b);
+      tma_load_4d(vd + kTileBytes / 2, &tv, vf, 64, kt * kBN, kvh, b);
+      ++n;
+    }
+    // Let every issued copy land before the CTA may leave (bounded).
+    for (int r = (n > kStages ? n - kStages : 0); r < n; ++r) {
+      const int s = r % kStages;
+      wait_bar(smem_u32(&ctl->k_full[s]), (r / kStages) & 1, abort_flag, nullptr);
+      wait_bar(smem_u32(&ctl->v_full[s]), (r / kStages) & 1, abort_flag, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);
+    bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
+    // Walk the nonempty tiles with one tile of look-ahead for S.
+    int kt_cur = kt_lo - 1, kt_next = kt_lo - 1;
+    auto next_tile = [&](int from) {
+      for (int kt = from + 1; kt <= kt_hi; ++kt)
+        if (fwd_class(a.ct, a.m, a.T, b, h, qt, kt) != kEmpty) return kt;
+      return kt_hi + 1;
+    };
+    auto issue_s = [&](int n) -> bool {
+      const int s = n % kStages;
+      if (!wait_bar(smem_u32(&ctl->k_full[s]), (n / kStages) & 1, abort_flag, a.status)) return false;
+      if (!wait_bar(smem_u32(&ctl->s_empty[n & 1]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint32_t d = tS + (n & 1) * 128;
+      const uint32_t qa = sbase + kFwdQ, ka = sbase + kFwdK + s * kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+        mma_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS, kk > 0);
+      }
+      mma_commit(smem_u32(&ctl->s_full[n & 1]));
+      return true;
+    };
+    if (ok) {
+      kt_next = next_tile(kt_cur);
+      int n = 0;
+      if (kt_next <= kt_hi) ok = issue_s(0);
+      while (ok && kt_next <= kt_hi) {
+        kt_cur = kt_next;
+        kt_next = next_tile(kt_cur);
+        if (kt_next <= kt_hi && !issue_s(n + 1)) break;
+        const int s = n % kStages;
+        if (!wait_bar(smem_u32(&ctl->p_full), n & 1, abort_flag, a.status)) break;
+        if (!wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t pa = sbase + kFwdP, va = sbase + kFwdV + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t poff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+          mma_ss(tO, smem_desc_sw128(pa + poff, 16, 1024), smem_desc_sw128(va + kk * 2048, kTileBytes / 2, 1024),
+                 idPV, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&ctl->o_done));
+        mma_commit(smem_u32(&ctl->kv_empty[s]));
+        ++n;
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax warpgroup: thread t owns query row q0 + t
+    const int t = threadIdx.x - 128;
+    const int row = q0 + t;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;  // base-2 running max and running sum
+    int n = 0;
+    bool ok = true;
+    const uint32_t pbase = sbase + kFwdP;
+    for (int kt = kt_lo; kt <= kt_hi && ok; ++kt) {
+      const uint8_t cls = fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
+      if (cls == kEmpty) continue;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[n & 1]), (n >> 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + lane_off + (n & 1) * 128 + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * a.scale_log2;
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->s_empty[n & 1]));
+      if (cls == kPartial) {
+        const int64_t j0 = (int64_t)kt * kBN;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int64_t j = j0 + c;
+          if (!(j < a.T && row < a.T && allowed(a.m, b, h, row, j))) s[c] = -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      float m_new = m_run;
+      if (mx > -INFINITY && (m_run == -INFINITY || mx > m_run + kRescaleThreshold)) m_new = fmaxf(mx, m_run);
+      const float alpha = (m_new == m_run) ? 1.f : ex2(m_run - m_new);  // 0 when m_run = -inf
+      const float msub = m_new == -INFINITY ? 0.f : m_new;
+      float sum = 0.f;
+      uint32_t pk[64];
+      if (a.m.dropout) {
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const int64_t j = (int64_t)kt * kBN + c4 * 4;
+          const uint4 w = philox4x32_10(make_uint4((uint32_t)(j >> 2), (uint32_t)row, (uint32_t)h, (uint32_t)b),
+                                        a.m.seed_lo, a.m.seed_hi);
+          float p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            p[e] = ex2(s[c4 * 4 + e] - msub);
+            sum += p[e];
+          }
+          // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
+          p[0] = w.x >= a.m.keep_thr ? p[0] : 0.f;
+          p[1] = w.y >= a.m.keep_thr ? p[1] : 0.f;
+          p[2] = w.z >= a.m.keep_thr ? p[2] : 0.f;
+          p[3] = w.w >= a.m.keep_thr ? p[3] : 0.f;
+          pk[c4 * 2] = pack_bf16(p[0], p[1]);
+          pk[c4 * 2 + 1] = pack_bf16(p[2], p[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          const float p0 = ex2(s[2 * c2] - msub), p1 = ex2(s[2 * c2 + 1] - msub);
+          sum += p0 + p1;
+          pk[c2] = pack_bf16(p0, p1);
+        }
+      }
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+      // PV of the previous tile must finish before O is rescaled and P reused.
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_done), (n - 1) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + lane_off + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tO + lane_off + c * 32, r);
+          }
+          tmem_wait_st();
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const uint32_t addr = pbase + (cc >> 3) * (kTileBytes / 2) + sw128_offset(t, (cc & 7) * 16);
+        st_shared_v4(addr, pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->p_full));
+      ++n;
+    }
+    // ---------------- epilogue: Y = u / (l + exp(z - m)), LSE = m + ln(...)
+    float o_row[128];
+    bool have_o = false;
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_done), (n - 1) & 1, abort_flag, a.status));
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o_row[c * 32 + e] = __uint_as_float(r[e]);
+        }
+        have_o = true;
+      }
+    }
+    if (ok && row < a.T) {
+      const bool has_sink = a.m.sink != nullptr;
+      const float z2 = has_sink ? a.m.sink[h] * kLog2e : -INFINITY;
+      float lse2, oscale;
+      if (m_run == -INFINITY || !have_o) {
+        lse2 = has_sink ? z2 : -INFINITY;
+        oscale = 0.f;
+      } else {
+        const float M = has_sink ? fmaxf(m_run, z2) : m_run;
+        const float tot = l_run * exp2f(m_run - M) + (has_sink ? exp2f(z2 - M) : 0.f);
+        oscale = exp2f(m_run - M) / tot;
+        if (a.m.dropout) oscale *= a.m.inv_keep;
+        lse2 = M + log2f(tot);
+      }
+      __nv_bfloat16* orow = a.o + b * a.so[0] + h * a.so[1] + (int64_t)row * a.so[2];
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8) {
+        uint4 v;
+        v.x = pack_bf16(have_o ? o_row[c8 * 8 + 0] * oscale : 0.f, have_o ? o_row[c8 * 8 + 1] * oscale : 0.f);
+        v.y = pack_bf16(have_o ? o_row[c8 * 8 + 2] * oscale : 0.f, have_o ? o_row[c8 * 8 + 3] * oscale : 0.f);
+        v.z = pack_bf16(have_o ? o_row[c8 * 8 + 4] * oscale : 0.f, have_o ? o_row[c8 * 8 + 5] * oscale : 0.f);
+        v.w = pack_bf16(have_o ? o_row[c8 * 8 + 6] * oscale : 0.f, have_o ? o_row[c8 * 8 + 7] * oscale : 0.f);
+        *reinterpret_cast<uint4*>(orow + c8 * 8) = v;
+      }
+      a.lse[b * a.sl[0] + h * a.sl[1] + (int64_t)row * a.sl[2]] = lse2 / kLog2e;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------- reverse
+
+struct BwdArgs {
+  MaskP m;
+  ClassTable ct;
+  int B, Hq, Hkv, T, Tpad;
+  float scale_log2;
+  const float* lse2;    // [B*Hq, Tpad] base-2 LSE (+inf on rows without keys)
+  const float* dpad;    // [B*Hq, Tpad] delta, zero on padding rows
+  float* dq_acc;        // [B, Hq, T, 128] fp32
+  __nv_bfloat16* dk;
+  int64_t sdk[3];
+  __nv_bfloat16* dv;
+  int64_t sdv[3];
+  float scale;
+  uint32_t* status;
+};
+
+constexpr uint32_t kHalfQ = kBMb * 64 * 2;  // 8 KB: 64 rows x 64 bf16
+constexpr uint32_t kQTile = kBMb * kD * 2;  // 16 KB: 64 rows x 128 bf16
+constexpr uint32_t kBwdK = 0;
+constexpr uint32_t kBwdV = kBwdK + kTileBytes;
+constexpr uint32_t kBwdQ = kBwdV + kTileBytes;              // kStages x 16 KB
+constexpr uint32_t kBwdG = kBwdQ + kStages * kQTile;        // kStages x 16 KB
+constexpr uint32_t kBwdPT = kBwdG + kStages * kQTile;       // 128 keys x 64 q bf16 = 16 KB
+constexpr uint32_t kBwdDS = kBwdPT + kBN * kBMb * 2;        // 16 KB
+constexpr uint32_t kBwdDQ = kBwdDS + kBN * kBMb * 2;        // 64 x 128 fp32 = 32 KB
+constexpr uint32_t kBwdStat = kBwdDQ + kBMb * kD * 4;       // kStages x (64 lse2 + 64 delta) fp32
+constexpr uint32_t kBwdCtl = kBwdStat + kStages * 512;
+constexpr uint32_t kBwdSmem = kBwdCtl + 1024 + 1024;
+
+struct BwdCtl {
+  uint64_t kv_full;
+  uint64_t q_full[kStages], q_empty[kStages];
+  uint64_t st_full, st_empty;
+  uint64_t ds_full, pds_empty;
+  uint64_t dq_full, dq_empty;
+  uint64_t acc_done;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+// Query-slice range [lo, hi] that can hold rows seeing keys [k0, k0 + 128).
+__device__ __forceinline__ void bwd_query_slices(const MaskP& m, int T, int k0, int& lo, int& hi) {
+  const int nqs = (T + kBMb - 1) / kBMb;
+  lo = 0;
+  hi = nqs - 1;
+  if (m.flags & ATTN_MASK_CAUSAL) lo = k0 / kBMb;
+  if (m.flags & ATTN_MASK_WINDOW) {
+    const int64_t last = (int64_t)k0 + kBN - 1 + m.window - 1;
+    if (last < T) hi = (int)(last / kBMb);
+  }
+}
+
+__device__ __forceinline__ void red_bulk_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(gdst)),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void wg_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(256, 1)
+bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  BwdCtl* ctl = reinterpret_cast<BwdCtl*>(smem + kBwdCtl);
+  volatile uint32_t* abort_flag = &ctl->abort_flag;
+  float* stat = reinterpret_cast<float*>(smem + kBwdStat);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int group = a.Hq / a.Hkv;
+  const int bkv = blockIdx.x % (a.B * a.Hkv);
+  const int kt = (int)(blockIdx.x / (a.B * a.Hkv));  // earliest key tiles (most work) first
+  const int kvh = bkv % a.Hkv, b = bkv / a.Hkv;
+  const int k0 = kt * kBN;
+  int qs_lo, qs_hi;
+  bwd_query_slices(a.m, a.T, k0, qs_lo, qs_hi);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&ctl->kv_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl->q_full[s]), 1);
+      mbar_init(smem_u32(&ctl->q_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->st_full), 1);
+    mbar_init(smem_u32(&ctl->st_empty), 128);
+    mbar_init(smem_u32(&ctl->ds_full), 128);
+    mbar_init(smem_u32(&ctl->pds_empty), 1);
+    mbar_init(smem_u32(&ctl->dq_full), 1);
+    mbar_init(smem_u32(&ctl->dq_empty), 128);
+    mbar_init(smem_u32(&ctl->acc_done), 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  // TMEM columns: S^T 0..63, dP^T 64..127, dV 128..255, dK 256..383, dQ^T 384..447
+  const uint32_t tST = tmem, tDPT = tmem + 64, tDV = tmem + 128, tDK = tmem + 256, tDQ = tmem + 384;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&tg);
+    const uint32_t kvf = smem_u32(&ctl->kv_full);
+    mbar_expect_tx(kvf, 2 * kTileBytes);
+    tma_load_4d(sbase + kBwdK, &tk, kvf, 0, k0, kvh, b);
+    tma_load_4d(sbase + kBwdK + kTileBytes / 2, &tk, kvf, 64, k0, kvh, b);
+    tma_load_4d(sbase + kBwdV, &tv, kvf, 0, k0, kvh, b);
+    tma_load_4d(sbase + kBwdV + kTileBytes / 2, &tv, kvf, 64, k0, kvh, b);
+    int n = 0;
+    bool ok = true;
+    for (int hh = 0; hh < group && ok; ++hh) {
+      const int h = kvh * group + hh;
+      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
+        if (lookup_class(a.ct, a.m, a.T, b, h, qs, kt) == kEmpty) continue;
+        const int s = n % kStages;
+        if (!(ok = wait_bar(smem_u32(&ctl->q_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, a.status))) break;
+        const uint32_t qf = smem_u32(&ctl->q_full[s]);
+        mbar_expect_tx(qf, 2 * kQTile + 512);
+        const uint32_t qd = sbase + kBwdQ + s * kQTile, gd = sbase + kBwdG + s * kQTile;
+        tma_load_4d(qd, &tq, qf, 0, qs * kBMb, h, b);
+        tma_load_4d(qd + kHalfQ, &tq, qf, 64, qs * kBMb, h, b);
+        tma_load_4d(gd, &tg, qf, 0, qs * kBMb, h, b);
+        tma_load_4d(gd + kHalfQ, &tg, qf, 64, qs * kBMb, h, b);
+        const int64_t roff = ((int64_t)b * a.Hq + h) * a.Tpad + (int64_t)qs * kBMb;
+        bulk_load(sbase + kBwdStat + s * 512, a.lse2 + roff, 256, qf);
+        bulk_load(sbase + kBwdStat + s * 512 + 256, a.dpad + roff, 256, qf);
+        ++n;
+      }
+    }
+    for (int r = (n > kStages ? n - kStages : 0); r < n; ++r)
+      wait_bar(smem_u32(&ctl->q_full[r % kStages]), (r / kStages) & 1, abort_flag, nullptr);
+    wait_bar(kvf, 0, abort_flag, nullptr);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idST = idesc_bf16(128, 64, 0, 0);   // K Q^T, V dO^T
+    constexpr uint32_t idACC = idesc_bf16(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
+    constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
+    bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
+    int n = 0;
+    for (int hh = 0; hh < group && ok; ++hh) {
+      const int h = kvh * group + hh;
+      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
+        if (lookup_class(a.ct, a.m, a.T, b, h, qs, kt) == kEmpty) continue;
+        const int s = n % kStages;
+        if (!(ok = wait_bar(smem_u32(&ctl->q_full[s]), (n / kStages) & 1, abort_flag, a.status))) break;
+        if (!(ok = wait_bar(smem_u32(&ctl->st_empty), (n & 1) ^ 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
+          mma_ss(tST, smem_desc_sw128(sbase + kBwdK + koff, 16, 1024), smem_desc_sw128(qa + qoff, 16, 1024), idST,
+                 kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
+          mma_ss(tDPT, smem_desc_sw128(sbase + kBwdV + koff, 16, 1024), smem_desc_sw128(ga + qoff, 16, 1024),
+                 idST, kk > 0);
+        }
+        mma_commit(smem_u32(&ctl->st_full));
+        if (!(ok = wait_bar(smem_u32(&ctl->ds_full), n & 1, abort_flag, a.status))) break;
+        if (!(ok = wait_bar(smem_u32(&ctl->dq_empty), (n & 1) ^ 1, abort_flag, a.status))) break;
+        tc_fence_after();
+        const uint32_t pta = sbase + kBwdPT, dsa = sbase + kBwdDS;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = 64 query rows
+          mma_ss(tDV, smem_desc_sw128(pta + kk * 32, 16, 1024), smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kHalfQ, 1024), idACC,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = 128 keys
+          mma_ss(tDQ, smem_desc_sw128(sbase + kBwdK + kk * 2048, kTileBytes / 2, 1024),
+                 smem_desc_sw128(dsa + kk * 2048, kHalfQ, 1024), idDQ, kk > 0);
+        }
+        mma_commit(smem_u32(&ctl->q_empty[s]));
+        mma_commit(smem_u32(&ctl->pds_empty));
+        mma_commit(smem_u32(&ctl->dq_full));
+        ++n;
+      }
+    }
+    mma_commit(smem_u32(&ctl->acc_done));
+  } else if (warp >= 4) {
+    // ---------------- compute warpgroup: thread t owns key row k0 + t
+    // (and, for the dQ^T readback, head-dimension index t)
+    const int t = threadIdx.x - 128;
+    const int64_t j = (int64_t)k0 + t;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float* dq_stage = reinterpret_cast<float*>(smem + kBwdDQ);
+    int n = 0;
+    bool ok = true;
+    for (int hh = 0; hh < group && ok; ++hh) {
+      const int h = kvh * group + hh;
+      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
+        const uint8_t cls = lookup_class(a.ct, a.m, a.T, b, h, qs, kt);
+        if (cls == kEmpty) continue;
+        const int s = n % kStages;
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full), n & 1, abort_flag, a.status)))) break;
+        if (!(ok = __all_sync(0xffffffffu,
+                              wait_bar(smem_u32(&ctl->q_full[s]), (n / kStages) & 1, abort_flag, a.status))))
+          break;
+        tc_fence_after();
+        float sv[64], dp[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tST + lane_off + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
+          tmem_ld32(tDPT + lane_off + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) dp[c * 32 + e] = __uint_as_float(r[e]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl->st_empty));
+        const float* lse2 = stat + s * 128;
+        const float* dl = lse2 + 64;
+        const int64_t i0 = (int64_t)qs * kBMb;
+        uint32_t ppk[32], dpk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          float pt[2], ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * c2 + e;
+            const int64_t i = i0 + c;
+            bool alw = true;
+            if (cls == kPartial) alw = i < a.T && j < a.T && allowed(a.m, b, h, i, j);
+            float p = alw ? ex2(sv[c] * a.scale_log2 - lse2[c]) : 0.f;
+            float dpv = dp[c];
+            float ptil = p;
+            if (a.m.dropout) {
+              // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
+              const bool keep = dropout_keep(a.m, b, h, i, j);
+              ptil = keep ? p : 0.f;
+              dpv = keep ? dpv * a.m.inv_keep : 0.f;
+            }
+            pt[e] = ptil;
+            ds[e] = p * (dpv - dl[c]);
+          }
+          ppk[c2] = pack_bf16(pt[0], pt[1]);
+          dpk[c2] = pack_bf16(ds[0], ds[1]);
+        }
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty), (n & 1) ^ 1, abort_flag, a.status))))
+          break;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const uint32_t off = sw128_offset(t, cc * 16);
+          st_shared_v4(sbase + kBwdPT + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
+          st_shared_v4(sbase + kBwdDS + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl->ds_full));
+        // dQ^T tile: thread t holds head-dimension t for 64 query rows.
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_full), n & 1, abort_flag, a.status)))) break;
+        tc_fence_after();
+        // The previous step's bulk reduce must have read the staging buffer.
+        if (t == 0) bulk_wait_read0();
+        wg_sync();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tDQ + lane_off + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) dq_stage[(c * 32 + e) * kD + t] = __uint_as_float(r[e]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl->dq_empty));
+        fence_proxy_async_smem();
+        wg_sync();
+        if (t == 0) {
+          const int rows = (int)((a.T - i0) < kBMb ? (a.T - i0) : kBMb);
+          float* dst = a.dq_acc + (((int64_t)b * a.Hq + h) * a.T + i0) * kD;
+          red_bulk_add_f32(dst, sbase + kBwdDQ, (uint32_t)rows * kD * 4);
+          bulk_commit();
+        }
+        ++n;
+      }
+    }
+    if (t == 0) bulk_wait0();
+    // ---------------- epilogue: dK = c * sum gamma^T Q, dV = sum P~^T dO
+    bool have = false;
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->acc_done), 0, abort_flag, a.status));
+      if (ok) tc_fence_after();
+      have = ok;
+    }
+    const float dv_scale = a.m.dropout ? a.m.inv_keep : 1.f;
+    if (ok || n == 0) {
+      __nv_bfloat16* dkr = a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2];
+      __nv_bfloat16* dvr = a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rk[32], rv[32];
+        if (have) {
+          tmem_ld32(tDK + lane_off + c * 32, rk);
+          tmem_ld32(tDV + lane_off + c * 32, rv);
+          tmem_wait_ld();
+        }
+        if (j < a.T) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 vk, vv;
+            uint32_t* pk = &vk.x;
+            uint32_t* pv = &vv.x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int idx = c8 * 8 + e * 2;
+              pk[e] = have ? pack_bf16(__uint_as_float(rk[idx]) * a.scale, __uint_as_float(rk[idx + 1]) * a.scale)
+                           : 0u;
+              pv[e] = have ? pack_bf16(__uint_as_float(rv[idx]) * dv_scale, __uint_as_float(rv[idx + 1]) * dv_scale)
+                           : 0u;
+            }
+            *reinterpret_cast<uint4*>(dkr + c * 32 + c8 * 8) = vk;
+            *reinterpret_cast<uint4*>(dvr + c * 32 + c8 * 8) = vv;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Reverse-pass preparation, one warp per (b, h, row < Tpad): delta from the
+// stored O and dO, the base-2 LSE, and a zeroed dQ accumulator row.
+__global__ void __launch_bounds__(256)
+bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2, const __nv_bfloat16* g,
+                   int64_t sg0, int64_t sg1, int64_t sg2, const float* lse, int64_t sl0, int64_t sl1, int64_t sl2,
+                   int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta, float* dq_acc) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (int64_t)B * Hq * Tpad) return;
+  const int i = (int)(w % Tpad);
+  const int64_t bh = w / Tpad;
+  const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+  if (i >= T) {
+    if (lane == 0) {
+      lse2[w] = INFINITY;
+      dpad[w] = 0.f;
+    }
+    return;
+  }
+  const __nv_bfloat16* orow = o + b * so0 + h * so1 + (int64_t)i * so2;
+  const __nv_bfloat16* grow = g + b * sg0 + h * sg1 + (int64_t)i * sg2;
+  const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
+  const uint2 gv = *reinterpret_cast<const uint2*>(grow + lane * 4);
+  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+  const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float2 a2 = __bfloat1622float2(o2[e]), b2 = __bfloat1622float2(g2[e]);
+    s = fmaf(a2.x, b2.x, s);
+    s = fmaf(a2.y, b2.y, s);
+  }
+  s = warp_sum(s);
+  float4* dqr = reinterpret_cast<float4*>(dq_acc + (bh * T + i) * kD);
+  dqr[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    const float L = lse[b * sl0 + h * sl1 + (int64_t)i * sl2];
+    lse2[w] = L == -INFINITY ? INFINITY : L * kLog2e;
+    dpad[w] = s;
+    delta[bh * T + i] = s;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, __nv_bfloat16* dq, int64_t s0, int64_t s1,
+                 int64_t s2) {
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e >= (int64_t)B * Hq * T * kD) return;
+  const int c = (int)(e % kD);
+  const int64_t r = e / kD;
+  const int i = (int)(r % T);
+  const int h = (int)((r / T) % Hq);
+  const int b = (int)(r / ((int64_t)T * Hq));
+  const float4 v = *reinterpret_cast<const float4*>(dq_acc + e);
+  uint2 out;
+  out.x = pack_bf16(v.x * scale, v.y * scale);
+  out.y = pack_bf16(v.z * scale, v.w * scale);
+  *reinterpret_cast<uint2*>(dq + b * s0 + h * s1 + (int64_t)i * s2 + c) = out;
+}
+
+// ----------------------------------------------------------- host helpers
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 4-D bf16 map over (d, T, H, B) with a (64, rows, 1, 1) box and 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int T, int H, int B, int64_t st, int64_t sh, int64_t sb,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)st * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tma_ok(const attn_tensor* t) {
+  if (!t || t->dtype != ATTN_BF16 || t->ndim != 4 || t->stride[3] != 1) return false;
+  if (reinterpret_cast<uintptr_t>(t->data) % 16) return false;
+  for (int i = 0; i < 3; ++i) {
+    if ((t->stride[i] * 2) % 16) return false;
+    if (t->stride[i] <= 0 && t->shape[i] > 1) return false;
+  }
+  return true;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
+  static bool done[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done[which][dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < 64) done[which][dev] = true;
+  return e;
+}
+
+size_t class_bytes(int B, int Hq, int T, const attn_mask* m) {
+  if (!m || !(m->flags & ATTN_MASK_BLOCK)) return 0;
+  const int nb = m->bm_stride_b ? B : 1, nh = m->bm_stride_h ? Hq : 1;
+  const size_t nqs = (T + kBMb - 1) / kBMb, nkt = (T + kBN - 1) / kBN;
+  return align_up((size_t)nb * nh * nqs * nkt, 256);
+}
+
+ClassTable build_class_table(const DenseP& p, void* ws, cudaStream_t st, cudaError_t& err) {
+  ClassTable ct;
+  ct.cls = nullptr;
+  ct.nb = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sb ? p.B : 1;
+  ct.nh = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sh ? p.Hq : 1;
+  ct.nqs = (p.T + kBMb - 1) / kBMb;
+  ct.nkt = (p.T + kBN - 1) / kBN;
+  err = cudaSuccess;
+  if (!(p.m.flags & ATTN_MASK_BLOCK)) return ct;
+  uint8_t* out = static_cast<uint8_t*>(ws);
+  const int64_t n = (int64_t)ct.nb * ct.nh * ct.nqs * ct.nkt;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  classify_kernel<<<blocks, 256, 0, st>>>(p.m, p.T, p.B, p.Hq, ct, out);
+  err = cudaGetLastError();
+  ct.cls = out;
+  return ct;
+}
+
+}  // namespace
+
+size_t sm100_fwd_workspace_bytes(int B, int Hq, int T, const attn_mask* m) { return class_bytes(B, Hq, T, m); }
+
+size_t sm100_bwd_extra_workspace_bytes(int B, int Hq, int Hkv, int T, const attn_mask* m) {
+  (void)Hkv;
+  const size_t Tpad = (size_t)((T + kBN - 1) / kBN) * kBN;
+  return 2 * align_up((size_t)B * Hq * Tpad * sizeof(float), 256) + class_bytes(B, Hq, T, m);
+}
+
+bool sm100_dense_supported(const DenseP& p, const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
+                           const attn_tensor* o) {
+  if (p.d != kD || p.dv != kD || p.T < 1) return false;
+  if (!tma_ok(q) || !tma_ok(k) || !tma_ok(v) || !tma_ok(o)) return false;
+  if (!encode_fn()) return false;
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0;
+}
+
+bool sm100_dense_bwd_supported(const DenseP&, const attn_tensor* do_, const attn_tensor* dq, const attn_tensor* dk,
+                               const attn_tensor* dv) {
+  return tma_ok(do_) && tma_ok(dq) && tma_ok(dk) && tma_ok(dv);
+}
+
+cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float* lse, const int64_t sl[3], void* ws,
+                            uint32_t* status, cudaStream_t st) {
+  cudaError_t err;
+  ClassTable ct = build_class_table(p, ws, st, err);
+  if (err != cudaSuccess) return err;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM) ||
+      !make_map(&mk, p.k, p.T, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
+      !make_map(&mv, p.v, p.T, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN))
+    return cudaErrorInvalidValue;
+  FwdArgs a;
+  a.m = p.m;
+  a.ct = ct;
+  a.B = p.B;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.T = p.T;
+  a.scale_log2 = p.scale * kLog2e;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  for (int i = 0; i < 3; ++i) {
+    a.so[i] = so[i];
+    a.sl[i] = sl[i];
+  }
+  a.lse = lse;
+  a.status = status;
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(fwd_kernel), kFwdSmem, 0)) != cudaSuccess) return err;
+  const int nqt = (p.T + kBM - 1) / kBM;
+  fwd_kernel<<<nqt * p.B * p.Hq, 256, kFwdSmem, st>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3], const void* g, const int64_t sg[3],
+                            const float* lse, const int64_t sl[3], float* delta, float* dq_acc, void* dq,
+                            const int64_t sdq[3], void* dk, const int64_t sdk[3], void* dv, const int64_t sdv[3],
+                            void* ws_extra, uint32_t* status, cudaStream_t st) {
+  const int Tpad = ((p.T + kBN - 1) / kBN) * kBN;
+  const size_t padb = align_up((size_t)p.B * p.Hq * Tpad * sizeof(float), 256);
+  float* lse2 = static_cast<float*>(ws_extra);
+  float* dpad = reinterpret_cast<float*>(static_cast<char*>(ws_extra) + padb);
+  cudaError_t err;
+  ClassTable ct = build_class_table(p, static_cast<char*>(ws_extra) + 2 * padb, st, err);
+  if (err != cudaSuccess) return err;
+  const int64_t rows = (int64_t)p.B * p.Hq * Tpad;
+  bwd_prepare_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), so[0], so[1], so[2], static_cast<const __nv_bfloat16*>(g), sg[0], sg[1],
+      sg[2], lse, sl[0], sl[1], sl[2], p.B, p.Hq, p.T, Tpad, lse2, dpad, delta, dq_acc);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  CUtensorMap mq, mk, mv, mg;
+  if (!make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
+      !make_map(&mk, p.k, p.T, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
+      !make_map(&mv, p.v, p.T, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN) ||
+      !make_map(&mg, g, p.T, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb))
+    return cudaErrorInvalidValue;
+  BwdArgs a;
+  a.m = p.m;
+  a.ct = ct;
+  a.B = p.B;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.T = p.T;
+  a.Tpad = Tpad;
+  a.scale_log2 = p.scale * kLog2e;
+  a.lse2 = lse2;
+  a.dpad = dpad;
+  a.dq_acc = dq_acc;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  for (int i = 0; i < 3; ++i) {
+    a.sdk[i] = sdk[i];
+    a.sdv[i] = sdv[i];
+  }
+  a.scale = p.scale;
+  a.status = status;
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
+  const int nkt = (p.T + kBN - 1) / kBN;
+  bwd_kernel<<<nkt * p.B * p.Hkv, 256, kBwdSmem, st>>>(mq, mk, mv, mg, a);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int64_t n4 = (int64_t)p.B * p.Hq * p.T * kD / 4;
+  dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.T, p.scale,
+                                                                 static_cast<__nv_bfloat16*>(dq), sdq[0], sdq[1],
+                                                                 sdq[2]);
+  return cudaGetLastError();
 }
 
 }  // namespace attn

@@ -168,15 +168,19 @@ def test_worked_examples_on_gpu():
     assert np.allclose(o[0, 0, 3].cpu().numpy(), gd["tiled_output_row3"], rtol=1e-6)
     # Sink: o = 0.7, dS = (0.65, -0.51), dz = -0.14 (dense realisation).
     e = ex["sink"]
-    q = _f32([[1.0]])[None, None]
+    # The dense layout has as many query rows as keys: a second query row with
+    # zero upstream gradient contributes nothing to any gradient.
+    q = _f32([[1.0], [0.3]])[None, None]
     k = _f32([[math.log(e["p"][0])], [math.log(e["p"][1])]])[None, None]
     v = _f32([[e["v"][0]], [e["v"][1]]])[None, None]
-    g = _f32([[e["g"]]])[None, None]
+    g = _f32([[e["g"]], [0.0]])[None, None]
     al = eta.AllowedSet(sink=_f32([math.log(e["p_sink"])]))
     o, lse = eta.attn_fwd(q, k, v, al, 1.0)
     dq, dk, dv, ds = eta.attn_bwd(q, k, v, o, g, lse, al, 1.0)
-    assert abs(o.item() - e["o"]) <= 1e-6
+    assert abs(o[0, 0, 0, 0].item() - e["o"]) <= 1e-6
+    assert abs(lse[0, 0, 0].item()) <= 1e-6
     assert np.allclose(dk.flatten().cpu().numpy(), e["dS"], atol=1e-6)
+    assert np.allclose(dv.flatten().cpu().numpy(), e["p"], atol=1e-6)
     assert abs(ds.item() - e["dz"]) <= 1e-6
 
 
@@ -191,7 +195,7 @@ def test_dropout_replay_example_on_gpu():
     o, lse = eta.attn_fwd(q, k, v, al, 1.0)
     dq, dk, dv, _ = eta.attn_bwd(q, k, v, o, g, lse, al, 1.0)
     assert abs(o[0, 0, 0, 0].item() - 2.0) <= 1e-6
-    assert np.allclose(dv.flatten().cpu().numpy(), e["dv"], atol=1e-6)
+    assert np.allclose(dv.flatten().cpu().numpy(), np.ravel(e["dv"]), atol=1e-6)
 
 
 def _topk_small(dtype, seed, Tq=40, Tkv=300, H=8, Dqk=96, Dv=64, topk=128, lo=20, hi=128, sink=True):

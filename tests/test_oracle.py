@@ -420,3 +420,49 @@ def test_oracle_detects_planted_mistakes():
     finally:
         A.backward = orig
     assert np.abs(good.dq).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Row/column-restricted evaluation equals the full definition
+# ---------------------------------------------------------------------------
+
+def test_sampled_rows_and_columns_match_full_oracle():
+    from oracle import sampled as S
+    rng = np.random.default_rng(17)
+    B, Hq, Hkv, T, d, dv = 1, 4, 2, 37, 6, 5
+    q = rng.standard_normal((B, Hq, T, d))
+    k = rng.standard_normal((B, Hkv, T, d))
+    v = rng.standard_normal((B, Hkv, T, dv))
+    g = rng.standard_normal((B, Hq, T, dv))
+    sink = rng.standard_normal(Hq)
+    rho, seed, c = 0.2, 77, 0.45
+    bm = rng.random((5, 5)) < 0.6
+    np.fill_diagonal(bm, True)
+    kw = dict(causal=True, window_left=11, block_mask=bm, block_q=8, block_k=8)
+    allow = A.allowed_dense(T, T, **kw)
+    keep = P.dropout_keep(seed, rho, B, Hq, T, T)
+    fw = A.forward(q, k, v, allow, c, sink=sink, keep=keep, rho=rho)
+    bw = A.backward(q, k, v, g, allow, c, sink=sink, keep=keep, rho=rho)
+    rows = np.array([0, 3, 17, 36])
+    cols = np.array([1, 20, 36])
+    gq = Hq // Hkv
+    for h in range(Hq):
+        ar = S.allowed_at(rows, np.arange(T), **kw)
+        assert np.array_equal(ar, allow[rows])
+        kr = S.keep_at(seed, rho, 0, h, rows, np.arange(T))
+        assert np.array_equal(kr, keep[0, h][rows])
+        y, lse, delta, dq = S.rows_forward_backward(q[0, h], k[0, h // gq], v[0, h // gq], g[0, h], rows, ar, c,
+                                                    z=sink[h], keep_rows=kr, rho=rho)
+        assert np.allclose(y, fw.y[0, h][rows], atol=1e-13)
+        assert np.allclose(lse, fw.lse[0, h][rows], atol=1e-13)
+        assert np.allclose(dq, bw.dq[0, h][rows], atol=1e-12)
+        assert np.allclose(delta, bw.delta[0, h][rows], atol=1e-12)
+    for kvh in range(Hkv):
+        heads = [kvh * gq + hh for hh in range(gq)]
+        dk, dvv = S.cols_backward(
+            [q[0, h] for h in heads], [g[0, h] for h in heads], k[0, kvh], v[0, kvh], cols,
+            lambda hh, r, cc: S.allowed_at(r, cc, **kw),
+            [fw.lse[0, h] for h in heads], [bw.delta[0, h] for h in heads], c,
+            keep_fn=lambda hh, r, cc, hs=heads: S.keep_at(seed, rho, 0, hs[hh], r, cc), rho=rho)
+        assert np.allclose(dk, bw.dk[0, kvh][cols], atol=1e-12)
+        assert np.allclose(dvv, bw.dv[0, kvh][cols], atol=1e-12)
