@@ -15,7 +15,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "AllowedSet", "AttnError", "attn_fwd", "attn_bwd", "attn_fwd_workspace_size",
+    "AllowedSet", "AttnError", "attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_fwd_workspace_size",
     "attn_bwd_workspace_size", "attn_get_status", "attn_status_string", "attn_version",
     "library_path", "load_library",
 ]
@@ -87,6 +87,8 @@ def load_library():
     lib.attn_fwd.argtypes = [T, T, T, M, ctypes.c_float, T, T, vp, sz, vp]
     lib.attn_bwd.restype = ctypes.c_int
     lib.attn_bwd.argtypes = [T, T, T, T, T, T, M, ctypes.c_float, T, T, T, vp, vp, sz, vp]
+    lib.attn_bwd_noalloc.restype = ctypes.c_int
+    lib.attn_bwd_noalloc.argtypes = [T, T, T, T, T, T, M, ctypes.c_float, T, T, T, vp, vp]
     lib.attn_get_status.restype = ctypes.c_int
     lib.attn_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     _LIB = lib
@@ -262,6 +264,26 @@ def attn_bwd(q, k, v, o, do, lse, allowed: AllowedSet | None = None, scale: floa
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_bwd")
     return dq, dk, (None if topk else dv), dsink
+
+
+def attn_bwd_noalloc(q, k, v, o, do, lse, allowed: AllowedSet | None = None, scale: float | None = None, *,
+                     dq, dk, dv=None, dsink=None, stream=None):
+    """Reverse pass whose scratch is the library's fixed 64 MiB device array
+    (for callers that cannot allocate device memory). The caller passes every
+    output buffer; nothing is allocated here or in the library. Returns
+    (dq, dk, dv, dsink)."""
+    lib = load_library()
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    m = allowed.to_c() if allowed else None
+    cq, ck, cv, co, cdo, cl = (_tensor(x) for x in (q, k, v, o, do, lse))
+    cdq, cdk, cdv = _tensor(dq), _tensor(dk), _tensor(dv)
+    rc = lib.attn_bwd_noalloc(_ref(cq), _ref(ck), _ref(cv), _ref(co), _ref(cdo), _ref(cl), _ref(m),
+                              ctypes.c_float(scale), _ref(cdq), _ref(cdk), _ref(cdv),
+                              dsink.data_ptr() if dsink is not None else None, _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd_noalloc")
+    return dq, dk, dv, dsink
 
 
 def attn_get_status(workspace: torch.Tensor, stream=None) -> int:

@@ -160,6 +160,31 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k,
                      attn_tensor* dk, attn_tensor* dv, float* dsink,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* Reverse pass without any device allocation, for callers that cannot call
+ * cudaMalloc: a host framework that owns every byte of device memory through
+ * its own allocator and budget, a plugin that may not allocate behind that
+ * framework's back, or a latency-bound loop where an allocation (which can
+ * synchronise the device) is not allowed. The pages have no counterpart to
+ * this entry point; it exists only for such callers.
+ *
+ * Same arguments and results as attn_bwd, minus the workspace: the scratch
+ * space is a fixed 64 MiB array inside the library's device memory (one per
+ * GPU that loads the library, held until the process exits). A problem whose
+ * attn_bwd_workspace_size exceeds 64 MiB is rejected with
+ * ATTN_ERR_WORKSPACE before anything is enqueued. The first call on each
+ * device looks up the array's device address with that device current; make
+ * that first call before any stream capture. Every call shares the one array
+ * and it keeps the previous call's contents (the pass clears what must start
+ * at zero itself), so calls whose GPU work overlaps in time, on different
+ * streams or from different threads, race on it: serialise them. The status
+ * word lives in that array too and cannot be read with attn_get_status. */
+attn_status attn_bwd_noalloc(const attn_tensor* q, const attn_tensor* k,
+                             const attn_tensor* v, const attn_tensor* o,
+                             const attn_tensor* do_, const attn_tensor* lse,
+                             const attn_mask* mask, float scale, attn_tensor* dq,
+                             attn_tensor* dk, attn_tensor* dv, float* dsink,
+                             void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word at the
  * start of `workspace`. *device_bits receives the ATTN_DEVERR_* bits (0 when
  * clean). Returns ATTN_ERR_DEVICE when any bit was set. */
