@@ -59,27 +59,29 @@ def allowed_pairs(case: W.DenseCase) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms; summary()
+    keeps the samples whose timestamps fall inside the timed window."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.window = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -89,18 +91,35 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
+    @staticmethod
+    def _epoch(stamp: str):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(stamp, fmt).timestamp()
+            except ValueError:
+                continue
+        return None
+
     def summary(self):
-        rows = [[c.strip() for c in ln.split(",")] for ln in getattr(self, "lines", [])]
-        rows = [r for r in rows if len(r) >= 9]
-        if not rows:
+        rows = [[c.strip() for c in ln.split(",")] for ln in self.lines]
+        rows = [r for r in rows if len(r) >= 10]
+        inside = rows
+        where = "all samples"
+        if self.window and rows:
+            t0, t1 = self.window
+            sel = [r for r in rows if (lambda e: e is not None and t0 - 0.05 <= e <= t1 + 0.05)(self._epoch(r[0]))]
+            if sel:
+                inside, where = sel, "timed window"
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        num = lambda x: x.replace(".", "", 1).isdigit()
+        sm = [float(r[2]) for r in inside if num(r[2])]
+        mx = [float(r[3]) for r in inside if num(r[3])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
-        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({names[k] for r in inside for k in range(4) if r[6 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside), "sampled": where}
 
 
 def cpu_baseline(case: W.DenseCase, budget_s: float = 12.0):
@@ -156,7 +175,7 @@ def run_reference(args, case, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="causal_8k", choices=["causal_8k", "causal_2k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -199,6 +218,8 @@ def main():
         eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
         eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
 
+    clk = ClockSampler(local).start()
+    time.sleep(0.5)  # nvidia-smi needs a moment before its first sample
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
@@ -209,7 +230,8 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    t_wall0 = time.time()
+    if True:
         for s in range(n_ev):
             flush.fill_(s & 0xFF)
             e0, e1, e2 = ev[s]
@@ -219,6 +241,9 @@ def main():
             eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
             e2.record(stream)
         torch.cuda.synchronize()
+    t_wall1 = time.time()
+    clk.stop()
+    clk.window = (t_wall0, t_wall1)
     if world > 1:
         dist.barrier()
     t_fwd = [a.elapsed_time(b) for a, b, _ in ev]

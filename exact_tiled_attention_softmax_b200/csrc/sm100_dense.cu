@@ -137,7 +137,8 @@ struct FwdArgs {
   MaskP m;
   ClassTable ct;
   int B, Hq, Hkv, T;
-  float scale_log2;  // c * log2(e)
+  int block_aligned;  // block mask constant over every (64-row slice, 128-key tile)
+  float scale_log2;   // c * log2(e)
   __nv_bfloat16* o;
   int64_t so[3];
   float* lse;
@@ -150,20 +151,21 @@ constexpr uint32_t kTileBytes = kBN * kD * 2;  // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t kFwdQ = 0;
 constexpr uint32_t kFwdK = kFwdQ + kTileBytes;
 constexpr uint32_t kFwdV = kFwdK + kStages * kTileBytes;
-constexpr uint32_t kFwdP = kFwdV + kStages * kTileBytes;
-constexpr uint32_t kFwdCtl = kFwdP + kTileBytes;
+constexpr uint32_t kFwdP = kFwdV + kStages * kTileBytes;  // 2 buffers
+constexpr uint32_t kFwdCtl = kFwdP + 2 * kTileBytes;
 constexpr uint32_t kFwdSmem = kFwdCtl + 1024 + 1024;  // control block + alignment slack
 
 struct FwdCtl {
   uint64_t q_full;
   uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, o_done;
+  uint64_t p_full[2], p_free[2];
+  uint64_t o_done, o_final;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
 
-// Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
+// Key-tile range that can hold allowed keys for rows [q0, q0 + 128).
 __device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int& lo, int& hi) {
   const int nkt = (T + kBN - 1) / kBN;
   lo = 0;
@@ -175,6 +177,61 @@ __device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int
   if (m.flags & ATTN_MASK_WINDOW) {
     const int64_t first = (int64_t)q0 - m.window + 1;
     lo = first > 0 ? (int)(first / kBN) : 0;
+  }
+}
+
+// Bits lo..hi (inclusive, within [0, 63]) of a 64-bit word; 0 when lo > hi.
+__device__ __forceinline__ uint64_t range_bits64(int64_t lo, int64_t hi) {
+  if (lo > hi || hi < 0 || lo > 63) return 0ull;
+  lo = lo < 0 ? 0 : lo;
+  hi = hi > 63 ? 63 : hi;
+  const uint64_t upto = hi >= 63 ? ~0ull : ((1ull << (hi + 1)) - 1ull);
+  return upto & ~((1ull << lo) - 1ull);
+}
+
+// Allowed keys of row i inside key tile [j0, j0 + 128) as two 64-bit words
+// (bit c <-> key j0 + c). The causal/window conditions give one interval;
+// a block mask that is constant over (64-row slice, 128-key tile) blocks is
+// already folded into the tile class, otherwise it is looked up per key.
+__device__ __forceinline__ void fwd_row_bits(const FwdArgs& a, int b, int h, int64_t i, int64_t j0, uint8_t slice_cls,
+                                             uint64_t& w0, uint64_t& w1) {
+  w0 = w1 = 0ull;
+  if (i >= a.T || slice_cls == kEmpty) return;
+  int64_t lo = j0, hi = j0 + kBN - 1;
+  if (hi > a.T - 1) hi = a.T - 1;
+  if (a.m.flags & ATTN_MASK_CAUSAL) hi = i < hi ? i : hi;
+  if (a.m.flags & ATTN_MASK_WINDOW) lo = i - a.m.window + 1 > lo ? i - a.m.window + 1 : lo;
+  if (lo > hi) return;
+  w0 = range_bits64(lo - j0, hi - j0);
+  w1 = range_bits64(lo - j0 - 64, hi - j0 - 64);
+  if ((a.m.flags & ATTN_MASK_BLOCK) && !a.block_aligned) {
+    const uint8_t* row = a.m.bm + b * a.m.bm_sb + h * a.m.bm_sh + (i / a.m.bq) * a.m.bm_sq;
+    uint64_t b0 = 0, b1 = 0;
+#pragma unroll 1
+    for (int c = 0; c < 64; ++c) {
+      if (j0 + c < a.T && row[(j0 + c) / a.m.bk]) b0 |= 1ull << c;
+      if (j0 + 64 + c < a.T && row[(j0 + 64 + c) / a.m.bk]) b1 |= 1ull << c;
+    }
+    w0 &= b0;
+    w1 &= b1;
+  }
+}
+
+// Keep bits xi for row i and keys [j0, j0 + 128): 32 Philox blocks of 4 keys.
+__device__ __forceinline__ void fwd_keep_bits(const MaskP& m, int b, int h, int64_t i, int64_t j0, uint64_t& k0,
+                                              uint64_t& k1) {
+  k0 = k1 = 0ull;
+#pragma unroll 1
+  for (int g = 0; g < 32; ++g) {
+    const int64_t j = j0 + 4 * g;
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)(j >> 2), (uint32_t)i, (uint32_t)h, (uint32_t)b), m.seed_lo,
+                                  m.seed_hi);
+    const uint64_t nib = (uint64_t)(w.x >= m.keep_thr) | ((uint64_t)(w.y >= m.keep_thr) << 1) |
+                         ((uint64_t)(w.z >= m.keep_thr) << 2) | ((uint64_t)(w.w >= m.keep_thr) << 3);
+    if (g < 16)
+      k0 |= nib << (4 * g);
+    else
+      k1 |= nib << (4 * (g - 16));
   }
 }
 
@@ -207,9 +264,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->s_full[s]), 1);
       mbar_init(smem_u32(&ctl->s_empty[s]), 128);
+      mbar_init(smem_u32(&ctl->p_full[s]), 128);
+      mbar_init(smem_u32(&ctl->p_free[s]), 1);
     }
-    mbar_init(smem_u32(&ctl->p_full), 128);
     mbar_init(smem_u32(&ctl->o_done), 1);
+    mbar_init(smem_u32(&ctl->o_final), 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -258,8 +317,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);
     bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
-    // Walk the nonempty tiles with one tile of look-ahead for S.
-    int kt_cur = kt_lo - 1, kt_next = kt_lo - 1;
     auto next_tile = [&](int from) {
       for (int kt = from + 1; kt <= kt_hi; ++kt)
         if (fwd_class(a.ct, a.m, a.T, b, h, qt, kt) != kEmpty) return kt;
@@ -280,19 +337,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       mma_commit(smem_u32(&ctl->s_full[n & 1]));
       return true;
     };
+    int n = 0;
     if (ok) {
-      kt_next = next_tile(kt_cur);
-      int n = 0;
+      int kt_next = next_tile(kt_lo - 1);
       if (kt_next <= kt_hi) ok = issue_s(0);
       while (ok && kt_next <= kt_hi) {
-        kt_cur = kt_next;
-        kt_next = next_tile(kt_cur);
-        if (kt_next <= kt_hi && !issue_s(n + 1)) break;
+        kt_next = next_tile(kt_next);
+        const bool last = kt_next > kt_hi;
+        if (!last && !issue_s(n + 1)) break;
         const int s = n % kStages;
-        if (!wait_bar(smem_u32(&ctl->p_full), n & 1, abort_flag, a.status)) break;
+        if (!wait_bar(smem_u32(&ctl->p_full[n & 1]), (n >> 1) & 1, abort_flag, a.status)) break;
         if (!wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t pa = sbase + kFwdP, va = sbase + kFwdV + s * kTileBytes;
+        const uint32_t pa = sbase + kFwdP + (n & 1) * kTileBytes, va = sbase + kFwdV + s * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t poff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
@@ -300,43 +357,48 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                  idPV, (n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(smem_u32(&ctl->o_done));
+        mma_commit(smem_u32(&ctl->p_free[n & 1]));
         mma_commit(smem_u32(&ctl->kv_empty[s]));
+        if (last) mma_commit(smem_u32(&ctl->o_final));
         ++n;
       }
     }
   } else if (warp >= 4) {
     // ---------------- softmax warpgroup: thread t owns query row q0 + t
     const int t = threadIdx.x - 128;
-    const int row = q0 + t;
+    const int64_t row = q0 + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;  // base-2 running max and running sum
     int n = 0;
     bool ok = true;
-    const uint32_t pbase = sbase + kFwdP;
     for (int kt = kt_lo; kt <= kt_hi && ok; ++kt) {
       const uint8_t cls = fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
       if (cls == kEmpty) continue;
+      uint64_t mw0 = ~0ull, mw1 = ~0ull;
+      if (cls == kPartial) {
+        mw0 = mw1 = 0ull;
+        if (row < a.T) {
+          const uint8_t scls = lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), kt);
+          fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, scls, mw0, mw1);
+        }
+      }
+      uint64_t kb0 = ~0ull, kb1 = ~0ull;
+      if (a.m.dropout) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[n & 1]), (n >> 1) & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      float s[128];
+      uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + lane_off + (n & 1) * 128 + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * a.scale_log2;
-      }
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + (n & 1) * 128 + c * 32, r[c]);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl->s_empty[n & 1]));
-      if (cls == kPartial) {
-        const int64_t j0 = (int64_t)kt * kBN;
+      float s[128];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int64_t j = j0 + c;
-          if (!(j < a.T && row < a.T && allowed(a.m, b, h, row, j))) s[c] = -INFINITY;
-        }
+      for (int c = 0; c < 128; ++c) {
+        const uint64_t w = c < 64 ? mw0 : mw1;
+        const float v = __uint_as_float(r[c >> 5][c & 31]) * a.scale_log2;
+        s[c] = ((w >> (c & 63)) & 1ull) ? v : -INFINITY;
       }
       float mx = -INFINITY;
 #pragma unroll
@@ -347,54 +409,37 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const float msub = m_new == -INFINITY ? 0.f : m_new;
       float sum = 0.f;
       uint32_t pk[64];
-      if (a.m.dropout) {
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
-          const int64_t j = (int64_t)kt * kBN + c4 * 4;
-          const uint4 w = philox4x32_10(make_uint4((uint32_t)(j >> 2), (uint32_t)row, (uint32_t)h, (uint32_t)b),
-                                        a.m.seed_lo, a.m.seed_hi);
-          float p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            p[e] = ex2(s[c4 * 4 + e] - msub);
-            sum += p[e];
-          }
-          // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
-          p[0] = w.x >= a.m.keep_thr ? p[0] : 0.f;
-          p[1] = w.y >= a.m.keep_thr ? p[1] : 0.f;
-          p[2] = w.z >= a.m.keep_thr ? p[2] : 0.f;
-          p[3] = w.w >= a.m.keep_thr ? p[3] : 0.f;
-          pk[c4 * 2] = pack_bf16(p[0], p[1]);
-          pk[c4 * 2 + 1] = pack_bf16(p[2], p[3]);
-        }
-      } else {
-#pragma unroll
-        for (int c2 = 0; c2 < 64; ++c2) {
-          const float p0 = ex2(s[2 * c2] - msub), p1 = ex2(s[2 * c2 + 1] - msub);
-          sum += p0 + p1;
-          pk[c2] = pack_bf16(p0, p1);
-        }
+      for (int c2 = 0; c2 < 64; ++c2) {
+        const float p0 = ex2(s[2 * c2] - msub), p1 = ex2(s[2 * c2 + 1] - msub);
+        sum += p0 + p1;
+        // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
+        const uint64_t kw = c2 < 32 ? kb0 : kb1;
+        const int bit = (2 * c2) & 63;
+        pk[c2] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
       }
       l_run = l_run * alpha + sum;
       m_run = m_new;
-      // PV of the previous tile must finish before O is rescaled and P reused.
-      if (n > 0) {
+      // The PV that last read this P buffer (two tiles back) must be done.
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->p_free[n & 1]), ((n >> 1) & 1) ^ 1, abort_flag, a.status));
+      if (!ok) break;
+      if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O must hold every earlier PV before it is rescaled.
         ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_done), (n - 1) & 1, abort_flag, a.status));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + c * 32, r);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(tO + lane_off + c * 32, r);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + lane_off + c * 32, o);
         }
+        tmem_wait_st();
       }
+      const uint32_t pbase = sbase + kFwdP + (n & 1) * kTileBytes;
 #pragma unroll
       for (int cc = 0; cc < 16; ++cc) {
         const uint32_t addr = pbase + (cc >> 3) * (kTileBytes / 2) + sw128_offset(t, (cc & 7) * 16);
@@ -402,24 +447,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->p_full));
+      mbar_arrive(smem_u32(&ctl->p_full[n & 1]));
       ++n;
     }
     // ---------------- epilogue: Y = u / (l + exp(z - m)), LSE = m + ln(...)
-    float o_row[128];
     bool have_o = false;
+    uint32_t orow_bits[4][32];
     if (ok && n > 0) {
-      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_done), (n - 1) & 1, abort_flag, a.status));
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_final), 0, abort_flag, a.status));
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + lane_off + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o_row[c * 32 + e] = __uint_as_float(r[e]);
-        }
+        for (int c = 0; c < 4; ++c) tmem_ld32(tO + lane_off + c * 32, orow_bits[c]);
+        tmem_wait_ld();
         have_o = true;
       }
     }
@@ -437,17 +477,20 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (a.m.dropout) oscale *= a.m.inv_keep;
         lse2 = M + log2f(tot);
       }
-      __nv_bfloat16* orow = a.o + b * a.so[0] + h * a.so[1] + (int64_t)row * a.so[2];
+      __nv_bfloat16* orow = a.o + b * a.so[0] + h * a.so[1] + row * a.so[2];
 #pragma unroll
       for (int c8 = 0; c8 < 16; ++c8) {
-        uint4 v;
-        v.x = pack_bf16(have_o ? o_row[c8 * 8 + 0] * oscale : 0.f, have_o ? o_row[c8 * 8 + 1] * oscale : 0.f);
-        v.y = pack_bf16(have_o ? o_row[c8 * 8 + 2] * oscale : 0.f, have_o ? o_row[c8 * 8 + 3] * oscale : 0.f);
-        v.z = pack_bf16(have_o ? o_row[c8 * 8 + 4] * oscale : 0.f, have_o ? o_row[c8 * 8 + 5] * oscale : 0.f);
-        v.w = pack_bf16(have_o ? o_row[c8 * 8 + 6] * oscale : 0.f, have_o ? o_row[c8 * 8 + 7] * oscale : 0.f);
-        *reinterpret_cast<uint4*>(orow + c8 * 8) = v;
+        uint32_t pkd[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c8 * 8 + 2 * e;
+          const float v0 = have_o ? __uint_as_float(orow_bits[c >> 5][c & 31]) * oscale : 0.f;
+          const float v1 = have_o ? __uint_as_float(orow_bits[(c + 1) >> 5][(c + 1) & 31]) * oscale : 0.f;
+          pkd[e] = pack_bf16(v0, v1);
+        }
+        *reinterpret_cast<uint4*>(orow + c8 * 8) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
       }
-      a.lse[b * a.sl[0] + h * a.sl[1] + (int64_t)row * a.sl[2]] = lse2 / kLog2e;
+      a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
     }
   }
   tc_fence_before();
@@ -464,6 +507,7 @@ struct BwdArgs {
   MaskP m;
   ClassTable ct;
   int B, Hq, Hkv, T, Tpad;
+  int block_aligned;
   float scale_log2;
   const float* lse2;    // [B*Hq, Tpad] base-2 LSE (+inf on rows without keys)
   const float* dpad;    // [B*Hq, Tpad] delta, zero on padding rows
@@ -478,23 +522,25 @@ struct BwdArgs {
 
 constexpr uint32_t kHalfQ = kBMb * 64 * 2;  // 8 KB: 64 rows x 64 bf16
 constexpr uint32_t kQTile = kBMb * kD * 2;  // 16 KB: 64 rows x 128 bf16
+constexpr uint32_t kPTile = kBN * kBMb * 2; // 16 KB: 128 keys x 64 queries bf16
 constexpr uint32_t kBwdK = 0;
 constexpr uint32_t kBwdV = kBwdK + kTileBytes;
-constexpr uint32_t kBwdQ = kBwdV + kTileBytes;              // kStages x 16 KB
-constexpr uint32_t kBwdG = kBwdQ + kStages * kQTile;        // kStages x 16 KB
-constexpr uint32_t kBwdPT = kBwdG + kStages * kQTile;       // 128 keys x 64 q bf16 = 16 KB
-constexpr uint32_t kBwdDS = kBwdPT + kBN * kBMb * 2;        // 16 KB
-constexpr uint32_t kBwdDQ = kBwdDS + kBN * kBMb * 2;        // 64 x 128 fp32 = 32 KB
-constexpr uint32_t kBwdStat = kBwdDQ + kBMb * kD * 4;       // kStages x (64 lse2 + 64 delta) fp32
-constexpr uint32_t kBwdCtl = kBwdStat + kStages * 512;
+constexpr uint32_t kBwdQ = kBwdV + kTileBytes;          // 2 stages
+constexpr uint32_t kBwdG = kBwdQ + 2 * kQTile;          // 2 stages
+constexpr uint32_t kBwdPT = kBwdG + 2 * kQTile;         // 2 buffers
+constexpr uint32_t kBwdDS = kBwdPT + 2 * kPTile;        // 2 buffers
+constexpr uint32_t kBwdDQ = kBwdDS + 2 * kPTile;        // 32 query rows x 128 fp32 = 16 KB
+constexpr uint32_t kBwdStat = kBwdDQ + 32 * kD * 4;     // 2 stages x (64 lse2 + 64 delta) fp32
+constexpr uint32_t kBwdCtl = kBwdStat + 2 * 512;
 constexpr uint32_t kBwdSmem = kBwdCtl + 1024 + 1024;
+constexpr int kBwdThreads = 320;  // producer, MMA, compute warpgroup (warps 2-5), dQ warpgroup (6-9)
 
 struct BwdCtl {
   uint64_t kv_full;
-  uint64_t q_full[kStages], q_empty[kStages];
-  uint64_t st_full, st_empty;
-  uint64_t ds_full, pds_empty;
-  uint64_t dq_full, dq_empty;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t st_full[2], st_empty[2];
+  uint64_t ds_full[2], pds_empty[2];
+  uint64_t dq_full[2], dq_empty[2];
   uint64_t acc_done;
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -512,6 +558,48 @@ __device__ __forceinline__ void bwd_query_slices(const MaskP& m, int T, int k0, 
   }
 }
 
+// The next nonempty (query head in group, query slice) after (hh, qs).
+__device__ __forceinline__ bool bwd_next_step(const BwdArgs& a, int b, int kvh, int kt, int group, int qs_lo,
+                                              int qs_hi, int& hh, int& qs, uint8_t& cls) {
+  if (qs_lo > qs_hi) return false;
+  while (true) {
+    if (++qs > qs_hi) {
+      if (++hh >= group) return false;
+      qs = qs_lo;
+    }
+    cls = lookup_class(a.ct, a.m, a.T, b, kvh * group + hh, qs, kt);
+    if (cls != kEmpty) return true;
+  }
+}
+
+// Allowed query rows i0..i0+63 for key j, as a 64-bit word (bit c <-> i0 + c).
+__device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h, int64_t i0, int64_t j) {
+  if (j >= a.T) return 0ull;
+  int64_t lo = i0, hi = i0 + kBMb - 1;
+  if (hi > a.T - 1) hi = a.T - 1;
+  if (a.m.flags & ATTN_MASK_CAUSAL) lo = j > lo ? j : lo;
+  if (a.m.flags & ATTN_MASK_WINDOW) hi = j + a.m.window - 1 < hi ? j + a.m.window - 1 : hi;
+  uint64_t w = range_bits64(lo - i0, hi - i0);
+  if (w && (a.m.flags & ATTN_MASK_BLOCK) && !a.block_aligned) {
+    const uint8_t* base = a.m.bm + b * a.m.bm_sb + h * a.m.bm_sh + j / a.m.bk;
+    uint64_t bb = 0;
+#pragma unroll 1
+    for (int c = 0; c < kBMb; ++c)
+      if (i0 + c < a.T && base[((i0 + c) / a.m.bq) * a.m.bm_sq]) bb |= 1ull << c;
+    w &= bb;
+  }
+  return w;
+}
+
+// Keep bits xi for key j and query rows i0..i0+63.
+__device__ __forceinline__ uint64_t bwd_keep_bits(const MaskP& m, int b, int h, int64_t i0, int64_t j) {
+  uint64_t w = 0;
+#pragma unroll 1
+  for (int c = 0; c < kBMb; ++c)
+    if (dropout_keep(m, b, h, i0 + c, j)) w |= 1ull << c;
+  return w;
+}
+
 __device__ __forceinline__ void red_bulk_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
   asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
                    reinterpret_cast<uint64_t>(gdst)),
@@ -523,9 +611,9 @@ __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void wg_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void dq_group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -533,7 +621,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const uint32_t sbase = smem_u32(smem);
   BwdCtl* ctl = reinterpret_cast<BwdCtl*>(smem + kBwdCtl);
   volatile uint32_t* abort_flag = &ctl->abort_flag;
-  float* stat = reinterpret_cast<float*>(smem + kBwdStat);
+  const float* stat = reinterpret_cast<const float*>(smem + kBwdStat);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int group = a.Hq / a.Hkv;
@@ -546,16 +634,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->kv_full), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->q_full[s]), 1);
       mbar_init(smem_u32(&ctl->q_empty[s]), 1);
+      mbar_init(smem_u32(&ctl->st_full[s]), 1);
+      mbar_init(smem_u32(&ctl->st_empty[s]), 128);
+      mbar_init(smem_u32(&ctl->ds_full[s]), 128);
+      mbar_init(smem_u32(&ctl->pds_empty[s]), 1);
+      mbar_init(smem_u32(&ctl->dq_full[s]), 1);
+      mbar_init(smem_u32(&ctl->dq_empty[s]), 128);
     }
-    mbar_init(smem_u32(&ctl->st_full), 1);
-    mbar_init(smem_u32(&ctl->st_empty), 128);
-    mbar_init(smem_u32(&ctl->ds_full), 128);
-    mbar_init(smem_u32(&ctl->pds_empty), 1);
-    mbar_init(smem_u32(&ctl->dq_full), 1);
-    mbar_init(smem_u32(&ctl->dq_empty), 128);
     mbar_init(smem_u32(&ctl->acc_done), 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
@@ -568,8 +656,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  // TMEM columns: S^T 0..63, dP^T 64..127, dV 128..255, dK 256..383, dQ^T 384..447
-  const uint32_t tST = tmem, tDPT = tmem + 64, tDV = tmem + 128, tDK = tmem + 256, tDQ = tmem + 384;
+  // TMEM columns: two S^T | dP^T buffers (0..127, 128..255; dQ^T of a step
+  // reuses the S^T half of its buffer), dV 256..383, dK 384..511.
+  const uint32_t tDV = tmem + 256, tDK = tmem + 384;
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -583,189 +672,156 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     tma_load_4d(sbase + kBwdK + kTileBytes / 2, &tk, kvf, 64, k0, kvh, b);
     tma_load_4d(sbase + kBwdV, &tv, kvf, 0, k0, kvh, b);
     tma_load_4d(sbase + kBwdV + kTileBytes / 2, &tv, kvf, 64, k0, kvh, b);
-    int n = 0;
-    bool ok = true;
-    for (int hh = 0; hh < group && ok; ++hh) {
+    int n = 0, hh = 0, qs = qs_lo - 1;
+    uint8_t cls;
+    while (bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
       const int h = kvh * group + hh;
-      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
-        if (lookup_class(a.ct, a.m, a.T, b, h, qs, kt) == kEmpty) continue;
-        const int s = n % kStages;
-        if (!(ok = wait_bar(smem_u32(&ctl->q_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, a.status))) break;
-        const uint32_t qf = smem_u32(&ctl->q_full[s]);
-        mbar_expect_tx(qf, 2 * kQTile + 512);
-        const uint32_t qd = sbase + kBwdQ + s * kQTile, gd = sbase + kBwdG + s * kQTile;
-        tma_load_4d(qd, &tq, qf, 0, qs * kBMb, h, b);
-        tma_load_4d(qd + kHalfQ, &tq, qf, 64, qs * kBMb, h, b);
-        tma_load_4d(gd, &tg, qf, 0, qs * kBMb, h, b);
-        tma_load_4d(gd + kHalfQ, &tg, qf, 64, qs * kBMb, h, b);
-        const int64_t roff = ((int64_t)b * a.Hq + h) * a.Tpad + (int64_t)qs * kBMb;
-        bulk_load(sbase + kBwdStat + s * 512, a.lse2 + roff, 256, qf);
-        bulk_load(sbase + kBwdStat + s * 512 + 256, a.dpad + roff, 256, qf);
-        ++n;
-      }
+      const int s = n & 1;
+      if (!wait_bar(smem_u32(&ctl->q_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+      const uint32_t qf = smem_u32(&ctl->q_full[s]);
+      mbar_expect_tx(qf, 2 * kQTile + 512);
+      const uint32_t qd = sbase + kBwdQ + s * kQTile, gd = sbase + kBwdG + s * kQTile;
+      tma_load_4d(qd, &tq, qf, 0, qs * kBMb, h, b);
+      tma_load_4d(qd + kHalfQ, &tq, qf, 64, qs * kBMb, h, b);
+      tma_load_4d(gd, &tg, qf, 0, qs * kBMb, h, b);
+      tma_load_4d(gd + kHalfQ, &tg, qf, 64, qs * kBMb, h, b);
+      const int64_t roff = ((int64_t)b * a.Hq + h) * a.Tpad + (int64_t)qs * kBMb;
+      bulk_load(sbase + kBwdStat + s * 512, a.lse2 + roff, 256, qf);
+      bulk_load(sbase + kBwdStat + s * 512 + 256, a.dpad + roff, 256, qf);
+      ++n;
     }
-    for (int r = (n > kStages ? n - kStages : 0); r < n; ++r)
-      wait_bar(smem_u32(&ctl->q_full[r % kStages]), (r / kStages) & 1, abort_flag, nullptr);
+    for (int r = (n > 2 ? n - 2 : 0); r < n; ++r)
+      wait_bar(smem_u32(&ctl->q_full[r & 1]), (r >> 1) & 1, abort_flag, nullptr);
     wait_bar(kvf, 0, abort_flag, nullptr);
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: S^T/dP^T of step n+1 go ahead of the
+    // dV, dK, dQ^T products of step n so the tensor core overlaps the
+    // compute warpgroup.
     constexpr uint32_t idST = idesc_bf16(128, 64, 0, 0);   // K Q^T, V dO^T
     constexpr uint32_t idACC = idesc_bf16(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
     constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
     bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
-    int n = 0;
-    for (int hh = 0; hh < group && ok; ++hh) {
-      const int h = kvh * group + hh;
-      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
-        if (lookup_class(a.ct, a.m, a.T, b, h, qs, kt) == kEmpty) continue;
-        const int s = n % kStages;
-        if (!(ok = wait_bar(smem_u32(&ctl->q_full[s]), (n / kStages) & 1, abort_flag, a.status))) break;
-        if (!(ok = wait_bar(smem_u32(&ctl->st_empty), (n & 1) ^ 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
+    auto issue_st = [&](int m) -> bool {
+      const int s = m & 1;
+      const uint32_t par = (m >> 1) & 1;
+      if (!wait_bar(smem_u32(&ctl->q_full[s]), par, abort_flag, a.status)) return false;
+      if (!wait_bar(smem_u32(&ctl->st_empty[s]), par ^ 1, abort_flag, a.status)) return false;
+      if (!wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
+      const uint32_t dst = tmem + s * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
-          mma_ss(tST, smem_desc_sw128(sbase + kBwdK + koff, 16, 1024), smem_desc_sw128(qa + qoff, 16, 1024), idST,
-                 kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
-          mma_ss(tDPT, smem_desc_sw128(sbase + kBwdV + koff, 16, 1024), smem_desc_sw128(ga + qoff, 16, 1024),
-                 idST, kk > 0);
-        }
-        mma_commit(smem_u32(&ctl->st_full));
-        if (!(ok = wait_bar(smem_u32(&ctl->ds_full), n & 1, abort_flag, a.status))) break;
-        if (!(ok = wait_bar(smem_u32(&ctl->dq_empty), (n & 1) ^ 1, abort_flag, a.status))) break;
-        tc_fence_after();
-        const uint32_t pta = sbase + kBwdPT, dsa = sbase + kBwdDS;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = 64 query rows
-          mma_ss(tDV, smem_desc_sw128(pta + kk * 32, 16, 1024), smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kHalfQ, 1024), idACC,
-                 (n > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 keys
-          mma_ss(tDQ, smem_desc_sw128(sbase + kBwdK + kk * 2048, kTileBytes / 2, 1024),
-                 smem_desc_sw128(dsa + kk * 2048, kHalfQ, 1024), idDQ, kk > 0);
-        }
-        mma_commit(smem_u32(&ctl->q_empty[s]));
-        mma_commit(smem_u32(&ctl->pds_empty));
-        mma_commit(smem_u32(&ctl->dq_full));
-        ++n;
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+        const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
+        mma_ss(dst, smem_desc_sw128(sbase + kBwdK + koff, 16, 1024), smem_desc_sw128(qa + qoff, 16, 1024), idST,
+               kk > 0);
       }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+        const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
+        mma_ss(dst + 64, smem_desc_sw128(sbase + kBwdV + koff, 16, 1024), smem_desc_sw128(ga + qoff, 16, 1024),
+               idST, kk > 0);
+      }
+      mma_commit(smem_u32(&ctl->st_full[s]));
+      return true;
+    };
+    int hh = 0, qs = qs_lo - 1, n = 0;
+    uint8_t cls;
+    bool have = ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls);
+    if (have) ok = issue_st(0);
+    while (ok && have) {
+      int nh = hh, nq = qs;
+      uint8_t ncls;
+      const bool next = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
+      if (next && !(ok = issue_st(n + 1))) break;
+      const int s = n & 1;
+      if (!(ok = wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
+      const uint32_t pta = sbase + kBwdPT + s * kPTile, dsa = sbase + kBwdDS + s * kPTile;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows
+        mma_ss(tDV, smem_desc_sw128(pta + kk * 32, 16, 1024), smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC,
+               (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kHalfQ, 1024), idACC,
+               (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
+        mma_ss(tmem + s * 128, smem_desc_sw128(sbase + kBwdK + kk * 2048, kTileBytes / 2, 1024),
+               smem_desc_sw128(dsa + kk * 2048, kHalfQ, 1024), idDQ, kk > 0);
+      mma_commit(smem_u32(&ctl->q_empty[s]));
+      mma_commit(smem_u32(&ctl->pds_empty[s]));
+      mma_commit(smem_u32(&ctl->dq_full[s]));
+      hh = nh;
+      qs = nq;
+      have = next;
+      ++n;
     }
     mma_commit(smem_u32(&ctl->acc_done));
-  } else if (warp >= 4) {
+  } else if (warp >= 2 && warp < 6) {
     // ---------------- compute warpgroup: thread t owns key row k0 + t
-    // (and, for the dQ^T readback, head-dimension index t)
-    const int t = threadIdx.x - 128;
+    const int t = ((warp & 3) << 5) | lane;
     const int64_t j = (int64_t)k0 + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float* dq_stage = reinterpret_cast<float*>(smem + kBwdDQ);
-    int n = 0;
+    int n = 0, hh = 0, qs = qs_lo - 1;
+    uint8_t cls;
     bool ok = true;
-    for (int hh = 0; hh < group && ok; ++hh) {
+    while (ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
       const int h = kvh * group + hh;
-      for (int qs = qs_lo; qs <= qs_hi; ++qs) {
-        const uint8_t cls = lookup_class(a.ct, a.m, a.T, b, h, qs, kt);
-        if (cls == kEmpty) continue;
-        const int s = n % kStages;
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full), n & 1, abort_flag, a.status)))) break;
-        if (!(ok = __all_sync(0xffffffffu,
-                              wait_bar(smem_u32(&ctl->q_full[s]), (n / kStages) & 1, abort_flag, a.status))))
-          break;
-        tc_fence_after();
-        float sv[64], dp[64];
+      const int s = n & 1;
+      const uint32_t par = (n >> 1) & 1;
+      const int64_t i0 = (int64_t)qs * kBMb;
+      const uint64_t allow = cls == kPartial ? bwd_col_bits(a, b, h, i0, j) : ~0ull;
+      const uint64_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0, j) : ~0ull;
+      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->q_full[s]), par, abort_flag, a.status)))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty[s]), par ^ 1, abort_flag, a.status))))
+        break;
+      tc_fence_after();
+      const float* lse2 = stat + s * 128;
+      const float* dl = lse2 + 64;
+      const uint32_t pt_base = sbase + kBwdPT + s * kPTile, ds_base = sbase + kBwdDS + s * kPTile;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tST + lane_off + c * 32, r);
-          tmem_wait_ld();
+      for (int half = 0; half < 2; ++half) {
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tmem + lane_off + s * 128 + half * 32, rs);
+        tmem_ld32(tmem + lane_off + s * 128 + 64 + half * 32, rp);
+        tmem_wait_ld();
+        uint32_t ppk[16], dpk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
-          tmem_ld32(tDPT + lane_off + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) dp[c * 32 + e] = __uint_as_float(r[e]);
-        }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&ctl->st_empty));
-        const float* lse2 = stat + s * 128;
-        const float* dl = lse2 + 64;
-        const int64_t i0 = (int64_t)qs * kBMb;
-        uint32_t ppk[32], dpk[32];
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
+        for (int c2 = 0; c2 < 16; ++c2) {
           float pt[2], ds[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int c = 2 * c2 + e;
-            const int64_t i = i0 + c;
-            bool alw = true;
-            if (cls == kPartial) alw = i < a.T && j < a.T && allowed(a.m, b, h, i, j);
-            float p = alw ? ex2(sv[c] * a.scale_log2 - lse2[c]) : 0.f;
-            float dpv = dp[c];
-            float ptil = p;
-            if (a.m.dropout) {
-              // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
-              const bool keep = dropout_keep(a.m, b, h, i, j);
-              ptil = keep ? p : 0.f;
-              dpv = keep ? dpv * a.m.inv_keep : 0.f;
-            }
-            pt[e] = ptil;
+            const int c = half * 32 + 2 * c2 + e;
+            const float p = ((allow >> c) & 1ull) ? ex2(fmaf(__uint_as_float(rs[2 * c2 + e]), a.scale_log2, -lse2[c]))
+                                                   : 0.f;
+            const bool kp = (keep >> c) & 1ull;
+            // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
+            pt[e] = kp ? p : 0.f;
+            const float dpv = kp ? __uint_as_float(rp[2 * c2 + e]) * (a.m.dropout ? a.m.inv_keep : 1.f) : 0.f;
             ds[e] = p * (dpv - dl[c]);
           }
           ppk[c2] = pack_bf16(pt[0], pt[1]);
           dpk[c2] = pack_bf16(ds[0], ds[1]);
         }
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty), (n & 1) ^ 1, abort_flag, a.status))))
-          break;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const uint32_t off = sw128_offset(t, cc * 16);
-          st_shared_v4(sbase + kBwdPT + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
-          st_shared_v4(sbase + kBwdDS + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t off = sw128_offset(t, (half * 4 + cc) * 16);
+          st_shared_v4(pt_base + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
+          st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&ctl->ds_full));
-        // dQ^T tile: thread t holds head-dimension t for 64 query rows.
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_full), n & 1, abort_flag, a.status)))) break;
-        tc_fence_after();
-        // The previous step's bulk reduce must have read the staging buffer.
-        if (t == 0) bulk_wait_read0();
-        wg_sync();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tDQ + lane_off + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) dq_stage[(c * 32 + e) * kD + t] = __uint_as_float(r[e]);
-        }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&ctl->dq_empty));
-        fence_proxy_async_smem();
-        wg_sync();
-        if (t == 0) {
-          const int rows = (int)((a.T - i0) < kBMb ? (a.T - i0) : kBMb);
-          float* dst = a.dq_acc + (((int64_t)b * a.Hq + h) * a.T + i0) * kD;
-          red_bulk_add_f32(dst, sbase + kBwdDQ, (uint32_t)rows * kD * 4);
-          bulk_commit();
-        }
-        ++n;
       }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->st_empty[s]));
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&ctl->ds_full[s]));
+      ++n;
     }
-    if (t == 0) bulk_wait0();
     // ---------------- epilogue: dK = c * sum gamma^T Q, dV = sum P~^T dO
     bool have = false;
     if (ok && n > 0) {
@@ -788,9 +844,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (j < a.T) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
-            uint4 vk, vv;
-            uint32_t* pk = &vk.x;
-            uint32_t* pv = &vv.x;
+            uint32_t pk[4], pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int idx = c8 * 8 + e * 2;
@@ -799,12 +853,53 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               pv[e] = have ? pack_bf16(__uint_as_float(rv[idx]) * dv_scale, __uint_as_float(rv[idx + 1]) * dv_scale)
                            : 0u;
             }
-            *reinterpret_cast<uint4*>(dkr + c * 32 + c8 * 8) = vk;
-            *reinterpret_cast<uint4*>(dvr + c * 32 + c8 * 8) = vv;
+            *reinterpret_cast<uint4*>(dkr + c * 32 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dvr + c * 32 + c8 * 8) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
           }
         }
       }
     }
+  } else if (warp >= 6) {
+    // ---------------- dQ warpgroup: thread t owns head-dimension index t of
+    // the dQ^T tile and stages it row-major for a bulk reduce-add.
+    const int t = ((warp & 3) << 5) | lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    float* stage = reinterpret_cast<float*>(smem + kBwdDQ);
+    int n = 0, hh = 0, qs = qs_lo - 1;
+    uint8_t cls;
+    bool ok = true;
+    while (ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
+      const int h = kvh * group + hh;
+      const int s = n & 1;
+      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_full[s]), (n >> 1) & 1, abort_flag, a.status))))
+        break;
+      tc_fence_after();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tmem + lane_off + s * 128, r0);
+      tmem_ld32(tmem + lane_off + s * 128 + 32, r1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->dq_empty[s]));
+      const int64_t i0 = (int64_t)qs * kBMb;
+      const int rows = (int)((a.T - i0) < kBMb ? (a.T - i0) : kBMb);
+      float* dst = a.dq_acc + (((int64_t)b * a.Hq + h) * a.T + i0) * kD;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (t == 0) bulk_wait_read0();  // the previous reduce has read the stage
+        dq_group_sync();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) stage[e * kD + t] = __uint_as_float(half ? r1[e] : r0[e]);
+        fence_proxy_async_smem();
+        dq_group_sync();
+        const int hr = rows - half * 32 < 32 ? rows - half * 32 : 32;
+        if (t == 0 && hr > 0) {
+          red_bulk_add_f32(dst + (int64_t)half * 32 * kD, sbase + kBwdDQ, (uint32_t)hr * kD * 4);
+          bulk_commit();
+        }
+      }
+      ++n;
+    }
+    if (t == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -902,6 +997,13 @@ bool make_map(CUtensorMap* map, const void* base, int T, int H, int B, int64_t s
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A block mask is constant over every (64-row slice, 128-key tile) when its
+// block sizes are multiples of those; then the tile class already says all.
+int block_aligned(const MaskP& m) {
+  if (!(m.flags & ATTN_MASK_BLOCK)) return 1;
+  return (m.bq % kBMb == 0 && m.bk % kBN == 0) ? 1 : 0;
+}
+
 bool tma_ok(const attn_tensor* t) {
   if (!t || t->dtype != ATTN_BF16 || t->ndim != 4 || t->stride[3] != 1) return false;
   if (reinterpret_cast<uintptr_t>(t->data) % 16) return false;
@@ -989,6 +1091,7 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   FwdArgs a;
   a.m = p.m;
   a.ct = ct;
+  a.block_aligned = block_aligned(p.m);
   a.B = p.B;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
@@ -1032,6 +1135,7 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   BwdArgs a;
   a.m = p.m;
   a.ct = ct;
+  a.block_aligned = block_aligned(p.m);
   a.B = p.B;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
@@ -1051,7 +1155,7 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
   const int nkt = (p.T + kBN - 1) / kBN;
-  bwd_kernel<<<nkt * p.B * p.Hkv, 256, kBwdSmem, st>>>(mq, mk, mv, mg, a);
+  bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, a);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n4 = (int64_t)p.B * p.Hq * p.T * kD / 4;
   dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.T, p.scale,

@@ -18,6 +18,6 @@ philox     Philox4x32-10 (Salmon et al., SC'11) and the dropout keep-mask
 from .attention import (  # noqa: F401
     BackwardResult, ForwardResult, TileCard, allowed_dense, backward,
     block_summary, forward, merge_summaries, tiled_forward, topk_allowed,
-    topk_backward, topk_forward,
+    topk_backward, topk_dsink, topk_forward,
 )
 from .philox import dropout_keep, keep_threshold, philox4x32  # noqa: F401

@@ -120,7 +120,9 @@ def _row_softmax(s: np.ndarray, allow: np.ndarray, z: float):
     finite = np.isfinite(m)
     shift = np.where(finite, m, 0.0)
     e = np.where(allow, np.exp(sm - shift[:, None]), 0.0)
-    e_sink = np.exp(z - shift) if np.isfinite(z) else np.zeros_like(shift)
+    z = np.broadcast_to(np.asarray(z, dtype=np.float64), shift.shape)   # one z per row
+    has_z = np.isfinite(z)
+    e_sink = np.where(has_z, np.exp(np.where(has_z, z, 0.0) - shift), 0.0)
     total = e.sum(axis=-1) + e_sink
     safe = np.where(finite, total, 1.0)
     p = np.where(finite[:, None], e / safe[:, None], 0.0)
@@ -235,17 +237,17 @@ def topk_forward(q, kv, idx, length, dv: int, scale: float, sink=None):
     o = np.zeros((t_q, H, dv))
     lse = np.full((t_q, H), NEG_INF)
     p_sink = np.zeros((t_q, H))
+    z = np.full(H, NEG_INF) if sink is None else np.asarray(sink, dtype=np.float64)
     for t in range(t_q):
+        # All heads of one token at once: the matrix form of the DSA note, section 5.
         sel = np.asarray(idx[t, :length[t]], dtype=np.int64)
         ksel = kv[sel]                       # [L, Dqk]
         vsel = kv[sel, :dv]                  # [L, dv]
         s = scale * (q[t] @ ksel.T)          # [H, L]
-        for h in range(H):
-            z = NEG_INF if sink is None else float(sink[h])
-            p, ps, l = _row_softmax(s[h:h + 1], np.ones((1, len(sel)), bool), z)
-            o[t, h] = p[0] @ vsel
-            lse[t, h] = l[0]
-            p_sink[t, h] = ps[0]
+        p, ps, l = _row_softmax(s, np.ones(s.shape, bool), z)
+        o[t] = p @ vsel
+        lse[t] = l
+        p_sink[t] = ps
     return o, lse, p_sink
 
 
@@ -267,18 +269,13 @@ def topk_backward(q, kv, idx, length, dv: int, scale: float, d_o, sink=None,
     dq = np.zeros_like(q)
     dkv = np.zeros_like(kv)
     dsink = np.zeros(H) if sink is not None else None
+    z = np.full(H, NEG_INF) if sink is None else np.asarray(sink, dtype=np.float64)
     for t in range(t_q):
         sel = np.asarray(idx[t, :length[t]], dtype=np.int64)
         ksel = kv[sel]
         vsel = kv[sel, :dv]
         s = scale * (q[t] @ ksel.T)                          # [H, L]
-        p = np.empty_like(s)
-        ps = np.empty(H)
-        for h in range(H):
-            z = NEG_INF if sink is None else float(sink[h])
-            pr, psr, _ = _row_softmax(s[h:h + 1], np.ones((1, len(sel)), bool), z)
-            p[h] = pr[0]
-            ps[h] = psr[0]
+        p, ps, _ = _row_softmax(s, np.ones(s.shape, bool), z)
         dP = d_o[t] @ vsel.T                                 # [H, L]
         D = np.sum(d_o[t] * o[t], axis=-1)                   # [H]
         gam = scale * p * (dP - D[:, None])                  # G = c dS
@@ -289,6 +286,14 @@ def topk_backward(q, kv, idx, length, dv: int, scale: float, d_o, sink=None,
         if dsink is not None:
             dsink += -ps * D
     return dq, dkv, dsink
+
+
+def topk_dsink(q, kv, idx, length, dv: int, scale: float, d_o, sink):
+    """dz_h = -sum_t p_sink[t, h] D[t, h] with D = <dO, O> (DSA note,
+    section 3.5), from the forward pass alone."""
+    o, _, p_sink = topk_forward(q, kv, idx, length, dv, scale, sink)
+    D = np.sum(np.asarray(d_o, dtype=np.float64) * o, axis=-1)     # [Tq, H]
+    return -np.sum(p_sink * D, axis=0)
 
 
 # ---------------------------------------------------------------------------

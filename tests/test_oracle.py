@@ -334,6 +334,7 @@ def test_topk_equals_dense_with_selected_sets():
     dkv_dense[:, :Dv] += bw.dv[0, 0]
     assert np.allclose(dkv, dkv_dense, atol=1e-12)
     assert np.allclose(dsink, bw.dsink, atol=1e-12)
+    assert np.allclose(A.topk_dsink(q, kv, idx, ln, Dv, c, d_o, sink), bw.dsink, atol=1e-12)
 
 
 def test_topk_lists_are_causal_and_distinct():
