@@ -148,36 +148,42 @@ struct FwdArgs {
 
 // Shared-memory map of the forward kernel (offsets from a 1024-aligned base).
 constexpr uint32_t kTileBytes = kBN * kD * 2;  // 32 KB: 128 rows x 128 bf16
-constexpr uint32_t kFwdQ = 0;
-constexpr uint32_t kFwdK = kFwdQ + kTileBytes;
+constexpr int kFwdRows = 2 * kBM;              // two 128-row query tiles per CTA
+constexpr uint32_t kFwdQ = 0;                  // 2 tiles
+constexpr uint32_t kFwdK = kFwdQ + 2 * kTileBytes;
 constexpr uint32_t kFwdV = kFwdK + kStages * kTileBytes;
-constexpr uint32_t kFwdP = kFwdV + kStages * kTileBytes;  // 2 buffers
-constexpr uint32_t kFwdCtl = kFwdP + 2 * kTileBytes;
+constexpr uint32_t kFwdCtl = kFwdV + kStages * kTileBytes;
 constexpr uint32_t kFwdSmem = kFwdCtl + 1024 + 1024;  // control block + alignment slack
+constexpr int kFwdThreads = 320;  // producer, MMA issuer, softmax warpgroups (warps 2-5, 6-9)
 
 struct FwdCtl {
   uint64_t q_full;
   uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_free[2];
-  uint64_t o_done, o_final;
+  uint64_t s_full[2], p_full[2];  // one pair per softmax warpgroup
+  uint64_t o_final;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
 
-// Key-tile range that can hold allowed keys for rows [q0, q0 + 128).
-__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int& lo, int& hi) {
+// Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
+__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int rows, int& lo, int& hi) {
   const int nkt = (T + kBN - 1) / kBN;
   lo = 0;
   hi = nkt - 1;
   if (m.flags & ATTN_MASK_CAUSAL) {
-    const int last = (q0 + kBM - 1 < T - 1 ? q0 + kBM - 1 : T - 1) / kBN;
+    const int last = (q0 + rows - 1 < T - 1 ? q0 + rows - 1 : T - 1) / kBN;
     hi = last < hi ? last : hi;
   }
   if (m.flags & ATTN_MASK_WINDOW) {
     const int64_t first = (int64_t)q0 - m.window + 1;
     lo = first > 0 ? (int)(first / kBN) : 0;
   }
+}
+
+// Class of (128-row query tile qt, key tile kt); tiles past T are empty.
+__device__ __forceinline__ uint8_t wg_class(const FwdArgs& a, int b, int h, int qt, int kt) {
+  if (qt * kBM >= a.T) return kEmpty;
+  return fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
 }
 
 // Bits lo..hi (inclusive, within [0, 63]) of a 64-bit word; 0 when lo > hi.
@@ -235,7 +241,13 @@ __device__ __forceinline__ void fwd_keep_bits(const MaskP& m, int b, int h, int6
   }
 }
 
-__global__ void __launch_bounds__(256, 1)
+// Two query tiles per CTA, one softmax warpgroup each, alternating on the
+// tensor core: while one warpgroup turns its S tile into P, the MMA issuer
+// runs the other warpgroup's P V and next S. P (bf16 pairs) is written back
+// into the warpgroup's own S columns of TMEM and read from there by the PV
+// MMA; S of the next tile lands in the same columns only after that PV, in
+// issue order.
+__global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -245,14 +257,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   volatile uint32_t* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqt = (a.T + kBM - 1) / kBM;
+  const int nct = (a.T + kFwdRows - 1) / kFwdRows;
   const int bh = blockIdx.x % (a.B * a.Hq);
-  const int qt = nqt - 1 - (int)(blockIdx.x / (a.B * a.Hq));  // longest query tiles first
+  const int ct = nct - 1 - (int)(blockIdx.x / (a.B * a.Hq));  // longest query tiles first
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int kvh = h / (a.Hq / a.Hkv);
-  const int q0 = qt * kBM;
+  const int q0 = ct * kFwdRows;
+  const int qt0 = 2 * ct, qt1 = 2 * ct + 1;
   int kt_lo, kt_hi;
-  fwd_key_tiles(a.m, a.T, q0, kt_lo, kt_hi);
+  fwd_key_tiles(a.m, a.T, q0, kFwdRows, kt_lo, kt_hi);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->q_full), 1);
@@ -263,11 +276,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->s_full[s]), 1);
-      mbar_init(smem_u32(&ctl->s_empty[s]), 128);
       mbar_init(smem_u32(&ctl->p_full[s]), 128);
-      mbar_init(smem_u32(&ctl->p_free[s]), 1);
     }
-    mbar_init(smem_u32(&ctl->o_done), 1);
     mbar_init(smem_u32(&ctl->o_final), 1);
     ctl->abort_flag = 0;
     fence_barrier_init();
@@ -280,7 +290,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 256;  // S buffers at columns 0 and 128, O at 256
+  // TMEM columns: S/P of warpgroup w at 128 w, O of warpgroup w at 256 + 128 w.
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -288,12 +298,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
     const uint32_t qf = smem_u32(&ctl->q_full);
-    mbar_expect_tx(qf, kTileBytes);
-    tma_load_4d(sbase + kFwdQ, &tq, qf, 0, q0, h, b);
-    tma_load_4d(sbase + kFwdQ + kTileBytes / 2, &tq, qf, 64, q0, h, b);
+    mbar_expect_tx(qf, 2 * kTileBytes);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      tma_load_4d(sbase + kFwdQ + w * kTileBytes, &tq, qf, 0, q0 + w * kBM, h, b);
+      tma_load_4d(sbase + kFwdQ + w * kTileBytes + kTileBytes / 2, &tq, qf, 64, q0 + w * kBM, h, b);
+    }
     int n = 0;
     for (int kt = kt_lo; kt <= kt_hi; ++kt) {
-      if (fwd_class(a.ct, a.m, a.T, b, h, qt, kt) == kEmpty) continue;
+      if (wg_class(a, b, h, qt0, kt) == kEmpty && wg_class(a, b, h, qt1, kt) == kEmpty) continue;
       const int s = n % kStages;
       if (!wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, a.status)) break;
       const uint32_t kf = smem_u32(&ctl->k_full[s]), vf = smem_u32(&ctl->v_full[s]);
@@ -306,7 +319,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tma_load_4d(vd + kTileBytes / 2, &tv, vf, 64, kt * kBN, kvh, b);
       ++n;
     }
-    // Let every issued copy land before the CTA may leave (bounded).
     for (int r = (n > kStages ? n - kStages : 0); r < n; ++r) {
       const int s = r % kStages;
       wait_bar(smem_u32(&ctl->k_full[s]), (r / kStages) & 1, abort_flag, nullptr);
@@ -317,62 +329,80 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);
     bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
-    auto next_tile = [&](int from) {
-      for (int kt = from + 1; kt <= kt_hi; ++kt)
-        if (fwd_class(a.ct, a.m, a.T, b, h, qt, kt) != kEmpty) return kt;
+    auto next_tile = [&](int from, uint8_t& c0, uint8_t& c1) {
+      for (int kt = from + 1; kt <= kt_hi; ++kt) {
+        c0 = wg_class(a, b, h, qt0, kt);
+        c1 = wg_class(a, b, h, qt1, kt);
+        if (c0 != kEmpty || c1 != kEmpty) return kt;
+      }
       return kt_hi + 1;
     };
-    auto issue_s = [&](int n) -> bool {
-      const int s = n % kStages;
-      if (!wait_bar(smem_u32(&ctl->k_full[s]), (n / kStages) & 1, abort_flag, a.status)) return false;
-      if (!wait_bar(smem_u32(&ctl->s_empty[n & 1]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
-      tc_fence_after();
-      const uint32_t d = tS + (n & 1) * 128;
-      const uint32_t qa = sbase + kFwdQ, ka = sbase + kFwdK + s * kTileBytes;
+    auto issue_s = [&](int w, int stage) {
+      const uint32_t qa = sbase + kFwdQ + w * kTileBytes, ka = sbase + kFwdK + stage * kTileBytes;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-        mma_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS, kk > 0);
+        mma_ss(tmem + w * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS,
+               kk > 0);
       }
-      mma_commit(smem_u32(&ctl->s_full[n & 1]));
-      return true;
+      mma_commit(smem_u32(&ctl->s_full[w]));
     };
+    uint8_t c[2], nc[2];
+    int kt_cur = next_tile(kt_lo - 1, c[0], c[1]);
+    int npv[2] = {0, 0};
     int n = 0;
-    if (ok) {
-      int kt_next = next_tile(kt_lo - 1);
-      if (kt_next <= kt_hi) ok = issue_s(0);
-      while (ok && kt_next <= kt_hi) {
-        kt_next = next_tile(kt_next);
-        const bool last = kt_next > kt_hi;
-        if (!last && !issue_s(n + 1)) break;
-        const int s = n % kStages;
-        if (!wait_bar(smem_u32(&ctl->p_full[n & 1]), (n >> 1) & 1, abort_flag, a.status)) break;
-        if (!wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status)) break;
+    if (ok && kt_cur <= kt_hi) {
+      ok = wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, a.status);
+      if (ok) {
         tc_fence_after();
-        const uint32_t pa = sbase + kFwdP + (n & 1) * kTileBytes, va = sbase + kFwdV + s * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t poff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-          mma_ss(tO, smem_desc_sw128(pa + poff, 16, 1024), smem_desc_sw128(va + kk * 2048, kTileBytes / 2, 1024),
-                 idPV, (n > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&ctl->o_done));
-        mma_commit(smem_u32(&ctl->p_free[n & 1]));
-        mma_commit(smem_u32(&ctl->kv_empty[s]));
-        if (last) mma_commit(smem_u32(&ctl->o_final));
-        ++n;
+        for (int w = 0; w < 2; ++w)
+          if (c[w] != kEmpty) issue_s(w, 0);
       }
     }
-  } else if (warp >= 4) {
-    // ---------------- softmax warpgroup: thread t owns query row q0 + t
-    const int t = threadIdx.x - 128;
-    const int64_t row = q0 + t;
+    while (ok && kt_cur <= kt_hi) {
+      const int kt_nx = next_tile(kt_cur, nc[0], nc[1]);
+      const int s = n % kStages, s1 = (n + 1) % kStages;
+      const bool more = kt_nx <= kt_hi;
+      for (int w = 0; w < 2 && ok; ++w) {
+        if (c[w] != kEmpty) {
+          if (!(ok = wait_bar(smem_u32(&ctl->p_full[w]), npv[w] & 1, abort_flag, a.status))) break;
+          if (!(ok = wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          const uint32_t va = sbase + kFwdV + s * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // A = P in TMEM: 16 keys = 8 packed columns per step
+            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8,
+                   smem_desc_sw128(va + kk * 2048, kTileBytes / 2, 1024), idPV, (npv[w] > 0 || kk > 0) ? 1u : 0u);
+          ++npv[w];
+        }
+        if (more && nc[w] != kEmpty) {
+          if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, a.status))) break;
+          tc_fence_after();
+          issue_s(w, s1);
+        }
+      }
+      if (!ok) break;
+      mma_commit(smem_u32(&ctl->kv_empty[s]));
+      kt_cur = kt_nx;
+      c[0] = nc[0];
+      c[1] = nc[1];
+      ++n;
+    }
+    mma_commit(smem_u32(&ctl->o_final));
+  } else if (warp >= 2) {
+    // ---------------- softmax warpgroups: thread t of warpgroup w owns query row
+    // q0 + 128 w + t (TMEM lane t of that warpgroup's S/P and O columns).
+    const int w = (warp - 2) >> 2;
+    const int qt = 2 * ct + w;
+    const int t = ((warp & 3) << 5) | lane;
+    const int64_t row = (int64_t)q0 + w * kBM + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + w * 128, tO = tmem + lane_off + 256 + w * 128;
     float m_run = -INFINITY, l_run = 0.f;  // base-2 running max and running sum
     int n = 0;
     bool ok = true;
     for (int kt = kt_lo; kt <= kt_hi && ok; ++kt) {
-      const uint8_t cls = fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
+      const uint8_t cls = wg_class(a, b, h, qt, kt);
       if (cls == kEmpty) continue;
       uint64_t mw0 = ~0ull, mw1 = ~0ull;
       if (cls == kPartial) {
@@ -384,86 +414,78 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       uint64_t kb0 = ~0ull, kb1 = ~0ull;
       if (a.m.dropout) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
-      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[n & 1]), (n >> 1) & 1, abort_flag, a.status));
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[w]), n & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + (n & 1) * 128 + c * 32, r[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->s_empty[n & 1]));
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const uint64_t w = c < 64 ? mw0 : mw1;
-        const float v = __uint_as_float(r[c >> 5][c & 31]) * a.scale_log2;
-        s[c] = ((w >> (c & 63)) & 1ull) ? v : -INFINITY;
-      }
+      // Pass 1 over the S row: the masked maximum (64 columns per TMEM load).
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tS + hf * 64, r0);
+        tmem_ld32(tS + hf * 64 + 32, r1);
+        tmem_wait_ld();
+        const uint64_t mw = hf ? mw1 : mw0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if ((mw >> e) & 1ull) mx = fmaxf(mx, __uint_as_float(r0[e]) * a.scale_log2);
+          if ((mw >> (32 + e)) & 1ull) mx = fmaxf(mx, __uint_as_float(r1[e]) * a.scale_log2);
+        }
+      }
       float m_new = m_run;
       if (mx > -INFINITY && (m_run == -INFINITY || mx > m_run + kRescaleThreshold)) m_new = fmaxf(mx, m_run);
       const float alpha = (m_new == m_run) ? 1.f : ex2(m_run - m_new);  // 0 when m_run = -inf
       const float msub = m_new == -INFINITY ? 0.f : m_new;
-      float sum = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c2 = 0; c2 < 64; ++c2) {
-        const float p0 = ex2(s[2 * c2] - msub), p1 = ex2(s[2 * c2 + 1] - msub);
-        sum += p0 + p1;
-        // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
-        const uint64_t kw = c2 < 32 ? kb0 : kb1;
-        const int bit = (2 * c2) & 63;
-        pk[c2] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
-      }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-      // The PV that last read this P buffer (two tiles back) must be done.
-      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->p_free[n & 1]), ((n >> 1) & 1) ^ 1, abort_flag, a.status));
-      if (!ok) break;
+      // Every earlier P V of this warpgroup has completed (the S commit covers
+      // them), so O can be rescaled in place.
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O must hold every earlier PV before it is rescaled.
-        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_done), (n - 1) & 1, abort_flag, a.status));
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + lane_off + c * 32, o);
+          tmem_st32(tO + c * 32, o);
         }
-        tmem_wait_st();
       }
-      const uint32_t pbase = sbase + kFwdP + (n & 1) * kTileBytes;
+      // Pass 2: p = 2^(s - m), written back as bf16 pairs over the first 64
+      // columns (P chunk q covers S columns already read).
+      float sum = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t r[32];
+        tmem_ld32(tS + q * 32, r);
+        tmem_wait_ld();
+        const uint64_t mw = q < 2 ? mw0 : mw1;
+        const uint64_t kw = q < 2 ? kb0 : kb1;
+        uint32_t pk[16];
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const uint32_t addr = pbase + (cc >> 3) * (kTileBytes / 2) + sw128_offset(t, (cc & 7) * 16);
-        st_shared_v4(addr, pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+        for (int e = 0; e < 16; ++e) {
+          const int bit = (q * 32 + 2 * e) & 63;
+          const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * a.scale_log2 - msub) : 0.f;
+          const float p1 = ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * a.scale_log2 - msub) : 0.f;
+          sum += p0 + p1;
+          // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
+          pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+        }
+        tmem_st16(tS + q * 16, pk);
       }
-      fence_proxy_async_smem();
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->p_full[n & 1]));
+      mbar_arrive(smem_u32(&ctl->p_full[w]));
       ++n;
     }
     // ---------------- epilogue: Y = u / (l + exp(z - m)), LSE = m + ln(...)
     bool have_o = false;
-    uint32_t orow_bits[4][32];
     if (ok && n > 0) {
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->o_final), 0, abort_flag, a.status));
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tO + lane_off + c * 32, orow_bits[c]);
-        tmem_wait_ld();
-        have_o = true;
-      }
+      if (ok) tc_fence_after();
+      have_o = ok;
     }
-    if (ok && row < a.T) {
+    if (ok) {
       const bool has_sink = a.m.sink != nullptr;
       const float z2 = has_sink ? a.m.sink[h] * kLog2e : -INFINITY;
       float lse2, oscale;
@@ -479,18 +501,26 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       __nv_bfloat16* orow = a.o + b * a.so[0] + h * a.so[1] + row * a.so[2];
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        uint32_t pkd[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c8 * 8 + 2 * e;
-          const float v0 = have_o ? __uint_as_float(orow_bits[c >> 5][c & 31]) * oscale : 0.f;
-          const float v1 = have_o ? __uint_as_float(orow_bits[(c + 1) >> 5][(c + 1) & 31]) * oscale : 0.f;
-          pkd[e] = pack_bf16(v0, v1);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
         }
-        *reinterpret_cast<uint4*>(orow + c8 * 8) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+        if (row < a.T) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t pkd[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int idx = c8 * 8 + 2 * e;
+              pkd[e] = have_o ? pack_bf16(__uint_as_float(o[idx]) * oscale, __uint_as_float(o[idx + 1]) * oscale) : 0u;
+            }
+            *reinterpret_cast<uint4*>(orow + c * 32 + c8 * 8) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+          }
+        }
       }
-      a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
+      if (row < a.T) a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
     }
   }
   tc_fence_before();
@@ -533,7 +563,9 @@ constexpr uint32_t kBwdDQ = kBwdDS + 2 * kPTile;        // 32 query rows x 128 f
 constexpr uint32_t kBwdStat = kBwdDQ + 32 * kD * 4;     // 2 stages x (64 lse2 + 64 delta) fp32
 constexpr uint32_t kBwdCtl = kBwdStat + 2 * 512;
 constexpr uint32_t kBwdSmem = kBwdCtl + 1024 + 1024;
-constexpr int kBwdThreads = 320;  // producer, MMA, compute warpgroup (warps 2-5), dQ warpgroup (6-9)
+// Warps: 0 TMA producer, 1 MMA issuer, 2-3 idle, 4-7 and 8-11 the two compute
+// warpgroups (query columns 0-31 and 32-63 of each step), 12-15 dQ warpgroup.
+constexpr int kBwdThreads = 512;
 
 struct BwdCtl {
   uint64_t kv_full;
@@ -591,12 +623,12 @@ __device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h,
   return w;
 }
 
-// Keep bits xi for key j and query rows i0..i0+63.
-__device__ __forceinline__ uint64_t bwd_keep_bits(const MaskP& m, int b, int h, int64_t i0, int64_t j) {
-  uint64_t w = 0;
+// Keep bits xi for key j and query rows i0..i0+31.
+__device__ __forceinline__ uint32_t bwd_keep_bits(const MaskP& m, int b, int h, int64_t i0, int64_t j) {
+  uint32_t w = 0;
 #pragma unroll 1
-  for (int c = 0; c < kBMb; ++c)
-    if (dropout_keep(m, b, h, i0 + c, j)) w |= 1ull << c;
+  for (int c = 0; c < 32; ++c)
+    if (dropout_keep(m, b, h, i0 + c, j)) w |= 1u << c;
   return w;
 }
 
@@ -638,8 +670,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       mbar_init(smem_u32(&ctl->q_full[s]), 1);
       mbar_init(smem_u32(&ctl->q_empty[s]), 1);
       mbar_init(smem_u32(&ctl->st_full[s]), 1);
-      mbar_init(smem_u32(&ctl->st_empty[s]), 128);
-      mbar_init(smem_u32(&ctl->ds_full[s]), 128);
+      mbar_init(smem_u32(&ctl->st_empty[s]), 256);
+      mbar_init(smem_u32(&ctl->ds_full[s]), 256);
       mbar_init(smem_u32(&ctl->pds_empty[s]), 1);
       mbar_init(smem_u32(&ctl->dq_full[s]), 1);
       mbar_init(smem_u32(&ctl->dq_empty[s]), 128);
@@ -762,8 +794,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       ++n;
     }
     mma_commit(smem_u32(&ctl->acc_done));
-  } else if (warp >= 2 && warp < 6) {
-    // ---------------- compute warpgroup: thread t owns key row k0 + t
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------- compute warpgroups: thread t owns key row k0 + t; warpgroup
+    // hf handles query columns 32 hf .. 32 hf + 31 of each step.
+    const int hf = (warp - 4) >> 2;
     const int t = ((warp & 3) << 5) | lane;
     const int64_t j = (int64_t)k0 + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -775,91 +809,98 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const int s = n & 1;
       const uint32_t par = (n >> 1) & 1;
       const int64_t i0 = (int64_t)qs * kBMb;
-      const uint64_t allow = cls == kPartial ? bwd_col_bits(a, b, h, i0, j) : ~0ull;
-      const uint64_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0, j) : ~0ull;
+      const bool general = cls == kPartial || a.m.dropout;
+      const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
+      const uint32_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j) : ~0u;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->q_full[s]), par, abort_flag, a.status)))) break;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty[s]), par ^ 1, abort_flag, a.status))))
         break;
       tc_fence_after();
-      const float* lse2 = stat + s * 128;
-      const float* dl = lse2 + 64;
-      const uint32_t pt_base = sbase + kBwdPT + s * kPTile, ds_base = sbase + kBwdDS + s * kPTile;
+      uint32_t rs[32], rp[32];
+      tmem_ld32(tmem + lane_off + s * 128 + hf * 32, rs);
+      tmem_ld32(tmem + lane_off + s * 128 + 64 + hf * 32, rp);
+      const float* lse2 = stat + s * 128 + hf * 32;
+      const float* dl = stat + s * 128 + 64 + hf * 32;
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->st_empty[s]));
+      uint32_t ppk[16], dpk[16];
+      if (!general) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t rs[32], rp[32];
-        tmem_ld32(tmem + lane_off + s * 128 + half * 32, rs);
-        tmem_ld32(tmem + lane_off + s * 128 + 64 + half * 32, rp);
-        tmem_wait_ld();
-        uint32_t ppk[16], dpk[16];
+        for (int c2 = 0; c2 < 16; ++c2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + 2 * c2);
+          const float2 d2 = *reinterpret_cast<const float2*>(dl + 2 * c2);
+          const float p0 = ex2(fmaf(__uint_as_float(rs[2 * c2]), a.scale_log2, -l2.x));
+          const float p1 = ex2(fmaf(__uint_as_float(rs[2 * c2 + 1]), a.scale_log2, -l2.y));
+          ppk[c2] = pack_bf16(p0, p1);
+          dpk[c2] = pack_bf16(p0 * (__uint_as_float(rp[2 * c2]) - d2.x), p1 * (__uint_as_float(rp[2 * c2 + 1]) - d2.y));
+        }
+      } else {
+        const float inv = a.m.dropout ? a.m.inv_keep : 1.f;
 #pragma unroll
         for (int c2 = 0; c2 < 16; ++c2) {
           float pt[2], ds[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int c = half * 32 + 2 * c2 + e;
-            const float p = ((allow >> c) & 1ull) ? ex2(fmaf(__uint_as_float(rs[2 * c2 + e]), a.scale_log2, -lse2[c]))
-                                                   : 0.f;
-            const bool kp = (keep >> c) & 1ull;
+            const int c = 2 * c2 + e;
+            const float p = ((allow >> c) & 1u) ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, -lse2[c])) : 0.f;
+            const bool kp = (keep >> c) & 1u;
             // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
             pt[e] = kp ? p : 0.f;
-            const float dpv = kp ? __uint_as_float(rp[2 * c2 + e]) * (a.m.dropout ? a.m.inv_keep : 1.f) : 0.f;
+            const float dpv = kp ? __uint_as_float(rp[c]) * inv : 0.f;
             ds[e] = p * (dpv - dl[c]);
           }
           ppk[c2] = pack_bf16(pt[0], pt[1]);
           dpk[c2] = pack_bf16(ds[0], ds[1]);
         }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t off = sw128_offset(t, (half * 4 + cc) * 16);
-          st_shared_v4(pt_base + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
-          st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
-        }
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->st_empty[s]));
+      const uint32_t pt_base = sbase + kBwdPT + s * kPTile, ds_base = sbase + kBwdDS + s * kPTile;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t off = sw128_offset(t, (hf * 4 + cc) * 16);
+        st_shared_v4(pt_base + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
+        st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
+      }
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&ctl->ds_full[s]));
       ++n;
     }
-    // ---------------- epilogue: dK = c * sum gamma^T Q, dV = sum P~^T dO
+    // ---------------- epilogue: warpgroup 0 writes dK = c * sum gamma^T Q,
+    // warpgroup 1 writes dV = sum P~^T dO.
     bool have = false;
     if (ok && n > 0) {
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->acc_done), 0, abort_flag, a.status));
       if (ok) tc_fence_after();
       have = ok;
     }
-    const float dv_scale = a.m.dropout ? a.m.inv_keep : 1.f;
+    const float osc = hf == 0 ? a.scale : (a.m.dropout ? a.m.inv_keep : 1.f);
     if (ok || n == 0) {
-      __nv_bfloat16* dkr = a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2];
-      __nv_bfloat16* dvr = a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
+      __nv_bfloat16* orow = hf == 0 ? a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2]
+                                    : a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
+      const uint32_t tacc = (hf == 0 ? tDK : tDV) + lane_off;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t rk[32], rv[32];
+        uint32_t r[32];
         if (have) {
-          tmem_ld32(tDK + lane_off + c * 32, rk);
-          tmem_ld32(tDV + lane_off + c * 32, rv);
+          tmem_ld32(tacc + c * 32, r);
           tmem_wait_ld();
         }
         if (j < a.T) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t pk[4], pv[4];
+            uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int idx = c8 * 8 + e * 2;
-              pk[e] = have ? pack_bf16(__uint_as_float(rk[idx]) * a.scale, __uint_as_float(rk[idx + 1]) * a.scale)
-                           : 0u;
-              pv[e] = have ? pack_bf16(__uint_as_float(rv[idx]) * dv_scale, __uint_as_float(rv[idx + 1]) * dv_scale)
-                           : 0u;
+              pk[e] = have ? pack_bf16(__uint_as_float(r[idx]) * osc, __uint_as_float(r[idx + 1]) * osc) : 0u;
             }
-            *reinterpret_cast<uint4*>(dkr + c * 32 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(dvr + c * 32 + c8 * 8) = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+            *reinterpret_cast<uint4*>(orow + c * 32 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
         }
       }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 12) {
     // ---------------- dQ warpgroup: thread t owns head-dimension index t of
     // the dQ^T tile and stages it row-major for a bulk reduce-add.
     const int t = ((warp & 3) << 5) | lane;
@@ -1105,8 +1146,8 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   a.lse = lse;
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(fwd_kernel), kFwdSmem, 0)) != cudaSuccess) return err;
-  const int nqt = (p.T + kBM - 1) / kBM;
-  fwd_kernel<<<nqt * p.B * p.Hq, 256, kFwdSmem, st>>>(mq, mk, mv, a);
+  const int nct = (p.T + kFwdRows - 1) / kFwdRows;
+  fwd_kernel<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
