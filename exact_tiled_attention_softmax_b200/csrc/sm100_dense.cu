@@ -257,9 +257,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   volatile uint32_t* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Longest query tiles (most keys under a causal mask) first over the whole
+  // grid: the tail of the launch is made of the shortest tiles.
   const int nct = (a.T + kFwdRows - 1) / kFwdRows;
   const int bh = blockIdx.x % (a.B * a.Hq);
-  const int ct = nct - 1 - (int)(blockIdx.x / (a.B * a.Hq));  // longest query tiles first
+  const int ct = nct - 1 - (int)(blockIdx.x / (a.B * a.Hq));
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int kvh = h / (a.Hq / a.Hkv);
   const int q0 = ct * kFwdRows;
@@ -417,19 +419,38 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[w]), n & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      // Pass 1 over the S row: the masked maximum (64 columns per TMEM load).
+      const bool fast = cls == kFull && !a.m.dropout;
+      // Pass 1 over the S row: the (masked) maximum, 64 columns per TMEM load.
       float mx = -INFINITY;
+      if (fast) {
+        // Every key allowed: extremum of the raw scores, scaled once.
+        float hi = -INFINITY, lo = INFINITY;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tS + hf * 64, r0);
-        tmem_ld32(tS + hf * 64 + 32, r1);
-        tmem_wait_ld();
-        const uint64_t mw = hf ? mw1 : mw0;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tS + hf * 64, r0);
+          tmem_ld32(tS + hf * 64 + 32, r1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if ((mw >> e) & 1ull) mx = fmaxf(mx, __uint_as_float(r0[e]) * a.scale_log2);
-          if ((mw >> (32 + e)) & 1ull) mx = fmaxf(mx, __uint_as_float(r1[e]) * a.scale_log2);
+          for (int e = 0; e < 32; ++e) {
+            hi = fmaxf(hi, fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+            lo = fminf(lo, fminf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
+          }
+        }
+        mx = a.scale_log2 >= 0.f ? hi * a.scale_log2 : lo * a.scale_log2;
+      } else {
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tS + hf * 64, r0);
+          tmem_ld32(tS + hf * 64 + 32, r1);
+          tmem_wait_ld();
+          const uint64_t mw = hf ? mw1 : mw0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if ((mw >> e) & 1ull) mx = fmaxf(mx, __uint_as_float(r0[e]) * a.scale_log2);
+            if ((mw >> (32 + e)) & 1ull) mx = fmaxf(mx, __uint_as_float(r1[e]) * a.scale_log2);
+          }
         }
       }
       float m_new = m_run;
@@ -452,24 +473,44 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       // Pass 2: p = 2^(s - m), written back as bf16 pairs over the first 64
       // columns (P chunk q covers S columns already read).
       float sum = 0.f;
+      if (fast) {
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tS + q * 32, r);
-        tmem_wait_ld();
-        const uint64_t mw = q < 2 ? mw0 : mw1;
-        const uint64_t kw = q < 2 ? kb0 : kb1;
-        uint32_t pk[16];
+        for (int q = 0; q < 4; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tS + q * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int bit = (q * 32 + 2 * e) & 63;
-          const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * a.scale_log2 - msub) : 0.f;
-          const float p1 = ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * a.scale_log2 - msub) : 0.f;
-          sum += p0 + p1;
-          // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
-          pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -msub));
+            const float p1 = ex2(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -msub));
+            sum += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + q * 16, pk);
         }
-        tmem_st16(tS + q * 16, pk);
+      } else {
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t r[32];
+          tmem_ld32(tS + q * 32, r);
+          tmem_wait_ld();
+          const uint64_t mw = q < 2 ? mw0 : mw1;
+          const uint64_t kw = q < 2 ? kb0 : kb1;
+          const int base = (q & 1) * 32;
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int bit = base + 2 * e;
+            const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * a.scale_log2 - msub) : 0.f;
+            const float p1 =
+                ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * a.scale_log2 - msub) : 0.f;
+            sum += p0 + p1;
+            // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
+            pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+          }
+          tmem_st16(tS + q * 16, pk);
+        }
       }
       l_run = l_run * alpha + sum;
       m_run = m_new;
@@ -555,21 +596,22 @@ constexpr uint32_t kQTile = kBMb * kD * 2;  // 16 KB: 64 rows x 128 bf16
 constexpr uint32_t kPTile = kBN * kBMb * 2; // 16 KB: 128 keys x 64 queries bf16
 constexpr uint32_t kBwdK = 0;
 constexpr uint32_t kBwdV = kBwdK + kTileBytes;
-constexpr uint32_t kBwdQ = kBwdV + kTileBytes;          // 2 stages
-constexpr uint32_t kBwdG = kBwdQ + 2 * kQTile;          // 2 stages
-constexpr uint32_t kBwdPT = kBwdG + 2 * kQTile;         // 2 buffers
-constexpr uint32_t kBwdDS = kBwdPT + 2 * kPTile;        // 2 buffers
-constexpr uint32_t kBwdDQ = kBwdDS + 2 * kPTile;        // 32 query rows x 128 fp32 = 16 KB
-constexpr uint32_t kBwdStat = kBwdDQ + 32 * kD * 4;     // 2 stages x (64 lse2 + 64 delta) fp32
-constexpr uint32_t kBwdCtl = kBwdStat + 2 * 512;
-constexpr uint32_t kBwdSmem = kBwdCtl + 1024 + 1024;
+constexpr int kQStages = 3;                             // Q / dO / LSE / delta ring depth
+constexpr int kBwdBand = 8;                             // (b, K/V head) pairs per scheduling band
+constexpr uint32_t kBwdQ = kBwdV + kTileBytes;          // kQStages x 16 KB
+constexpr uint32_t kBwdG = kBwdQ + kQStages * kQTile;   // kQStages x 16 KB
+constexpr uint32_t kBwdDS = kBwdG + kQStages * kQTile;  // 2 buffers of gamma^T (P^T lives in TMEM)
+constexpr uint32_t kBwdDQ = kBwdDS + 2 * kPTile;        // 4 warps x (64 rows x 32 fp32) = 32 KB
+constexpr uint32_t kBwdStat = kBwdDQ + 4 * kBMb * 32 * 4;  // kQStages x (64 lse2 + 64 delta) fp32
+constexpr uint32_t kBwdCtl = kBwdStat + kQStages * 512;
+constexpr uint32_t kBwdSmem = kBwdCtl + 256 + 1024;     // control block + alignment slack
 // Warps: 0 TMA producer, 1 MMA issuer, 2-3 idle, 4-7 and 8-11 the two compute
 // warpgroups (query columns 0-31 and 32-63 of each step), 12-15 dQ warpgroup.
 constexpr int kBwdThreads = 512;
 
 struct BwdCtl {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[kQStages], q_empty[kQStages];
   uint64_t st_full[2], st_empty[2];
   uint64_t ds_full[2], pds_empty[2];
   uint64_t dq_full[2], dq_empty[2];
@@ -632,10 +674,12 @@ __device__ __forceinline__ uint32_t bwd_keep_bits(const MaskP& m, int b, int h, 
   return w;
 }
 
-__device__ __forceinline__ void red_bulk_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(gdst)),
-               "r"(ssrc), "r"(bytes)
+// Element-wise add of a shared-memory box into global memory through a tensor
+// map; boxes reaching past the tensor's extent are clipped.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t ssrc, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(ssrc), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -643,11 +687,11 @@ __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void dq_group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, const BwdArgs a) {
+           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
+           const __grid_constant__ CUtensorMap tdq, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -657,8 +701,17 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int group = a.Hq / a.Hkv;
-  const int bkv = blockIdx.x % (a.B * a.Hkv);
-  const int kt = (int)(blockIdx.x / (a.B * a.Hkv));  // earliest key tiles (most work) first
+  // Bands of kBwdBand (b, K/V head) pairs: within a band the earliest key tiles
+  // (most work under a causal mask) go first; the CTAs resident at any time
+  // then share a few heads' dQ accumulator rows and Q/dO in L2.
+  const int nkt_all = (a.T + kBN - 1) / kBN;
+  const int nbkv = a.B * a.Hkv;
+  const int band = (int)(blockIdx.x / ((int64_t)kBwdBand * nkt_all));
+  const int band0 = band * kBwdBand;
+  const int bw = nbkv - band0 < kBwdBand ? nbkv - band0 : kBwdBand;
+  const int within = (int)(blockIdx.x - (int64_t)band0 * nkt_all);
+  const int kt = within / bw;
+  const int bkv = band0 + within % bw;
   const int kvh = bkv % a.Hkv, b = bkv / a.Hkv;
   const int k0 = kt * kBN;
   int qs_lo, qs_hi;
@@ -666,9 +719,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->kv_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(smem_u32(&ctl->q_full[s]), 1);
       mbar_init(smem_u32(&ctl->q_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->st_full[s]), 1);
       mbar_init(smem_u32(&ctl->st_empty[s]), 256);
       mbar_init(smem_u32(&ctl->ds_full[s]), 256);
@@ -688,8 +743,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  // TMEM columns: two S^T | dP^T buffers (0..127, 128..255; dQ^T of a step
-  // reuses the S^T half of its buffer), dV 256..383, dK 384..511.
+  // TMEM columns: two S^T | dP^T buffers (0..127, 128..255). In a step's
+  // buffer, P~^T (bf16 pairs) is written over the dP^T half once read, and
+  // dQ^T reuses the S^T half. dV 256..383, dK 384..511.
   const uint32_t tDV = tmem + 256, tDK = tmem + 384;
 
   if (warp == 0 && lane == 0) {
@@ -708,8 +764,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     uint8_t cls;
     while (bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
       const int h = kvh * group + hh;
-      const int s = n & 1;
-      if (!wait_bar(smem_u32(&ctl->q_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+      const int s = n % kQStages;
+      if (!wait_bar(smem_u32(&ctl->q_empty[s]), ((n / kQStages) & 1) ^ 1, abort_flag, a.status)) break;
       const uint32_t qf = smem_u32(&ctl->q_full[s]);
       mbar_expect_tx(qf, 2 * kQTile + 512);
       const uint32_t qd = sbase + kBwdQ + s * kQTile, gd = sbase + kBwdG + s * kQTile;
@@ -722,8 +778,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       bulk_load(sbase + kBwdStat + s * 512 + 256, a.dpad + roff, 256, qf);
       ++n;
     }
-    for (int r = (n > 2 ? n - 2 : 0); r < n; ++r)
-      wait_bar(smem_u32(&ctl->q_full[r & 1]), (r >> 1) & 1, abort_flag, nullptr);
+    for (int r = (n > kQStages ? n - kQStages : 0); r < n; ++r)
+      wait_bar(smem_u32(&ctl->q_full[r % kQStages]), (r / kQStages) & 1, abort_flag, nullptr);
     wait_bar(kvf, 0, abort_flag, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S^T/dP^T of step n+1 go ahead of the
@@ -734,13 +790,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
     bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
     auto issue_st = [&](int m) -> bool {
-      const int s = m & 1;
+      const int s = m & 1, sq = m % kQStages;
       const uint32_t par = (m >> 1) & 1;
-      if (!wait_bar(smem_u32(&ctl->q_full[s]), par, abort_flag, a.status)) return false;
+      if (!wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)) return false;
       if (!wait_bar(smem_u32(&ctl->st_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       if (!wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       tc_fence_after();
-      const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
+      const uint32_t qa = sbase + kBwdQ + sq * kQTile, ga = sbase + kBwdG + sq * kQTile;
       const uint32_t dst = tmem + s * 128;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
@@ -768,15 +824,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint8_t ncls;
       const bool next = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
       if (next && !(ok = issue_st(n + 1))) break;
-      const int s = n & 1;
+      const int s = n & 1, sq = n % kQStages;
       if (!(ok = wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      const uint32_t qa = sbase + kBwdQ + s * kQTile, ga = sbase + kBwdG + s * kQTile;
-      const uint32_t pta = sbase + kBwdPT + s * kPTile, dsa = sbase + kBwdDS + s * kPTile;
+      const uint32_t qa = sbase + kBwdQ + sq * kQTile, ga = sbase + kBwdG + sq * kQTile;
+      const uint32_t dsa = sbase + kBwdDS + s * kPTile;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows
-        mma_ss(tDV, smem_desc_sw128(pta + kk * 32, 16, 1024), smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC,
-               (n > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows; A = P~^T from TMEM (16 rows = 8 columns)
+        mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
+               smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kHalfQ, 1024), idACC,
@@ -785,7 +841,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
         mma_ss(tmem + s * 128, smem_desc_sw128(sbase + kBwdK + kk * 2048, kTileBytes / 2, 1024),
                smem_desc_sw128(dsa + kk * 2048, kHalfQ, 1024), idDQ, kk > 0);
-      mma_commit(smem_u32(&ctl->q_empty[s]));
+      mma_commit(smem_u32(&ctl->q_empty[sq]));
       mma_commit(smem_u32(&ctl->pds_empty[s]));
       mma_commit(smem_u32(&ctl->dq_full[s]));
       hh = nh;
@@ -806,25 +862,25 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     bool ok = true;
     while (ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
       const int h = kvh * group + hh;
-      const int s = n & 1;
+      const int s = n & 1, sq = n % kQStages;
       const uint32_t par = (n >> 1) & 1;
       const int64_t i0 = (int64_t)qs * kBMb;
       const bool general = cls == kPartial || a.m.dropout;
       const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
       const uint32_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j) : ~0u;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
-      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->q_full[s]), par, abort_flag, a.status)))) break;
+      if (!(ok = __all_sync(0xffffffffu,
+                            wait_bar(smem_u32(&ctl->q_full[sq]), (n / kQStages) & 1, abort_flag, a.status))))
+        break;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty[s]), par ^ 1, abort_flag, a.status))))
         break;
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tmem + lane_off + s * 128 + hf * 32, rs);
       tmem_ld32(tmem + lane_off + s * 128 + 64 + hf * 32, rp);
-      const float* lse2 = stat + s * 128 + hf * 32;
-      const float* dl = stat + s * 128 + 64 + hf * 32;
+      const float* lse2 = stat + sq * 128 + hf * 32;
+      const float* dl = stat + sq * 128 + 64 + hf * 32;
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->st_empty[s]));
       uint32_t ppk[16], dpk[16];
       if (!general) {
 #pragma unroll
@@ -855,13 +911,17 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           dpk[c2] = pack_bf16(ds[0], ds[1]);
         }
       }
-      const uint32_t pt_base = sbase + kBwdPT + s * kPTile, ds_base = sbase + kBwdDS + s * kPTile;
+      // P~^T as bf16 pairs over this warpgroup's own dP^T columns (already read).
+      tmem_st16(tmem + lane_off + s * 128 + 64 + hf * 32, ppk);
+      const uint32_t ds_base = sbase + kBwdDS + s * kPTile;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const uint32_t off = sw128_offset(t, (hf * 4 + cc) * 16);
-        st_shared_v4(pt_base + off, ppk[cc * 4], ppk[cc * 4 + 1], ppk[cc * 4 + 2], ppk[cc * 4 + 3]);
         st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl->st_empty[s]));
       fence_proxy_async_smem();
       mbar_arrive(smem_u32(&ctl->ds_full[s]));
       ++n;
@@ -901,11 +961,15 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
     }
   } else if (warp >= 12) {
-    // ---------------- dQ warpgroup: thread t owns head-dimension index t of
-    // the dQ^T tile and stages it row-major for a bulk reduce-add.
-    const int t = ((warp & 3) << 5) | lane;
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    float* stage = reinterpret_cast<float*>(smem + kBwdDQ);
+    // ---------------- dQ warpgroup: warp wq reads head-dimension indices
+    // 32 wq .. 32 wq + 31 of the dQ^T tile (its TMEM lanes), stages them as a
+    // [64 rows][32] fp32 box and adds the box into the fp32 accumulator with
+    // a TMA reduce; rows past T are clipped by the tensor map.
+    const int wq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t stage_s = sbase + kBwdDQ + wq * (kBMb * 32 * 4);
+    float* stage = reinterpret_cast<float*>(smem + kBwdDQ + wq * (kBMb * 32 * 4));
+    if (lane == 0) tma_prefetch_desc(&tdq);
     int n = 0, hh = 0, qs = qs_lo - 1;
     uint8_t cls;
     bool ok = true;
@@ -921,26 +985,22 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl->dq_empty[s]));
-      const int64_t i0 = (int64_t)qs * kBMb;
-      const int rows = (int)((a.T - i0) < kBMb ? (a.T - i0) : kBMb);
-      float* dst = a.dq_acc + (((int64_t)b * a.Hq + h) * a.T + i0) * kD;
+      if (lane == 0) bulk_wait_read0();  // the previous reduce has read this warp's box
+      __syncwarp();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (t == 0) bulk_wait_read0();  // the previous reduce has read the stage
-        dq_group_sync();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) stage[e * kD + t] = __uint_as_float(half ? r1[e] : r0[e]);
-        fence_proxy_async_smem();
-        dq_group_sync();
-        const int hr = rows - half * 32 < 32 ? rows - half * 32 : 32;
-        if (t == 0 && hr > 0) {
-          red_bulk_add_f32(dst + (int64_t)half * 32 * kD, sbase + kBwdDQ, (uint32_t)hr * kD * 4);
-          bulk_commit();
-        }
+      for (int e = 0; e < 32; ++e) {
+        stage[e * 32 + lane] = __uint_as_float(r0[e]);
+        stage[(32 + e) * 32 + lane] = __uint_as_float(r1[e]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&tdq, stage_s, 32 * wq, qs * kBMb, b * a.Hq + h);
+        bulk_commit();
       }
       ++n;
     }
-    if (t == 0) bulk_wait0();
+    if (lane == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -1043,6 +1103,20 @@ bool make_map(CUtensorMap* map, const void* base, int T, int H, int B, int64_t s
 int block_aligned(const MaskP& m) {
   if (!(m.flags & ATTN_MASK_BLOCK)) return 1;
   return (m.bq % kBMb == 0 && m.bk % kBN == 0) ? 1 : 0;
+}
+
+// 3-D fp32 map over the dQ accumulator [B*Hq][T][128] with a (32, 64, 1) box,
+// no swizzle: the reduce-add target of the reverse kernel.
+bool make_dq_map(CUtensorMap* map, float* base, int T, int BH) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)kD * 4, (cuuint64_t)T * kD * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)kBMb, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool tma_ok(const attn_tensor* t) {
@@ -1167,8 +1241,9 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
       static_cast<const __nv_bfloat16*>(o), so[0], so[1], so[2], static_cast<const __nv_bfloat16*>(g), sg[0], sg[1],
       sg[2], lse, sl[0], sl[1], sl[2], p.B, p.Hq, p.T, Tpad, lse2, dpad, delta, dq_acc);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  CUtensorMap mq, mk, mv, mg;
-  if (!make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
+  CUtensorMap mq, mk, mv, mg, mdq;
+  if (!make_dq_map(&mdq, dq_acc, p.T, p.B * p.Hq) ||
+      !make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
       !make_map(&mk, p.k, p.T, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
       !make_map(&mv, p.v, p.T, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN) ||
       !make_map(&mg, g, p.T, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb))
@@ -1196,7 +1271,7 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
   const int nkt = (p.T + kBN - 1) / kBN;
-  bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, a);
+  bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n4 = (int64_t)p.B * p.Hq * p.T * kD / 4;
   dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.T, p.scale,
