@@ -55,8 +55,12 @@ def _run_gpu(c):
         block_q=c["block"] or 128, block_k=c["block"] or 128,
         sink=to_dev(c["sink"], torch.float32) if c["sink"] is not None else None,
         dropout_p=c["dropout"], dropout_seed=c["seed"])
-    o, lse = eta.attn_fwd(q, k, v, allowed, c["scale"])
-    dq, dk, dv, dsink = eta.attn_bwd(q, k, v, o, g, lse, allowed, c["scale"])
+    wf = torch.empty(eta.attn_fwd_workspace_size(q, k, v, allowed), dtype=torch.uint8, device="cuda")
+    wb = torch.empty(eta.attn_bwd_workspace_size(q, k, v, allowed), dtype=torch.uint8, device="cuda")
+    o, lse = eta.attn_fwd(q, k, v, allowed, c["scale"], workspace=wf)
+    assert eta.attn_get_status(wf) == 0, "device status after attn_fwd"
+    dq, dk, dv, dsink = eta.attn_bwd(q, k, v, o, g, lse, allowed, c["scale"], workspace=wb)
+    assert eta.attn_get_status(wb) == 0, "device status after attn_bwd"
     torch.cuda.synchronize()
     return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, dsink=dsink, inputs=(q, k, v, g), allowed=allowed)
 
