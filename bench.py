@@ -122,6 +122,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside), "sampled": where}
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the ncu capture
+    recorded in profiles/dram_traffic.json, or None when the kernel source
+    has changed since that capture (its SHA-256 no longer matches)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)[kernel][workload]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if digest != rec["source_sha256"]:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 def cpu_baseline(case: W.DenseCase, budget_s: float = 12.0):
     """The float64 oracle, as it stands, on a bounded sample of the workload:
     whole (b, h) slices of the same shape, one after another, until the time
@@ -227,6 +244,13 @@ def main():
     n_ev = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    # Events around the main kernel of each call (fwd_kernel, bwd_kernel),
+    # recorded by the library itself on the launching stream.
+    kev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n_ev)]
+    for evs in kev:
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -235,9 +259,12 @@ def main():
         for s in range(n_ev):
             flush.fill_(s & 0xFF)
             e0, e1, e2 = ev[s]
+            k0, k1, k2, k3 = kev[s]
             e0.record(stream)
+            eta.attn_set_kernel_events(k0, k1)
             eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
             e1.record(stream)
+            eta.attn_set_kernel_events(k2, k3)
             eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
             e2.record(stream)
         torch.cuda.synchronize()
@@ -248,6 +275,8 @@ def main():
         dist.barrier()
     t_fwd = [a.elapsed_time(b) for a, b, _ in ev]
     t_bwd = [b.elapsed_time(c) for _, b, c in ev]
+    t_fwd_kernel = [k0.elapsed_time(k1) for k0, k1, _, _ in kev]
+    t_bwd_kernel = [k2.elapsed_time(k3) for _, _, k2, k3 in kev]
     total_ms = sum(f + b for f, b in zip(t_fwd, t_bwd))
     if world > 1:
         tt = torch.tensor([total_ms], device=dev)
@@ -291,9 +320,13 @@ def main():
     peak = float(peaks["bf16_tflops"])
     bwd_ms = statistics.mean(t_bwd)
     bwd_flops = pairs * (6 * case.d + 4 * case.dv)
-    achieved = bwd_flops / (bwd_ms / 1e3) / 1e12
     fwd_ms = statistics.mean(t_fwd)
-    fwd_achieved = pairs * (2 * case.d + 2 * case.dv) / (fwd_ms / 1e3) / 1e12
+    fwd_flops = pairs * (2 * case.d + 2 * case.dv)
+    fwd_achieved = fwd_flops / (fwd_ms / 1e3) / 1e12
+    bwd_kernel_ms = statistics.mean(t_bwd_kernel)
+    fwd_kernel_ms = statistics.mean(t_fwd_kernel)
+    achieved = bwd_flops / (bwd_kernel_ms / 1e3) / 1e12
+    traffic = recorded_traffic("bwd_kernel", case.name)
 
     if rank == 0:
         clocks = clk.summary()
@@ -307,10 +340,16 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "pct_of_peak": {"measured_bf16_burst": 100 * value / world / peak,
                             "nvidia_dense_bf16_spec_2250": 100 * value / world / 2250.0},
-            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_achieved, "bwd_tflops": achieved,
-            "roofline": {"bound": "tensor", "kernel": "attn_bwd (prepare + bwd_kernel + dq_finish)",
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_achieved,
+            "bwd_tflops": bwd_flops / (bwd_ms / 1e3) / 1e12,
+            "kernels": {"fwd_kernel": {"ms": fwd_kernel_ms, "tflops": fwd_flops / (fwd_kernel_ms / 1e3) / 1e12},
+                        "bwd_kernel": {"ms": bwd_kernel_ms, "tflops": achieved}},
+            "roofline": {"bound": "tensor", "kernel": "bwd_kernel",
                          "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                         "traffic": None, "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"},
+                         "traffic": traffic,
+                         "work_per_launch": f"{bwd_flops:.4e} flops = {pairs} allowed pairs x "
+                                            f"{6 * case.d + 4 * case.dv} (6d + 4dv)",
+                         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"},
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 4 * args.steps,

@@ -16,8 +16,8 @@ import torch
 
 __all__ = [
     "AllowedSet", "AttnError", "attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_fwd_workspace_size",
-    "attn_bwd_workspace_size", "attn_get_status", "attn_status_string", "attn_version",
-    "library_path", "load_library",
+    "attn_bwd_workspace_size", "attn_get_status", "attn_set_kernel_events", "attn_status_string",
+    "attn_version", "library_path", "load_library",
 ]
 
 ATTN_OK = 0
@@ -91,6 +91,8 @@ def load_library():
     lib.attn_bwd_noalloc.argtypes = [T, T, T, T, T, T, M, ctypes.c_float, T, T, T, vp, vp]
     lib.attn_get_status.restype = ctypes.c_int
     lib.attn_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.attn_set_kernel_events.restype = ctypes.c_int
+    lib.attn_set_kernel_events.argtypes = [vp, vp]
     _LIB = lib
     return lib
 
@@ -293,3 +295,17 @@ def attn_get_status(workspace: torch.Tensor, stream=None) -> int:
     if rc not in (ATTN_OK, ATTN_ERR_DEVICE):
         raise AttnError(rc, "attn_get_status")
     return int(bits.value)
+
+
+def attn_set_kernel_events(begin: "torch.cuda.Event | None", end: "torch.cuda.Event | None") -> None:
+    """Have the next attn_fwd / attn_bwd call on this thread record `begin`
+    and `end` around its main kernel (timing events created with
+    enable_timing=True). Each event is recorded once here first so that its
+    CUDA handle exists; None, None cancels."""
+    if begin is None or end is None:
+        load_library().attn_set_kernel_events(None, None)
+        return
+    for ev in (begin, end):
+        if not ev.cuda_event:
+            ev.record()
+    load_library().attn_set_kernel_events(ctypes.c_void_p(begin.cuda_event), ctypes.c_void_p(end.cuda_event))

@@ -150,8 +150,36 @@ size_t bwd_topk_bytes(const Topk& s) {
 
 }  // namespace
 
+namespace attn {
+
+namespace {
+thread_local cudaEvent_t g_kernel_ev[2] = {nullptr, nullptr};
+}  // namespace
+
+void main_kernel_begin(cudaStream_t st) {
+  if (g_kernel_ev[0]) cudaEventRecord(g_kernel_ev[0], st);
+}
+
+void main_kernel_end(cudaStream_t st) {
+  if (g_kernel_ev[1]) cudaEventRecord(g_kernel_ev[1], st);
+  g_kernel_ev[0] = g_kernel_ev[1] = nullptr;
+}
+
+// A pending event pair applies to one call only, whichever way it returns.
+struct ForgetKernelEvents {
+  ~ForgetKernelEvents() { g_kernel_ev[0] = g_kernel_ev[1] = nullptr; }
+};
+
+}  // namespace attn
+
 #pragma GCC visibility push(default)
 extern "C" {
+
+attn_status attn_set_kernel_events(void* begin, void* end) {
+  attn::g_kernel_ev[0] = static_cast<cudaEvent_t>(begin);
+  attn::g_kernel_ev[1] = static_cast<cudaEvent_t>(end);
+  return ATTN_OK;
+}
 
 int attn_version(void) { return ATTN_VERSION; }
 
@@ -193,6 +221,8 @@ size_t attn_bwd_workspace_size(const attn_tensor* q, const attn_tensor* k, const
 attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
                      const attn_mask* mask, float scale, attn_tensor* o, attn_tensor* lse,
                      void* workspace, size_t workspace_bytes, void* stream) {
+  attn::ForgetKernelEvents forget_events;
+
   attn_status st = check_mask(mask);
   if (st != ATTN_OK) return st;
   if (!o || !lse || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -227,12 +257,14 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.Dv = s.Dv;
     p.scale = scale;
     p.sink = mask->sink;
+    main_kernel_begin(cs);
     cudaError_t e = q->dtype == ATTN_F32
         ? launch_topk_fwd_rows<float>(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
                                       lse->stride[0], lse->stride[1], status, cs)
         : launch_topk_fwd_rows<__nv_bfloat16>(p, o->data, o->stride[0], o->stride[1],
                                               static_cast<float*>(lse->data), lse->stride[0], lse->stride[1],
                                               status, cs);
+    main_kernel_end(cs);
     return cuda_status(e);
   }
 
@@ -270,8 +302,10 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     return cuda_status(sm100_dense_fwd(p, o->data, so, lsep, sl, static_cast<char*>(workspace) + kStatusBytes,
                                        status, cs));
   }
+  main_kernel_begin(cs);
   cudaError_t e = q->dtype == ATTN_F32 ? launch_dense_fwd_rows<float>(p, o->data, so, lsep, sl, cs)
                                        : launch_dense_fwd_rows<__nv_bfloat16>(p, o->data, so, lsep, sl, cs);
+  main_kernel_end(cs);
   return cuda_status(e);
 }
 
@@ -279,6 +313,8 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
                      const attn_tensor* do_, const attn_tensor* lse, const attn_mask* mask, float scale,
                      attn_tensor* dq, attn_tensor* dk, attn_tensor* dv, float* dsink, void* workspace,
                      size_t workspace_bytes, void* stream) {
+  attn::ForgetKernelEvents forget_events;
+
   attn_status st = check_mask(mask);
   if (st != ATTN_OK) return st;
   if (!o || !do_ || !lse || !dq || !dk || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
@@ -327,18 +363,22 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     cudaError_t e;
     if (q->dtype == ATTN_F32) {
       e = launch_rows_delta<float>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
+      main_kernel_begin(cs);
       if (e == cudaSuccess)
         e = launch_topk_bwd_rows<float>(p, do_->data, do_->stride[0], do_->stride[1],
                                         static_cast<const float*>(lse->data), lse->stride[0], lse->stride[1],
                                         delta, dq->data, dq->stride[0], dq->stride[1], acc, dk->data,
                                         dk->stride[0], status, cs);
+      main_kernel_end(cs);
     } else {
       e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
+      main_kernel_begin(cs);
       if (e == cudaSuccess)
         e = launch_topk_bwd_rows<__nv_bfloat16>(p, do_->data, do_->stride[0], do_->stride[1],
                                                 static_cast<const float*>(lse->data), lse->stride[0],
                                                 lse->stride[1], delta, dq->data, dq->stride[0], dq->stride[1],
                                                 acc, dk->data, dk->stride[0], status, cs);
+      main_kernel_end(cs);
     }
     if (e == cudaSuccess && want_dsink)
       e = launch_dsink(mask->sink, static_cast<const float*>(lse->data), delta, s.Tq, s.H, 1, lse->stride[0],
@@ -395,14 +435,18 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
                         dv->data, sdv, extra, status, cs);
   } else if (q->dtype == ATTN_F32) {
     e = launch_rows_delta<float>(o->data, do_->data, s.B, s.Hq, s.T, so, sg, s.dv, delta, cs);
+    main_kernel_begin(cs);
     if (e == cudaSuccess)
       e = launch_dense_bwd_rows<float>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk, dv->data,
                                        sdv, cs);
+    main_kernel_end(cs);
   } else {
     e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, s.B, s.Hq, s.T, so, sg, s.dv, delta, cs);
+    main_kernel_begin(cs);
     if (e == cudaSuccess)
       e = launch_dense_bwd_rows<__nv_bfloat16>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk,
                                                dv->data, sdv, cs);
+    main_kernel_end(cs);
   }
   if (e == cudaSuccess && want_dsink)
     e = launch_dsink(mask->sink, lsep, delta, s.B, s.Hq, s.T, sl[0], sl[1], sl[2], true, dsink, cs);

@@ -133,4 +133,9 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Caller-supplied timing events around the main kernel of the next call on
+// this host thread (attn_set_kernel_events); no-ops when none is pending.
+void main_kernel_begin(cudaStream_t st);
+void main_kernel_end(cudaStream_t st);
+
 }  // namespace attn

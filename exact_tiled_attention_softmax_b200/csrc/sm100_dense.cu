@@ -1221,7 +1221,9 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(fwd_kernel), kFwdSmem, 0)) != cudaSuccess) return err;
   const int nct = (p.T + kFwdRows - 1) / kFwdRows;
+  main_kernel_begin(st);
   fwd_kernel<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
+  main_kernel_end(st);
   return cudaGetLastError();
 }
 
@@ -1271,7 +1273,9 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
   const int nkt = (p.T + kBN - 1) / kBN;
+  main_kernel_begin(st);
   bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
+  main_kernel_end(st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n4 = (int64_t)p.B * p.Hq * p.T * kD / 4;
   dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.T, p.scale,

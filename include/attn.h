@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 100 /* major * 100 + minor */
+#define ATTN_VERSION 101 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -189,6 +189,16 @@ attn_status attn_bwd_noalloc(const attn_tensor* q, const attn_tensor* k,
  * start of `workspace`. *device_bits receives the ATTN_DEVERR_* bits (0 when
  * clean). Returns ATTN_ERR_DEVICE when any bit was set. */
 attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits);
+
+/* Kernel timing without a profiler. `begin` and `end` are cudaEvent_t
+ * handles created and owned by the caller. The next attn_fwd or attn_bwd
+ * call made from the same host thread records `begin` on its stream just
+ * before its main kernel (the tensor-core kernel, or the row-wise kernels
+ * that do the attention arithmetic) and `end` just after it, then forgets
+ * both, whether or not the call launched anything; the small setup and
+ * finishing kernels around it (tile classes, delta, the dq cast) fall
+ * outside the pair. NULL, NULL cancels a pending pair. Always ATTN_OK. */
+attn_status attn_set_kernel_events(void* begin, void* end);
 
 /* Static, human-readable text for a status code. */
 const char* attn_status_string(attn_status status);
