@@ -41,6 +41,12 @@ constexpr int kBMb = 64;         // reverse query rows per step
 constexpr int kStages = 2;       // K/V ring depth (forward), Q/dO ring depth (reverse)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // move the running max only past 2^8
+constexpr int kPolyEvery = 0;              // forward: every k-th pair of exponentials on the FMA pipe (0: none)
+
+// Does pair e of a 16-pair chunk take its exponentials on the FMA pipe?
+__host__ __device__ constexpr bool poly_pair(int e) {
+  return kPolyEvery > 0 && e % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
+}
 
 enum : uint8_t { kEmpty = 0, kFull = 1, kPartial = 2 };
 
@@ -163,6 +169,9 @@ struct FwdCtl {
   uint64_t o_final;
   uint32_t tmem_base;
   uint32_t abort_flag;
+  // Per K/V stage, written by the producer before the stage's loads: bit w =
+  // the tile has allowed keys for query tile w, bit 2 = another tile follows.
+  uint32_t tinfo[kStages];
 };
 
 // Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
@@ -184,6 +193,19 @@ __device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int
 __device__ __forceinline__ uint8_t wg_class(const FwdArgs& a, int b, int h, int qt, int kt) {
   if (qt * kBM >= a.T) return kEmpty;
   return fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
+}
+
+// First key tile after `from` (up to kt_hi) with allowed keys for either
+// query tile of the CTA (qt0, qt0 + 1); kt_hi + 1 when none. flags: bit w
+// set when query tile qt0 + w has allowed keys there.
+__device__ __forceinline__ int fwd_next_tile(const FwdArgs& a, int b, int h, int qt0, int kt_hi, int from,
+                                             uint32_t& flags) {
+  for (int kt = from + 1; kt <= kt_hi; ++kt) {
+    flags = (wg_class(a, b, h, qt0, kt) != kEmpty ? 1u : 0u) | (wg_class(a, b, h, qt0 + 1, kt) != kEmpty ? 2u : 0u);
+    if (flags) return kt;
+  }
+  flags = 0;
+  return kt_hi + 1;
 }
 
 // Bits lo..hi (inclusive, within [0, 63]) of a 64-bit word; 0 when lo > hi.
@@ -241,6 +263,135 @@ __device__ __forceinline__ void fwd_keep_bits(const MaskP& m, int b, int h, int6
   }
 }
 
+// New running maximum after a tile whose (scaled, base-2) maximum is mx:
+// moved only when mx exceeds it by more than the threshold (or on the first
+// tile with an allowed key). Returns the factor alpha = 2^(m_old - m_new) that
+// rescales the earlier terms (0 when there were none, 1 when m stays).
+__device__ __forceinline__ float move_max(float mx, float& m_run) {
+  float m_new = m_run;
+  if (mx > -INFINITY && (m_run == -INFINITY || mx > m_run + kRescaleThreshold)) m_new = fmaxf(mx, m_run);
+  const float alpha = (m_new == m_run) ? 1.f : ex2(m_run - m_new);
+  m_run = m_new;
+  return alpha;
+}
+
+// One S row (128 keys, all allowed, no dropout) of the calling thread's TMEM
+// lane -> P (bf16 pairs written over the row's first 64 columns), with the
+// running summary (m_run, l_run) updated. The row stays in registers between
+// the maximum and the exponentials (one TMEM wait); x = s c log2(e) - m is
+// formed on packed fp32 pairs and every kPolyEvery-th pair of exponentials
+// runs on the FMA pipe instead of MUFU. Returns alpha.
+__device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2, float& m_run, float& l_run) {
+  uint32_t s0[32], s1[32], s2[32], s3[32];
+  tmem_ld32(tS, s0);
+  tmem_ld32(tS + 32, s1);
+  tmem_ld32(tS + 64, s2);
+  tmem_ld32(tS + 96, s3);
+  tmem_wait_ld();
+  // Extremum of the raw scores, scaled once.
+  float mx;
+  if (scale_log2 >= 0.f) {
+    float e0 = -INFINITY, e1 = -INFINITY, e2 = -INFINITY, e3 = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      e0 = max3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+      e1 = max3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+      e2 = max3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
+      e3 = max3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
+    }
+    mx = max3f(e0, e1, fmaxf(e2, e3)) * scale_log2;
+  } else {
+    float e0 = INFINITY, e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      e0 = min3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+      e1 = min3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+      e2 = min3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
+      e3 = min3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
+    }
+    mx = min3f(e0, e1, fminf(e2, e3)) * scale_log2;
+  }
+  const float alpha = move_max(mx, m_run);
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
+  uint64_t acc0 = 0ull, acc1 = 0ull;  // two packed partial sums (pairs of +0.0f)
+  auto chunk = [&](const uint32_t (&r)[32], int q) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sc2, nm2);
+      float x0, x1;
+      f2_unpack(x, x0, x1);
+      const uint64_t pp = poly_pair(e)
+                              ? exp2_fma2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)))
+                              : f2_pack(ex2(x0), ex2(x1));
+      if (e & 1)
+        acc1 = f2_add(acc1, pp);
+      else
+        acc0 = f2_add(acc0, pp);
+      float p0, p1;
+      f2_unpack(pp, p0, p1);
+      pk[e] = pack_bf16(p0, p1);
+    }
+    tmem_st16(tS + q * 16, pk);
+  };
+  chunk(s0, 0);
+  chunk(s1, 1);
+  chunk(s2, 2);
+  chunk(s3, 3);
+  float a0, a1, b0, b1;
+  f2_unpack(acc0, a0, a1);
+  f2_unpack(acc1, b0, b1);
+  l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
+  return alpha;
+}
+
+// The general row: allowed-key bits (mw0, mw1) and dropout keep bits
+// (kb0, kb1) per key; two TMEM passes of 64 columns for the maximum, then 32
+// columns per pass for the exponentials. The sum and the maximum use
+// every allowed key (undropped); P carries only the kept ones (the 1/(1-rho)
+// factor is applied to O in fp32 at the end). Returns alpha.
+__device__ __forceinline__ float softmax_masked_tile(uint32_t tS, float scale_log2, uint64_t mw0, uint64_t mw1,
+                                                     uint64_t kb0, uint64_t kb1, float& m_run, float& l_run) {
+  float mx = -INFINITY;
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tS + hf * 64, r0);
+    tmem_ld32(tS + hf * 64 + 32, r1);
+    tmem_wait_ld();
+    const uint64_t mw = hf ? mw1 : mw0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      if ((mw >> e) & 1ull) mx = fmaxf(mx, __uint_as_float(r0[e]) * scale_log2);
+      if ((mw >> (32 + e)) & 1ull) mx = fmaxf(mx, __uint_as_float(r1[e]) * scale_log2);
+    }
+  }
+  const float alpha = move_max(mx, m_run);
+  const float msub = m_run == -INFINITY ? 0.f : m_run;
+  float sum = 0.f;
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t r[32];
+    tmem_ld32(tS + q * 32, r);
+    tmem_wait_ld();
+    const uint64_t mw = q < 2 ? mw0 : mw1;
+    const uint64_t kw = q < 2 ? kb0 : kb1;
+    const int base = (q & 1) * 32;
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int bit = base + 2 * e;
+      const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * scale_log2 - msub) : 0.f;
+      const float p1 = ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * scale_log2 - msub) : 0.f;
+      sum += p0 + p1;
+      pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+    }
+    tmem_st16(tS + q * 16, pk);
+  }
+  l_run = l_run * alpha + sum;
+  return alpha;
+}
+
 // Two query tiles per CTA, one softmax warpgroup each, alternating on the
 // tensor core: while one warpgroup turns its S tile into P, the MMA issuer
 // runs the other warpgroup's P V and next S. P (bf16 pairs) is written back
@@ -265,7 +416,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int kvh = h / (a.Hq / a.Hkv);
   const int q0 = ct * kFwdRows;
-  const int qt0 = 2 * ct, qt1 = 2 * ct + 1;
+  const int qt0 = 2 * ct;
   int kt_lo, kt_hi;
   fwd_key_tiles(a.m, a.T, q0, kFwdRows, kt_lo, kt_hi);
 
@@ -306,11 +457,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tma_load_4d(sbase + kFwdQ + w * kTileBytes, &tq, qf, 0, q0 + w * kBM, h, b);
       tma_load_4d(sbase + kFwdQ + w * kTileBytes + kTileBytes / 2, &tq, qf, 64, q0 + w * kBM, h, b);
     }
+    // The tile walk (and its mask classes) runs here, ahead of the MMA
+    // issuer, which reads each stage's flags from tinfo.
     int n = 0;
-    for (int kt = kt_lo; kt <= kt_hi; ++kt) {
-      if (wg_class(a, b, h, qt0, kt) == kEmpty && wg_class(a, b, h, qt1, kt) == kEmpty) continue;
+    uint32_t fl;
+    for (int kt = fwd_next_tile(a, b, h, qt0, kt_hi, kt_lo - 1, fl); kt <= kt_hi;) {
+      uint32_t nfl;
+      const int nk = fwd_next_tile(a, b, h, qt0, kt_hi, kt, nfl);
       const int s = n % kStages;
       if (!wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, a.status)) break;
+      ctl->tinfo[s] = fl | (nk <= kt_hi ? 4u : 0u);  // published by the release of the arrive below
       const uint32_t kf = smem_u32(&ctl->k_full[s]), vf = smem_u32(&ctl->v_full[s]);
       const uint32_t kd = sbase + kFwdK + s * kTileBytes, vd = sbase + kFwdV + s * kTileBytes;
       mbar_expect_tx(kf, kTileBytes);
@@ -320,6 +476,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tma_load_4d(vd, &tv, vf, 0, kt * kBN, kvh, b);
       tma_load_4d(vd + kTileBytes / 2, &tv, vf, 64, kt * kBN, kvh, b);
       ++n;
+      kt = nk;
+      fl = nfl;
     }
     for (int r = (n > kStages ? n - kStages : 0); r < n; ++r) {
       const int s = r % kStages;
@@ -331,63 +489,66 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);
     bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
-    auto next_tile = [&](int from, uint8_t& c0, uint8_t& c1) {
-      for (int kt = from + 1; kt <= kt_hi; ++kt) {
-        c0 = wg_class(a, b, h, qt0, kt);
-        c1 = wg_class(a, b, h, qt1, kt);
-        if (c0 != kEmpty || c1 != kEmpty) return kt;
-      }
-      return kt_hi + 1;
-    };
+    // Descriptors of every operand tile, formed once; a K step adds its byte
+    // offset >> 4 to the start-address field.
+    uint64_t dQ[2], dK[kStages], dV[kStages];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) dQ[i] = smem_desc_sw128(sbase + kFwdQ + i * kTileBytes, 16, 1024);
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) {
+      dK[i] = smem_desc_sw128(sbase + kFwdK + i * kTileBytes, 16, 1024);
+      dV[i] = smem_desc_sw128(sbase + kFwdV + i * kTileBytes, kTileBytes / 2, 1024);
+    }
     auto issue_s = [&](int w, int stage) {
-      const uint32_t qa = sbase + kFwdQ + w * kTileBytes, ka = sbase + kFwdK + stage * kTileBytes;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-        mma_ss(tmem + w * 128, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idS,
-               kk > 0);
+        const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+        mma_ss(tmem + w * 128, dQ[w] + off, dK[stage] + off, idS, kk > 0);
       }
       mma_commit(smem_u32(&ctl->s_full[w]));
     };
-    uint8_t c[2], nc[2];
-    int kt_cur = next_tile(kt_lo - 1, c[0], c[1]);
+    uint32_t fl0;
+    const bool any = fwd_next_tile(a, b, h, qt0, kt_hi, kt_lo - 1, fl0) <= kt_hi;
+    uint32_t info = 0;
     int npv[2] = {0, 0};
     int n = 0;
-    if (ok && kt_cur <= kt_hi) {
+    if (ok && any) {
       ok = wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, a.status);
       if (ok) {
         tc_fence_after();
+        info = ctl->tinfo[0];
         for (int w = 0; w < 2; ++w)
-          if (c[w] != kEmpty) issue_s(w, 0);
+          if ((info >> w) & 1u) issue_s(w, 0);
       }
     }
-    while (ok && kt_cur <= kt_hi) {
-      const int kt_nx = next_tile(kt_cur, nc[0], nc[1]);
+    while (ok && any) {
       const int s = n % kStages, s1 = (n + 1) % kStages;
-      const bool more = kt_nx <= kt_hi;
+      const bool more = info & 4u;
+      uint32_t ninfo = 0;
       for (int w = 0; w < 2 && ok; ++w) {
-        if (c[w] != kEmpty) {
+        if ((info >> w) & 1u) {
           if (!(ok = wait_bar(smem_u32(&ctl->p_full[w]), npv[w] & 1, abort_flag, a.status))) break;
           if (!(ok = wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status))) break;
           tc_fence_after();
-          const uint32_t va = sbase + kFwdV + s * kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // A = P in TMEM: 16 keys = 8 packed columns per step
-            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8,
-                   smem_desc_sw128(va + kk * 2048, kTileBytes / 2, 1024), idPV, (npv[w] > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dV[s] + (uint64_t)(kk * (2048 >> 4)), idPV,
+                   (npv[w] > 0 || kk > 0) ? 1u : 0u);
           ++npv[w];
         }
-        if (more && nc[w] != kEmpty) {
-          if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, a.status))) break;
-          tc_fence_after();
-          issue_s(w, s1);
+        if (more) {
+          if (w == 0) {
+            if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, a.status))) break;
+            tc_fence_after();
+            ninfo = ctl->tinfo[s1];
+          }
+          if ((ninfo >> w) & 1u) issue_s(w, s1);
         }
       }
       if (!ok) break;
       mma_commit(smem_u32(&ctl->kv_empty[s]));
-      kt_cur = kt_nx;
-      c[0] = nc[0];
-      c[1] = nc[1];
+      if (!more) break;
+      info = ninfo;
       ++n;
     }
     mma_commit(smem_u32(&ctl->o_final));
@@ -403,62 +564,40 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     float m_run = -INFINITY, l_run = 0.f;  // base-2 running max and running sum
     int n = 0;
     bool ok = true;
+    // Tile classes, 32 key tiles per round: lane l holds tile cbase + l
+    // (bits 0-1: this query tile, bits 2-3: this warp's 64-row slice).
+    int cbase = kt_lo - 32;
+    uint32_t cword = 0;
     for (int kt = kt_lo; kt <= kt_hi && ok; ++kt) {
-      const uint8_t cls = wg_class(a, b, h, qt, kt);
+      if (kt - cbase >= 32) {
+        cbase = kt;
+        const int mk = kt + lane;
+        cword = 0;
+        if (mk <= kt_hi) {
+          cword = wg_class(a, b, h, qt, mk);
+          if (cword == kPartial) cword |= (uint32_t)lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), mk) << 2;
+        }
+      }
+      const uint32_t cv = __shfl_sync(0xffffffffu, cword, kt - cbase);
+      const uint8_t cls = cv & 3u;
       if (cls == kEmpty) continue;
       uint64_t mw0 = ~0ull, mw1 = ~0ull;
       if (cls == kPartial) {
         mw0 = mw1 = 0ull;
-        if (row < a.T) {
-          const uint8_t scls = lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), kt);
-          fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, scls, mw0, mw1);
-        }
+        if (row < a.T) fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, (uint8_t)(cv >> 2), mw0, mw1);
       }
       uint64_t kb0 = ~0ull, kb1 = ~0ull;
       if (a.m.dropout) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[w]), n & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      const bool fast = cls == kFull && !a.m.dropout;
-      // Pass 1 over the S row: the (masked) maximum, 64 columns per TMEM load.
-      float mx = -INFINITY;
-      if (fast) {
-        // Every key allowed: extremum of the raw scores, scaled once.
-        float hi = -INFINITY, lo = INFINITY;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tS + hf * 64, r0);
-          tmem_ld32(tS + hf * 64 + 32, r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            hi = fmaxf(hi, fmaxf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
-            lo = fminf(lo, fminf(__uint_as_float(r0[e]), __uint_as_float(r1[e])));
-          }
-        }
-        mx = a.scale_log2 >= 0.f ? hi * a.scale_log2 : lo * a.scale_log2;
-      } else {
-#pragma unroll 1
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tS + hf * 64, r0);
-          tmem_ld32(tS + hf * 64 + 32, r1);
-          tmem_wait_ld();
-          const uint64_t mw = hf ? mw1 : mw0;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if ((mw >> e) & 1ull) mx = fmaxf(mx, __uint_as_float(r0[e]) * a.scale_log2);
-            if ((mw >> (32 + e)) & 1ull) mx = fmaxf(mx, __uint_as_float(r1[e]) * a.scale_log2);
-          }
-        }
-      }
-      float m_new = m_run;
-      if (mx > -INFINITY && (m_run == -INFINITY || mx > m_run + kRescaleThreshold)) m_new = fmaxf(mx, m_run);
-      const float alpha = (m_new == m_run) ? 1.f : ex2(m_run - m_new);  // 0 when m_run = -inf
-      const float msub = m_new == -INFINITY ? 0.f : m_new;
+      float alpha;
+      if (cls == kFull && !a.m.dropout)
+        alpha = softmax_full_tile(tS, a.scale_log2, m_run, l_run);
+      else
+        alpha = softmax_masked_tile(tS, a.scale_log2, mw0, mw1, kb0, kb1, m_run, l_run);
       // Every earlier P V of this warpgroup has completed (the S commit covers
-      // them), so O can be rescaled in place.
+      // them) and the next one waits for p_full: O can be rescaled in place.
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -470,50 +609,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           tmem_st32(tO + c * 32, o);
         }
       }
-      // Pass 2: p = 2^(s - m), written back as bf16 pairs over the first 64
-      // columns (P chunk q covers S columns already read).
-      float sum = 0.f;
-      if (fast) {
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tS + q * 32, r);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(fmaf(__uint_as_float(r[2 * e]), a.scale_log2, -msub));
-            const float p1 = ex2(fmaf(__uint_as_float(r[2 * e + 1]), a.scale_log2, -msub));
-            sum += p0 + p1;
-            pk[e] = pack_bf16(p0, p1);
-          }
-          tmem_st16(tS + q * 16, pk);
-        }
-      } else {
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tS + q * 32, r);
-          tmem_wait_ld();
-          const uint64_t mw = q < 2 ? mw0 : mw1;
-          const uint64_t kw = q < 2 ? kb0 : kb1;
-          const int base = (q & 1) * 32;
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int bit = base + 2 * e;
-            const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * a.scale_log2 - msub) : 0.f;
-            const float p1 =
-                ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * a.scale_log2 - msub) : 0.f;
-            sum += p0 + p1;
-            // xi only; the constant 1/(1-rho) is applied to O in fp32 at the end.
-            pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
-          }
-          tmem_st16(tS + q * 16, pk);
-        }
-      }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl->p_full[w]));

@@ -227,7 +227,13 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
 }
 
-// Per-warpgroup register reallocation (all warps of an aligned warpgroup).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Per-warpgroup register reallocation (every warp of an aligned warpgroup).
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -237,10 +243,57 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Two fp32 lanes in one 64-bit register, for the packed f32x2 FMA path.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_fma on two lanes at once (same arithmetic; x >= -125 is the caller's
+// to ensure, e.g. by a clamp before the call).
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
+  const uint64_t kRound2 = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t kNegRound2 = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t t = f2_add(x, kRound2);
+  const uint64_t n = f2_add(t, kNegRound2);                  // rint(x)
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x);    // x - rint(x), exact
+  uint64_t p = f2_fma(f2_pack(0.05459282547235489f, 0.05459282547235489f), f,
+                      f2_pack(0.24221783876419067f, 0.24221783876419067f));
+  p = f2_fma(p, f, f2_pack(0.6933686137199402f, 0.6933686137199402f));
+  p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+  // 2^n into the exponent field: the bits of t are 0x4B400000 + n, and
+  // 0x4B400000 << 23 vanishes modulo 2^32, so (bits(t) << 23) = n << 23.
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
 }  // namespace sm100
