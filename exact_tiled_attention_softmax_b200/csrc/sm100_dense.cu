@@ -491,19 +491,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
     // Descriptors of every operand tile, formed once; a K step adds its byte
     // offset >> 4 to the start-address field.
-    uint64_t dQ[2], dK[kStages], dV[kStages];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) dQ[i] = smem_desc_sw128(sbase + kFwdQ + i * kTileBytes, 16, 1024);
-#pragma unroll
-    for (int i = 0; i < kStages; ++i) {
-      dK[i] = smem_desc_sw128(sbase + kFwdK + i * kTileBytes, 16, 1024);
-      dV[i] = smem_desc_sw128(sbase + kFwdV + i * kTileBytes, kTileBytes / 2, 1024);
-    }
+    const uint64_t dQ0 = smem_desc_sw128(sbase + kFwdQ, 16, 1024), dK0 = smem_desc_sw128(sbase + kFwdK, 16, 1024);
+    const uint64_t dV0 = smem_desc_sw128(sbase + kFwdV, kTileBytes / 2, 1024);
+    constexpr uint64_t kTileStep = kTileBytes >> 4;  // one 32 KB tile further
+    auto dQ = [&](int i) { return dQ0 + (uint64_t)i * kTileStep; };
+    auto dK = [&](int i) { return dK0 + (uint64_t)i * kTileStep; };
+    auto dV = [&](int i) { return dV0 + (uint64_t)i * kTileStep; };
     auto issue_s = [&](int w, int stage) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-        mma_ss(tmem + w * 128, dQ[w] + off, dK[stage] + off, idS, kk > 0);
+        mma_ss(tmem + w * 128, dQ(w) + off, dK(stage) + off, idS, kk > 0);
       }
       mma_commit(smem_u32(&ctl->s_full[w]));
     };
@@ -532,7 +530,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // A = P in TMEM: 16 keys = 8 packed columns per step
-            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dV[s] + (uint64_t)(kk * (2048 >> 4)), idPV,
+            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dV(s) + (uint64_t)(kk * (2048 >> 4)), idPV,
                    (npv[w] > 0 || kk > 0) ? 1u : 0u);
           ++npv[w];
         }
@@ -713,6 +711,10 @@ struct BwdCtl {
   uint64_t acc_done;
   uint32_t tmem_base;
   uint32_t abort_flag;
+  // Per Q/dO stage, written by the producer before the stage's loads:
+  // word 0 = query slice | class << 28 | (another step follows) << 30,
+  // word 1 = query head within the group.
+  uint32_t qinfo[kQStages][2];
 };
 
 // Query-slice range [lo, hi] that can hold rows seeing keys [k0, k0 + 128).
@@ -855,12 +857,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     tma_load_4d(sbase + kBwdK + kTileBytes / 2, &tk, kvf, 64, k0, kvh, b);
     tma_load_4d(sbase + kBwdV, &tv, kvf, 0, k0, kvh, b);
     tma_load_4d(sbase + kBwdV + kTileBytes / 2, &tv, kvf, 64, k0, kvh, b);
+    // The step walk (query head, query slice, class) runs here, ahead of the
+    // MMA issuer and the compute warpgroups, which read it from qinfo.
     int n = 0, hh = 0, qs = qs_lo - 1;
     uint8_t cls;
-    while (bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
+    bool have = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls);
+    while (have) {
+      int nh = hh, nq = qs;
+      uint8_t ncls;
+      const bool next = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
       const int h = kvh * group + hh;
       const int s = n % kQStages;
       if (!wait_bar(smem_u32(&ctl->q_empty[s]), ((n / kQStages) & 1) ^ 1, abort_flag, a.status)) break;
+      ctl->qinfo[s][0] = (uint32_t)qs | ((uint32_t)cls << 28) | (next ? 1u << 30 : 0u);
+      ctl->qinfo[s][1] = (uint32_t)hh;  // both published by the release of the arrive below
       const uint32_t qf = smem_u32(&ctl->q_full[s]);
       mbar_expect_tx(qf, 2 * kQTile + 512);
       const uint32_t qd = sbase + kBwdQ + s * kQTile, gd = sbase + kBwdG + s * kQTile;
@@ -872,6 +882,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       bulk_load(sbase + kBwdStat + s * 512, a.lse2 + roff, 256, qf);
       bulk_load(sbase + kBwdStat + s * 512 + 256, a.dpad + roff, 256, qf);
       ++n;
+      hh = nh;
+      qs = nq;
+      cls = ncls;
+      have = next;
     }
     for (int r = (n > kQStages ? n - kQStages : 0); r < n; ++r)
       wait_bar(smem_u32(&ctl->q_full[r % kQStages]), (r / kQStages) & 1, abort_flag, nullptr);
@@ -884,64 +898,75 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     constexpr uint32_t idACC = idesc_bf16(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
     constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
     bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
-    auto issue_st = [&](int m) -> bool {
+    // Descriptors formed once; a K step adds its byte offset >> 4.
+    const uint64_t dK = smem_desc_sw128(sbase + kBwdK, 16, 1024), dV = smem_desc_sw128(sbase + kBwdV, 16, 1024);
+    const uint64_t dKmn = smem_desc_sw128(sbase + kBwdK, kTileBytes / 2, 1024);
+    // Stage i of a ring: the stage-0 descriptor plus i * (stage bytes >> 4).
+    const uint64_t dQk0 = smem_desc_sw128(sbase + kBwdQ, 16, 1024), dGk0 = smem_desc_sw128(sbase + kBwdG, 16, 1024);
+    const uint64_t dQmn0 = smem_desc_sw128(sbase + kBwdQ, kHalfQ, 1024);
+    const uint64_t dGmn0 = smem_desc_sw128(sbase + kBwdG, kHalfQ, 1024);
+    const uint64_t dDS0 = smem_desc_sw128(sbase + kBwdDS, 16, 1024);
+    const uint64_t dDSmn0 = smem_desc_sw128(sbase + kBwdDS, kHalfQ, 1024);
+    auto dQk = [&](int i) { return dQk0 + (uint64_t)(i * (kQTile >> 4)); };
+    auto dGk = [&](int i) { return dGk0 + (uint64_t)(i * (kQTile >> 4)); };
+    auto dQmn = [&](int i) { return dQmn0 + (uint64_t)(i * (kQTile >> 4)); };
+    auto dGmn = [&](int i) { return dGmn0 + (uint64_t)(i * (kQTile >> 4)); };
+    auto dDS = [&](int i) { return dDS0 + (uint64_t)(i * (kPTile >> 4)); };
+    auto dDSmn = [&](int i) { return dDSmn0 + (uint64_t)(i * (kPTile >> 4)); };
+    // Issue S^T and dP^T of step m; returns its qinfo word 0 (0 on abort).
+    auto issue_st = [&](int m, uint32_t& info) -> bool {
       const int s = m & 1, sq = m % kQStages;
       const uint32_t par = (m >> 1) & 1;
       if (!wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)) return false;
+      info = ctl->qinfo[sq][0];
       if (!wait_bar(smem_u32(&ctl->st_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       if (!wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       tc_fence_after();
-      const uint32_t qa = sbase + kBwdQ + sq * kQTile, ga = sbase + kBwdG + sq * kQTile;
       const uint32_t dst = tmem + s * 128;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-        const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
-        mma_ss(dst, smem_desc_sw128(sbase + kBwdK + koff, 16, 1024), smem_desc_sw128(qa + qoff, 16, 1024), idST,
-               kk > 0);
+        const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+        const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+        mma_ss(dst, dK + koff, dQk(sq) + qoff, idST, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-        const uint32_t qoff = (kk >> 2) * kHalfQ + (kk & 3) * 32;
-        mma_ss(dst + 64, smem_desc_sw128(sbase + kBwdV + koff, 16, 1024), smem_desc_sw128(ga + qoff, 16, 1024),
-               idST, kk > 0);
+        const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+        const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+        mma_ss(dst + 64, dV + koff, dGk(sq) + qoff, idST, kk > 0);
       }
       mma_commit(smem_u32(&ctl->st_full[s]));
       return true;
     };
-    int hh = 0, qs = qs_lo - 1, n = 0;
-    uint8_t cls;
-    bool have = ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls);
-    if (have) ok = issue_st(0);
+    int hh0 = 0, qs0 = qs_lo - 1, n = 0;
+    uint8_t cls0;
+    bool have = ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh0, qs0, cls0);
+    uint32_t info = 0;
+    if (have) ok = issue_st(0, info);
     while (ok && have) {
-      int nh = hh, nq = qs;
-      uint8_t ncls;
-      const bool next = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
-      if (next && !(ok = issue_st(n + 1))) break;
+      const bool next = info & (1u << 30);
+      uint32_t ninfo = 0;
+      if (next && !(ok = issue_st(n + 1, ninfo))) break;
       const int s = n & 1, sq = n % kQStages;
       if (!(ok = wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
-      const uint32_t qa = sbase + kBwdQ + sq * kQTile, ga = sbase + kBwdG + sq * kQTile;
-      const uint32_t dsa = sbase + kBwdDS + s * kPTile;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows; A = P~^T from TMEM (16 rows = 8 columns)
-        mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8,
-               smem_desc_sw128(ga + kk * 2048, kHalfQ, 1024), idACC, (n > 0 || kk > 0) ? 1u : 0u);
+        mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8, dGmn(sq) + (uint64_t)(kk * (2048 >> 4)),
+               idACC, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tDK, smem_desc_sw128(dsa + kk * 32, 16, 1024), smem_desc_sw128(qa + kk * 2048, kHalfQ, 1024), idACC,
+        mma_ss(tDK, dDS(s) + (uint64_t)(kk * (32 >> 4)), dQmn(sq) + (uint64_t)(kk * (2048 >> 4)), idACC,
                (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
-        mma_ss(tmem + s * 128, smem_desc_sw128(sbase + kBwdK + kk * 2048, kTileBytes / 2, 1024),
-               smem_desc_sw128(dsa + kk * 2048, kHalfQ, 1024), idDQ, kk > 0);
+        mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
+               kk > 0);
       mma_commit(smem_u32(&ctl->q_empty[sq]));
       mma_commit(smem_u32(&ctl->pds_empty[s]));
       mma_commit(smem_u32(&ctl->dq_full[s]));
-      hh = nh;
-      qs = nq;
       have = next;
+      info = ninfo;
       ++n;
     }
     mma_commit(smem_u32(&ctl->acc_done));
@@ -952,21 +977,31 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     const int t = ((warp & 3) << 5) | lane;
     const int64_t j = (int64_t)k0 + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    int n = 0, hh = 0, qs = qs_lo - 1;
-    uint8_t cls;
+    int n = 0;
     bool ok = true;
-    while (ok && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls)) {
-      const int h = kvh * group + hh;
+    bool more;
+    {
+      int hh0 = 0, qs0 = qs_lo - 1;
+      uint8_t cls0;
+      more = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh0, qs0, cls0);
+    }
+    while (ok && more) {
       const int s = n & 1, sq = n % kQStages;
       const uint32_t par = (n >> 1) & 1;
+      // The stage's step info arrives with its Q/dO tiles, long before S^T.
+      if (!(ok = __all_sync(0xffffffffu,
+                            wait_bar(smem_u32(&ctl->q_full[sq]), (n / kQStages) & 1, abort_flag, a.status))))
+        break;
+      const uint32_t info = ctl->qinfo[sq][0];
+      const int h = kvh * group + (int)ctl->qinfo[sq][1];
+      const int qs = (int)(info & 0x0fffffffu);
+      const uint8_t cls = (uint8_t)((info >> 28) & 3u);
+      more = info & (1u << 30);
       const int64_t i0 = (int64_t)qs * kBMb;
       const bool general = cls == kPartial || a.m.dropout;
       const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
       const uint32_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j) : ~0u;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
-      if (!(ok = __all_sync(0xffffffffu,
-                            wait_bar(smem_u32(&ctl->q_full[sq]), (n / kQStages) & 1, abort_flag, a.status))))
-        break;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty[s]), par ^ 1, abort_flag, a.status))))
         break;
       tc_fence_after();
