@@ -429,7 +429,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->s_full[s]), 1);
-      mbar_init(smem_u32(&ctl->p_full[s]), 128);
+      mbar_init(smem_u32(&ctl->p_full[s]), 4);  // one arrival per softmax warp
     }
     mbar_init(smem_u32(&ctl->o_final), 1);
     ctl->abort_flag = 0;
@@ -609,7 +609,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->p_full[w]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->p_full[w]));
       ++n;
     }
     // ---------------- epilogue: Y = u / (l + exp(z - m)), LSE = m + ln(...)
@@ -822,11 +823,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->st_full[s]), 1);
-      mbar_init(smem_u32(&ctl->st_empty[s]), 256);
-      mbar_init(smem_u32(&ctl->ds_full[s]), 256);
+      mbar_init(smem_u32(&ctl->st_empty[s]), 8);  // one arrival per compute warp
+      mbar_init(smem_u32(&ctl->ds_full[s]), 8);
       mbar_init(smem_u32(&ctl->pds_empty[s]), 1);
       mbar_init(smem_u32(&ctl->dq_full[s]), 1);
-      mbar_init(smem_u32(&ctl->dq_empty[s]), 128);
+      mbar_init(smem_u32(&ctl->dq_empty[s]), 4);  // one arrival per dQ warp
     }
     mbar_init(smem_u32(&ctl->acc_done), 1);
     ctl->abort_flag = 0;
@@ -1051,9 +1052,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->st_empty[s]));
       fence_proxy_async_smem();
-      mbar_arrive(smem_u32(&ctl->ds_full[s]));
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&ctl->st_empty[s]));
+        mbar_arrive(smem_u32(&ctl->ds_full[s]));
+      }
       ++n;
     }
     // ---------------- epilogue: warpgroup 0 writes dK = c * sum gamma^T Q,
@@ -1114,8 +1118,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tmem_ld32(tmem + lane_off + s * 128 + 32, r1);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(&ctl->dq_empty[s]));
-      if (lane == 0) bulk_wait_read0();  // the previous reduce has read this warp's box
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&ctl->dq_empty[s]));
+        bulk_wait_read0();  // the previous reduce has read this warp's box
+      }
       __syncwarp();
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
