@@ -109,6 +109,7 @@ struct ClassTable {
 
 __device__ __forceinline__ uint8_t lookup_class(const ClassTable& ct, const MaskP& m, int T, int b, int h, int qs,
                                                 int kt) {
+  if ((int64_t)qs * kBMb >= T) return kEmpty;  // slices past the last row are not in the table
   if (!ct.cls) return tile_class(m, T, b, h, qs, kt);
   const int sb = ct.nb > 1 ? b : 0, sh = ct.nh > 1 ? h : 0;
   return ct.cls[(((int64_t)sb * ct.nh + sh) * ct.nqs + qs) * ct.nkt + kt];
@@ -573,7 +574,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         cword = 0;
         if (mk <= kt_hi) {
           cword = wg_class(a, b, h, qt, mk);
-          if (cword == kPartial) cword |= (uint32_t)lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), mk) << 2;
+          if (cword == kPartial)
+            cword |= ((uint32_t)lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), mk) & 3u) << 2;
         }
       }
       const uint32_t cv = __shfl_sync(0xffffffffu, cword, kt - cbase);
@@ -1014,14 +1016,21 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tmem_wait_ld();
       uint32_t ppk[16], dpk[16];
       if (!general) {
+        // LSE and delta of the 32 columns: broadcast 16-byte loads.
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          const float2 l2 = *reinterpret_cast<const float2*>(lse2 + 2 * c2);
-          const float2 d2 = *reinterpret_cast<const float2*>(dl + 2 * c2);
-          const float p0 = ex2(fmaf(__uint_as_float(rs[2 * c2]), a.scale_log2, -l2.x));
-          const float p1 = ex2(fmaf(__uint_as_float(rs[2 * c2 + 1]), a.scale_log2, -l2.y));
-          ppk[c2] = pack_bf16(p0, p1);
-          dpk[c2] = pack_bf16(p0 * (__uint_as_float(rp[2 * c2]) - d2.x), p1 * (__uint_as_float(rp[2 * c2 + 1]) - d2.y));
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * c4);
+          const float4 d4 = *reinterpret_cast<const float4*>(dl + 4 * c4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c2 = 2 * c4 + e;
+            const float p0 = ex2(fmaf(__uint_as_float(rs[2 * c2]), a.scale_log2, -lv[2 * e]));
+            const float p1 = ex2(fmaf(__uint_as_float(rs[2 * c2 + 1]), a.scale_log2, -lv[2 * e + 1]));
+            ppk[c2] = pack_bf16(p0, p1);
+            dpk[c2] = pack_bf16(p0 * (__uint_as_float(rp[2 * c2]) - dv4[2 * e]),
+                                p1 * (__uint_as_float(rp[2 * c2 + 1]) - dv4[2 * e + 1]));
+          }
         }
       } else {
         const float inv = a.m.dropout ? a.m.inv_keep : 1.f;
