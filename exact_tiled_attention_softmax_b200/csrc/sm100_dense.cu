@@ -676,8 +676,8 @@ struct BwdArgs {
   int B, Hq, Hkv, T, Tpad;
   int block_aligned;
   float scale_log2;
-  const float* lse2;    // [B*Hq, Tpad] base-2 LSE (+inf on rows without keys)
-  const float* dpad;    // [B*Hq, Tpad] delta, zero on padding rows
+  const float* lse2;    // [B*Hq, Tpad] minus the base-2 LSE (-inf on rows without keys)
+  const float* dpad;    // [B*Hq, Tpad] minus delta, zero on padding rows
   float* dq_acc;        // [B, Hq, T, 128] fp32
   __nv_bfloat16* dk;
   int64_t sdk[3];
@@ -708,8 +708,11 @@ constexpr int kBwdThreads = 512;
 struct BwdCtl {
   uint64_t kv_full;
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t st_full[2], st_empty[2];
-  uint64_t ds_full[2], pds_empty[2];
+  // Buffer reuse needs no "empty" barriers for S^T/dP^T, P~^T and gamma^T:
+  // the MMA issuer writes S^T(n + 2) only after ds_full(n), and st_full(n + 2)
+  // commits after the dV, dK, dQ^T products of step n that read them.
+  uint64_t st_full[2];
+  uint64_t ds_full[2];
   uint64_t dq_full[2], dq_empty[2];
   uint64_t acc_done;
   uint32_t tmem_base;
@@ -825,9 +828,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->st_full[s]), 1);
-      mbar_init(smem_u32(&ctl->st_empty[s]), 8);  // one arrival per compute warp
       mbar_init(smem_u32(&ctl->ds_full[s]), 8);
-      mbar_init(smem_u32(&ctl->pds_empty[s]), 1);
       mbar_init(smem_u32(&ctl->dq_full[s]), 1);
       mbar_init(smem_u32(&ctl->dq_empty[s]), 4);  // one arrival per dQ warp
     }
@@ -922,7 +923,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint32_t par = (m >> 1) & 1;
       if (!wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)) return false;
       info = ctl->qinfo[sq][0];
-      if (!wait_bar(smem_u32(&ctl->st_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       if (!wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       tc_fence_after();
       const uint32_t dst = tmem + s * 128;
@@ -966,7 +966,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
                kk > 0);
       mma_commit(smem_u32(&ctl->q_empty[sq]));
-      mma_commit(smem_u32(&ctl->pds_empty[s]));
       mma_commit(smem_u32(&ctl->dq_full[s]));
       have = next;
       info = ninfo;
@@ -1005,31 +1004,36 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
       const uint32_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j) : ~0u;
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
-      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->pds_empty[s]), par ^ 1, abort_flag, a.status))))
-        break;
       tc_fence_after();
       uint32_t rs[32], rp[32];
       tmem_ld32(tmem + lane_off + s * 128 + hf * 32, rs);
       tmem_ld32(tmem + lane_off + s * 128 + 64 + hf * 32, rp);
-      const float* lse2 = stat + sq * 128 + hf * 32;
-      const float* dl = stat + sq * 128 + 64 + hf * 32;
+      const float* nl = stat + sq * 128 + hf * 32;       // -LSE (base 2) of the 32 columns
+      const float* nd = stat + sq * 128 + 64 + hf * 32;  // -delta
       tmem_wait_ld();
       uint32_t ppk[16], dpk[16];
       if (!general) {
-        // LSE and delta of the 32 columns: broadcast 16-byte loads.
+        // Pairs of columns on packed fp32: x = s c log2(e) - LSE, p = 2^x,
+        // gamma = p (dP - delta); -LSE and -delta come as broadcast 16-byte loads.
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * c4);
-          const float4 d4 = *reinterpret_cast<const float4*>(dl + 4 * c4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          const float4 l4 = *reinterpret_cast<const float4*>(nl + 4 * c4);
+          const float4 d4 = *reinterpret_cast<const float4*>(nd + 4 * c4);
+          const uint64_t lp[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+          const uint64_t dp[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int c2 = 2 * c4 + e;
-            const float p0 = ex2(fmaf(__uint_as_float(rs[2 * c2]), a.scale_log2, -lv[2 * e]));
-            const float p1 = ex2(fmaf(__uint_as_float(rs[2 * c2 + 1]), a.scale_log2, -lv[2 * e + 1]));
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
             ppk[c2] = pack_bf16(p0, p1);
-            dpk[c2] = pack_bf16(p0 * (__uint_as_float(rp[2 * c2]) - dv4[2 * e]),
-                                p1 * (__uint_as_float(rp[2 * c2 + 1]) - dv4[2 * e + 1]));
+            const uint64_t g = f2_mul(f2_pack(p0, p1),
+                                      f2_add(f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1])), dp[e]));
+            float g0, g1;
+            f2_unpack(g, g0, g1);
+            dpk[c2] = pack_bf16(g0, g1);
           }
         }
       } else {
@@ -1040,12 +1044,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int c = 2 * c2 + e;
-            const float p = ((allow >> c) & 1u) ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, -lse2[c])) : 0.f;
+            const float p = ((allow >> c) & 1u) ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, nl[c])) : 0.f;
             const bool kp = (keep >> c) & 1u;
             // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
             pt[e] = kp ? p : 0.f;
             const float dpv = kp ? __uint_as_float(rp[c]) * inv : 0.f;
-            ds[e] = p * (dpv - dl[c]);
+            ds[e] = p * (dpv + nd[c]);
           }
           ppk[c2] = pack_bf16(pt[0], pt[1]);
           dpk[c2] = pack_bf16(ds[0], ds[1]);
@@ -1063,10 +1067,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&ctl->st_empty[s]));
-        mbar_arrive(smem_u32(&ctl->ds_full[s]));
-      }
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->ds_full[s]));
       ++n;
     }
     // ---------------- epilogue: warpgroup 0 writes dK = c * sum gamma^T Q,
@@ -1157,7 +1158,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 }
 
 // Reverse-pass preparation, one warp per (b, h, row < Tpad): delta from the
-// stored O and dO, the base-2 LSE, and a zeroed dQ accumulator row.
+// stored O and dO (kept, and negated in the padded array), the negated base-2
+// LSE, and a zeroed dQ accumulator row.
 __global__ void __launch_bounds__(256)
 bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2, const __nv_bfloat16* g,
                    int64_t sg0, int64_t sg1, int64_t sg2, const float* lse, int64_t sl0, int64_t sl1, int64_t sl2,
@@ -1170,7 +1172,7 @@ bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2
   const int h = (int)(bh % Hq), b = (int)(bh / Hq);
   if (i >= T) {
     if (lane == 0) {
-      lse2[w] = INFINITY;
+      lse2[w] = -INFINITY;
       dpad[w] = 0.f;
     }
     return;
@@ -1193,8 +1195,8 @@ bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2
   dqr[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
     const float L = lse[b * sl0 + h * sl1 + (int64_t)i * sl2];
-    lse2[w] = L == -INFINITY ? INFINITY : L * kLog2e;
-    dpad[w] = s;
+    lse2[w] = L == -INFINITY ? -INFINITY : -L * kLog2e;  // negated: the reverse adds them
+    dpad[w] = -s;
     delta[bh * T + i] = s;
   }
 }

@@ -275,6 +275,12 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return r;
 }
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // exp2_fma on two lanes at once (same arithmetic; x >= -125 is the caller's
 // to ensure, e.g. by a clamp before the call).
 __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
