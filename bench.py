@@ -48,14 +48,28 @@ def load_peaks():
 
 
 def allowed_pairs(case: W.DenseCase) -> int:
-    """Sum over (b, h, i) of |A_i| for the causal / window workloads."""
+    """Sum over (b, h, i) of |A_i|: causal / window in closed form, a block
+    mask counted block pair by block pair."""
     T = case.T
-    if case.block_size:
-        raise ValueError("block-mask workloads need the mask to count pairs")
     i = np.arange(T, dtype=np.int64)
     lo = np.zeros(T, np.int64) if not case.window_left else np.maximum(0, i - case.window_left + 1)
     hi = i if case.causal else np.full(T, T - 1, np.int64)
-    return int(case.B * case.Hq * np.sum(hi - lo + 1))
+    if not case.block_size:
+        return int(case.B * case.Hq * np.sum(hi - lo + 1))
+    bm = W.block_mask(case)
+    bs = case.block_size
+    total = 0
+    for kb in range(bm.shape[1]):
+        c0, c1 = kb * bs, min(T, (kb + 1) * bs) - 1
+        rows = np.nonzero(np.repeat(bm[:, kb], bs)[:T])[0]
+        cnt = np.minimum(hi[rows], c1) - np.maximum(lo[rows], c0) + 1
+        total += int(np.sum(np.maximum(cnt, 0)))
+    return int(case.B * case.Hq * total)
+
+
+def fp32_alu_peak_tflops(sm_mhz: float) -> float:
+    """Dense fp32 FFMA rate: 148 SMs x 128 lanes x 2 flops x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 class ClockSampler:
@@ -189,22 +203,89 @@ def run_reference(args, case, rank, world):
     print(json.dumps(line), flush=True)
 
 
+class Problem:
+    """One workload on the device: the fwd and bwd calls through the public
+    binding, their inputs (for the end-to-end copies) and outputs, and the
+    algorithmic work per step."""
+
+    def __init__(self, name, pairs, fwd_fpp, bwd_fpp, inputs, outputs, fwd, bwd, config, bound, launches):
+        self.name, self.pairs, self.fwd_fpp, self.bwd_fpp = name, pairs, fwd_fpp, bwd_fpp
+        self.inputs, self.outputs, self.fwd, self.bwd = inputs, outputs, fwd, bwd
+        self.config, self.bound, self.launches = config, bound, launches
+
+
+def dense_problem(case: W.DenseCase, dev, torch, eta) -> Problem:
+    q, k, v, g = W.dense_inputs(case)
+    tq, tk, tv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v, g))
+    bm = W.block_mask(case)
+    allowed = eta.AllowedSet(causal=case.causal, window_left=case.window_left,
+                             block_mask=torch.from_numpy(bm).to(dev) if bm is not None else None,
+                             block_q=case.block_size or 128, block_k=case.block_size or 128,
+                             dropout_p=case.dropout_p, dropout_seed=case.dropout_seed)
+    o = torch.empty_like(tq)
+    lse = torch.empty(tq.shape[:-1], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+    ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
+    mask = "causal" + (f" & window {case.window_left}" if case.window_left else "") + \
+        (f" & {case.block_size}-blocks p={case.block_p_keep}" if case.block_size else "") + \
+        (f", dropout {case.dropout_p}" if case.dropout_p else "")
+    config = {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "T": case.T, "d": case.d,
+              "dv": case.dv, "mask": mask}
+    return Problem(case.name, allowed_pairs(case), 2 * case.d + 2 * case.dv, 6 * case.d + 4 * case.dv,
+                   [tq, tk, tv, tg], [dq, dk, dv],
+                   lambda: eta.attn_fwd(tq, tk, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
+                   lambda: eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, case.scale, dq=dq, dk=dk, dv=dv,
+                                        workspace=ws_b),
+                   config, "tensor",
+                   # fwd_kernel; prepare, bwd_kernel, dq_finish; plus a tile-class pass per call
+                   # when a block mask is present
+                   4 + (2 if bm is not None else 0))
+
+
+def topk_problem(case: W.TopkCase, dev, torch, eta) -> Problem:
+    q, kv, g, idx, ln, sink = W.topk_inputs(case)
+    tq, tkv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, kv, g))
+    allowed = eta.AllowedSet(topk_idxs=torch.from_numpy(idx).to(dev), topk_length=torch.from_numpy(ln).to(dev),
+                             sink=torch.from_numpy(sink).to(dev))
+    tv = tkv[:, :case.Dv]
+    o = torch.empty((case.Tq, case.H, case.Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((case.Tq, case.H), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(tq)
+    dkv = torch.empty_like(tkv)
+    dsink = torch.empty(case.H, dtype=torch.float32, device=dev)
+    ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tkv, tv, allowed), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tkv, tv, allowed), dtype=torch.uint8, device=dev)
+    config = {"workload": case.name, "Tq": case.Tq, "Tkv": case.Tkv, "H": case.H, "Dqk": case.Dqk, "Dv": case.Dv,
+              "mask": f"top-k lists, lengths U[{case.len_lo},{case.len_hi}], sink"}
+    return Problem(case.name, case.H * int(ln.astype(np.int64).sum()), 2 * case.Dqk + 2 * case.Dv,
+                   6 * case.Dqk + 4 * case.Dv, [tq, tkv, tg], [dq, dkv],
+                   lambda: eta.attn_fwd(tq, tkv, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
+                   lambda: eta.attn_bwd(tq, tkv, tv, o, tg, lse, allowed, case.scale, dq=dq, dk=dkv, dv=None,
+                                        dsink=dsink, workspace=ws_b),
+                   config, "alu",
+                   # fwd rows; delta, dQ rows, dKV pairs, fixed-point cast, dSink
+                   6)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="causal_8k", choices=["causal_8k", "causal_2k"])
+    ap.add_argument("--workload", default="causal_8k",
+                    choices=["causal_8k", "causal_2k", "window_block_8k", "gqa_dropout_16k", "topk_shared_kv"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    case = W.WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        run_reference(args, case, rank, world)
+        if args.workload not in ("causal_8k", "causal_2k"):
+            raise SystemExit("--impl reference times the oracle on the causal workloads")
+        run_reference(args, W.WORKLOADS[args.workload], rank, world)
         return
 
     import torch
@@ -219,21 +300,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     eta.load_library()
 
-    q, k, v, g = W.dense_inputs(case)
-    tq, tk, tv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v, g))
-    allowed = eta.AllowedSet(causal=case.causal, window_left=case.window_left)
-    scale = case.scale
-    o = torch.empty_like(tq)
-    lse = torch.empty(tq.shape[:-1], dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
-    ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
+    if args.workload in W.TOPK_WORKLOADS:
+        prob = topk_problem(W.TOPK_WORKLOADS[args.workload], dev, torch, eta)
+    else:
+        prob = dense_problem(W.WORKLOADS[args.workload], dev, torch, eta)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
-        eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        prob.fwd()
+        prob.bwd()
 
     clk = ClockSampler(local).start()
     time.sleep(0.5)  # nvidia-smi needs a moment before its first sample
@@ -242,10 +318,9 @@ def main():
     torch.cuda.synchronize()
 
     n_ev = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
-    # Events around the main kernel of each call (fwd_kernel, bwd_kernel),
-    # recorded by the library itself on the launching stream.
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n_ev)]
+    # Events around the main kernel of each call, recorded by the library
+    # itself on the launching stream.
     kev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n_ev)]
     for evs in kev:
         for e in evs:
@@ -255,19 +330,18 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    if True:
-        for s in range(n_ev):
-            flush.fill_(s & 0xFF)
-            e0, e1, e2 = ev[s]
-            k0, k1, k2, k3 = kev[s]
-            e0.record(stream)
-            eta.attn_set_kernel_events(k0, k1)
-            eta.attn_fwd(tq, tk, tv, allowed, scale, out=o, lse=lse, workspace=ws_f)
-            e1.record(stream)
-            eta.attn_set_kernel_events(k2, k3)
-            eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, scale, dq=dq, dk=dk, dv=dv, workspace=ws_b)
-            e2.record(stream)
-        torch.cuda.synchronize()
+    for s in range(n_ev):
+        flush.fill_(s & 0xFF)
+        e0, e1, e2 = ev[s]
+        k0, k1, k2, k3 = kev[s]
+        e0.record(stream)
+        eta.attn_set_kernel_events(k0, k1)
+        prob.fwd()
+        e1.record(stream)
+        eta.attn_set_kernel_events(k2, k3)
+        prob.bwd()
+        e2.record(stream)
+    torch.cuda.synchronize()
     t_wall1 = time.time()
     clk.stop()
     clk.window = (t_wall0, t_wall1)
@@ -283,28 +357,25 @@ def main():
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         total_ms = float(tt.item())
     ms_step = total_ms / n_ev
-    pairs = allowed_pairs(case)
-    flops_step = pairs * case.flops_per_pair
+    pairs = prob.pairs
+    flops_step = pairs * (prob.fwd_fpp + prob.bwd_fpp)
     value = world * flops_step * n_ev / (total_ms / 1e3) / 1e12
 
     # End to end through the public API: pinned host inputs in, results out.
-    hq, hk, hv, hg = (x.to("cpu").pin_memory() for x in (tq, tk, tv, tg))
-    hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (dq, dk, dv))
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
-    d2h = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
+    hosts_in = [x.to("cpu").pin_memory() for x in prob.inputs]
+    hosts_out = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in prob.outputs]
+    h2d = sum(x.numel() * x.element_size() for x in hosts_in)
+    d2h = sum(x.numel() * x.element_size() for x in hosts_out)
     e2e_ms = []
     for s in range(n_ev + 2):
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.fill_(s & 0xFF)
         a0.record(stream)
-        tq.copy_(hq, non_blocking=True)
-        tk.copy_(hk, non_blocking=True)
-        tv.copy_(hv, non_blocking=True)
-        tg.copy_(hg, non_blocking=True)
+        for d_, h_ in zip(prob.inputs, hosts_in):
+            d_.copy_(h_, non_blocking=True)
         step()
-        hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True)
-        hdv.copy_(dv, non_blocking=True)
+        for h_, d_ in zip(hosts_out, prob.outputs):
+            h_.copy_(d_, non_blocking=True)
         a1.record(stream)
         torch.cuda.synchronize()
         if s >= 2:
@@ -317,44 +388,46 @@ def main():
     e2e_value = world * flops_step * len(e2e_ms) / (e2e_total / 1e3) / 1e12
 
     peaks, peak_src = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    bwd_ms = statistics.mean(t_bwd)
-    bwd_flops = pairs * (6 * case.d + 4 * case.dv)
-    fwd_ms = statistics.mean(t_fwd)
-    fwd_flops = pairs * (2 * case.d + 2 * case.dv)
-    fwd_achieved = fwd_flops / (fwd_ms / 1e3) / 1e12
-    bwd_kernel_ms = statistics.mean(t_bwd_kernel)
-    fwd_kernel_ms = statistics.mean(t_fwd_kernel)
+    bwd_flops, fwd_flops = pairs * prob.bwd_fpp, pairs * prob.fwd_fpp
+    fwd_ms, bwd_ms = statistics.mean(t_fwd), statistics.mean(t_bwd)
+    fwd_kernel_ms, bwd_kernel_ms = statistics.mean(t_fwd_kernel), statistics.mean(t_bwd_kernel)
     achieved = bwd_flops / (bwd_kernel_ms / 1e3) / 1e12
-    traffic = recorded_traffic("bwd_kernel", case.name)
 
     if rank == 0:
         clocks = clk.summary()
+        if prob.bound == "tensor":
+            peak = float(peaks["bf16_tflops"])
+            kname = "bwd_kernel"
+            src = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
+        else:
+            peak = fp32_alu_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)
+            kname = "row-wise reverse kernels (CUDA cores, fp32 FFMA)"
+            src = "derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock"
+        config = dict(prob.config)
+        config.update({"allowed_pairs": pairs, "flops_per_pair": prob.fwd_fpp + prob.bwd_fpp,
+                       "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas x{world}"})
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": case.name, "B": case.B, "H": case.Hq, "T": case.T, "d": case.d,
-                       "dv": case.dv, "mask": "causal", "allowed_pairs": pairs,
-                       "flops_per_pair": case.flops_per_pair, "l2": "flushed (256 MB write) before every step",
-                       "parallelism": f"replicas x{world}"},
-            "pct_of_peak": {"measured_bf16_burst": 100 * value / world / peak,
+            "config": config,
+            "pct_of_peak": {"measured_bf16_burst": 100 * value / world / float(peaks["bf16_tflops"]),
                             "nvidia_dense_bf16_spec_2250": 100 * value / world / 2250.0},
-            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_achieved,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_flops / (fwd_ms / 1e3) / 1e12,
             "bwd_tflops": bwd_flops / (bwd_ms / 1e3) / 1e12,
-            "kernels": {"fwd_kernel": {"ms": fwd_kernel_ms, "tflops": fwd_flops / (fwd_kernel_ms / 1e3) / 1e12},
-                        "bwd_kernel": {"ms": bwd_kernel_ms, "tflops": achieved}},
-            "roofline": {"bound": "tensor", "kernel": "bwd_kernel",
+            "kernels": {"fwd_main": {"ms": fwd_kernel_ms, "tflops": fwd_flops / (fwd_kernel_ms / 1e3) / 1e12},
+                        "bwd_main": {"ms": bwd_kernel_ms, "tflops": achieved}},
+            "roofline": {"bound": prob.bound, "kernel": kname,
                          "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                         "traffic": traffic,
-                         "work_per_launch": f"{bwd_flops:.4e} flops = {pairs} allowed pairs x "
-                                            f"{6 * case.d + 4 * case.dv} (6d + 4dv)",
-                         "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"},
+                         "traffic": recorded_traffic("bwd_kernel", prob.name) if prob.bound == "tensor" else None,
+                         "work_per_launch": f"{bwd_flops:.4e} flops = {pairs} allowed pairs x {prob.bwd_fpp}",
+                         "peak_source": src},
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": prob.launches * args.steps,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.workload == "causal_8k":
+            case = W.WORKLOADS["causal_8k"]
             line["cpu_baseline"] = cpu_baseline(W.DenseCase(
                 "causal_8k_slice", 1, 1, 1, case.T, case.d, case.dv, "bf16", case.scale, causal=True,
                 seed=case.seed))
