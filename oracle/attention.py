@@ -116,7 +116,7 @@ def _row_softmax(s: np.ndarray, allow: np.ndarray, z: float):
     grid": inactive rows remain zero and undergo no division).
     """
     sm = np.where(allow, s, NEG_INF)
-    m = np.maximum(sm.max(axis=-1), z)
+    m = np.maximum(sm.max(axis=-1, initial=NEG_INF), z)  # a row of no columns is empty too
     finite = np.isfinite(m)
     shift = np.where(finite, m, 0.0)
     e = np.where(allow, np.exp(sm - shift[:, None]), 0.0)

@@ -467,3 +467,20 @@ def test_sampled_rows_and_columns_match_full_oracle():
             keep_fn=lambda hh, r, cc, hs=heads: S.keep_at(seed, rho, 0, hs[hh], r, cc), rho=rho)
         assert np.allclose(dk, bw.dk[0, kvh][cols], atol=1e-12)
         assert np.allclose(dvv, bw.dv[0, kvh][cols], atol=1e-12)
+
+
+def test_topk_empty_list_gives_zero_output_and_sink_lse():
+    """An empty selection is an empty allowed set: Y = 0 and LSE = z with a
+    sink, -inf without one; the other tokens are unaffected."""
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((2, 3, 8))
+    kv = rng.standard_normal((10, 8))
+    idx = np.array([[1, 4, 7], [0, 0, 0]], dtype=np.int32)
+    ln = np.array([3, 0], dtype=np.int32)
+    z = np.array([0.5, -1.0, 2.0])
+    o, lse, ps = oracle.topk_forward(q, kv, idx, ln, 4, 0.3, z)
+    assert np.all(o[1] == 0.0) and np.allclose(lse[1], z) and np.allclose(ps[1], 1.0)
+    o2, lse2, _ = oracle.topk_forward(q, kv, idx, ln, 4, 0.3, None)
+    assert np.all(o2[1] == 0.0) and np.all(np.isneginf(lse2[1]))
+    o1, lse1, _ = oracle.topk_forward(q[:1], kv, idx[:1], ln[:1], 4, 0.3, z)
+    assert np.allclose(o1[0], o[0]) and np.allclose(lse1[0], lse[0])
