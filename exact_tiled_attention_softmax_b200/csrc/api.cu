@@ -7,6 +7,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "sm100_dense.h"
+#include "sm100_topk.h"
 
 using namespace attn;
 
@@ -257,6 +258,9 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.Dv = s.Dv;
     p.scale = scale;
     p.sink = mask->sink;
+    if (sm100_topk_supported(p, q, k, o))
+      return cuda_status(sm100_topk_fwd(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
+                                        lse->stride[0], lse->stride[1], status, cs));
     main_kernel_begin(cs);
     cudaError_t e = q->dtype == ATTN_F32
         ? launch_topk_fwd_rows<float>(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),

@@ -1,0 +1,107 @@
+"""GPU parity of the tensor-core top-k forward (64 heads, Dqk = 576, Dv = 512,
+bf16: the shape the DSA note's kernel targets) against the float64 oracle.
+
+Cases span several 64-key tiles with ragged last tiles, an empty list, the
+sink, the lazy running-max move (later tiles with much larger scores), and a
+listed index outside [0, Tkv) that must be skipped and flagged."""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+import exact_tiled_attention_softmax_b200 as eta  # noqa: E402
+from exact_tiled_attention_softmax_b200 import workloads as W  # noqa: E402
+import oracle  # noqa: E402
+from tests.parity_util import BF16_O_ABS, to_dev, to_np  # noqa: E402
+
+H, DQK, DV = 64, 576, 512
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    eta.load_library()
+
+
+def _case(seed, Tq=24, Tkv=700, topk=256, lo=1, hi=256, sink=True, grow=False):
+    rng = np.random.default_rng(seed)
+    q = W.round_to_bf16(rng.standard_normal((Tq, H, DQK), dtype=np.float32))
+    kv = W.round_to_bf16(rng.standard_normal((Tkv, DQK), dtype=np.float32))
+    idx, ln = W.topk_lists(Tq, Tkv, topk, lo, hi, seed + 1)
+    if grow:
+        # The last 64 columns (they enter the scores only, never V) of the
+        # rows in the upper half of the index range are 16x larger (exact in
+        # bf16) and every list is sorted: later tiles raise the running max
+        # by far more than 2^8 while O stays of unit scale.
+        kv[Tkv // 2:, DV:] *= 16.0
+        for t in range(Tq):
+            idx[t, :ln[t]] = np.sort(idx[t, :ln[t]])
+    sk = rng.standard_normal(H).astype(np.float32) if sink else None
+    return q, kv, idx, ln, sk
+
+
+def _run(q, kv, idx, ln, sk, scale):
+    qd, kvd = to_dev(q, torch.bfloat16), to_dev(kv, torch.bfloat16)
+    al = eta.AllowedSet(topk_idxs=to_dev(idx, torch.int32), topk_length=to_dev(ln, torch.int32),
+                        sink=to_dev(sk, torch.float32) if sk is not None else None)
+    ws = torch.empty(eta.attn_fwd_workspace_size(qd, kvd, kvd[:, :DV], al), dtype=torch.uint8, device="cuda")
+    o, lse = eta.attn_fwd(qd, kvd, kvd[:, :DV], al, scale, workspace=ws)
+    status = eta.attn_get_status(ws)
+    torch.cuda.synchronize()
+    return to_np(o), to_np(lse), status
+
+
+def _check(o, lse, o_ref, lse_ref, per_row_scale=False):
+    err = np.abs(o - o_ref)
+    if per_row_scale:
+        # Nearly one-hot rows: O is a single V row of magnitude up to ~4, and
+        # the bf16 rounding of P (2^-9 relative per term, against an l summed
+        # in fp32) and of O itself both scale with |O|.
+        err = err / np.maximum(1.0, np.abs(o_ref).max(axis=-1, keepdims=True))
+    assert err.max() <= BF16_O_ABS, err.max()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse), fin)
+    assert np.abs(lse[fin] - lse_ref[fin]).max(initial=0) <= 1e-3
+
+
+@pytest.mark.parametrize("sink", [True, False])
+def test_topk_tc_ragged_tiles(sink):
+    q, kv, idx, ln, sk = _case(71, sink=sink)
+    ln[5] = 0        # empty list: O = 0, LSE = z or -inf
+    ln[6] = 64       # exactly one tile
+    ln[7] = 65       # one key into the second tile
+    scale = 1 / math.sqrt(DQK)
+    o, lse, status = _run(q, kv, idx, ln, sk, scale)
+    assert status == 0
+    o_ref, lse_ref, _ = oracle.topk_forward(q, kv, idx, ln, DV, scale,
+                                            sk.astype(np.float64) if sk is not None else None)
+    _check(o, lse, o_ref, lse_ref)
+
+
+def test_topk_tc_running_max_moves():
+    q, kv, idx, ln, sk = _case(72, grow=True, lo=128, hi=256)
+    scale = 1 / math.sqrt(DQK)
+    o, lse, status = _run(q, kv, idx, ln, sk, scale)
+    assert status == 0
+    o_ref, lse_ref, _ = oracle.topk_forward(q, kv, idx, ln, DV, scale, sk.astype(np.float64))
+    _check(o, lse, o_ref, lse_ref, per_row_scale=True)
+
+
+def test_topk_tc_bad_index_skipped_and_flagged():
+    q, kv, idx, ln, sk = _case(73, lo=100, hi=200)
+    bad_t = 3
+    idx[bad_t, 10] = kv.shape[0] + 5   # outside [0, Tkv), inside the valid length
+    scale = 1 / math.sqrt(DQK)
+    o, lse, status = _run(q, kv, idx, ln, sk, scale)
+    assert status & eta.ATTN_DEVERR_TOPK_INDEX
+    # The reference drops the bad entry (the list shifts left by one).
+    idx_ref, ln_ref = idx.copy(), ln.copy()
+    idx_ref[bad_t, 10:-1] = idx[bad_t, 11:]
+    ln_ref[bad_t] -= 1
+    o_ref, lse_ref, _ = oracle.topk_forward(q, kv, idx_ref, ln_ref, DV, scale, sk.astype(np.float64))
+    _check(o, lse, o_ref, lse_ref)
