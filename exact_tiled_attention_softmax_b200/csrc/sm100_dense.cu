@@ -768,13 +768,31 @@ __device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h,
   return w;
 }
 
-// Keep bits xi for key j and query rows i0..i0+31.
+// Keep bits xi for key j and query rows i0..i0+31 (bit c <-> row i0 + c).
+// One Philox block (j >> 2, i, h, b) holds the words of keys 4(j >> 2) .. +3,
+// i.e. of the four lanes that share j >> 2 (keys k0 + t with k0 a multiple of
+// 4). Those lanes split the 32 rows, 8 blocks each, and trade their keep
+// nibbles, so every block is evaluated once. Whole warp, converged.
 __device__ __forceinline__ uint32_t bwd_keep_bits(const MaskP& m, int b, int h, int64_t i0, int64_t j) {
-  uint32_t w = 0;
+  const int lane = threadIdx.x & 31, e = lane & 3;
+  uint32_t nib = 0;  // 4 keep bits (keys 4(j >> 2) + 0..3) per row, rows 8e .. 8e+7
 #pragma unroll 1
-  for (int c = 0; c < 32; ++c)
-    if (dropout_keep(m, b, h, i0 + c, j)) w |= 1u << c;
-  return w;
+  for (int c = 0; c < 8; ++c) {
+    const uint4 w = philox4x32_10(make_uint4((uint32_t)(j >> 2), (uint32_t)(i0 + 8 * e + c), (uint32_t)h, (uint32_t)b),
+                                  m.seed_lo, m.seed_hi);
+    nib |= ((uint32_t)(w.x >= m.keep_thr) | ((uint32_t)(w.y >= m.keep_thr) << 1) |
+            ((uint32_t)(w.z >= m.keep_thr) << 2) | ((uint32_t)(w.w >= m.keep_thr) << 3))
+           << (4 * c);
+  }
+  const int base = lane & ~3, word = (int)(j & 3);
+  uint32_t keep = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t nq = __shfl_sync(0xffffffffu, nib, base + q);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) keep |= ((nq >> (4 * c + word)) & 1u) << (8 * q + c);
+  }
+  return keep;
 }
 
 // Element-wise add of a shared-memory box into global memory through a tensor
