@@ -263,8 +263,8 @@ def topk_problem(case: W.TopkCase, dev, torch, eta) -> Problem:
                    lambda: eta.attn_fwd(tq, tkv, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
                    lambda: eta.attn_bwd(tq, tkv, tv, o, tg, lse, allowed, case.scale, dq=dq, dk=dkv, dv=None,
                                         dsink=dsink, workspace=ws_b),
-                   config, "alu",
-                   # fwd rows; delta, dQ rows, dKV pairs, fixed-point cast, dSink
+                   config, "tensor",
+                   # forward; delta, dQ + G/P, dKV contributions, fixed-point cast, dSink
                    6)
 
 
@@ -397,7 +397,8 @@ def main():
         clocks = clk.summary()
         if prob.bound == "tensor":
             peak = float(peaks["bf16_tflops"])
-            kname = "bwd_kernel"
+            kname = "bwd_kernel" if args.workload not in W.TOPK_WORKLOADS else \
+                "top-k reverse kernels (dQ + G/P, dKV contributions)"
             src = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
         else:
             peak = fp32_alu_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)

@@ -142,10 +142,12 @@ size_t bwd_dense_bytes(const Dense& s) {
   return n;
 }
 
-size_t bwd_topk_bytes(const Topk& s) {
+size_t bwd_topk_bytes(const Topk& s, const attn_tensor* q, const attn_mask* m) {
   size_t n = kStatusBytes;
   n += align_up((size_t)s.Tq * s.H * sizeof(float), 256);                       // delta
   n += align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);      // 32.32 dKV
+  if (q->dtype == ATTN_BF16)                                                    // G, P rows (tensor-core path)
+    n += align_up(attn::sm100_topk_bwd_scratch_bytes(s.Tq, s.H, s.Dqk, s.Dv, m->topk_max), 256);
   return n;
 }
 
@@ -212,7 +214,7 @@ size_t attn_bwd_workspace_size(const attn_tensor* q, const attn_tensor* k, const
   if (flags_of(mask) & ATTN_MASK_TOPK) {
     Topk s;
     if (check_topk(q, k, v, s) != ATTN_OK) return kStatusBytes;
-    return bwd_topk_bytes(s);
+    return bwd_topk_bytes(s, q, mask);
   }
   Dense s;
   if (check_dense(q, k, v, s) != ATTN_OK) return kStatusBytes;
@@ -341,7 +343,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       return ATTN_ERR_INVALID_ARG;
     if (!inner_contiguous(o) || !inner_contiguous(do_) || !inner_contiguous(dq) || !inner_contiguous(dk))
       return ATTN_ERR_INVALID_ARG;
-    if ((st = check_workspace(workspace, workspace_bytes, bwd_topk_bytes(s))) != ATTN_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes, bwd_topk_bytes(s, q, mask))) != ATTN_OK) return st;
     if (cudaMemsetAsync(status, 0, kStatusBytes, cs) != cudaSuccess) return ATTN_ERR_CUDA;
     float* delta = reinterpret_cast<float*>(ws + kStatusBytes);
     unsigned long long* acc = reinterpret_cast<unsigned long long*>(
@@ -374,6 +376,18 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
                                         delta, dq->data, dq->stride[0], dq->stride[1], acc, dk->data,
                                         dk->stride[0], status, cs);
       main_kernel_end(cs);
+    } else if (sm100_topk_bwd_supported(p, q, k, o, do_, dq)) {
+      // Tensor cores: dQ and the per-token dKV contributions; the fixed-point
+      // accumulator starts at zero and is cast to dKV at the end.
+      char* scratch = ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256) +
+                      align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);
+      e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
+      if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * (size_t)s.Tkv * s.Dqk, cs);
+      if (e == cudaSuccess)
+        e = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], static_cast<const float*>(lse->data),
+                           lse->stride[0], lse->stride[1], delta, dq->data, dq->stride[0], dq->stride[1], acc,
+                           scratch, status, cs);
+      if (e == cudaSuccess) e = launch_fixed_to_out<__nv_bfloat16>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
     } else {
       e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
       main_kernel_begin(cs);

@@ -28,6 +28,9 @@ cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, in
                                  const float* lse, int64_t sl_t, int64_t sl_h, const float* delta,
                                  void* dq, int64_t sd_t, int64_t sd_h, unsigned long long* acc_fixed,
                                  void* dkv, int64_t sdkv, uint32_t* status, cudaStream_t st);
+template <typename T>
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int cols, void* out, int64_t so,
+                                cudaStream_t st);
 cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta, int n_outer, int n_heads,
                          int n_inner, int64_t sl_outer, int64_t sl_head, int64_t sl_inner,
                          bool delta_head_major, float* dsink, cudaStream_t st);

@@ -514,6 +514,14 @@ cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, in
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int cols, void* out, int64_t so,
+                                cudaStream_t st) {
+  const int64_t n = (int64_t)rows * cols;
+  if (n > 0) fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(acc, rows, cols, static_cast<T*>(out), so);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta, int n_outer, int n_heads,
                          int n_inner, int64_t sl_outer, int64_t sl_head, int64_t sl_inner,
                          bool delta_head_major, float* dsink, cudaStream_t st) {
@@ -538,7 +546,8 @@ cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta
   template cudaError_t launch_topk_bwd_rows<T>(const TopkP&, const void*, int64_t, int64_t,             \
                                                const float*, int64_t, int64_t, const float*, void*,     \
                                                int64_t, int64_t, unsigned long long*, void*, int64_t,   \
-                                               uint32_t*, cudaStream_t);
+                                               uint32_t*, cudaStream_t);                               \
+  template cudaError_t launch_fixed_to_out<T>(const unsigned long long*, int, int, void*, int64_t, cudaStream_t);
 
 ATTN_INSTANTIATE(float)
 ATTN_INSTANTIATE(__nv_bfloat16)

@@ -367,6 +367,521 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
   }
 }
 
+// ------------------------------------------------------------- reverse
+
+// Reverse, first kernel (one CTA per query token): recompute S = Q K^T,
+// P = 2^(S c log2(e) - LSE2) on the listed keys, dP = dO V^T, and
+// G = c P (dP - delta) (DSA note, sections 3.3-3.4, 8); accumulate
+// dQ = G K_sel in TMEM over the tiles, and store G and P as bf16 rows
+// [token][head][listed position] for the dKV kernel.
+//   upper half: S cols 0-63, dP 64-127, Q 128-415, dQ[:, 512:576] 416-479
+//   lower half: dQ[:, 0:512] cols 0-511
+constexpr int kBStages = 2;
+constexpr uint32_t kBKV = 0;
+constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads x 64 columns
+constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys bf16
+constexpr uint32_t kBCtl = kBG + kTH * 128;
+constexpr uint32_t kBSmem = kBCtl + 512 + 1024;
+constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
+
+struct TopkBwdCtl {
+  uint64_t kv_full[kBStages], kv_empty[kBStages];
+  uint64_t do_full, q_ready, st_full, st_empty, g_full, g_free, dq_done;
+  uint32_t vmask[kBStages][2];
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct TopkBwdArgs {
+  const __nv_bfloat16* q;
+  int64_t sq_t, sq_h;
+  const int32_t* idx;
+  int64_t idx_stride;
+  int32_t topk_max, topk_pad;
+  const int32_t* len;
+  int Tq, Tkv;
+  float scale, scale_log2;
+  const float* lse;
+  int64_t sl_t, sl_h;
+  const float* delta;  // [Tq, 64]
+  __nv_bfloat16* dq;
+  int64_t sd_t, sd_h;
+  __nv_bfloat16* g_scr;  // [Tq, 64, topk_pad]
+  __nv_bfloat16* p_scr;
+  uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kTThreads, 1)
+topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constant__ CUtensorMap tdo,
+                   const TopkBwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  TopkBwdCtl* ctl = reinterpret_cast<TopkBwdCtl*>(smem + kBCtl);
+  volatile uint32_t* abort_flag = &ctl->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int n_keys = a.len ? min(max(a.len[t], 0), a.topk_max) : a.topk_max;
+  const int ntiles = (n_keys + kTK - 1) / kTK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(smem_u32(&ctl->kv_full[s]), 1);
+      mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->do_full), 1);
+    mbar_init(smem_u32(&ctl->q_ready), 4);
+    mbar_init(smem_u32(&ctl->st_full), 1);
+    mbar_init(smem_u32(&ctl->st_empty), 4);
+    mbar_init(smem_u32(&ctl->g_full), 4);
+    mbar_init(smem_u32(&ctl->g_free), 1);
+    mbar_init(smem_u32(&ctl->dq_done), 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- producer: dO once (8 planes), then the KV gathers.
+    if (lane == 0) {
+      tma_prefetch_desc(&tkv);
+      tma_prefetch_desc(&tdo);
+      const uint32_t df = smem_u32(&ctl->do_full);
+      mbar_expect_tx(df, 8 * kTPlane);
+      for (int c = 0; c < 8; ++c) tma_load_3d(sbase + kBDO + c * kTPlane, &tdo, df, 64 * c, 0, t);
+    }
+    __syncwarp();
+    const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
+    int n = 0;
+    for (; n < ntiles; ++n) {
+      const int s = n % kBStages;
+      if (!__all_sync(0xffffffffu,
+                      wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kBStages) & 1) ^ 1, abort_flag, a.status)))
+        break;
+      int row[2];
+      bool valid[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int pos = n * kTK + 2 * lane + e;
+        const int j = pos < n_keys ? list[pos] : -1;
+        valid[e] = pos < n_keys && j >= 0 && j < a.Tkv;
+        if (pos < n_keys && !valid[e]) set_status(a.status, ATTN_DEVERR_TOPK_INDEX);
+        row[e] = valid[e] ? j : 0;
+      }
+      const uint32_t vm0 = __ballot_sync(0xffffffffu, valid[0]), vm1 = __ballot_sync(0xffffffffu, valid[1]);
+      const uint32_t kf = smem_u32(&ctl->kv_full[s]);
+      if (lane == 0) {
+        ctl->vmask[s][0] = vm0;
+        ctl->vmask[s][1] = vm1;
+        mbar_expect_tx(kf, kTTile);
+      }
+      __syncwarp();
+      const int g = lane & 15;
+      const int r0 = __shfl_sync(0xffffffffu, row[0], 2 * g), r1 = __shfl_sync(0xffffffffu, row[1], 2 * g);
+      const int r2 = __shfl_sync(0xffffffffu, row[0], 2 * g + 1), r3 = __shfl_sync(0xffffffffu, row[1], 2 * g + 1);
+      if (lane < 16) {
+        const uint32_t dst = sbase + kBKV + s * kTTile + g * 512;
+#pragma unroll 1
+        for (int c = 0; c < kTPlanes; ++c) gather4(dst + c * kTPlane, &tkv, kf, 64 * c, r0, r1, r2, r3);
+      }
+    }
+    if (lane == 0) {
+      for (int r = (n > kBStages ? n - kBStages : 0); r < n; ++r)
+        wait_bar(smem_u32(&ctl->kv_full[r % kBStages]), (r / kBStages) & 1, abort_flag, nullptr);
+      wait_bar(smem_u32(&ctl->do_full), 0, abort_flag, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: S(n), dP(n) as soon as the compute warps
+    // have read S(n-1), dP(n-1); dQ += G(n) K(n) once G(n) is in shared memory.
+    constexpr uint32_t idS = idesc_bf16(64, kTK, 0, 0);
+    constexpr uint32_t idDQ = idesc_bf16(64, 256, 0, 1);
+    constexpr uint32_t idDQ64 = idesc_bf16(64, 64, 0, 1);
+    const uint64_t dKV0 = smem_desc_sw128(sbase + kBKV, 16, 1024);
+    const uint64_t dKmn0 = smem_desc_sw128(sbase + kBKV, kTPlane, 1024);
+    const uint64_t dDO = smem_desc_sw128(sbase + kBDO, 16, 1024);
+    const uint64_t dG = smem_desc_sw128(sbase + kBG, 16, 1024);
+    constexpr uint64_t kStageStep = kTTile >> 4;
+    bool ok = wait_bar(smem_u32(&ctl->q_ready), 0, abort_flag, a.status) &&
+              wait_bar(smem_u32(&ctl->do_full), 0, abort_flag, a.status);
+    auto issue_sdp = [&](int m) -> bool {
+      const int s = m % kBStages;
+      if (!wait_bar(smem_u32(&ctl->kv_full[s]), (m / kBStages) & 1, abort_flag, a.status)) return false;
+      if (m > 0 && !wait_bar(smem_u32(&ctl->st_empty), (m - 1) & 1, abort_flag, a.status)) return false;
+      tc_fence_after();
+      const uint64_t dk = dKV0 + (uint64_t)s * kStageStep;
+#pragma unroll
+      for (int kk = 0; kk < kTD / 16; ++kk)  // S = Q K^T, A = Q from TMEM
+        mma_ts(tmem + kUpper, tmem + kUpper + kQCol + kk * 8,
+               dk + (uint64_t)(((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < kTDV / 16; ++kk) {  // dP = dO V^T, both K-major over the first 8 planes
+        const uint32_t off = ((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4;
+        mma_ss(tmem + kUpper + kDPCol, dDO + (uint64_t)off, dk + (uint64_t)off, idS, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(smem_u32(&ctl->st_full));
+      return true;
+    };
+    if (ok && ntiles > 0) ok = issue_sdp(0);
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int s = n % kBStages;
+      if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
+      if (!(ok = wait_bar(smem_u32(&ctl->g_full), n & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      const uint64_t dk = dKmn0 + (uint64_t)s * kStageStep;
+#pragma unroll
+      for (int kk = 0; kk < kTK / 16; ++kk) {  // dQ += G K: B = K rows as [keys x d], d contiguous
+        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+        mma_ss(tmem, dG + (uint64_t)(kk * 2), dk + (uint64_t)((kk * 2048) >> 4), idDQ, acc);
+        mma_ss(tmem + 256, dG + (uint64_t)(kk * 2), dk + (uint64_t)((4 * kTPlane + kk * 2048) >> 4), idDQ, acc);
+        mma_ss(tmem + kUpper + kDQHiCol, dG + (uint64_t)(kk * 2), dk + (uint64_t)((8 * kTPlane + kk * 2048) >> 4),
+               idDQ64, acc);
+      }
+      mma_commit(smem_u32(&ctl->g_free));
+      mma_commit(smem_u32(&ctl->kv_empty[s]));
+    }
+    mma_commit(smem_u32(&ctl->dq_done));
+  } else if (warp >= 2) {
+    // ---------------- compute warps: lane l >= 16 of quarter qt owns row
+    // h = 16 qt + l - 16 of S, dP and dQ[:, 512:576]; lane l < 16 the same
+    // head's dQ[:, 0:512].
+    const int qt = warp & 3;
+    const bool upper = lane >= 16;
+    const int h = 16 * qt + (lane & 15);
+    const uint32_t tq = tmem + ((uint32_t)(32 * qt) << 16);
+    {
+      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (int64_t)t * a.sq_t + (int64_t)h * a.sq_h);
+#pragma unroll 1
+      for (int c = 0; c < kTD / 64; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 x = upper ? qrow[c * 8 + v] : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * v] = x.x;
+          r[4 * v + 1] = x.y;
+          r[4 * v + 2] = x.z;
+          r[4 * v + 3] = x.w;
+        }
+        tmem_st32(tq + kQCol + 32 * c, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->q_ready));
+    }
+    const float L = a.lse[(int64_t)t * a.sl_t + (int64_t)h * a.sl_h];
+    const float lse2 = L * kLog2e;
+    const float dl = a.delta[(int64_t)t * kTH + h];
+    const bool live = L != -INFINITY;
+    const uint32_t g_row = sbase + kBG + h * 128;
+    __nv_bfloat16* gs = a.g_scr + ((int64_t)t * kTH + h) * a.topk_pad;
+    __nv_bfloat16* ps = a.p_scr + ((int64_t)t * kTH + h) * a.topk_pad;
+    bool ok = true;
+    for (int n = 0; n < ntiles && ok; ++n) {
+      const int s = n % kBStages;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full), n & 1, abort_flag, a.status));
+      if (ok)
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(smem_u32(&ctl->kv_full[s]), (n / kBStages) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      tmem_ld32(tq, s0);
+      tmem_ld32(tq + 32, s1);
+      tmem_ld32(tq + kDPCol, d0);
+      tmem_ld32(tq + kDPCol + 32, d1);
+      const uint32_t vm[2] = {ctl->vmask[s][0], ctl->vmask[s][1]};
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->st_empty));  // S and dP may be overwritten
+      uint32_t gp[32], pp[32];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        float pv[4], gv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = (u < 2 ? 2 * e + u : 32 + 2 * e + u - 2);
+          const uint32_t sv = u < 2 ? s0[2 * e + u] : s1[2 * e + u - 2];
+          const uint32_t dv = u < 2 ? d0[2 * e + u] : d1[2 * e + u - 2];
+          const float p = (live && key_valid(vm, k)) ? ex2(__uint_as_float(sv) * a.scale_log2 - lse2) : 0.f;
+          pv[u] = p;
+          gv[u] = a.scale * p * (__uint_as_float(dv) - dl);
+        }
+        pp[e] = pack_bf16(pv[0], pv[1]);
+        pp[16 + e] = pack_bf16(pv[2], pv[3]);
+        gp[e] = pack_bf16(gv[0], gv[1]);
+        gp[16 + e] = pack_bf16(gv[2], gv[3]);
+      }
+      // G's shared-memory tile is free once dQ += G(n-1) K(n-1) has completed.
+      if (n > 0)
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->g_free), (n - 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      if (upper) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(g_row + ((c ^ (h & 7)) << 4), gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
+        uint4* gd = reinterpret_cast<uint4*>(gs + n * kTK);
+        uint4* pd = reinterpret_cast<uint4*>(ps + n * kTK);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          gd[c] = make_uint4(gp[4 * c], gp[4 * c + 1], gp[4 * c + 2], gp[4 * c + 3]);
+          pd[c] = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->g_full));
+    }
+    // ---------------- epilogue: dQ rows (lower lanes: columns 0-511, upper
+    // lanes: 512-575 from the upper half). G already carries the scale c.
+    bool have = false;
+    if (ok && ntiles > 0) {
+      have = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_done), 0, abort_flag, a.status));
+      if (have) tc_fence_after();
+    }
+    if (ok) {
+      __nv_bfloat16* drow = a.dq + (int64_t)t * a.sd_t + (int64_t)h * a.sd_h;
+      auto put = [&](const uint32_t (&r)[32], int col0) {
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int idx = c8 * 8 + 2 * e;
+            pk[e] = have ? pack_bf16(__uint_as_float(r[idx]), __uint_as_float(r[idx + 1])) : 0u;
+          }
+          *reinterpret_cast<uint4*>(drow + col0 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      };
+#pragma unroll 1
+      for (int c = 0; c < kTDV / 32; ++c) {
+        uint32_t r[32];
+        if (have) {
+          tmem_ld32(tq + 32 * c, r);
+          tmem_wait_ld();
+        }
+        if (!upper) put(r, 32 * c);
+      }
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        if (have) {
+          tmem_ld32(tq + kDQHiCol + 32 * c, r);
+          tmem_wait_ld();
+        }
+        if (upper) put(r, kTDV + 32 * c);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Reverse, second kernel (one CTA per query token): the token's
+// contribution to dKV for each listed row j (DSA note, sections 8-9),
+// C_j = sum_h G[h, j] Q[h, :] + [sum_h P[h, j] dO[h, :], 0], as
+// C^T = Q^T G + dO^T P on the tensor cores (M = 128 columns of Dqk per
+// chunk, N = 64 listed keys, K = 64 heads), then added into the signed
+// 32.32 fixed-point dKV accumulator with 64-bit integer atomics: integer
+// addition is associative, so dKV is bitwise reproducible.
+//   TMEM: chunk c = 0..3 (columns 128c..128c+127 of Dqk) at columns 64c,
+//   chunk 4 (columns 512-575, M = 64, lower half) at 256.
+constexpr uint32_t kCQ = 0;                        // Q: 9 planes of 64 heads x 64 columns
+constexpr uint32_t kCDO = kCQ + kTPlanes * kTPlane;  // dO: 8 planes
+constexpr uint32_t kCGP = kCDO + 8 * kTPlane;        // 2 stages x (G, P) tiles of 64 heads x 64 keys
+constexpr uint32_t kCRow = kCGP + 2 * 2 * kTPlane;   // 2 stages x 64 KV rows (-1: not listed / invalid)
+constexpr uint32_t kCCtl = kCRow + 2 * kTK * 4;
+constexpr uint32_t kCSmem = kCCtl + 256 + 1024;
+
+struct TopkDkvCtl {
+  uint64_t qdo_full, gp_full[2], gp_empty[2], c_full, c_empty;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct TopkDkvArgs {
+  const int32_t* idx;
+  int64_t idx_stride;
+  int32_t topk_max;
+  const int32_t* len;
+  int Tq, Tkv, Dqk;
+  unsigned long long* acc;  // [Tkv, Dqk] signed 32.32 fixed point
+  uint32_t* status;
+};
+
+__global__ void __launch_bounds__(kTThreads, 1)
+topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
+                    const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tp,
+                    const TopkDkvArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  TopkDkvCtl* ctl = reinterpret_cast<TopkDkvCtl*>(smem + kCCtl);
+  int32_t* krow = reinterpret_cast<int32_t*>(smem + kCRow);
+  volatile uint32_t* abort_flag = &ctl->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int n_keys = a.len ? min(max(a.len[t], 0), a.topk_max) : a.topk_max;
+  const int ntiles = (n_keys + kTK - 1) / kTK;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&ctl->qdo_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&ctl->gp_full[s]), 1);
+      mbar_init(smem_u32(&ctl->gp_empty[s]), 4);  // released by the draining warps: krow is theirs too
+    }
+    mbar_init(smem_u32(&ctl->c_full), 1);
+    mbar_init(smem_u32(&ctl->c_empty), 4);  // one arrival per draining warp
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- producer: Q and dO of the token once, then per tile
+    // the G and P tiles and the listed rows.
+    if (lane == 0 && ntiles > 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tdo);
+      tma_prefetch_desc(&tg);
+      tma_prefetch_desc(&tp);
+      const uint32_t f = smem_u32(&ctl->qdo_full);
+      mbar_expect_tx(f, (kTPlanes + 8) * kTPlane);
+      for (int c = 0; c < kTPlanes; ++c) tma_load_3d(sbase + kCQ + c * kTPlane, &tq, f, 64 * c, 0, t);
+      for (int c = 0; c < 8; ++c) tma_load_3d(sbase + kCDO + c * kTPlane, &tdo, f, 64 * c, 0, t);
+    }
+    __syncwarp();
+    const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
+    int n = 0;
+    for (; n < ntiles; ++n) {
+      const int s = n & 1;
+      if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)))
+        break;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int k = 2 * lane + e, pos = n * kTK + k;
+        const int j = pos < n_keys ? list[pos] : -1;
+        krow[s * kTK + k] = (j >= 0 && j < a.Tkv) ? j : -1;  // the first kernel flagged invalid entries
+      }
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t f = smem_u32(&ctl->gp_full[s]);
+        mbar_expect_tx(f, 2 * kTPlane);  // its release publishes krow with the tiles
+        tma_load_3d(sbase + kCGP + (2 * s) * kTPlane, &tg, f, n * kTK, 0, t);
+        tma_load_3d(sbase + kCGP + (2 * s + 1) * kTPlane, &tp, f, n * kTK, 0, t);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {
+      for (int r = (n > 2 ? n - 2 : 0); r < n; ++r)
+        wait_bar(smem_u32(&ctl->gp_full[r & 1]), (r >> 1) & 1, abort_flag, nullptr);
+      if (ntiles > 0) wait_bar(smem_u32(&ctl->qdo_full), 0, abort_flag, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer: C^T = Q^T G + dO^T P per tile.
+    constexpr uint32_t id128 = idesc_bf16(128, kTK, 1, 1);
+    constexpr uint32_t id64 = idesc_bf16(64, kTK, 1, 1);
+    const uint64_t dQ0 = smem_desc_sw128(sbase + kCQ, kTPlane, 1024);    // [heads x d], d contiguous
+    const uint64_t dDO0 = smem_desc_sw128(sbase + kCDO, kTPlane, 1024);
+    const uint64_t dGP0 = smem_desc_sw128(sbase + kCGP, kTPlane, 1024);  // [heads x keys], keys contiguous
+    bool ok = ntiles == 0 || wait_bar(smem_u32(&ctl->qdo_full), 0, abort_flag, a.status);
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int s = n & 1;
+      if (!(ok = wait_bar(smem_u32(&ctl->gp_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
+      if (n > 0 && !(ok = wait_bar(smem_u32(&ctl->c_empty), (n - 1) & 1, abort_flag, a.status))) break;
+      tc_fence_after();
+      const uint64_t dG = dGP0 + (uint64_t)((2 * s) * (kTPlane >> 4)), dP = dG + (uint64_t)(kTPlane >> 4);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int kk = 0; kk < kTH / 16; ++kk)  // K = 16 heads = 16 rows of every plane per step
+          mma_ss(tmem + 64 * c, dQ0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128),
+                 id128, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kTH / 16; ++kk)
+          mma_ss(tmem + 64 * c, dDO0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dP + (uint64_t)(kk * 128),
+                 id128, 1u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kTH / 16; ++kk)  // columns 512-575: Q part only, M = 64
+        mma_ss(tmem + 256, dQ0 + (uint64_t)((8 * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128), id64,
+               kk > 0 ? 1u : 0u);
+      mma_commit(smem_u32(&ctl->c_full));
+    }
+  } else if (warp >= 2) {
+    // ---------------- drain: lane l of quarter qt holds column 128 c + 32 qt + l
+    // of chunk c (and 512 + 16 qt + l of chunk 4 when l < 16) for all 64 keys.
+    const int qt = warp & 3;
+    const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
+    bool ok = true, sat = false;
+    for (int n = 0; n < ntiles && ok; ++n) {
+      const int s = n & 1;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full), n & 1, abort_flag, a.status));
+      if (ok)  // the listed rows come with the stage's tiles
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_full[s]), (n >> 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      const int32_t* rows = krow + s * kTK;
+#pragma unroll 1
+      for (int c = 0; c < 5; ++c) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tq4 + 64 * c, v0);
+        tmem_ld32(tq4 + 64 * c + 32, v1);
+        tmem_wait_ld();
+        const int col = c < 4 ? 128 * c + 32 * qt + lane : 512 + 16 * qt + lane;
+        if (c == 4 && lane >= 16) continue;
+        auto add = [&](const uint32_t (&v)[32], int k0) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int j = rows[k0 + k];
+            if (j < 0) continue;
+            float x = __uint_as_float(v[k]);
+            const float lim = 1073741824.f;  // 2^30: |x| 2^32 stays below 2^62
+            if (!(fabsf(x) < lim)) {
+              sat = true;
+              x = x != x ? 0.f : copysignf(lim, x);
+            }
+            atomicAdd(a.acc + (int64_t)j * a.Dqk + col, (unsigned long long)__float2ll_rn(x * 4294967296.f));
+          }
+        };
+        add(v0, 0);
+        add(v1, 32);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&ctl->c_empty));
+        mbar_arrive(smem_u32(&ctl->gp_empty[s]));  // c_full(n) implies the MMAs are done with G and P
+      }
+    }
+    if (__any_sync(0xffffffffu, sat) && lane == 0) set_status(a.status, ATTN_DEVERR_OVERFLOW);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 topk_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -383,7 +898,110 @@ bool aligned16(const void* p, int64_t stride_elems) {
   return reinterpret_cast<uintptr_t>(p) % 16 == 0 && (stride_elems * 2) % 16 == 0;
 }
 
+// 3-D bf16 map (inner, 64, Tq) with (64, 64, 1) boxes and 128-byte swizzle:
+// one token's 64 rows of a 64-column plane per load.
+bool make_map3(CUtensorMap* map, const void* base, int64_t inner, int Tq, int64_t s_row, int64_t s_tok) {
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)kTH, (cuuint64_t)Tq};
+  cuuint64_t strides[2] = {(cuuint64_t)s_row * 2, (cuuint64_t)s_tok * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kTH, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return topk_encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_kv_gather_map(CUtensorMap* map, const TopkP& p) {
+  cuuint64_t dims[2] = {(cuuint64_t)p.Dqk, (cuuint64_t)p.Tkv};
+  cuuint64_t strides[1] = {(cuuint64_t)p.skv * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  return topk_encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.kv), dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t raise_smem(const void* fn, uint32_t bytes, int which) {
+  static bool done[3][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done[which][dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < 64) done[which][dev] = true;
+  return e;
+}
+
 }  // namespace
+
+int sm100_topk_pad(int topk_max) { return ((topk_max + kTK - 1) / kTK) * kTK; }
+
+size_t sm100_topk_bwd_scratch_bytes(int Tq, int H, int Dqk, int Dv, int topk_max) {
+  if (H != kTH || Dqk != kTD || Dv != kTDV) return 0;
+  return 2 * (size_t)Tq * kTH * sm100_topk_pad(topk_max) * sizeof(__nv_bfloat16);
+}
+
+bool sm100_topk_bwd_supported(const TopkP& p, const attn_tensor* q, const attn_tensor* kv, const attn_tensor* o,
+                              const attn_tensor* do_, const attn_tensor* dq) {
+  if (!sm100_topk_supported(p, q, kv, o)) return false;
+  if (do_->dtype != ATTN_BF16 || dq->dtype != ATTN_BF16) return false;
+  return aligned16(do_->data, do_->stride[0]) && aligned16(do_->data, do_->stride[1]) &&
+         aligned16(dq->data, dq->stride[0]) && aligned16(dq->data, dq->stride[1]);
+}
+
+cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t sg_h, const float* lse,
+                           int64_t sl_t, int64_t sl_h, const float* delta, void* dq, int64_t sd_t, int64_t sd_h,
+                           unsigned long long* acc, void* scratch, uint32_t* status, cudaStream_t st) {
+  const int pad = sm100_topk_pad(p.topk_max);
+  __nv_bfloat16* g_scr = static_cast<__nv_bfloat16*>(scratch);
+  __nv_bfloat16* p_scr = g_scr + (size_t)p.Tq * kTH * pad;
+  CUtensorMap mkv, mdo, mq, mg, mp;
+  if (!make_kv_gather_map(&mkv, p) || !make_map3(&mdo, g, kTDV, p.Tq, sg_h, sg_t) ||
+      !make_map3(&mq, p.q, kTD, p.Tq, p.sq_h, p.sq_t) || !make_map3(&mg, g_scr, pad, p.Tq, pad, (int64_t)kTH * pad) ||
+      !make_map3(&mp, p_scr, pad, p.Tq, pad, (int64_t)kTH * pad))
+    return cudaErrorInvalidValue;
+  TopkBwdArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(p.q);
+  a.sq_t = p.sq_t;
+  a.sq_h = p.sq_h;
+  a.idx = p.idx;
+  a.idx_stride = p.idx_stride;
+  a.topk_max = p.topk_max;
+  a.topk_pad = pad;
+  a.len = p.len;
+  a.Tq = p.Tq;
+  a.Tkv = p.Tkv;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  a.lse = lse;
+  a.sl_t = sl_t;
+  a.sl_h = sl_h;
+  a.delta = delta;
+  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.sd_t = sd_t;
+  a.sd_h = sd_h;
+  a.g_scr = g_scr;
+  a.p_scr = p_scr;
+  a.status = status;
+  TopkDkvArgs c;
+  c.idx = p.idx;
+  c.idx_stride = p.idx_stride;
+  c.topk_max = p.topk_max;
+  c.len = p.len;
+  c.Tq = p.Tq;
+  c.Tkv = p.Tkv;
+  c.Dqk = p.Dqk;
+  c.acc = acc;
+  c.status = status;
+  cudaError_t e;
+  if ((e = raise_smem(reinterpret_cast<const void*>(topk_bwd_dq_kernel), kBSmem, 1)) != cudaSuccess) return e;
+  if ((e = raise_smem(reinterpret_cast<const void*>(topk_bwd_dkv_kernel), kCSmem, 2)) != cudaSuccess) return e;
+  main_kernel_begin(st);
+  topk_bwd_dq_kernel<<<p.Tq, kTThreads, kBSmem, st>>>(mkv, mdo, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  topk_bwd_dkv_kernel<<<p.Tq, kTThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
+  main_kernel_end(st);
+  return cudaGetLastError();
+}
 
 bool sm100_topk_supported(const TopkP& p, const attn_tensor* q, const attn_tensor* kv, const attn_tensor* o) {
   if (q->dtype != ATTN_BF16 || kv->dtype != ATTN_BF16 || o->dtype != ATTN_BF16) return false;
@@ -403,14 +1021,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   // 2-D map over the KV rows: 64-column boxes one row high (the gather4 form)
   // with 128-byte swizzle, matching the planes the MMAs read.
   CUtensorMap map;
-  cuuint64_t dims[2] = {(cuuint64_t)p.Dqk, (cuuint64_t)p.Tkv};
-  cuuint64_t strides[1] = {(cuuint64_t)p.skv * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t es[2] = {1, 1};
-  if (topk_encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.kv), dims, strides, box, es,
-                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (!make_kv_gather_map(&map, p)) return cudaErrorInvalidValue;
   TopkArgs a;
   a.q = static_cast<const __nv_bfloat16*>(p.q);
   a.sq_t = p.sq_t;
@@ -430,16 +1041,8 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   a.sl_t = sl_t;
   a.sl_h = sl_h;
   a.status = status;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = raise_smem(reinterpret_cast<const void*>(topk_fwd_kernel), kTSmem, 0);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_done[dev]) {
-    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(topk_fwd_kernel),
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTSmem);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_done[dev] = true;
-  }
   main_kernel_begin(st);
   topk_fwd_kernel<<<p.Tq, kTThreads, kTSmem, st>>>(map, a);
   main_kernel_end(st);

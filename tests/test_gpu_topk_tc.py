@@ -105,3 +105,31 @@ def test_topk_tc_bad_index_skipped_and_flagged():
     ln_ref[bad_t] -= 1
     o_ref, lse_ref, _ = oracle.topk_forward(q, kv, idx_ref, ln_ref, DV, scale, sk.astype(np.float64))
     _check(o, lse, o_ref, lse_ref)
+
+
+def test_topk_tc_backward_matches_oracle_and_is_reproducible():
+    from tests.parity_util import BF16_GRAD_REL, rel_fro
+    q, kv, idx, ln, sk = _case(74)
+    ln[5] = 0
+    ln[6] = 64
+    ln[7] = 65
+    rng = np.random.default_rng(75)
+    g = W.round_to_bf16(rng.standard_normal((q.shape[0], H, DV), dtype=np.float32))
+    scale = 1 / math.sqrt(DQK)
+    qd, kvd, gd = to_dev(q, torch.bfloat16), to_dev(kv, torch.bfloat16), to_dev(g, torch.bfloat16)
+    al = eta.AllowedSet(topk_idxs=to_dev(idx, torch.int32), topk_length=to_dev(ln, torch.int32),
+                        sink=to_dev(sk, torch.float32))
+    o, lse = eta.attn_fwd(qd, kvd, kvd[:, :DV], al, scale)
+    ws = torch.empty(eta.attn_bwd_workspace_size(qd, kvd, kvd[:, :DV], al), dtype=torch.uint8, device="cuda")
+    dq, dkv, _, ds = eta.attn_bwd(qd, kvd, kvd[:, :DV], o, gd, lse, al, scale, workspace=ws)
+    assert eta.attn_get_status(ws) == 0
+    sink64 = sk.astype(np.float64)
+    o_ref, _, _ = oracle.topk_forward(q, kv, idx, ln, DV, scale, sink64)
+    dq_ref, dkv_ref, ds_ref = oracle.topk_backward(q, kv, idx, ln, DV, scale, g, sink64, o=o_ref)
+    assert rel_fro(to_np(dq), dq_ref) <= BF16_GRAD_REL
+    assert rel_fro(to_np(dkv), dkv_ref) <= BF16_GRAD_REL
+    assert np.abs(to_np(ds) - ds_ref).max() <= 2e-2 * max(1.0, np.abs(ds_ref).max())
+    assert np.all(to_np(dq)[5] == 0.0)  # the empty list's token
+    dq2, dkv2, _, ds2 = eta.attn_bwd(qd, kvd, kvd[:, :DV], o, gd, lse, al, scale, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(dkv2, dkv) and torch.equal(ds2, ds)
