@@ -215,7 +215,8 @@ def attn_bwd_workspace_size(q, k, v, allowed: AllowedSet | None = None) -> int:
 
 def attn_fwd(q, k, v, allowed: AllowedSet | None = None, scale: float | None = None, *,
              out=None, lse=None, workspace=None, stream=None):
-    """Forward pass. Dense: q [B,Hq,T,d], k [B,Hkv,T,d], v [B,Hkv,T,dv].
+    """Forward pass. Dense: q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v [B,Hkv,Tk,dv];
+    with Tq != Tk query row i sits at key position i + Tk - Tq.
     Top-k: q [Tq,H,Dqk], k = KV [Tkv,Dqk], v = KV[:, :Dv].
     Returns (o, lse); lse is fp32, natural log, sink-inclusive."""
     lib = load_library()

@@ -14,7 +14,7 @@ using namespace attn;
 namespace {
 
 struct Dense {
-  int B, Hq, Hkv, T, d, dv;
+  int B, Hq, Hkv, Tq, Tk, d, dv;
 };
 
 bool inner_contiguous(const attn_tensor* t) { return t->ndim >= 1 && t->stride[t->ndim - 1] == 1; }
@@ -86,17 +86,17 @@ attn_status check_dense(const attn_tensor* q, const attn_tensor* k, const attn_t
   if (!dims_fit_int(q) || !dims_fit_int(k) || !dims_fit_int(v)) return ATTN_ERR_INVALID_ARG;
   s.B = (int)q->shape[0];
   s.Hq = (int)q->shape[1];
-  s.T = (int)q->shape[2];
+  s.Tq = (int)q->shape[2];
+  s.Tk = (int)k->shape[2];
   s.d = (int)q->shape[3];
   s.Hkv = (int)k->shape[1];
   s.dv = (int)v->shape[3];
-  if (k->shape[0] != s.B || v->shape[0] != s.B || k->shape[2] != s.T || v->shape[2] != s.T)
-    return ATTN_ERR_INVALID_ARG;
+  if (k->shape[0] != s.B || v->shape[0] != s.B || v->shape[2] != s.Tk) return ATTN_ERR_INVALID_ARG;
   if (k->shape[3] != s.d || v->shape[1] != s.Hkv) return ATTN_ERR_INVALID_ARG;
   if (s.Hq < 1 || s.Hkv < 1 || s.Hq % s.Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (s.d < 1 || s.dv < 1) return ATTN_ERR_INVALID_ARG;
   if (s.d > 576 || s.dv > 576) return ATTN_ERR_UNSUPPORTED;
-  if (!q->data || !k->data || !v->data) return (s.B && s.T) ? ATTN_ERR_INVALID_ARG : ATTN_OK;
+  if (!q->data || !k->data || !v->data) return (s.B && s.Tq && s.Tk) ? ATTN_ERR_INVALID_ARG : ATTN_OK;
   if (!inner_contiguous(q) || !inner_contiguous(k) || !inner_contiguous(v)) return ATTN_ERR_INVALID_ARG;
   if (!valid_dtype(q->dtype) || k->dtype != q->dtype || v->dtype != q->dtype) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
@@ -135,7 +135,7 @@ attn_status check_workspace(void* ws, size_t have, size_t need) {
 }
 
 size_t bwd_dense_bytes(const Dense& s) {
-  const size_t rows = (size_t)s.B * s.Hq * s.T;
+  const size_t rows = (size_t)s.B * s.Hq * s.Tq;
   size_t n = kStatusBytes;
   n += align_up(rows * sizeof(float), 256);                       // delta
   n += align_up(rows * (size_t)s.d * sizeof(float), 256);         // dQ accumulator
@@ -204,7 +204,7 @@ size_t attn_fwd_workspace_size(const attn_tensor* q, const attn_tensor* k, const
   size_t n = kStatusBytes;
   if (!(flags_of(mask) & ATTN_MASK_TOPK)) {
     Dense s;
-    if (check_dense(q, k, v, s) == ATTN_OK) n += sm100_fwd_workspace_bytes(s.B, s.Hq, s.T, mask);
+    if (check_dense(q, k, v, s) == ATTN_OK) n += sm100_fwd_workspace_bytes(s.B, s.Hq, s.Tq, s.Tk, mask);
   }
   return n;
 }
@@ -218,7 +218,7 @@ size_t attn_bwd_workspace_size(const attn_tensor* q, const attn_tensor* k, const
   }
   Dense s;
   if (check_dense(q, k, v, s) != ATTN_OK) return kStatusBytes;
-  return bwd_dense_bytes(s) + sm100_bwd_extra_workspace_bytes(s.B, s.Hq, s.Hkv, s.T, mask);
+  return bwd_dense_bytes(s) + sm100_bwd_extra_workspace_bytes(s.B, s.Hq, s.Hkv, s.Tq, s.Tk, mask);
 }
 
 attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
@@ -276,13 +276,13 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
 
   Dense s;
   if ((st = check_dense(q, k, v, s)) != ATTN_OK) return st;
-  const int64_t os[4] = {s.B, s.Hq, s.T, s.dv}, ls[3] = {s.B, s.Hq, s.T};
+  const int64_t os[4] = {s.B, s.Hq, s.Tq, s.dv}, ls[3] = {s.B, s.Hq, s.Tq};
   if (!same_shape(o, 4, os) || !same_shape(lse, 3, ls) || o->dtype != q->dtype || !inner_contiguous(o))
     return ATTN_ERR_INVALID_ARG;
   const size_t need = attn_fwd_workspace_size(q, k, v, mask);
   if ((st = check_workspace(workspace, workspace_bytes, need)) != ATTN_OK) return st;
   if (cudaMemsetAsync(status, 0, kStatusBytes, cs) != cudaSuccess) return ATTN_ERR_CUDA;
-  if ((int64_t)s.B * s.Hq * s.T == 0) return ATTN_OK;
+  if ((int64_t)s.B * s.Hq * s.Tq == 0) return ATTN_OK;
   if (!o->data || !lse->data) return ATTN_ERR_INVALID_ARG;
   DenseP p;
   p.q = q->data;
@@ -296,11 +296,13 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.B = s.B;
   p.Hq = s.Hq;
   p.Hkv = s.Hkv;
-  p.T = s.T;
+  p.Tq = s.Tq;
+  p.Tk = s.Tk;
   p.d = s.d;
   p.dv = s.dv;
   p.scale = scale;
   p.m = mask_params(mask);
+  p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
   const int64_t so[3] = {o->stride[0], o->stride[1], o->stride[2]};
   const int64_t sl[3] = {lse->stride[0], lse->stride[1], lse->stride[2]};
   float* lsep = static_cast<float*>(lse->data);
@@ -407,8 +409,8 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   Dense s;
   if ((st = check_dense(q, k, v, s)) != ATTN_OK) return st;
   if (!dv) return ATTN_ERR_INVALID_ARG;
-  const int64_t os[4] = {s.B, s.Hq, s.T, s.dv}, ls[3] = {s.B, s.Hq, s.T}, qs[4] = {s.B, s.Hq, s.T, s.d},
-                ks[4] = {s.B, s.Hkv, s.T, s.d}, vs[4] = {s.B, s.Hkv, s.T, s.dv};
+  const int64_t os[4] = {s.B, s.Hq, s.Tq, s.dv}, ls[3] = {s.B, s.Hq, s.Tq}, qs[4] = {s.B, s.Hq, s.Tq, s.d},
+                ks[4] = {s.B, s.Hkv, s.Tk, s.d}, vs[4] = {s.B, s.Hkv, s.Tk, s.dv};
   if (!same_shape(o, 4, os) || !same_shape(do_, 4, os) || !same_shape(lse, 3, ls) || !same_shape(dq, 4, qs) ||
       !same_shape(dk, 4, ks) || !same_shape(dv, 4, vs))
     return ATTN_ERR_INVALID_ARG;
@@ -418,9 +420,9 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   const size_t need = attn_bwd_workspace_size(q, k, v, mask);
   if ((st = check_workspace(workspace, workspace_bytes, need)) != ATTN_OK) return st;
   if (cudaMemsetAsync(status, 0, kStatusBytes, cs) != cudaSuccess) return ATTN_ERR_CUDA;
-  if ((int64_t)s.B * s.Hq * s.T == 0) return ATTN_OK;
+  if ((int64_t)s.B * s.Hq * s.Tq == 0) return ATTN_OK;
   float* delta = reinterpret_cast<float*>(ws + kStatusBytes);
-  const size_t rows = (size_t)s.B * s.Hq * s.T;
+  const size_t rows = (size_t)s.B * s.Hq * s.Tq;
   float* dq_acc = reinterpret_cast<float*>(ws + kStatusBytes + align_up(rows * sizeof(float), 256));
   char* extra = ws + bwd_dense_bytes(s);
   DenseP p;
@@ -435,11 +437,13 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.B = s.B;
   p.Hq = s.Hq;
   p.Hkv = s.Hkv;
-  p.T = s.T;
+  p.Tq = s.Tq;
+  p.Tk = s.Tk;
   p.d = s.d;
   p.dv = s.dv;
   p.scale = scale;
   p.m = mask_params(mask);
+  p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
   const int64_t so[3] = {o->stride[0], o->stride[1], o->stride[2]};
   const int64_t sg[3] = {do_->stride[0], do_->stride[1], do_->stride[2]};
   const int64_t sl[3] = {lse->stride[0], lse->stride[1], lse->stride[2]};
@@ -452,14 +456,14 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     e = sm100_dense_bwd(p, o->data, so, do_->data, sg, lsep, sl, delta, dq_acc, dq->data, sdq, dk->data, sdk,
                         dv->data, sdv, extra, status, cs);
   } else if (q->dtype == ATTN_F32) {
-    e = launch_rows_delta<float>(o->data, do_->data, s.B, s.Hq, s.T, so, sg, s.dv, delta, cs);
+    e = launch_rows_delta<float>(o->data, do_->data, s.B, s.Hq, s.Tq, so, sg, s.dv, delta, cs);
     main_kernel_begin(cs);
     if (e == cudaSuccess)
       e = launch_dense_bwd_rows<float>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk, dv->data,
                                        sdv, cs);
     main_kernel_end(cs);
   } else {
-    e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, s.B, s.Hq, s.T, so, sg, s.dv, delta, cs);
+    e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, s.B, s.Hq, s.Tq, so, sg, s.dv, delta, cs);
     main_kernel_begin(cs);
     if (e == cudaSuccess)
       e = launch_dense_bwd_rows<__nv_bfloat16>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk,
@@ -467,7 +471,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     main_kernel_end(cs);
   }
   if (e == cudaSuccess && want_dsink)
-    e = launch_dsink(mask->sink, lsep, delta, s.B, s.Hq, s.T, sl[0], sl[1], sl[2], true, dsink, cs);
+    e = launch_dsink(mask->sink, lsep, delta, s.B, s.Hq, s.Tq, sl[0], sl[1], sl[2], true, dsink, cs);
   return cuda_status(e);
 }
 

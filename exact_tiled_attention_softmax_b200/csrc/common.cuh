@@ -18,7 +18,8 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Allowed-set descriptor as the kernels see it.
 struct MaskP {
   uint32_t flags;
-  int64_t window;  // W: j > i - W
+  int64_t qoff;    // query row i sits at key position i + qoff (Tk - Tq: bottom-right alignment)
+  int64_t window;  // W: j > i + qoff - W
   const uint8_t* bm;
   int32_t bq, bk;
   int64_t bm_sb, bm_sh, bm_sq;
@@ -35,7 +36,7 @@ struct DenseP {
   const void* k;
   const void* v;
   int64_t sq[3], sk[3], sv[3];
-  int B, Hq, Hkv, T, d, dv;
+  int B, Hq, Hkv, Tq, Tk, d, dv;
   float scale;
   MaskP m;
 };
@@ -61,8 +62,9 @@ __device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfl
 
 // The allowed-set predicate A_i (flags intersect).
 __device__ __forceinline__ bool allowed(const MaskP& m, int b, int h, int64_t i, int64_t j) {
-  if ((m.flags & ATTN_MASK_CAUSAL) && j > i) return false;
-  if ((m.flags & ATTN_MASK_WINDOW) && j <= i - m.window) return false;
+  const int64_t ip = i + m.qoff;  // the query's key position
+  if ((m.flags & ATTN_MASK_CAUSAL) && j > ip) return false;
+  if ((m.flags & ATTN_MASK_WINDOW) && j <= ip - m.window) return false;
   if (m.flags & ATTN_MASK_BLOCK) {
     const uint8_t* row = m.bm + b * m.bm_sb + h * m.bm_sh + (i / m.bq) * m.bm_sq;
     if (!row[j / m.bk]) return false;
@@ -73,11 +75,12 @@ __device__ __forceinline__ bool allowed(const MaskP& m, int b, int h, int64_t i,
 // Key range [lo, hi] that can hold allowed keys for query row i.
 __device__ __forceinline__ void key_range(const MaskP& m, int64_t i, int64_t n_k,
                                           int64_t& lo, int64_t& hi) {
+  const int64_t ip = i + m.qoff;
   lo = 0;
   hi = n_k - 1;
-  if (m.flags & ATTN_MASK_CAUSAL) hi = i < hi ? i : hi;
+  if (m.flags & ATTN_MASK_CAUSAL) hi = ip < hi ? ip : hi;
   if (m.flags & ATTN_MASK_WINDOW) {
-    int64_t w = i - m.window + 1;
+    int64_t w = ip - m.window + 1;
     lo = w > 0 ? w : 0;
   }
 }
@@ -87,9 +90,9 @@ __device__ __forceinline__ void query_range(const MaskP& m, int64_t j, int64_t n
                                             int64_t& lo, int64_t& hi) {
   lo = 0;
   hi = n_q - 1;
-  if (m.flags & ATTN_MASK_CAUSAL) lo = j;
+  if (m.flags & ATTN_MASK_CAUSAL) lo = j - m.qoff > 0 ? j - m.qoff : 0;
   if (m.flags & ATTN_MASK_WINDOW) {
-    int64_t w = j + m.window - 1;
+    int64_t w = j + m.window - 1 - m.qoff;
     hi = w < hi ? w : hi;
   }
 }

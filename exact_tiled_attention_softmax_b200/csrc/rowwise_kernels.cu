@@ -63,10 +63,10 @@ dense_fwd_rows(DenseP p, T* o, int64_t so0, int64_t so1, int64_t so2, float* lse
                int64_t sl1, int64_t sl2) {
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= (int64_t)p.B * p.Hq * p.T) return;
-  const int i = (int)(warp % p.T);
-  const int h = (int)((warp / p.T) % p.Hq);
-  const int b = (int)(warp / ((int64_t)p.T * p.Hq));
+  if (warp >= (int64_t)p.B * p.Hq * p.Tq) return;
+  const int i = (int)(warp % p.Tq);
+  const int h = (int)((warp / p.Tq) % p.Hq);
+  const int b = (int)(warp / ((int64_t)p.Tq * p.Hq));
   const int kvh = h / (p.Hq / p.Hkv);
   const T* Q = static_cast<const T*>(p.q) + b * p.sq[0] + h * p.sq[1] + (int64_t)i * p.sq[2];
   const T* Kb = static_cast<const T*>(p.k) + b * p.sk[0] + kvh * p.sk[1];
@@ -77,7 +77,7 @@ dense_fwd_rows(DenseP p, T* o, int64_t so0, int64_t so1, int64_t so2, float* lse
   for (int c = 0; c < NV; ++c) acc[c] = 0.f;
   float m = -INFINITY, l = 0.f;
   int64_t lo, hi;
-  key_range(p.m, i, p.T, lo, hi);
+  key_range(p.m, i, p.Tk, lo, hi);
   for (int64_t j = lo; j <= hi; ++j) {
     if (!allowed(p.m, b, h, i, j)) continue;  // empty keys leave the state untouched
     float kr[NQ];
@@ -176,10 +176,10 @@ dense_dq_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, const
               int64_t sd1, int64_t sd2) {
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= (int64_t)p.B * p.Hq * p.T) return;
-  const int i = (int)(warp % p.T);
-  const int h = (int)((warp / p.T) % p.Hq);
-  const int b = (int)(warp / ((int64_t)p.T * p.Hq));
+  if (warp >= (int64_t)p.B * p.Hq * p.Tq) return;
+  const int i = (int)(warp % p.Tq);
+  const int h = (int)((warp / p.Tq) % p.Hq);
+  const int b = (int)(warp / ((int64_t)p.Tq * p.Hq));
   const int kvh = h / (p.Hq / p.Hkv);
   const T* Kb = static_cast<const T*>(p.k) + b * p.sk[0] + kvh * p.sk[1];
   const T* Vb = static_cast<const T*>(p.v) + b * p.sv[0] + kvh * p.sv[1];
@@ -192,7 +192,7 @@ dense_dq_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, const
   const float dl = delta[warp];
   if (L != -INFINITY) {
     int64_t lo, hi;
-    key_range(p.m, i, p.T, lo, hi);
+    key_range(p.m, i, p.Tk, lo, hi);
     for (int64_t j = lo; j <= hi; ++j) {
       if (!allowed(p.m, b, h, i, j)) continue;
       float kr[NQ], vr[NV];
@@ -224,10 +224,10 @@ dense_dkv_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, cons
                int64_t sdk1, int64_t sdk2, T* dvp, int64_t sdv0, int64_t sdv1, int64_t sdv2) {
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= (int64_t)p.B * p.Hkv * p.T) return;
-  const int j = (int)(warp % p.T);
-  const int kvh = (int)((warp / p.T) % p.Hkv);
-  const int b = (int)(warp / ((int64_t)p.T * p.Hkv));
+  if (warp >= (int64_t)p.B * p.Hkv * p.Tk) return;
+  const int j = (int)(warp % p.Tk);
+  const int kvh = (int)((warp / p.Tk) % p.Hkv);
+  const int b = (int)(warp / ((int64_t)p.Tk * p.Hkv));
   const int group = p.Hq / p.Hkv;
   float kr[NQ], vr[NV], ak[NQ], av[NV];
   load_row(static_cast<const T*>(p.k) + b * p.sk[0] + kvh * p.sk[1] + (int64_t)j * p.sk[2], p.d, lane, kr);
@@ -237,7 +237,7 @@ dense_dkv_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, cons
 #pragma unroll
   for (int c = 0; c < NV; ++c) av[c] = 0.f;
   int64_t lo, hi;
-  query_range(p.m, j, p.T, lo, hi);
+  query_range(p.m, j, p.Tq, lo, hi);
   for (int hh = 0; hh < group; ++hh) {
     const int h = kvh * group + hh;
     const T* Qb = static_cast<const T*>(p.q) + b * p.sq[0] + h * p.sq[1];
@@ -258,7 +258,7 @@ dense_dkv_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, cons
         dp = keep ? dp * p.m.inv_keep : 0.f;
         pt = keep ? pij * p.m.inv_keep : 0.f;
       }
-      const float gam = pij * (dp - delta[((int64_t)b * p.Hq + h) * p.T + i]);
+      const float gam = pij * (dp - delta[((int64_t)b * p.Hq + h) * p.Tq + i]);
 #pragma unroll
       for (int c = 0; c < NQ; ++c) ak[c] = fmaf(gam, q[c], ak[c]);
 #pragma unroll
@@ -435,7 +435,7 @@ int width_class(int n) { return n <= 32 ? 1 : n <= 64 ? 2 : n <= 128 ? 4 : n <= 
 template <typename T>
 cudaError_t launch_dense_fwd_rows(const DenseP& p, void* o, const int64_t so[3], float* lse,
                                   const int64_t sl[3], cudaStream_t st) {
-  const int64_t rows = (int64_t)p.B * p.Hq * p.T;
+  const int64_t rows = (int64_t)p.B * p.Hq * p.Tq;
   if (rows == 0) return cudaSuccess;
   const int w = width_class(p.d > p.dv ? p.d : p.dv);
   ATTN_DISPATCH_WIDTH(w, dense_fwd_rows<T, NQ, NV><<<blocks_for_warps(rows), kWarps * 32, 0, st>>>(
@@ -478,7 +478,7 @@ cudaError_t launch_dense_bwd_rows(const DenseP& p, const void* g, const int64_t 
                                   void* dk, const int64_t sdk[3], void* dv, const int64_t sdv[3],
                                   cudaStream_t st) {
   const int w = width_class(p.d > p.dv ? p.d : p.dv);
-  const int64_t qrows = (int64_t)p.B * p.Hq * p.T, krows = (int64_t)p.B * p.Hkv * p.T;
+  const int64_t qrows = (int64_t)p.B * p.Hq * p.Tq, krows = (int64_t)p.B * p.Hkv * p.Tk;
   if (qrows == 0) return cudaSuccess;
   ATTN_DISPATCH_WIDTH(w,
       dense_dq_rows<T, NQ, NV><<<blocks_for_warps(qrows), kWarps * 32, 0, st>>>(

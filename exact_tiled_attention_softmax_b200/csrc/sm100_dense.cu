@@ -53,9 +53,9 @@ enum : uint8_t { kEmpty = 0, kFull = 1, kPartial = 2 };
 // ------------------------------------------------------------------ masks
 
 // Is every (i, j) of the rectangle [r0, r1] x [c0, c1] inside the
-// causal/window band, and is any? Row i allows [max(c0, i-W+1), min(c1, i)],
-// so some row qualifies iff i can be chosen with c0 <= i (causal) and
-// i <= c1 + W - 1 (window).
+// causal/window band, and is any? Rows are given as key positions (query row
+// + qoff). Row i allows [max(c0, i-W+1), min(c1, i)], so some row qualifies
+// iff i can be chosen with c0 <= i (causal) and i <= c1 + W - 1 (window).
 __device__ __forceinline__ void band_test(const MaskP& m, int64_t r0, int64_t r1, int64_t c0, int64_t c1, bool& any,
                                           bool& all) {
   const bool causal = m.flags & ATTN_MASK_CAUSAL, window = m.flags & ATTN_MASK_WINDOW;
@@ -69,14 +69,14 @@ __device__ __forceinline__ void band_test(const MaskP& m, int64_t r0, int64_t r1
 }
 
 // Class of the (64-row query slice qs, 128-key tile kt) pair.
-__device__ uint8_t tile_class(const MaskP& m, int T, int b, int h, int qs, int kt) {
-  const int64_t r0 = (int64_t)qs * kBMb, r1 = (r0 + kBMb < T ? r0 + kBMb : T) - 1;
-  const int64_t c0 = (int64_t)kt * kBN, c1e = c0 + kBN - 1, c1 = (c1e < T ? c1e : T - 1);
+__device__ uint8_t tile_class(const MaskP& m, int Tq, int Tk, int b, int h, int qs, int kt) {
+  const int64_t r0 = (int64_t)qs * kBMb, r1 = (r0 + kBMb < Tq ? r0 + kBMb : Tq) - 1;
+  const int64_t c0 = (int64_t)kt * kBN, c1e = c0 + kBN - 1, c1 = (c1e < Tk ? c1e : Tk - 1);
   if (r0 > r1 || c0 > c1) return kEmpty;
-  bool any = false, all = c1e <= T - 1;
+  bool any = false, all = c1e <= Tk - 1;
   if (!(m.flags & ATTN_MASK_BLOCK)) {
     bool a, f;
-    band_test(m, r0, r1, c0, c1, a, f);
+    band_test(m, r0 + m.qoff, r1 + m.qoff, c0, c1, a, f);
     any = a;
     all = all && f;
   } else {
@@ -88,7 +88,7 @@ __device__ uint8_t tile_class(const MaskP& m, int T, int b, int h, int qs, int k
         const int64_t cc0 = cb * m.bk > c0 ? cb * m.bk : c0;
         const int64_t cc1 = cb * m.bk + m.bk - 1 < c1 ? cb * m.bk + m.bk - 1 : c1;
         bool a, f;
-        band_test(m, rr0, rr1, cc0, cc1, a, f);
+        band_test(m, rr0 + m.qoff, rr1 + m.qoff, cc0, cc1, a, f);
         if (base[rb * m.bm_sq + cb]) {
           any = any || a;
           all = all && f;
@@ -107,32 +107,32 @@ struct ClassTable {
   int nqs, nkt;
 };
 
-__device__ __forceinline__ uint8_t lookup_class(const ClassTable& ct, const MaskP& m, int T, int b, int h, int qs,
-                                                int kt) {
-  if ((int64_t)qs * kBMb >= T) return kEmpty;  // slices past the last row are not in the table
-  if (!ct.cls) return tile_class(m, T, b, h, qs, kt);
+__device__ __forceinline__ uint8_t lookup_class(const ClassTable& ct, const MaskP& m, int Tq, int Tk, int b, int h,
+                                                int qs, int kt) {
+  if ((int64_t)qs * kBMb >= Tq) return kEmpty;  // slices past the last row are not in the table
+  if (!ct.cls) return tile_class(m, Tq, Tk, b, h, qs, kt);
   const int sb = ct.nb > 1 ? b : 0, sh = ct.nh > 1 ? h : 0;
   return ct.cls[(((int64_t)sb * ct.nh + sh) * ct.nqs + qs) * ct.nkt + kt];
 }
 
-__global__ void classify_kernel(MaskP m, int T, int B, int Hq, ClassTable ct, uint8_t* out) {
+__global__ void classify_kernel(MaskP m, int Tq, int Tk, int B, int Hq, ClassTable ct, uint8_t* out) {
   const int64_t n = (int64_t)ct.nb * ct.nh * ct.nqs * ct.nkt;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
     const int kt = (int)(e % ct.nkt);
     const int qs = (int)((e / ct.nkt) % ct.nqs);
     const int sh = (int)((e / ((int64_t)ct.nkt * ct.nqs)) % ct.nh);
     const int sb = (int)(e / ((int64_t)ct.nkt * ct.nqs * ct.nh));
-    out[e] = tile_class(m, T, sb, sh, qs, kt);
+    out[e] = tile_class(m, Tq, Tk, sb, sh, qs, kt);
   }
   (void)B;
   (void)Hq;
 }
 
 // Forward tile class for a 128-row query tile: merge its two 64-row slices.
-__device__ __forceinline__ uint8_t fwd_class(const ClassTable& ct, const MaskP& m, int T, int b, int h, int qt,
-                                             int kt) {
-  const uint8_t a = lookup_class(ct, m, T, b, h, 2 * qt, kt);
-  const uint8_t c = (2 * qt + 1) * kBMb < T ? lookup_class(ct, m, T, b, h, 2 * qt + 1, kt) : a;
+__device__ __forceinline__ uint8_t fwd_class(const ClassTable& ct, const MaskP& m, int Tq, int Tk, int b, int h,
+                                             int qt, int kt) {
+  const uint8_t a = lookup_class(ct, m, Tq, Tk, b, h, 2 * qt, kt);
+  const uint8_t c = (2 * qt + 1) * kBMb < Tq ? lookup_class(ct, m, Tq, Tk, b, h, 2 * qt + 1, kt) : a;
   if (a == kEmpty && c == kEmpty) return kEmpty;
   if (a == kFull && c == kFull) return kFull;
   return kPartial;
@@ -143,7 +143,7 @@ __device__ __forceinline__ uint8_t fwd_class(const ClassTable& ct, const MaskP& 
 struct FwdArgs {
   MaskP m;
   ClassTable ct;
-  int B, Hq, Hkv, T;
+  int B, Hq, Hkv, Tq, Tk;
   int block_aligned;  // block mask constant over every (64-row slice, 128-key tile)
   float scale_log2;   // c * log2(e)
   __nv_bfloat16* o;
@@ -176,24 +176,28 @@ struct FwdCtl {
 };
 
 // Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
-__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int T, int q0, int rows, int& lo, int& hi) {
-  const int nkt = (T + kBN - 1) / kBN;
+__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int Tq, int Tk, int q0, int rows, int& lo,
+                                              int& hi) {
+  const int nkt = (Tk + kBN - 1) / kBN;
   lo = 0;
   hi = nkt - 1;
   if (m.flags & ATTN_MASK_CAUSAL) {
-    const int last = (q0 + rows - 1 < T - 1 ? q0 + rows - 1 : T - 1) / kBN;
-    hi = last < hi ? last : hi;
+    const int64_t last = (int64_t)(q0 + rows - 1 < Tq - 1 ? q0 + rows - 1 : Tq - 1) + m.qoff;  // key position
+    if (last < 0)
+      hi = -1;
+    else if (last / kBN < hi)
+      hi = (int)(last / kBN);
   }
   if (m.flags & ATTN_MASK_WINDOW) {
-    const int64_t first = (int64_t)q0 - m.window + 1;
+    const int64_t first = (int64_t)q0 + m.qoff - m.window + 1;
     lo = first > 0 ? (int)(first / kBN) : 0;
   }
 }
 
-// Class of (128-row query tile qt, key tile kt); tiles past T are empty.
+// Class of (128-row query tile qt, key tile kt); tiles past Tq are empty.
 __device__ __forceinline__ uint8_t wg_class(const FwdArgs& a, int b, int h, int qt, int kt) {
-  if (qt * kBM >= a.T) return kEmpty;
-  return fwd_class(a.ct, a.m, a.T, b, h, qt, kt);
+  if (qt * kBM >= a.Tq) return kEmpty;
+  return fwd_class(a.ct, a.m, a.Tq, a.Tk, b, h, qt, kt);
 }
 
 // First key tile after `from` (up to kt_hi) with allowed keys for either
@@ -225,11 +229,12 @@ __device__ __forceinline__ uint64_t range_bits64(int64_t lo, int64_t hi) {
 __device__ __forceinline__ void fwd_row_bits(const FwdArgs& a, int b, int h, int64_t i, int64_t j0, uint8_t slice_cls,
                                              uint64_t& w0, uint64_t& w1) {
   w0 = w1 = 0ull;
-  if (i >= a.T || slice_cls == kEmpty) return;
+  if (i >= a.Tq || slice_cls == kEmpty) return;
+  const int64_t ip = i + a.m.qoff;  // the row's key position
   int64_t lo = j0, hi = j0 + kBN - 1;
-  if (hi > a.T - 1) hi = a.T - 1;
-  if (a.m.flags & ATTN_MASK_CAUSAL) hi = i < hi ? i : hi;
-  if (a.m.flags & ATTN_MASK_WINDOW) lo = i - a.m.window + 1 > lo ? i - a.m.window + 1 : lo;
+  if (hi > a.Tk - 1) hi = a.Tk - 1;
+  if (a.m.flags & ATTN_MASK_CAUSAL) hi = ip < hi ? ip : hi;
+  if (a.m.flags & ATTN_MASK_WINDOW) lo = ip - a.m.window + 1 > lo ? ip - a.m.window + 1 : lo;
   if (lo > hi) return;
   w0 = range_bits64(lo - j0, hi - j0);
   w1 = range_bits64(lo - j0 - 64, hi - j0 - 64);
@@ -238,8 +243,8 @@ __device__ __forceinline__ void fwd_row_bits(const FwdArgs& a, int b, int h, int
     uint64_t b0 = 0, b1 = 0;
 #pragma unroll 1
     for (int c = 0; c < 64; ++c) {
-      if (j0 + c < a.T && row[(j0 + c) / a.m.bk]) b0 |= 1ull << c;
-      if (j0 + 64 + c < a.T && row[(j0 + 64 + c) / a.m.bk]) b1 |= 1ull << c;
+      if (j0 + c < a.Tk && row[(j0 + c) / a.m.bk]) b0 |= 1ull << c;
+      if (j0 + 64 + c < a.Tk && row[(j0 + 64 + c) / a.m.bk]) b1 |= 1ull << c;
     }
     w0 &= b0;
     w1 &= b1;
@@ -411,7 +416,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Longest query tiles (most keys under a causal mask) first over the whole
   // grid: the tail of the launch is made of the shortest tiles.
-  const int nct = (a.T + kFwdRows - 1) / kFwdRows;
+  const int nct = (a.Tq + kFwdRows - 1) / kFwdRows;
   const int bh = blockIdx.x % (a.B * a.Hq);
   const int ct = nct - 1 - (int)(blockIdx.x / (a.B * a.Hq));
   const int h = bh % a.Hq, b = bh / a.Hq;
@@ -419,7 +424,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int q0 = ct * kFwdRows;
   const int qt0 = 2 * ct;
   int kt_lo, kt_hi;
-  fwd_key_tiles(a.m, a.T, q0, kFwdRows, kt_lo, kt_hi);
+  fwd_key_tiles(a.m, a.Tq, a.Tk, q0, kFwdRows, kt_lo, kt_hi);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->q_full), 1);
@@ -575,7 +580,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (mk <= kt_hi) {
           cword = wg_class(a, b, h, qt, mk);
           if (cword == kPartial)
-            cword |= ((uint32_t)lookup_class(a.ct, a.m, a.T, b, h, 2 * qt + (t >> 6), mk) & 3u) << 2;
+            cword |= ((uint32_t)lookup_class(a.ct, a.m, a.Tq, a.Tk, b, h, 2 * qt + (t >> 6), mk) & 3u) << 2;
         }
       }
       const uint32_t cv = __shfl_sync(0xffffffffu, cword, kt - cbase);
@@ -584,7 +589,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint64_t mw0 = ~0ull, mw1 = ~0ull;
       if (cls == kPartial) {
         mw0 = mw1 = 0ull;
-        if (row < a.T) fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, (uint8_t)(cv >> 2), mw0, mw1);
+        if (row < a.Tq) fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, (uint8_t)(cv >> 2), mw0, mw1);
       }
       uint64_t kb0 = ~0ull, kb1 = ~0ull;
       if (a.m.dropout) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
@@ -644,7 +649,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           tmem_ld32(tO + c * 32, o);
           tmem_wait_ld();
         }
-        if (row < a.T) {
+        if (row < a.Tq) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t pkd[4];
@@ -657,7 +662,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           }
         }
       }
-      if (row < a.T) a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
+      if (row < a.Tq) a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
     }
   }
   tc_fence_before();
@@ -673,12 +678,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 struct BwdArgs {
   MaskP m;
   ClassTable ct;
-  int B, Hq, Hkv, T, Tpad;
+  int B, Hq, Hkv, Tq, Tk, Tpad;
   int block_aligned;
   float scale_log2;
   const float* lse2;    // [B*Hq, Tpad] minus the base-2 LSE (-inf on rows without keys)
   const float* dpad;    // [B*Hq, Tpad] minus delta, zero on padding rows
-  float* dq_acc;        // [B, Hq, T, 128] fp32
+  float* dq_acc;        // [B, Hq, Tq, 128] fp32
   __nv_bfloat16* dk;
   int64_t sdk[3];
   __nv_bfloat16* dv;
@@ -724,14 +729,20 @@ struct BwdCtl {
 };
 
 // Query-slice range [lo, hi] that can hold rows seeing keys [k0, k0 + 128).
-__device__ __forceinline__ void bwd_query_slices(const MaskP& m, int T, int k0, int& lo, int& hi) {
-  const int nqs = (T + kBMb - 1) / kBMb;
+__device__ __forceinline__ void bwd_query_slices(const MaskP& m, int Tq, int k0, int& lo, int& hi) {
+  const int nqs = (Tq + kBMb - 1) / kBMb;
   lo = 0;
   hi = nqs - 1;
-  if (m.flags & ATTN_MASK_CAUSAL) lo = k0 / kBMb;
-  if (m.flags & ATTN_MASK_WINDOW) {
-    const int64_t last = (int64_t)k0 + kBN - 1 + m.window - 1;
-    if (last < T) hi = (int)(last / kBMb);
+  if (m.flags & ATTN_MASK_CAUSAL) {  // rows whose key position reaches k0
+    const int64_t first = (int64_t)k0 - m.qoff;
+    if (first > 0) lo = first / kBMb < nqs ? (int)(first / kBMb) : nqs;
+  }
+  if (m.flags & ATTN_MASK_WINDOW) {  // rows whose window still reaches the tile's last key
+    const int64_t last = (int64_t)k0 + kBN - 1 + m.window - 1 - m.qoff;
+    if (last < 0)
+      hi = -1;
+    else if (last < Tq)
+      hi = (int)(last / kBMb);
   }
 }
 
@@ -744,25 +755,26 @@ __device__ __forceinline__ bool bwd_next_step(const BwdArgs& a, int b, int kvh, 
       if (++hh >= group) return false;
       qs = qs_lo;
     }
-    cls = lookup_class(a.ct, a.m, a.T, b, kvh * group + hh, qs, kt);
+    cls = lookup_class(a.ct, a.m, a.Tq, a.Tk, b, kvh * group + hh, qs, kt);
     if (cls != kEmpty) return true;
   }
 }
 
 // Allowed query rows i0..i0+63 for key j, as a 64-bit word (bit c <-> i0 + c).
 __device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h, int64_t i0, int64_t j) {
-  if (j >= a.T) return 0ull;
+  if (j >= a.Tk) return 0ull;
   int64_t lo = i0, hi = i0 + kBMb - 1;
-  if (hi > a.T - 1) hi = a.T - 1;
-  if (a.m.flags & ATTN_MASK_CAUSAL) lo = j > lo ? j : lo;
-  if (a.m.flags & ATTN_MASK_WINDOW) hi = j + a.m.window - 1 < hi ? j + a.m.window - 1 : hi;
+  if (hi > a.Tq - 1) hi = a.Tq - 1;
+  if (a.m.flags & ATTN_MASK_CAUSAL) lo = j - a.m.qoff > lo ? j - a.m.qoff : lo;  // row i sees j iff i + qoff >= j
+  if (a.m.flags & ATTN_MASK_WINDOW)
+    hi = j + a.m.window - 1 - a.m.qoff < hi ? j + a.m.window - 1 - a.m.qoff : hi;
   uint64_t w = range_bits64(lo - i0, hi - i0);
   if (w && (a.m.flags & ATTN_MASK_BLOCK) && !a.block_aligned) {
     const uint8_t* base = a.m.bm + b * a.m.bm_sb + h * a.m.bm_sh + j / a.m.bk;
     uint64_t bb = 0;
 #pragma unroll 1
     for (int c = 0; c < kBMb; ++c)
-      if (i0 + c < a.T && base[((i0 + c) / a.m.bq) * a.m.bm_sq]) bb |= 1ull << c;
+      if (i0 + c < a.Tq && base[((i0 + c) / a.m.bq) * a.m.bm_sq]) bb |= 1ull << c;
     w &= bb;
   }
   return w;
@@ -825,7 +837,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   // Bands of kBwdBand (b, K/V head) pairs: within a band the earliest key tiles
   // (most work under a causal mask) go first; the CTAs resident at any time
   // then share a few heads' dQ accumulator rows and Q/dO in L2.
-  const int nkt_all = (a.T + kBN - 1) / kBN;
+  const int nkt_all = (a.Tk + kBN - 1) / kBN;
   const int nbkv = a.B * a.Hkv;
   const int band = (int)(blockIdx.x / ((int64_t)kBwdBand * nkt_all));
   const int band0 = band * kBwdBand;
@@ -836,7 +848,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int kvh = bkv % a.Hkv, b = bkv / a.Hkv;
   const int k0 = kt * kBN;
   int qs_lo, qs_hi;
-  bwd_query_slices(a.m, a.T, k0, qs_lo, qs_hi);
+  bwd_query_slices(a.m, a.Tq, k0, qs_lo, qs_hi);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->kv_full), 1);
@@ -1108,7 +1120,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           tmem_ld32(tacc + c * 32, r);
           tmem_wait_ld();
         }
-        if (j < a.T) {
+        if (j < a.Tk) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t pk[4];
@@ -1307,10 +1319,10 @@ cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
   return e;
 }
 
-size_t class_bytes(int B, int Hq, int T, const attn_mask* m) {
+size_t class_bytes(int B, int Hq, int Tq, int Tk, const attn_mask* m) {
   if (!m || !(m->flags & ATTN_MASK_BLOCK)) return 0;
   const int nb = m->bm_stride_b ? B : 1, nh = m->bm_stride_h ? Hq : 1;
-  const size_t nqs = (T + kBMb - 1) / kBMb, nkt = (T + kBN - 1) / kBN;
+  const size_t nqs = (Tq + kBMb - 1) / kBMb, nkt = (Tk + kBN - 1) / kBN;
   return align_up((size_t)nb * nh * nqs * nkt, 256);
 }
 
@@ -1319,14 +1331,14 @@ ClassTable build_class_table(const DenseP& p, void* ws, cudaStream_t st, cudaErr
   ct.cls = nullptr;
   ct.nb = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sb ? p.B : 1;
   ct.nh = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sh ? p.Hq : 1;
-  ct.nqs = (p.T + kBMb - 1) / kBMb;
-  ct.nkt = (p.T + kBN - 1) / kBN;
+  ct.nqs = (p.Tq + kBMb - 1) / kBMb;
+  ct.nkt = (p.Tk + kBN - 1) / kBN;
   err = cudaSuccess;
   if (!(p.m.flags & ATTN_MASK_BLOCK)) return ct;
   uint8_t* out = static_cast<uint8_t*>(ws);
   const int64_t n = (int64_t)ct.nb * ct.nh * ct.nqs * ct.nkt;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  classify_kernel<<<blocks, 256, 0, st>>>(p.m, p.T, p.B, p.Hq, ct, out);
+  classify_kernel<<<blocks, 256, 0, st>>>(p.m, p.Tq, p.Tk, p.B, p.Hq, ct, out);
   err = cudaGetLastError();
   ct.cls = out;
   return ct;
@@ -1334,17 +1346,19 @@ ClassTable build_class_table(const DenseP& p, void* ws, cudaStream_t st, cudaErr
 
 }  // namespace
 
-size_t sm100_fwd_workspace_bytes(int B, int Hq, int T, const attn_mask* m) { return class_bytes(B, Hq, T, m); }
+size_t sm100_fwd_workspace_bytes(int B, int Hq, int Tq, int Tk, const attn_mask* m) {
+  return class_bytes(B, Hq, Tq, Tk, m);
+}
 
-size_t sm100_bwd_extra_workspace_bytes(int B, int Hq, int Hkv, int T, const attn_mask* m) {
+size_t sm100_bwd_extra_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, const attn_mask* m) {
   (void)Hkv;
-  const size_t Tpad = (size_t)((T + kBN - 1) / kBN) * kBN;
-  return 2 * align_up((size_t)B * Hq * Tpad * sizeof(float), 256) + class_bytes(B, Hq, T, m);
+  const size_t Tpad = (size_t)((Tq + kBN - 1) / kBN) * kBN;
+  return 2 * align_up((size_t)B * Hq * Tpad * sizeof(float), 256) + class_bytes(B, Hq, Tq, Tk, m);
 }
 
 bool sm100_dense_supported(const DenseP& p, const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
                            const attn_tensor* o) {
-  if (p.d != kD || p.dv != kD || p.T < 1) return false;
+  if (p.d != kD || p.dv != kD || p.Tq < 1 || p.Tk < 1) return false;
   if (!tma_ok(q) || !tma_ok(k) || !tma_ok(v) || !tma_ok(o)) return false;
   if (!encode_fn()) return false;
   int dev = 0, major = 0, minor = 0;
@@ -1365,9 +1379,9 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   ClassTable ct = build_class_table(p, ws, st, err);
   if (err != cudaSuccess) return err;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM) ||
-      !make_map(&mk, p.k, p.T, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
-      !make_map(&mv, p.v, p.T, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN))
+  if (!make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM) ||
+      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
+      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN))
     return cudaErrorInvalidValue;
   FwdArgs a;
   a.m = p.m;
@@ -1376,7 +1390,8 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   a.B = p.B;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
-  a.T = p.T;
+  a.Tq = p.Tq;
+  a.Tk = p.Tk;
   a.scale_log2 = p.scale * kLog2e;
   a.o = static_cast<__nv_bfloat16*>(o);
   for (int i = 0; i < 3; ++i) {
@@ -1386,7 +1401,7 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   a.lse = lse;
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(fwd_kernel), kFwdSmem, 0)) != cudaSuccess) return err;
-  const int nct = (p.T + kFwdRows - 1) / kFwdRows;
+  const int nct = (p.Tq + kFwdRows - 1) / kFwdRows;
   main_kernel_begin(st);
   fwd_kernel<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
   main_kernel_end(st);
@@ -1397,7 +1412,7 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
                             const float* lse, const int64_t sl[3], float* delta, float* dq_acc, void* dq,
                             const int64_t sdq[3], void* dk, const int64_t sdk[3], void* dv, const int64_t sdv[3],
                             void* ws_extra, uint32_t* status, cudaStream_t st) {
-  const int Tpad = ((p.T + kBN - 1) / kBN) * kBN;
+  const int Tpad = ((p.Tq + kBN - 1) / kBN) * kBN;
   const size_t padb = align_up((size_t)p.B * p.Hq * Tpad * sizeof(float), 256);
   float* lse2 = static_cast<float*>(ws_extra);
   float* dpad = reinterpret_cast<float*>(static_cast<char*>(ws_extra) + padb);
@@ -1407,14 +1422,14 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   const int64_t rows = (int64_t)p.B * p.Hq * Tpad;
   bwd_prepare_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), so[0], so[1], so[2], static_cast<const __nv_bfloat16*>(g), sg[0], sg[1],
-      sg[2], lse, sl[0], sl[1], sl[2], p.B, p.Hq, p.T, Tpad, lse2, dpad, delta, dq_acc);
+      sg[2], lse, sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta, dq_acc);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   CUtensorMap mq, mk, mv, mg, mdq;
-  if (!make_dq_map(&mdq, dq_acc, p.T, p.B * p.Hq) ||
-      !make_map(&mq, p.q, p.T, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
-      !make_map(&mk, p.k, p.T, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
-      !make_map(&mv, p.v, p.T, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN) ||
-      !make_map(&mg, g, p.T, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb))
+  if (!make_dq_map(&mdq, dq_acc, p.Tq, p.B * p.Hq) ||
+      !make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
+      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
+      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN) ||
+      !make_map(&mg, g, p.Tq, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb))
     return cudaErrorInvalidValue;
   BwdArgs a;
   a.m = p.m;
@@ -1423,7 +1438,8 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.B = p.B;
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
-  a.T = p.T;
+  a.Tq = p.Tq;
+  a.Tk = p.Tk;
   a.Tpad = Tpad;
   a.scale_log2 = p.scale * kLog2e;
   a.lse2 = lse2;
@@ -1438,13 +1454,13 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.scale = p.scale;
   a.status = status;
   if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
-  const int nkt = (p.T + kBN - 1) / kBN;
+  const int nkt = (p.Tk + kBN - 1) / kBN;
   main_kernel_begin(st);
   bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
   main_kernel_end(st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  const int64_t n4 = (int64_t)p.B * p.Hq * p.T * kD / 4;
-  dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.T, p.scale,
+  const int64_t n4 = (int64_t)p.B * p.Hq * p.Tq * kD / 4;
+  dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.Tq, p.scale,
                                                                  static_cast<__nv_bfloat16*>(dq), sdq[0], sdq[1],
                                                                  sdq[2]);
   return cudaGetLastError();

@@ -8,8 +8,8 @@
 
 namespace attn {
 
-size_t sm100_fwd_workspace_bytes(int B, int Hq, int T, const attn_mask* m);
-size_t sm100_bwd_extra_workspace_bytes(int B, int Hq, int Hkv, int T, const attn_mask* m);
+size_t sm100_fwd_workspace_bytes(int B, int Hq, int Tq, int Tk, const attn_mask* m);
+size_t sm100_bwd_extra_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tk, const attn_mask* m);
 bool sm100_dense_supported(const DenseP& p, const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
                            const attn_tensor* o);
 bool sm100_dense_bwd_supported(const DenseP& p, const attn_tensor* do_, const attn_tensor* dq,

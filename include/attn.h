@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 101 /* major * 100 + minor */
+#define ATTN_VERSION 102 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -81,9 +81,12 @@ typedef struct attn_tensor {
   int64_t stride[4];
 } attn_tensor;
 
-/* Allowed-set flags. A_i is the intersection of every enabled set. */
-#define ATTN_MASK_CAUSAL 0x1u /* j <= i */
-#define ATTN_MASK_WINDOW 0x2u /* j >  i - window_left */
+/* Allowed-set flags. A_i is the intersection of every enabled set. With
+ * Tq query rows and Tk keys, query row i sits at key position
+ * p(i) = i + Tk - Tq (bottom-right alignment: the last query row sees the
+ * last key; p(i) = i when Tq = Tk). */
+#define ATTN_MASK_CAUSAL 0x1u /* j <= p(i) */
+#define ATTN_MASK_WINDOW 0x2u /* j >  p(i) - window_left */
 #define ATTN_MASK_BLOCK 0x4u  /* block_mask[i / block_q][j / block_k] != 0 */
 #define ATTN_MASK_TOPK 0x8u   /* j listed in topk_idxs[t][0 : topk_length[t]] */
 
@@ -121,8 +124,11 @@ typedef struct attn_mask {
 } attn_mask;
 
 /* Layouts
- *   Dense:  q [B,Hq,T,d], k [B,Hkv,T,d], v [B,Hkv,T,dv], o [B,Hq,T,dv],
- *           lse fp32 [B,Hq,T]. Any stride order (BHSD, BSHD, ...).
+ *   Dense:  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v [B,Hkv,Tk,dv], o [B,Hq,Tq,dv],
+ *           lse fp32 [B,Hq,Tq]; dq, do like q/o, dk, dv like k/v. Tq and Tk
+ *           may differ (a query block against a longer key cache); the
+ *           block mask grid is [ceil(Tq/block_q)][ceil(Tk/block_k)] indexed
+ *           by the query's own row. Any stride order (BHSD, BSHD, ...).
  *   Top-k (ATTN_MASK_TOPK, shared KV): q [Tq,H,Dqk], k = KV [Tkv,Dqk],
  *           v = the view KV[:, :Dv] (same data pointer and row stride as k),
  *           o [Tq,H,Dv], lse fp32 [Tq,H]. dk receives dKV [Tkv,Dqk]; dv is NULL.

@@ -248,3 +248,43 @@ def test_topk_bad_index_sets_status_and_returns():
     eta.attn_fwd(qd, kvd, kvd[:, :32], al, 0.125, workspace=ws)
     assert eta.attn_get_status(ws) & eta.ATTN_DEVERR_TOPK_INDEX
     assert eta.attn_get_status(ws) == 0  # read clears
+
+
+def _qk_case(B, Hq, Hkv, Tq, Tk, d, dv, dtype, seed, *, causal=True, window=0, block=0, dropout=0.0, sink=False):
+    rng = np.random.default_rng(seed)
+    f = (lambda s: W.round_to_bf16(rng.standard_normal(s, dtype=np.float32))) if dtype == "bf16" else \
+        (lambda s: rng.standard_normal(s, dtype=np.float32))
+    q, g = f((B, Hq, Tq, d)), f((B, Hq, Tq, dv))
+    k, v = f((B, Hkv, Tk, d)), f((B, Hkv, Tk, dv))
+    bm = None
+    if block:
+        bm = (rng.random((B, Hq, (Tq + block - 1) // block, (Tk + block - 1) // block)) < 0.6).astype(np.uint8)
+    sk = rng.standard_normal(Hq).astype(np.float32) if sink else None
+    return dict(q=q, k=k, v=v, g=g, bm=bm, sink=sk, scale=1 / math.sqrt(d), causal=causal, window=window,
+                block=block, dropout=dropout, seed=seed, dtype=dtype)
+
+
+@pytest.mark.parametrize("kind", ["causal_short_q", "causal_long_q", "window_block", "gqa_dropout_sink"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_query_block_against_longer_or_shorter_keys(kind, dtype):
+    """Tq != Tk with bottom-right alignment: query row i sits at key position
+    i + Tk - Tq (rows with no key position left get the empty-set result)."""
+    if kind == "causal_short_q":
+        c = _qk_case(2, 4, 2, 200, 330, 128, 128, dtype, 21)
+    elif kind == "causal_long_q":
+        c = _qk_case(1, 4, 4, 300, 130, 128, 128, dtype, 22)
+    elif kind == "window_block":
+        c = _qk_case(1, 3, 3, 130, 400, 128, 128, dtype, 23, window=100, block=64)
+    else:
+        c = _qk_case(2, 4, 2, 150, 290, 128, 128, dtype, 24, dropout=0.1, sink=True)
+    gpu = _run_gpu(c)
+    B, Hq, Tq = c["q"].shape[:3]
+    Tk = c["k"].shape[2]
+    allow = oracle.allowed_dense(Tq, Tk, causal=c["causal"], window_left=c["window"], block_mask=c["bm"],
+                                 block_q=c["block"] or 1, block_k=c["block"] or 1, query_offset=Tk - Tq)
+    keep = P.dropout_keep(c["seed"], c["dropout"], B, Hq, Tq, Tk) if c["dropout"] else None
+    q, k, v, g = (c[n].astype(np.float64) for n in ("q", "k", "v", "g"))
+    sink = c["sink"].astype(np.float64) if c["sink"] is not None else None
+    fw = oracle.forward(q, k, v, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"])
+    bw = oracle.backward(q, k, v, g, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"], y=fw.y)
+    _compare(c, gpu, fw, bw)
