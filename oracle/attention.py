@@ -58,7 +58,9 @@ NEG_INF = -np.inf
 
 def allowed_dense(t_q: int, t_k: int, *, causal: bool = False, window_left: int = 0,
                   block_mask: np.ndarray | None = None, block_q: int = 1,
-                  block_k: int = 1, query_offset: int = 0) -> np.ndarray:
+                  block_k: int = 1, query_offset: int = 0,
+                  lengths: np.ndarray | None = None,
+                  starts: np.ndarray | None = None) -> np.ndarray:
     """Boolean A as [.., t_q, t_k]: the intersection of the enabled sets.
 
     causal: j <= i + query_offset ("Accumulate attention without keeping the
@@ -70,6 +72,16 @@ def allowed_dense(t_q: int, t_k: int, *, causal: bool = False, window_left: int 
     block_mask [.., ceil(t_q/block_q), ceil(t_k/block_k)]: key j is allowed
     for query i iff block_mask[i // block_q, j // block_k] != 0.
     Leading dimensions of block_mask (batch, head) are kept in the result.
+
+    The row-interval layouts of the same page (section "Change attention
+    evaluation inside the existing model": the causal range intersected with
+    active lengths and packed-segment boundaries; the per-row lower bound
+    `starts` of section "Rescale earlier mass ..."):
+    lengths [B] (needs t_q == t_k): batch row b has L_b active cells; query
+    rows i >= L_b and keys j >= L_b are outside every set (L_b is clamped to
+    [0, t_k]). starts [B, t_q]: key j is allowed for query i of batch row b
+    only if j >= starts[b, i] (a packed segment's first cell). Either one
+    adds a batch axis: the result is [B, 1 or H, t_q, t_k].
     """
     i = np.arange(t_q)[:, None] + query_offset
     j = np.arange(t_k)[None, :]
@@ -83,6 +95,22 @@ def allowed_dense(t_q: int, t_k: int, *, causal: bool = False, window_left: int 
         rows = np.arange(t_q) // block_q
         cols = np.arange(t_k) // block_k
         allow = allow & bm[..., rows[:, None], cols[None, :]]
+    if lengths is not None or starts is not None:
+        n_b = len(lengths) if lengths is not None else np.asarray(starts).shape[0]
+        extra = np.ones((n_b, 1, t_q, t_k), dtype=bool)
+        if lengths is not None:
+            if t_q != t_k:
+                raise ValueError("lengths need t_q == t_k")
+            L = np.clip(np.asarray(lengths, dtype=np.int64), 0, t_k)[:, None, None, None]
+            extra &= (np.arange(t_q)[:, None] < L) & (np.arange(t_k)[None, :] < L)
+        if starts is not None:
+            st = np.asarray(starts, dtype=np.int64)[:, None, :, None]
+            extra &= j >= st
+        if allow.ndim == 2:
+            allow = allow[None, None]
+        elif allow.ndim == 3:
+            allow = allow[:, None]
+        allow = allow & extra
     return allow
 
 

@@ -484,3 +484,104 @@ def test_topk_empty_list_gives_zero_output_and_sink_lse():
     assert np.all(o2[1] == 0.0) and np.all(np.isneginf(lse2[1]))
     o1, lse1, _ = oracle.topk_forward(q[:1], kv, idx[:1], ln[:1], 4, 0.3, z)
     assert np.allclose(o1[0], o[0]) and np.allclose(lse1[0], lse[0])
+
+
+# ---------------------------------------------------------------------------
+# Row-interval layouts: a query block against a longer key range, packed
+# segments (per-row lower bound) and active lengths
+# ---------------------------------------------------------------------------
+
+def _rand(rng, *shape):
+    return rng.standard_normal(shape)
+
+
+def test_query_block_equals_trailing_rows_of_full_causal():
+    """Bottom-right alignment: the last Tq query rows of causal attention over
+    Tk cells, evaluated as a separate Tq-row block, give the same rows, LSE
+    and (with the upstream gradient zero on the other rows) the same K/V
+    gradients as the full Tk x Tk causal problem."""
+    rng = np.random.default_rng(301)
+    B, Hq, Hkv, Tk, Tq, d, dv = 2, 4, 2, 23, 9, 5, 3
+    q, k, v = _rand(rng, B, Hq, Tk, d), _rand(rng, B, Hkv, Tk, d), _rand(rng, B, Hkv, Tk, dv)
+    g = _rand(rng, B, Hq, Tk, dv)
+    g[:, :, :Tk - Tq] = 0.0
+    sink = _rand(rng, Hq)
+    full_allow = A.allowed_dense(Tk, Tk, causal=True, window_left=6)
+    blk_allow = A.allowed_dense(Tq, Tk, causal=True, window_left=6, query_offset=Tk - Tq)
+    fw_full = A.forward(q, k, v, full_allow, 0.4, sink=sink)
+    fw_blk = A.forward(q[:, :, Tk - Tq:], k, v, blk_allow, 0.4, sink=sink)
+    np.testing.assert_allclose(fw_blk.y, fw_full.y[:, :, Tk - Tq:], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(fw_blk.lse, fw_full.lse[:, :, Tk - Tq:], rtol=0, atol=1e-13)
+    bw_full = A.backward(q, k, v, g, full_allow, 0.4, sink=sink)
+    bw_blk = A.backward(q[:, :, Tk - Tq:], k, v, g[:, :, Tk - Tq:], blk_allow, 0.4, sink=sink)
+    np.testing.assert_allclose(bw_blk.dq, bw_full.dq[:, :, Tk - Tq:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(bw_blk.dk, bw_full.dk, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(bw_blk.dv, bw_full.dv, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(bw_blk.dsink, bw_full.dsink, rtol=0, atol=1e-12)
+    # Tq > Tk: the first Tq - Tk rows sit before the first key and are empty.
+    long_allow = A.allowed_dense(7, 4, causal=True, query_offset=4 - 7)
+    assert not long_allow[:3].any() and long_allow[3:].sum() == 10
+
+
+def test_packed_segments_equal_separate_sequences():
+    """Causal attention over packed segments (starts = each row's segment
+    start) equals causal attention over each segment on its own: outputs,
+    LSE, all three gradients, and a sink gradient that is the sum over the
+    segments."""
+    rng = np.random.default_rng(302)
+    B, Hq, Hkv, T, d, dv = 2, 4, 2, 41, 6, 5
+    bounds = [[0, 13, 29, 41], [0, 41]]
+    starts = np.zeros((B, T), dtype=np.int32)
+    for b, bd in enumerate(bounds):
+        for s0, s1 in zip(bd[:-1], bd[1:]):
+            starts[b, s0:s1] = s0
+    q, k, v = _rand(rng, B, Hq, T, d), _rand(rng, B, Hkv, T, d), _rand(rng, B, Hkv, T, dv)
+    g = _rand(rng, B, Hq, T, dv)
+    sink = _rand(rng, Hq)
+    allow = A.allowed_dense(T, T, causal=True, starts=starts)
+    assert allow.shape == (B, 1, T, T)
+    fw = A.forward(q, k, v, allow, 0.3, sink=sink)
+    bw = A.backward(q, k, v, g, allow, 0.3, sink=sink)
+    dsink = np.zeros(Hq)
+    for b, bd in enumerate(bounds):
+        for s0, s1 in zip(bd[:-1], bd[1:]):
+            sl = slice(s0, s1)
+            one = A.allowed_dense(s1 - s0, s1 - s0, causal=True)
+            f1 = A.forward(q[b:b + 1, :, sl], k[b:b + 1, :, sl], v[b:b + 1, :, sl], one, 0.3, sink=sink)
+            b1 = A.backward(q[b:b + 1, :, sl], k[b:b + 1, :, sl], v[b:b + 1, :, sl], g[b:b + 1, :, sl], one,
+                            0.3, sink=sink)
+            np.testing.assert_allclose(fw.y[b:b + 1, :, sl], f1.y, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(fw.lse[b:b + 1, :, sl], f1.lse, rtol=0, atol=1e-13)
+            for name in ("dq", "dk", "dv"):
+                np.testing.assert_allclose(getattr(bw, name)[b:b + 1, :, sl], getattr(b1, name), rtol=0, atol=1e-12)
+            dsink += b1.dsink
+    np.testing.assert_allclose(bw.dsink, dsink, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_lengths_equal_truncated_sequences(causal):
+    """Active lengths: rows and keys past L_b take no part. The active block
+    equals the attention of the truncated sequence, padding rows are empty
+    (Y = 0, LSE = -inf) and padding K/V rows get zero gradients."""
+    rng = np.random.default_rng(303 + causal)
+    B, Hq, Hkv, T, d, dv = 3, 2, 1, 19, 4, 3
+    lengths = np.array([19, 7, 0], dtype=np.int32)
+    q, k, v = _rand(rng, B, Hq, T, d), _rand(rng, B, Hkv, T, d), _rand(rng, B, Hkv, T, dv)
+    g = _rand(rng, B, Hq, T, dv)
+    allow = A.allowed_dense(T, T, causal=causal, lengths=lengths)
+    fw = A.forward(q, k, v, allow, 0.5)
+    bw = A.backward(q, k, v, g, allow, 0.5)
+    for b, L in enumerate(lengths):
+        assert np.all(fw.y[b, :, L:] == 0) and np.all(fw.lse[b, :, L:] == -np.inf)
+        assert np.all(bw.dq[b, :, L:] == 0) and np.all(bw.dk[b, :, L:] == 0) and np.all(bw.dv[b, :, L:] == 0)
+        if L == 0:
+            continue
+        one = A.allowed_dense(L, L, causal=causal)
+        f1 = A.forward(q[b:b + 1, :, :L], k[b:b + 1, :, :L], v[b:b + 1, :, :L], one, 0.5)
+        b1 = A.backward(q[b:b + 1, :, :L], k[b:b + 1, :, :L], v[b:b + 1, :, :L], g[b:b + 1, :, :L], one, 0.5)
+        np.testing.assert_allclose(fw.y[b:b + 1, :, :L], f1.y, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(fw.lse[b:b + 1, :, :L], f1.lse, rtol=0, atol=1e-13)
+        for name in ("dq", "dk", "dv"):
+            np.testing.assert_allclose(getattr(bw, name)[b:b + 1, :, :L], getattr(b1, name), rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        A.allowed_dense(4, 6, lengths=np.array([3]))
