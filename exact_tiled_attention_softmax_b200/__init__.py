@@ -38,6 +38,8 @@ ATTN_MASK_CAUSAL = 0x1
 ATTN_MASK_WINDOW = 0x2
 ATTN_MASK_BLOCK = 0x4
 ATTN_MASK_TOPK = 0x8
+ATTN_MASK_LENGTHS = 0x10
+ATTN_MASK_STARTS = 0x20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -59,7 +61,8 @@ class AttnMaskC(ctypes.Structure):
                 ("topk_idxs", ctypes.c_void_p), ("topk_stride", ctypes.c_int64),
                 ("topk_max", ctypes.c_int32), ("topk_length", ctypes.c_void_p),
                 ("sink", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
-                ("dropout_seed", ctypes.c_uint64)]
+                ("dropout_seed", ctypes.c_uint64), ("lengths", ctypes.c_void_p),
+                ("starts", ctypes.c_void_p), ("starts_stride_b", ctypes.c_int64)]
 
 
 _LIB = None
@@ -139,7 +142,9 @@ class AllowedSet:
 
     block_mask: uint8 [nq_blocks, nk_blocks], or with leading [B, H] dims
     (size-1 dims broadcast). topk_idxs int32 [Tq, >= topk_max],
-    topk_length int32 [Tq], sink float32 [Hq].
+    topk_length int32 [Tq], sink float32 [Hq]. lengths int32 [B] (active
+    cells per batch row, Tq == Tk); starts int32 [B, Tq] or [Tq] (lowest
+    allowed key of each query row, e.g. its packed segment's first cell).
     """
     causal: bool = False
     window_left: int = 0
@@ -152,6 +157,8 @@ class AllowedSet:
     sink: torch.Tensor | None = None
     dropout_p: float = 0.0
     dropout_seed: int = 0
+    lengths: torch.Tensor | None = None
+    starts: torch.Tensor | None = None
 
     def to_c(self) -> AttnMaskC:
         m = AttnMaskC()
@@ -179,6 +186,16 @@ class AllowedSet:
             m.topk_stride = self.topk_idxs.stride(0)
             m.topk_max = int(self.topk_max if self.topk_max is not None else self.topk_idxs.shape[1])
             m.topk_length = self.topk_length.data_ptr() if self.topk_length is not None else 0
+        if self.lengths is not None:
+            flags |= ATTN_MASK_LENGTHS
+            m.lengths = self.lengths.data_ptr()
+        if self.starts is not None:
+            st = self.starts
+            if st.stride(-1) != 1:
+                raise ValueError("starts rows must be contiguous")
+            flags |= ATTN_MASK_STARTS
+            m.starts = st.data_ptr()
+            m.starts_stride_b = st.stride(0) if st.dim() == 2 and st.shape[0] > 1 else 0
         if self.sink is not None:
             m.sink = self.sink.data_ptr()
         m.dropout_p = float(self.dropout_p)

@@ -39,7 +39,8 @@ uint32_t flags_of(const attn_mask* m) { return m ? m->flags : 0u; }
 // Validate the mask descriptor itself (not the tensors).
 attn_status check_mask(const attn_mask* m) {
   if (!m) return ATTN_OK;
-  const uint32_t known = ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK | ATTN_MASK_TOPK;
+  const uint32_t known = ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK | ATTN_MASK_TOPK |
+                         ATTN_MASK_LENGTHS | ATTN_MASK_STARTS;
   if (m->flags & ~known) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_WINDOW) && m->window_left < 1) return ATTN_ERR_INVALID_ARG;
   if (m->flags & ATTN_MASK_BLOCK) {
@@ -48,9 +49,12 @@ attn_status check_mask(const attn_mask* m) {
   }
   if (m->flags & ATTN_MASK_TOPK) {
     if (!m->topk_idxs || m->topk_max < 0 || m->topk_stride < m->topk_max) return ATTN_ERR_INVALID_ARG;
-    if (m->flags & (ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK)) return ATTN_ERR_UNSUPPORTED;
+    if (m->flags & (ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK | ATTN_MASK_LENGTHS | ATTN_MASK_STARTS))
+      return ATTN_ERR_UNSUPPORTED;
     if (m->dropout_p != 0.f) return ATTN_ERR_UNSUPPORTED;
   }
+  if ((m->flags & ATTN_MASK_LENGTHS) && !m->lengths) return ATTN_ERR_INVALID_ARG;
+  if ((m->flags & ATTN_MASK_STARTS) && (!m->starts || m->starts_stride_b < 0)) return ATTN_ERR_INVALID_ARG;
   if (!(m->dropout_p >= 0.f && m->dropout_p < 1.f)) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
@@ -59,7 +63,10 @@ MaskP mask_params(const attn_mask* m) {
   MaskP p;
   memset(&p, 0, sizeof(p));
   if (!m) return p;
-  p.flags = m->flags & (ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK);
+  p.flags = m->flags & (ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK | ATTN_MASK_LENGTHS | ATTN_MASK_STARTS);
+  p.lengths = (m->flags & ATTN_MASK_LENGTHS) ? m->lengths : nullptr;
+  p.starts = (m->flags & ATTN_MASK_STARTS) ? m->starts : nullptr;
+  p.st_sb = m->starts_stride_b;
   p.window = m->window_left;
   p.bm = m->block_mask;
   p.bq = m->block_q;
@@ -276,6 +283,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
 
   Dense s;
   if ((st = check_dense(q, k, v, s)) != ATTN_OK) return st;
+  if ((flags_of(mask) & ATTN_MASK_LENGTHS) && s.Tq != s.Tk) return ATTN_ERR_INVALID_ARG;
   const int64_t os[4] = {s.B, s.Hq, s.Tq, s.dv}, ls[3] = {s.B, s.Hq, s.Tq};
   if (!same_shape(o, 4, os) || !same_shape(lse, 3, ls) || o->dtype != q->dtype || !inner_contiguous(o))
     return ATTN_ERR_INVALID_ARG;
@@ -408,6 +416,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
 
   Dense s;
   if ((st = check_dense(q, k, v, s)) != ATTN_OK) return st;
+  if ((flags_of(mask) & ATTN_MASK_LENGTHS) && s.Tq != s.Tk) return ATTN_ERR_INVALID_ARG;
   if (!dv) return ATTN_ERR_INVALID_ARG;
   const int64_t os[4] = {s.B, s.Hq, s.Tq, s.dv}, ls[3] = {s.B, s.Hq, s.Tq}, qs[4] = {s.B, s.Hq, s.Tq, s.d},
                 ks[4] = {s.B, s.Hkv, s.Tk, s.d}, vs[4] = {s.B, s.Hkv, s.Tk, s.dv};

@@ -28,7 +28,22 @@ struct MaskP {
   uint32_t keep_thr;  // keep iff philox word >= keep_thr
   float inv_keep;     // 1 / (1 - rho)
   uint32_t seed_lo, seed_hi;
+  const int32_t* lengths;  // [B] active cells per batch row, or null
+  const int32_t* starts;   // (b, i) at starts[b * st_sb + i]: lowest allowed key, or null
+  int64_t st_sb;
 };
+
+// Active length of batch row b, clamped to [0, n] (n when not set).
+__device__ __forceinline__ int64_t active_len(const MaskP& m, int b, int64_t n) {
+  if (!m.lengths) return n;
+  const int64_t L = m.lengths[b];
+  return L < 0 ? 0 : (L > n ? n : L);
+}
+
+// Lowest allowed key of query row i of batch row b (0 when not set).
+__device__ __forceinline__ int64_t row_start(const MaskP& m, int b, int64_t i) {
+  return m.starts ? (int64_t)m.starts[b * m.st_sb + i] : 0;
+}
 
 // Dense problem: all strides in elements for (b, h, t); innermost stride 1.
 struct DenseP {
@@ -69,11 +84,16 @@ __device__ __forceinline__ bool allowed(const MaskP& m, int b, int h, int64_t i,
     const uint8_t* row = m.bm + b * m.bm_sb + h * m.bm_sh + (i / m.bq) * m.bm_sq;
     if (!row[j / m.bk]) return false;
   }
+  if (m.lengths) {
+    const int64_t L = active_len(m, b, INT64_MAX);
+    if (i >= L || j >= L) return false;
+  }
+  if (m.starts && j < row_start(m, b, i)) return false;
   return true;
 }
 
 // Key range [lo, hi] that can hold allowed keys for query row i.
-__device__ __forceinline__ void key_range(const MaskP& m, int64_t i, int64_t n_k,
+__device__ __forceinline__ void key_range(const MaskP& m, int b, int64_t i, int64_t n_k,
                                           int64_t& lo, int64_t& hi) {
   const int64_t ip = i + m.qoff;
   lo = 0;
@@ -83,10 +103,19 @@ __device__ __forceinline__ void key_range(const MaskP& m, int64_t i, int64_t n_k
     int64_t w = ip - m.window + 1;
     lo = w > 0 ? w : 0;
   }
+  if (m.lengths) {
+    const int64_t L = active_len(m, b, n_k);
+    if (i >= L) hi = -1;
+    if (L - 1 < hi) hi = L - 1;
+  }
+  if (m.starts) {
+    const int64_t s = row_start(m, b, i);
+    if (s > lo) lo = s;
+  }
 }
 
 // Query range [lo, hi] that can hold key j in its allowed set.
-__device__ __forceinline__ void query_range(const MaskP& m, int64_t j, int64_t n_q,
+__device__ __forceinline__ void query_range(const MaskP& m, int b, int64_t j, int64_t n_q,
                                             int64_t& lo, int64_t& hi) {
   lo = 0;
   hi = n_q - 1;
@@ -94,6 +123,11 @@ __device__ __forceinline__ void query_range(const MaskP& m, int64_t j, int64_t n
   if (m.flags & ATTN_MASK_WINDOW) {
     int64_t w = j + m.window - 1 - m.qoff;
     hi = w < hi ? w : hi;
+  }
+  if (m.lengths) {  // Tq = Tk here
+    const int64_t L = active_len(m, b, n_q);
+    if (j >= L) hi = -1;
+    if (L - 1 < hi) hi = L - 1;
   }
 }
 

@@ -77,7 +77,7 @@ dense_fwd_rows(DenseP p, T* o, int64_t so0, int64_t so1, int64_t so2, float* lse
   for (int c = 0; c < NV; ++c) acc[c] = 0.f;
   float m = -INFINITY, l = 0.f;
   int64_t lo, hi;
-  key_range(p.m, i, p.Tk, lo, hi);
+  key_range(p.m, b, i, p.Tk, lo, hi);
   for (int64_t j = lo; j <= hi; ++j) {
     if (!allowed(p.m, b, h, i, j)) continue;  // empty keys leave the state untouched
     float kr[NQ];
@@ -192,7 +192,7 @@ dense_dq_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, const
   const float dl = delta[warp];
   if (L != -INFINITY) {
     int64_t lo, hi;
-    key_range(p.m, i, p.Tk, lo, hi);
+    key_range(p.m, b, i, p.Tk, lo, hi);
     for (int64_t j = lo; j <= hi; ++j) {
       if (!allowed(p.m, b, h, i, j)) continue;
       float kr[NQ], vr[NV];
@@ -237,7 +237,7 @@ dense_dkv_rows(DenseP p, const T* g, int64_t sg0, int64_t sg1, int64_t sg2, cons
 #pragma unroll
   for (int c = 0; c < NV; ++c) av[c] = 0.f;
   int64_t lo, hi;
-  query_range(p.m, j, p.Tq, lo, hi);
+  query_range(p.m, b, j, p.Tq, lo, hi);
   for (int hh = 0; hh < group; ++hh) {
     const int h = kvh * group + hh;
     const T* Qb = static_cast<const T*>(p.q) + b * p.sq[0] + h * p.sq[1];

@@ -101,6 +101,41 @@ __device__ uint8_t tile_class(const MaskP& m, int Tq, int Tk, int b, int h, int 
   return any ? (all ? kFull : kPartial) : kEmpty;
 }
 
+// tile_class refined by the active lengths and per-row starts. Exact for
+// emptiness by length and for "every row's lowest key lies past the tile";
+// otherwise conservative (a tile may be marked partial and then masked row
+// by row). Only the class-table kernel evaluates it: a table always exists
+// when either is set.
+__device__ uint8_t tile_class_rows(const MaskP& m, int Tq, int Tk, int b, int h, int qs, int kt) {
+  const uint8_t base = tile_class(m, Tq, Tk, b, h, qs, kt);
+  if (base == kEmpty || !(m.lengths || m.starts)) return base;
+  bool all = base == kFull;
+  int64_t r0 = (int64_t)qs * kBMb, ra = (r0 + kBMb < Tq ? r0 + kBMb : Tq) - 1;
+  const int64_t c0 = (int64_t)kt * kBN, c1e = c0 + kBN - 1;
+  int64_t ca = c1e < Tk ? c1e : Tk - 1;
+  if (m.lengths) {
+    const int64_t L = active_len(m, b, Tk);
+    if (r0 >= L || c0 >= L) return kEmpty;
+    if (ra >= L) {
+      ra = L - 1;
+      all = false;
+    }
+    if (c1e >= L) all = false;
+    if (ca >= L) ca = L - 1;
+  }
+  if (m.starts) {
+    int64_t smin = INT64_MAX, smax = INT64_MIN;
+    for (int64_t r = r0; r <= ra; ++r) {
+      const int64_t s0 = row_start(m, b, r);
+      smin = s0 < smin ? s0 : smin;
+      smax = s0 > smax ? s0 : smax;
+    }
+    if (smin > ca) return kEmpty;
+    if (smax > c0) all = false;
+  }
+  return all ? kFull : kPartial;
+}
+
 struct ClassTable {
   const uint8_t* cls;  // null: compute analytically
   int nb, nh;          // slices along batch and head (1 = broadcast)
@@ -122,7 +157,7 @@ __global__ void classify_kernel(MaskP m, int Tq, int Tk, int B, int Hq, ClassTab
     const int qs = (int)((e / ct.nkt) % ct.nqs);
     const int sh = (int)((e / ((int64_t)ct.nkt * ct.nqs)) % ct.nh);
     const int sb = (int)(e / ((int64_t)ct.nkt * ct.nqs * ct.nh));
-    out[e] = tile_class(m, Tq, Tk, sb, sh, qs, kt);
+    out[e] = tile_class_rows(m, Tq, Tk, sb, sh, qs, kt);
   }
   (void)B;
   (void)Hq;
@@ -176,7 +211,7 @@ struct FwdCtl {
 };
 
 // Key-tile range that can hold allowed keys for rows [q0, q0 + rows).
-__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int Tq, int Tk, int q0, int rows, int& lo,
+__device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int b, int Tq, int Tk, int q0, int rows, int& lo,
                                               int& hi) {
   const int nkt = (Tk + kBN - 1) / kBN;
   lo = 0;
@@ -191,6 +226,13 @@ __device__ __forceinline__ void fwd_key_tiles(const MaskP& m, int Tq, int Tk, in
   if (m.flags & ATTN_MASK_WINDOW) {
     const int64_t first = (int64_t)q0 + m.qoff - m.window + 1;
     lo = first > 0 ? (int)(first / kBN) : 0;
+  }
+  if (m.lengths) {  // Tq = Tk here
+    const int64_t L = active_len(m, b, Tk);
+    if (q0 >= L)
+      hi = -1;
+    else if ((L - 1) / kBN < hi)
+      hi = (int)((L - 1) / kBN);
   }
 }
 
@@ -222,6 +264,29 @@ __device__ __forceinline__ uint64_t range_bits64(int64_t lo, int64_t hi) {
   return upto & ~((1ull << lo) - 1ull);
 }
 
+// Row i's key interval [lo, hi] narrowed by the active length and the row's
+// start (lo > hi when nothing is left). Kept out of line, with the few
+// fields it reads passed by value: the hot loops that mask partial tiles
+// stay as they are when neither is set.
+struct KeyInterval {
+  int64_t lo, hi;
+};
+
+__device__ __noinline__ KeyInterval clip_row_keys(const int32_t* lengths, const int32_t* starts, int64_t st_sb, int b,
+                                                  int64_t i, int64_t Tk, int64_t lo, int64_t hi) {
+  if (lengths) {
+    int64_t L = lengths[b];
+    L = L < 0 ? 0 : (L > Tk ? Tk : L);
+    if (i >= L) hi = -1;
+    hi = L - 1 < hi ? L - 1 : hi;
+  }
+  if (starts) {
+    const int64_t s0 = starts[b * st_sb + i];
+    lo = s0 > lo ? s0 : lo;
+  }
+  return KeyInterval{lo, hi};
+}
+
 // Allowed keys of row i inside key tile [j0, j0 + 128) as two 64-bit words
 // (bit c <-> key j0 + c). The causal/window conditions give one interval;
 // a block mask that is constant over (64-row slice, 128-key tile) blocks is
@@ -235,6 +300,11 @@ __device__ __forceinline__ void fwd_row_bits(const FwdArgs& a, int b, int h, int
   if (hi > a.Tk - 1) hi = a.Tk - 1;
   if (a.m.flags & ATTN_MASK_CAUSAL) hi = ip < hi ? ip : hi;
   if (a.m.flags & ATTN_MASK_WINDOW) lo = ip - a.m.window + 1 > lo ? ip - a.m.window + 1 : lo;
+  if (a.m.flags & (ATTN_MASK_LENGTHS | ATTN_MASK_STARTS)) {
+    const KeyInterval iv = clip_row_keys(a.m.lengths, a.m.starts, a.m.st_sb, b, i, a.Tk, lo, hi);
+    lo = iv.lo;
+    hi = iv.hi;
+  }
   if (lo > hi) return;
   w0 = range_bits64(lo - j0, hi - j0);
   w1 = range_bits64(lo - j0 - 64, hi - j0 - 64);
@@ -424,7 +494,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int q0 = ct * kFwdRows;
   const int qt0 = 2 * ct;
   int kt_lo, kt_hi;
-  fwd_key_tiles(a.m, a.Tq, a.Tk, q0, kFwdRows, kt_lo, kt_hi);
+  fwd_key_tiles(a.m, b, a.Tq, a.Tk, q0, kFwdRows, kt_lo, kt_hi);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->q_full), 1);
@@ -729,7 +799,7 @@ struct BwdCtl {
 };
 
 // Query-slice range [lo, hi] that can hold rows seeing keys [k0, k0 + 128).
-__device__ __forceinline__ void bwd_query_slices(const MaskP& m, int Tq, int k0, int& lo, int& hi) {
+__device__ __forceinline__ void bwd_query_slices(const MaskP& m, int b, int Tq, int k0, int& lo, int& hi) {
   const int nqs = (Tq + kBMb - 1) / kBMb;
   lo = 0;
   hi = nqs - 1;
@@ -743,6 +813,13 @@ __device__ __forceinline__ void bwd_query_slices(const MaskP& m, int Tq, int k0,
       hi = -1;
     else if (last < Tq)
       hi = (int)(last / kBMb);
+  }
+  if (m.lengths) {  // Tq = Tk here
+    const int64_t L = active_len(m, b, Tq);
+    if (k0 >= L)
+      hi = -1;
+    else if ((L - 1) / kBMb < hi)
+      hi = (int)((L - 1) / kBMb);
   }
 }
 
@@ -760,6 +837,28 @@ __device__ __forceinline__ bool bwd_next_step(const BwdArgs& a, int b, int kvh, 
   }
 }
 
+// Rows i0..i0+63 that the active length and the per-row starts allow to see
+// key j (bit c <-> i0 + c). Out of line, like clip_row_keys.
+__device__ __noinline__ uint64_t col_rows_allowed(const int32_t* lengths, const int32_t* starts, int64_t st_sb, int b,
+                                                  int64_t i0, int64_t j, int64_t Tq) {
+  int64_t hi = i0 + kBMb - 1 < Tq - 1 ? i0 + kBMb - 1 : Tq - 1;
+  if (lengths) {
+    int64_t L = lengths[b];
+    L = L < 0 ? 0 : (L > Tq ? Tq : L);
+    if (j >= L) return 0ull;
+    hi = L - 1 < hi ? L - 1 : hi;
+  }
+  uint64_t w = range_bits64(0, hi - i0);
+  if (w && starts) {
+    uint64_t sb = 0;
+#pragma unroll 1
+    for (int c = 0; c < kBMb; ++c)
+      if (i0 + c <= hi && starts[b * st_sb + i0 + c] <= j) sb |= 1ull << c;
+    w &= sb;
+  }
+  return w;
+}
+
 // Allowed query rows i0..i0+63 for key j, as a 64-bit word (bit c <-> i0 + c).
 __device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h, int64_t i0, int64_t j) {
   if (j >= a.Tk) return 0ull;
@@ -769,6 +868,7 @@ __device__ __forceinline__ uint64_t bwd_col_bits(const BwdArgs& a, int b, int h,
   if (a.m.flags & ATTN_MASK_WINDOW)
     hi = j + a.m.window - 1 - a.m.qoff < hi ? j + a.m.window - 1 - a.m.qoff : hi;
   uint64_t w = range_bits64(lo - i0, hi - i0);
+  if (w && (a.m.flags & (ATTN_MASK_LENGTHS | ATTN_MASK_STARTS))) w &= col_rows_allowed(a.m.lengths, a.m.starts, a.m.st_sb, b, i0, j, a.Tq);
   if (w && (a.m.flags & ATTN_MASK_BLOCK) && !a.block_aligned) {
     const uint8_t* base = a.m.bm + b * a.m.bm_sb + h * a.m.bm_sh + j / a.m.bk;
     uint64_t bb = 0;
@@ -848,7 +948,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   const int kvh = bkv % a.Hkv, b = bkv / a.Hkv;
   const int k0 = kt * kBN;
   int qs_lo, qs_hi;
-  bwd_query_slices(a.m, a.Tq, k0, qs_lo, qs_hi);
+  bwd_query_slices(a.m, b, a.Tq, k0, qs_lo, qs_hi);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->kv_full), 1);
@@ -1319,9 +1419,20 @@ cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
   return e;
 }
 
+constexpr uint32_t kTableFlags = ATTN_MASK_BLOCK | ATTN_MASK_LENGTHS | ATTN_MASK_STARTS;
+
+// A class table is kept per batch row when the block mask, the lengths or the
+// starts differ between batch rows, per head when the block mask does.
+int table_batches(uint32_t flags, int B, int64_t bm_sb, int64_t st_sb) {
+  const bool per_b = ((flags & ATTN_MASK_BLOCK) && bm_sb) || (flags & ATTN_MASK_LENGTHS) ||
+                     ((flags & ATTN_MASK_STARTS) && st_sb);
+  return per_b ? B : 1;
+}
+
 size_t class_bytes(int B, int Hq, int Tq, int Tk, const attn_mask* m) {
-  if (!m || !(m->flags & ATTN_MASK_BLOCK)) return 0;
-  const int nb = m->bm_stride_b ? B : 1, nh = m->bm_stride_h ? Hq : 1;
+  if (!m || !(m->flags & kTableFlags)) return 0;
+  const int nb = table_batches(m->flags, B, m->bm_stride_b, m->starts_stride_b);
+  const int nh = (m->flags & ATTN_MASK_BLOCK) && m->bm_stride_h ? Hq : 1;
   const size_t nqs = (Tq + kBMb - 1) / kBMb, nkt = (Tk + kBN - 1) / kBN;
   return align_up((size_t)nb * nh * nqs * nkt, 256);
 }
@@ -1329,12 +1440,12 @@ size_t class_bytes(int B, int Hq, int Tq, int Tk, const attn_mask* m) {
 ClassTable build_class_table(const DenseP& p, void* ws, cudaStream_t st, cudaError_t& err) {
   ClassTable ct;
   ct.cls = nullptr;
-  ct.nb = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sb ? p.B : 1;
+  ct.nb = table_batches(p.m.flags, p.B, p.m.bm_sb, p.m.st_sb);
   ct.nh = (p.m.flags & ATTN_MASK_BLOCK) && p.m.bm_sh ? p.Hq : 1;
   ct.nqs = (p.Tq + kBMb - 1) / kBMb;
   ct.nkt = (p.Tk + kBN - 1) / kBN;
   err = cudaSuccess;
-  if (!(p.m.flags & ATTN_MASK_BLOCK)) return ct;
+  if (!(p.m.flags & kTableFlags)) return ct;
   uint8_t* out = static_cast<uint8_t*>(ws);
   const int64_t n = (int64_t)ct.nb * ct.nh * ct.nqs * ct.nkt;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 102 /* major * 100 + minor */
+#define ATTN_VERSION 103 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -89,6 +89,8 @@ typedef struct attn_tensor {
 #define ATTN_MASK_WINDOW 0x2u /* j >  p(i) - window_left */
 #define ATTN_MASK_BLOCK 0x4u  /* block_mask[i / block_q][j / block_k] != 0 */
 #define ATTN_MASK_TOPK 0x8u   /* j listed in topk_idxs[t][0 : topk_length[t]] */
+#define ATTN_MASK_LENGTHS 0x10u /* i < lengths[b] and j < lengths[b] (needs Tq = Tk) */
+#define ATTN_MASK_STARTS 0x20u  /* j >= starts[b][i] */
 
 /* The allowed-set descriptor ("Tiled attention and its recomputed reverse
  * pass are exact": the fixed allowed sets A_i; causal, windowed and packed
@@ -121,6 +123,20 @@ typedef struct attn_mask {
    * stored. */
   float dropout_p;
   uint64_t dropout_seed;
+  /* Row-interval layouts ("Accumulate attention without keeping the full
+   * grid", section "Change attention evaluation inside the existing model":
+   * active lengths and packed-segment boundaries), dense calls only.
+   * ATTN_MASK_LENGTHS: int32 [B]; batch row b has lengths[b] active cells
+   * (values are clamped to [0, T]); query rows and keys past it belong to no
+   * set, so padding rows get the empty-set result. Requires Tq = Tk.
+   * ATTN_MASK_STARTS: int32, element (b, i) at starts[b*starts_stride_b + i]
+   * for query row i in [0, Tq) (a zero stride broadcasts over the batch);
+   * key j is allowed for that row only if j >= the element. With
+   * ATTN_MASK_CAUSAL and starts = each row's segment start this is causal
+   * attention inside packed segments. */
+  const int32_t* lengths;
+  const int32_t* starts;
+  int64_t starts_stride_b;
 } attn_mask;
 
 /* Layouts

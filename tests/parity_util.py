@@ -29,7 +29,8 @@ def rel_fro(a: np.ndarray, b: np.ndarray) -> float:
     return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
 
 
-def check_close(name: str, got: np.ndarray, want: np.ndarray, *, fp32: bool, grad: bool):
+def check_close(name: str, got: np.ndarray, want: np.ndarray, *, fp32: bool, grad: bool,
+                row_scale: bool = False):
     if fp32:
         err = float(np.abs(got - want).max()) if got.size else 0.0
         assert err <= FP32_ABS, f"{name}: max abs {err:.3e} > {FP32_ABS}"
@@ -37,6 +38,13 @@ def check_close(name: str, got: np.ndarray, want: np.ndarray, *, fp32: bool, gra
         err = rel_fro(got, want)
         assert err <= BF16_GRAD_REL, f"{name}: rel Frobenius {err:.3e} > {BF16_GRAD_REL}"
     else:
-        err = float(np.abs(got - want).max()) if got.size else 0.0
+        diff = np.abs(got - want)
+        if row_scale and got.size:
+            # Rows with a handful of allowed keys have |O| up to the largest
+            # |V| entry (about 3-4 for unit normals at d = 128); the bf16
+            # rounding of O (half an ulp, 2^-9 relative) and of the P operand
+            # both scale with it.
+            diff = diff / np.maximum(1.0, np.abs(want).max(axis=-1, keepdims=True))
+        err = float(diff.max()) if got.size else 0.0
         assert err <= BF16_O_ABS, f"{name}: max abs {err:.3e} > {BF16_O_ABS}"
     return err

@@ -140,3 +140,31 @@ def test_workspace_sizes_cover_scratch(lib):
     qt, kv, vt = _t([16, 4, 64]), _t([32, 64]), _t([32, 48], stride=[64, 1])
     bt = lib.attn_bwd_workspace_size(ctypes.byref(qt), ctypes.byref(kv), ctypes.byref(vt), ctypes.byref(m))
     assert bt >= 256 + 16 * 4 * 4 + 32 * 64 * 8
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of attn_tensor and attn_mask have the C layout:
+    a host C program built against the header prints each field's offset."""
+    import shutil
+    import subprocess
+    import exact_tiled_attention_softmax_b200 as eta
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    structs = {"attn_tensor": eta.AttnTensorC, "attn_mask": eta.AttnMaskC}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "attn.h"', "int main(void) {"]
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(line.split()[:2]): int(line.split()[2]) for line in out if line}
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)

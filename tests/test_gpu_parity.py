@@ -77,9 +77,9 @@ def _run_oracle(c):
     return fw, bw
 
 
-def _compare(c, gpu, fw, bw):
+def _compare(c, gpu, fw, bw, row_scale=False):
     fp32 = c["dtype"] == "f32"
-    check_close("O", to_np(gpu["o"]), fw.y, fp32=fp32, grad=False)
+    check_close("O", to_np(gpu["o"]), fw.y, fp32=fp32, grad=False, row_scale=row_scale)
     lse_g, lse_o = to_np(gpu["lse"]), fw.lse
     fin = np.isfinite(lse_o)
     assert np.array_equal(np.isfinite(lse_g), fin)
@@ -288,3 +288,88 @@ def test_query_block_against_longer_or_shorter_keys(kind, dtype):
     fw = oracle.forward(q, k, v, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"])
     bw = oracle.backward(q, k, v, g, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"], y=fw.y)
     _compare(c, gpu, fw, bw)
+
+
+def _segment_starts(bounds_per_batch, T):
+    st = np.zeros((len(bounds_per_batch), T), dtype=np.int32)
+    for b, bd in enumerate(bounds_per_batch):
+        for s0, s1 in zip(bd[:-1], bd[1:]):
+            st[b, s0:s1] = s0
+    return st
+
+
+def _run_layout_case(c, lengths=None, starts=None):
+    tdt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float32
+    q, k, v, g = (to_dev(c[n], tdt) for n in ("q", "k", "v", "g"))
+    allowed = eta.AllowedSet(
+        causal=c["causal"], window_left=c["window"],
+        block_mask=to_dev(c["bm"], torch.uint8) if c["bm"] is not None else None,
+        block_q=c["block"] or 128, block_k=c["block"] or 128,
+        sink=to_dev(c["sink"], torch.float32) if c["sink"] is not None else None,
+        dropout_p=c["dropout"], dropout_seed=c["seed"],
+        lengths=to_dev(lengths, torch.int32) if lengths is not None else None,
+        starts=to_dev(starts, torch.int32) if starts is not None else None)
+    wf = torch.empty(eta.attn_fwd_workspace_size(q, k, v, allowed), dtype=torch.uint8, device="cuda")
+    wb = torch.empty(eta.attn_bwd_workspace_size(q, k, v, allowed), dtype=torch.uint8, device="cuda")
+    o, lse = eta.attn_fwd(q, k, v, allowed, c["scale"], workspace=wf)
+    assert eta.attn_get_status(wf) == 0
+    dq, dk, dv, dsink = eta.attn_bwd(q, k, v, o, g, lse, allowed, c["scale"], workspace=wb)
+    assert eta.attn_get_status(wb) == 0
+    torch.cuda.synchronize()
+    gpu = dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv, dsink=dsink)
+    B, Hq, Tq = c["q"].shape[:3]
+    Tk = c["k"].shape[2]
+    allow = oracle.allowed_dense(Tq, Tk, causal=c["causal"], window_left=c["window"], block_mask=c["bm"],
+                                 block_q=c["block"] or 1, block_k=c["block"] or 1, query_offset=Tk - Tq,
+                                 lengths=lengths, starts=starts)
+    keep = P.dropout_keep(c["seed"], c["dropout"], B, Hq, Tq, Tk) if c["dropout"] else None
+    qq, kk, vv, gg = (c[n].astype(np.float64) for n in ("q", "k", "v", "g"))
+    sink = c["sink"].astype(np.float64) if c["sink"] is not None else None
+    fw = oracle.forward(qq, kk, vv, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"])
+    bw = oracle.backward(qq, kk, vv, gg, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"], y=fw.y)
+    _compare(c, gpu, fw, bw, row_scale=True)
+    return gpu
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_packed_segments(dtype):
+    """Causal attention inside packed segments (starts = the segment's first
+    cell), with GQA and a sink; boundaries fall inside and on tile edges."""
+    T = 600
+    c = _qk_case(2, 4, 2, T, T, 128, 128, dtype, 31, sink=True)
+    st = _segment_starts([[0, 70, 200, 256, 431, 600], [0, 128, 600]], T)
+    _run_layout_case(c, starts=st)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_active_lengths(dtype, causal):
+    """Active lengths per batch row (a full row, one ending inside a 64-row
+    slice and a 128-key tile, one empty) with dropout: padding rows are
+    empty, padding keys take no part."""
+    T = 300
+    c = _qk_case(3, 4, 2, T, T, 128, 128, dtype, 32, causal=causal, dropout=0.1)
+    gpu = _run_layout_case(c, lengths=np.array([300, 131, 0], dtype=np.int32))
+    o = to_np(gpu["o"])
+    assert np.all(o[1, :, 131:] == 0) and np.all(o[2] == 0)
+    assert np.all(to_np(gpu["dk"])[1, :, 131:] == 0) and np.all(to_np(gpu["dv"])[2] == 0)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_starts_with_window_block_and_longer_keys(dtype):
+    """Per-row lower bounds of arbitrary shape (not segments) together with a
+    window, a block mask and Tq < Tk."""
+    Tq, Tk = 200, 420
+    c = _qk_case(2, 2, 2, Tq, Tk, 128, 128, dtype, 33, window=300, block=64)
+    rng = np.random.default_rng(34)
+    pos = np.arange(Tq) + Tk - Tq
+    st = (pos[None, :] - rng.integers(0, 260, size=(2, Tq))).clip(0).astype(np.int32)
+    _run_layout_case(c, starts=st)
+
+
+def test_lengths_need_equal_query_and_key_counts():
+    q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 1, 16, 128, dtype=torch.bfloat16, device="cuda")
+    al = eta.AllowedSet(causal=True, lengths=torch.tensor([8], dtype=torch.int32, device="cuda"))
+    with pytest.raises(eta.AttnError):
+        eta.attn_fwd(q, k, k, al)
