@@ -11,13 +11,15 @@ Modules
 -------
 attention  dense masked attention, its analytic VJP, the shared-KV top-k
            variant, the running-summary recurrence with trace cards, and the
-           block-summary merge.
+           block-summary merge, and the LSE conventions (sink-inclusive,
+           KV-only with its logaddexp combination, base-2 scaled form).
 philox     Philox4x32-10 (Salmon et al., SC'11) and the dropout keep-mask
            convention built on it.
 """
 from .attention import (  # noqa: F401
     BackwardResult, ForwardResult, TileCard, allowed_dense, backward,
-    block_summary, forward, merge_summaries, tiled_forward, topk_allowed,
-    topk_backward, topk_dsink, topk_forward,
+    block_summary, combine_lse, forward, kv_only_lse, merge_summaries,
+    scaled_lse, tiled_forward, topk_allowed, topk_backward, topk_dsink,
+    topk_forward, topk_kv_only_lse,
 )
 from .philox import dropout_keep, keep_threshold, philox4x32  # noqa: F401

@@ -419,3 +419,55 @@ def merge_summaries(a, b):
     m = max(a[0], b[0])
     ea, eb = np.exp(a[0] - m), np.exp(b[0] - m)
     return m, ea * a[1] + eb * b[1], ea * np.asarray(a[2]) + eb * np.asarray(b[2])
+
+
+# ---------------------------------------------------------------------------
+# LSE conventions (DSA note, sections 7.1-7.3)
+# ---------------------------------------------------------------------------
+
+def _log_sum_exp_allowed(s: np.ndarray, allow: np.ndarray) -> np.ndarray:
+    """ln sum_{j allowed} exp(s_j) along the last axis; -inf for an empty row."""
+    sm = np.where(allow, s, NEG_INF)
+    m = sm.max(axis=-1, initial=NEG_INF)
+    shift = np.where(np.isfinite(m), m, 0.0)
+    tot = np.where(allow, np.exp(sm - shift[..., None]), 0.0).sum(axis=-1)
+    with np.errstate(divide="ignore"):
+        return np.where(tot > 0, shift + np.log(np.where(tot > 0, tot, 1.0)), NEG_INF)
+
+
+def kv_only_lse(q, k, allowed, scale: float) -> np.ndarray:
+    """LSE_kv = ln sum_{j in A_i} exp(s_ij), the sink left out (DSA note,
+    section 7.2). q [B,Hq,Tq,d], k [B,Hkv,Tk,d]; returns [B,Hq,Tq]."""
+    q, k = np.asarray(q, dtype=np.float64), np.asarray(k, dtype=np.float64)
+    B, Hq, Tq, _ = q.shape
+    Hkv, Tk = k.shape[1], k.shape[2]
+    allow = _bcast_allowed(allowed, B, Hq, Tq, Tk)
+    out = np.empty((B, Hq, Tq))
+    for b in range(B):
+        for h in range(Hq):
+            out[b, h] = _log_sum_exp_allowed(scale * (q[b, h] @ k[b, h // (Hq // Hkv)].T), allow[b, h])
+    return out
+
+
+def topk_kv_only_lse(q, kv, idx, length, scale: float) -> np.ndarray:
+    """LSE_kv of the shared-KV top-k layout: [Tq, H], each listed position
+    counted once, -inf for an empty list."""
+    q, kv = np.asarray(q, dtype=np.float64), np.asarray(kv, dtype=np.float64)
+    out = np.empty(q.shape[:2])
+    for t in range(q.shape[0]):
+        sel = np.asarray(idx[t, :length[t]], dtype=np.int64)
+        s = scale * (q[t] @ kv[sel].T)
+        out[t] = _log_sum_exp_allowed(s, np.ones(s.shape, bool))
+    return out
+
+
+def combine_lse(lse_kv: np.ndarray, z) -> np.ndarray:
+    """LSE_total = logaddexp(LSE_kv, z), the first step of a backward pass
+    that was handed a KV-only LSE while a sink is enabled (section 7.2)."""
+    return np.logaddexp(np.asarray(lse_kv, dtype=np.float64), z)
+
+
+def scaled_lse(lse: np.ndarray) -> np.ndarray:
+    """The base-2 stored form of section 7.3: scaled_LSE = -log2 Z for
+    LSE = ln Z (an empty row, LSE = -inf, gives +inf)."""
+    return -np.asarray(lse, dtype=np.float64) / np.log(2.0)

@@ -585,3 +585,61 @@ def test_lengths_equal_truncated_sequences(causal):
             np.testing.assert_allclose(getattr(bw, name)[b:b + 1, :, :L], getattr(b1, name), rtol=0, atol=1e-12)
     with pytest.raises(ValueError):
         A.allowed_dense(4, 6, lengths=np.array([3]))
+
+
+# ---------------------------------------------------------------------------
+# LSE conventions: sink-inclusive, KV-only, base-2 scaled
+# ---------------------------------------------------------------------------
+
+def test_lse_conventions_on_the_sink_example():
+    """The DSA note's sink example has Z = exp(z) + p1 + p2 = 1 (scores
+    ln p1, ln p2): LSE_total = 0, LSE_kv = ln(p1 + p2) = ln(1 - p_sink),
+    their logaddexp with z gives back 0, and scaled_LSE = -log2 Z = 0."""
+    ex = _golden("worked_examples.json")["sink"]
+    p1, p2 = ex["p"]
+    z = math.log(ex["p_sink"])
+    q = np.array([[1.0]])[None, None]
+    k = np.array([[math.log(p1)], [math.log(p2)]])[None, None]
+    allow = np.ones((1, 2), bool)
+    lkv = A.kv_only_lse(q, k, allow, 1.0)[0, 0, 0]
+    assert math.isclose(lkv, math.log(p1 + p2), rel_tol=1e-14)
+    assert math.isclose(lkv, math.log(1.0 - ex["p_sink"]), rel_tol=1e-12)
+    assert abs(A.combine_lse(lkv, z)) < 1e-15
+    assert A.scaled_lse(0.0) == 0.0
+    assert math.isclose(A.scaled_lse(math.log(8.0)), -3.0, rel_tol=1e-15)
+    assert A.scaled_lse(-np.inf) == np.inf
+    kv = np.array([[0.0, math.log(p1)], [0.0, math.log(p2)]])
+    lt = A.topk_kv_only_lse(np.array([[[0.0, 1.0]]]), kv, np.array([[0, 1]]), np.array([2]), 1.0)
+    assert math.isclose(lt[0, 0], math.log(p1 + p2), rel_tol=1e-14)
+
+
+def test_kv_only_lse_combines_to_the_sink_inclusive_lse():
+    """logaddexp(LSE_kv, z) equals the forward's sink-inclusive LSE (two
+    separate evaluations); without a sink the two conventions coincide; an
+    empty allowed set gives LSE_kv = -inf and LSE_total = z."""
+    rng = np.random.default_rng(311)
+    B, Hq, Hkv, T, d = 2, 4, 2, 17, 6
+    q, k, v = rng.standard_normal((B, Hq, T, d)), rng.standard_normal((B, Hkv, T, d)), \
+        rng.standard_normal((B, Hkv, T, 3))
+    allow = A.allowed_dense(T, T, causal=True, window_left=5)
+    allow = allow & (rng.random((B, Hq, T, T)) < 0.7)
+    allow[0, 0, 3] = False                          # one empty row
+    sink = rng.standard_normal(Hq) * 2
+    lkv = A.kv_only_lse(q, k, allow, 0.7)
+    fw = A.forward(q, k, v, allow, 0.7, sink=sink)
+    np.testing.assert_allclose(A.combine_lse(lkv, sink[None, :, None]), fw.lse, rtol=0, atol=1e-13)
+    assert lkv[0, 0, 3] == -np.inf and fw.lse[0, 0, 3] == sink[0]
+    fw0 = A.forward(q, k, v, allow, 0.7)
+    np.testing.assert_array_equal(np.isfinite(lkv), np.isfinite(fw0.lse))
+    fin = np.isfinite(lkv)
+    np.testing.assert_allclose(lkv[fin], fw0.lse[fin], rtol=0, atol=1e-13)
+    # Top-k layout: the same identity token by token.
+    Tkv, H = 40, 3
+    qt, kvt = rng.standard_normal((5, H, d)), rng.standard_normal((Tkv, d))
+    idx = np.stack([rng.permutation(Tkv)[:8] for _ in range(5)]).astype(np.int32)
+    ln = np.array([8, 3, 0, 5, 1], np.int32)
+    zt = rng.standard_normal(H)
+    lt = A.topk_kv_only_lse(qt, kvt, idx, ln, 0.5)
+    _, lse_t, _ = A.topk_forward(qt, kvt, idx, ln, 2, 0.5, zt)
+    np.testing.assert_allclose(A.combine_lse(lt, zt[None, :]), lse_t, rtol=0, atol=1e-13)
+    assert np.all(lt[2] == -np.inf)
