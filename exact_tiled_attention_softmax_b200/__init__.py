@@ -40,6 +40,8 @@ ATTN_MASK_BLOCK = 0x4
 ATTN_MASK_TOPK = 0x8
 ATTN_MASK_LENGTHS = 0x10
 ATTN_MASK_STARTS = 0x20
+ATTN_LSE_KV_ONLY = 0x1
+ATTN_LSE_NEG_LOG2 = 0x2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -62,7 +64,8 @@ class AttnMaskC(ctypes.Structure):
                 ("topk_max", ctypes.c_int32), ("topk_length", ctypes.c_void_p),
                 ("sink", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
                 ("dropout_seed", ctypes.c_uint64), ("lengths", ctypes.c_void_p),
-                ("starts", ctypes.c_void_p), ("starts_stride_b", ctypes.c_int64)]
+                ("starts", ctypes.c_void_p), ("starts_stride_b", ctypes.c_int64),
+                ("lse_format", ctypes.c_uint32)]
 
 
 _LIB = None
@@ -145,6 +148,8 @@ class AllowedSet:
     topk_length int32 [Tq], sink float32 [Hq]. lengths int32 [B] (active
     cells per batch row, Tq == Tk); starts int32 [B, Tq] or [Tq] (lowest
     allowed key of each query row, e.g. its packed segment's first cell).
+    lse_kv_only / lse_neg_log2 select the LSE format that attn_fwd writes
+    and attn_bwd expects: the sink left out, and/or stored as -log2 Z.
     """
     causal: bool = False
     window_left: int = 0
@@ -159,6 +164,8 @@ class AllowedSet:
     dropout_seed: int = 0
     lengths: torch.Tensor | None = None
     starts: torch.Tensor | None = None
+    lse_kv_only: bool = False
+    lse_neg_log2: bool = False
 
     def to_c(self) -> AttnMaskC:
         m = AttnMaskC()
@@ -198,6 +205,8 @@ class AllowedSet:
             m.starts_stride_b = st.stride(0) if st.dim() == 2 and st.shape[0] > 1 else 0
         if self.sink is not None:
             m.sink = self.sink.data_ptr()
+        m.lse_format = (ATTN_LSE_KV_ONLY if self.lse_kv_only else 0) | \
+            (ATTN_LSE_NEG_LOG2 if self.lse_neg_log2 else 0)
         m.dropout_p = float(self.dropout_p)
         m.dropout_seed = int(self.dropout_seed) & 0xFFFFFFFFFFFFFFFF
         m.flags = flags

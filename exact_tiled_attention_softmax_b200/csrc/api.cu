@@ -53,6 +53,7 @@ attn_status check_mask(const attn_mask* m) {
       return ATTN_ERR_UNSUPPORTED;
     if (m->dropout_p != 0.f) return ATTN_ERR_UNSUPPORTED;
   }
+  if (m->lse_format & ~(ATTN_LSE_KV_ONLY | ATTN_LSE_NEG_LOG2)) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_LENGTHS) && !m->lengths) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_STARTS) && (!m->starts || m->starts_stride_b < 0)) return ATTN_ERR_INVALID_ARG;
   if (!(m->dropout_p >= 0.f && m->dropout_p < 1.f)) return ATTN_ERR_INVALID_ARG;
@@ -67,6 +68,7 @@ MaskP mask_params(const attn_mask* m) {
   p.lengths = (m->flags & ATTN_MASK_LENGTHS) ? m->lengths : nullptr;
   p.starts = (m->flags & ATTN_MASK_STARTS) ? m->starts : nullptr;
   p.st_sb = m->starts_stride_b;
+  p.lse_fmt = m->lse_format;
   p.window = m->window_left;
   p.bm = m->block_mask;
   p.bq = m->block_q;
@@ -149,13 +151,21 @@ size_t bwd_dense_bytes(const Dense& s) {
   return n;
 }
 
+uint32_t lse_format_of(const attn_mask* m) { return m ? m->lse_format : 0u; }
+
+// Room for the reverse pass's natural-log, sink-inclusive copy of an LSE
+// given in another format (rows = the LSE's element count).
+size_t lse_copy_bytes(const attn_mask* m, size_t rows) {
+  return lse_format_of(m) ? align_up(rows * sizeof(float), 256) : 0;
+}
+
 size_t bwd_topk_bytes(const Topk& s, const attn_tensor* q, const attn_mask* m) {
   size_t n = kStatusBytes;
   n += align_up((size_t)s.Tq * s.H * sizeof(float), 256);                       // delta
   n += align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);      // 32.32 dKV
   if (q->dtype == ATTN_BF16)                                                    // G, P rows (tensor-core path)
     n += align_up(attn::sm100_topk_bwd_scratch_bytes(s.Tq, s.H, s.Dqk, s.Dv, m->topk_max), 256);
-  return n;
+  return n + lse_copy_bytes(m, (size_t)s.Tq * s.H);
 }
 
 }  // namespace
@@ -225,7 +235,8 @@ size_t attn_bwd_workspace_size(const attn_tensor* q, const attn_tensor* k, const
   }
   Dense s;
   if (check_dense(q, k, v, s) != ATTN_OK) return kStatusBytes;
-  return bwd_dense_bytes(s) + sm100_bwd_extra_workspace_bytes(s.B, s.Hq, s.Hkv, s.Tq, s.Tk, mask);
+  return bwd_dense_bytes(s) + sm100_bwd_extra_workspace_bytes(s.B, s.Hq, s.Hkv, s.Tq, s.Tk, mask) +
+         lse_copy_bytes(mask, (size_t)s.B * s.Hq * s.Tq);
 }
 
 attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tensor* v,
@@ -267,6 +278,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.Dv = s.Dv;
     p.scale = scale;
     p.sink = mask->sink;
+    p.lse_fmt = mask->lse_format;
     if (sm100_topk_supported(p, q, k, o))
       return cuda_status(sm100_topk_fwd(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
                                         lse->stride[0], lse->stride[1], status, cs));
@@ -375,14 +387,27 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.Dv = s.Dv;
     p.scale = scale;
     p.sink = mask->sink;
+    p.lse_fmt = mask->lse_format;
     const int64_t so[3] = {0, o->stride[0], o->stride[1]}, sg[3] = {0, do_->stride[0], do_->stride[1]};
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
+    const float* lsep = static_cast<const float*>(lse->data);
+    int64_t lst = lse->stride[0], lsh = lse->stride[1];
+    if (p.lse_fmt) {  // the reverse kernels read the natural-log, sink-inclusive LSE
+      const size_t rows = (size_t)s.Tq * s.H;
+      float* conv = reinterpret_cast<float*>(ws + bwd_topk_bytes(s, q, mask) - lse_copy_bytes(mask, rows));
+      const int64_t st3[3] = {0, lse->stride[0], lse->stride[1]};
+      if ((e = launch_lse_to_total(lsep, 1, s.Tq, s.H, st3, 2, mask->sink, p.lse_fmt, conv, cs)) != cudaSuccess)
+        return cuda_status(e);
+      lsep = conv;
+      lst = s.H;
+      lsh = 1;
+    }
     if (q->dtype == ATTN_F32) {
       e = launch_rows_delta<float>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
       main_kernel_begin(cs);
       if (e == cudaSuccess)
         e = launch_topk_bwd_rows<float>(p, do_->data, do_->stride[0], do_->stride[1],
-                                        static_cast<const float*>(lse->data), lse->stride[0], lse->stride[1],
+                                        lsep, lst, lsh,
                                         delta, dq->data, dq->stride[0], dq->stride[1], acc, dk->data,
                                         dk->stride[0], status, cs);
       main_kernel_end(cs);
@@ -394,8 +419,8 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
       if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * (size_t)s.Tkv * s.Dqk, cs);
       if (e == cudaSuccess)
-        e = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], static_cast<const float*>(lse->data),
-                           lse->stride[0], lse->stride[1], delta, dq->data, dq->stride[0], dq->stride[1], acc,
+        e = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta, dq->data,
+                           dq->stride[0], dq->stride[1], acc,
                            scratch, status, cs);
       if (e == cudaSuccess) e = launch_fixed_to_out<__nv_bfloat16>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
     } else {
@@ -403,14 +428,12 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       main_kernel_begin(cs);
       if (e == cudaSuccess)
         e = launch_topk_bwd_rows<__nv_bfloat16>(p, do_->data, do_->stride[0], do_->stride[1],
-                                                static_cast<const float*>(lse->data), lse->stride[0],
-                                                lse->stride[1], delta, dq->data, dq->stride[0], dq->stride[1],
+                                                lsep, lst, lsh, delta, dq->data, dq->stride[0], dq->stride[1],
                                                 acc, dk->data, dk->stride[0], status, cs);
       main_kernel_end(cs);
     }
     if (e == cudaSuccess && want_dsink)
-      e = launch_dsink(mask->sink, static_cast<const float*>(lse->data), delta, s.Tq, s.H, 1, lse->stride[0],
-                       lse->stride[1], 0, false, dsink, cs);
+      e = launch_dsink(mask->sink, lsep, delta, s.Tq, s.H, 1, lst, lsh, 0, false, dsink, cs);
     return cuda_status(e);
   }
 
@@ -455,12 +478,21 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
   const int64_t so[3] = {o->stride[0], o->stride[1], o->stride[2]};
   const int64_t sg[3] = {do_->stride[0], do_->stride[1], do_->stride[2]};
-  const int64_t sl[3] = {lse->stride[0], lse->stride[1], lse->stride[2]};
+  int64_t sl[3] = {lse->stride[0], lse->stride[1], lse->stride[2]};
   const int64_t sdq[3] = {dq->stride[0], dq->stride[1], dq->stride[2]};
   const int64_t sdk[3] = {dk->stride[0], dk->stride[1], dk->stride[2]};
   const int64_t sdv[3] = {dv->stride[0], dv->stride[1], dv->stride[2]};
   const float* lsep = static_cast<const float*>(lse->data);
   cudaError_t e;
+  if (p.m.lse_fmt) {  // the reverse kernels read the natural-log, sink-inclusive LSE
+    float* conv = reinterpret_cast<float*>(ws + need - lse_copy_bytes(mask, rows));
+    if ((e = launch_lse_to_total(lsep, s.B, s.Hq, s.Tq, sl, 1, mask->sink, p.m.lse_fmt, conv, cs)) != cudaSuccess)
+      return cuda_status(e);
+    lsep = conv;
+    sl[0] = (int64_t)s.Hq * s.Tq;
+    sl[1] = s.Tq;
+    sl[2] = 1;
+  }
   if (sm100_dense_supported(p, q, k, v, o) && sm100_dense_bwd_supported(p, do_, dq, dk, dv)) {
     e = sm100_dense_bwd(p, o->data, so, do_->data, sg, lsep, sl, delta, dq_acc, dq->data, sdq, dk->data, sdk,
                         dv->data, sdv, extra, status, cs);

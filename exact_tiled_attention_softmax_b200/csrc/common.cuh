@@ -31,6 +31,7 @@ struct MaskP {
   const int32_t* lengths;  // [B] active cells per batch row, or null
   const int32_t* starts;   // (b, i) at starts[b * st_sb + i]: lowest allowed key, or null
   int64_t st_sb;
+  uint32_t lse_fmt;        // ATTN_LSE_* bits of the LSE output
 };
 
 // Active length of batch row b, clamped to [0, n] (n when not set).
@@ -68,7 +69,28 @@ struct TopkP {
   int Tq, Tkv, H, Dqk, Dv;
   float scale;
   const float* sink;
+  uint32_t lse_fmt;  // ATTN_LSE_* bits of the LSE output
 };
+
+// The LSE value to store for a row, from base-2 quantities: lse2_total =
+// log2 of the sink-inclusive denominator, (m2, l2) = running maximum and
+// shifted sum of the allowed scores alone. Default: natural log, sink
+// included; ATTN_LSE_KV_ONLY: the sink left out; ATTN_LSE_NEG_LOG2: stored
+// as -log2 of the chosen denominator.
+__device__ __forceinline__ float stored_lse_log2(uint32_t fmt, float lse2_total, float m2, float l2) {
+  constexpr float log2e = 1.4426950408889634f;
+  float v = lse2_total;
+  if (fmt & ATTN_LSE_KV_ONLY) v = m2 == -INFINITY ? -INFINITY : m2 + log2f(l2);
+  return (fmt & ATTN_LSE_NEG_LOG2) ? -v : v / log2e;
+}
+
+// The same from natural-log quantities (lse_total, running max m, sum l).
+__device__ __forceinline__ float stored_lse_ln(uint32_t fmt, float lse_total, float m, float l) {
+  constexpr float log2e = 1.4426950408889634f;
+  float v = lse_total;
+  if (fmt & ATTN_LSE_KV_ONLY) v = m == -INFINITY ? -INFINITY : m + logf(l);
+  return (fmt & ATTN_LSE_NEG_LOG2) ? -v * log2e : v;
+}
 
 __device__ __forceinline__ float ld(const float* p) { return *p; }
 __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }

@@ -31,6 +31,8 @@ cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, in
 template <typename T>
 cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int cols, void* out, int64_t so,
                                 cudaStream_t st);
+cudaError_t launch_lse_to_total(const float* in, int n0, int n1, int n2, const int64_t s[3], int head_dim,
+                                const float* sink, uint32_t fmt, float* out, cudaStream_t st);
 cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta, int n_outer, int n_heads,
                          int n_inner, int64_t sl_outer, int64_t sl_head, int64_t sl_inner,
                          bool delta_head_major, float* dsink, cudaStream_t st);

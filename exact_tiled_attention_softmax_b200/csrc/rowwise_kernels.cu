@@ -37,7 +37,7 @@ __device__ __forceinline__ float dot_lanes(const float (&a)[N], const float (&b)
 // Finalise a row: fold the sink into the summary and write Y, LSE.
 template <typename T, int NV>
 __device__ __forceinline__ void finish_row(float m, float l, float (&acc)[NV], float z, bool has_sink,
-                                           T* orow, int dv, int lane, float* lse_out) {
+                                           T* orow, int dv, int lane, float* lse_out, uint32_t lse_fmt) {
   float lse;
   float scale_o;
   if (m == -INFINITY) {  // A_i empty: Y = 0, LSE = -inf or z
@@ -54,7 +54,7 @@ __device__ __forceinline__ void finish_row(float m, float l, float (&acc)[NV], f
     const int idx = lane + 32 * c;
     if (idx < dv) st(orow + idx, acc[c] * scale_o);
   }
-  if (lane == 0) *lse_out = lse;
+  if (lane == 0) *lse_out = stored_lse_ln(lse_fmt, lse, m, l);
 }
 
 template <typename T, int NQ, int NV>
@@ -101,7 +101,7 @@ dense_fwd_rows(DenseP p, T* o, int64_t so0, int64_t so1, int64_t so2, float* lse
   const bool has_sink = p.m.sink != nullptr;
   const float z = has_sink ? p.m.sink[h] : -INFINITY;
   finish_row<T, NV>(m, l, acc, z, has_sink, o + b * so0 + h * so1 + (int64_t)i * so2, p.dv, lane,
-                    lse + b * sl0 + h * sl1 + (int64_t)i * sl2);
+                    lse + b * sl0 + h * sl1 + (int64_t)i * sl2, p.m.lse_fmt);
 }
 
 template <typename T, int NQ, int NV>
@@ -147,7 +147,7 @@ topk_fwd_rows(TopkP p, T* o, int64_t so_t, int64_t so_h, float* lse, int64_t sl_
   const bool has_sink = p.sink != nullptr;
   const float z = has_sink ? p.sink[h] : -INFINITY;
   finish_row<T, NV>(m, l, acc, z, has_sink, o + (int64_t)t * so_t + (int64_t)h * so_h, p.Dv, lane,
-                    lse + (int64_t)t * sl_t + (int64_t)h * sl_h);
+                    lse + (int64_t)t * sl_t + (int64_t)h * sl_h, p.lse_fmt);
 }
 
 // delta_i = <G_i, Y_i> from the stored output, one warp per row. Rows are
@@ -519,6 +519,41 @@ cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int col
                                 cudaStream_t st) {
   const int64_t n = (int64_t)rows * cols;
   if (n > 0) fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(acc, rows, cols, static_cast<T*>(out), so);
+  return cudaGetLastError();
+}
+
+// An LSE in the caller's format -> the natural-log, sink-inclusive LSE that
+// the reverse kernels read ("DeepSeek Sparse Attention Forward and
+// Backward", sections 7.2-7.3): undo the -log2 scaling, then fold the sink
+// logit in as logaddexp(LSE_kv, z). Element (i0, i1, i2) of an
+// [n0, n1, n2] view with the given strides goes to out[(i0 n1 + i1) n2 + i2];
+// the head index is i1 (head_dim 1) or i2 (head_dim 2).
+__global__ void __launch_bounds__(256)
+lse_to_total_kernel(const float* in, int n0, int n1, int n2, int64_t s0, int64_t s1, int64_t s2, int head_dim,
+                    const float* sink, uint32_t fmt, float* out) {
+  constexpr float ln2 = 0.6931471805599453f;
+  const int64_t n = (int64_t)n0 * n1 * n2;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i2 = (int)(e % n2);
+    const int i1 = (int)((e / n2) % n1);
+    const int64_t i0 = e / ((int64_t)n1 * n2);
+    float v = in[i0 * s0 + i1 * s1 + i2 * s2];
+    if (fmt & ATTN_LSE_NEG_LOG2) v = -v * ln2;
+    if ((fmt & ATTN_LSE_KV_ONLY) && sink) {
+      const float z = sink[head_dim == 1 ? i1 : i2];
+      const float M = fmaxf(v, z);
+      v = M == -INFINITY ? -INFINITY : M + logf(expf(v - M) + expf(z - M));
+    }
+    out[e] = v;
+  }
+}
+
+cudaError_t launch_lse_to_total(const float* in, int n0, int n1, int n2, const int64_t s[3], int head_dim,
+                                const float* sink, uint32_t fmt, float* out, cudaStream_t st) {
+  const int64_t n = (int64_t)n0 * n1 * n2;
+  if (n == 0) return cudaSuccess;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  lse_to_total_kernel<<<blocks, 256, 0, st>>>(in, n0, n1, n2, s[0], s[1], s[2], head_dim, sink, fmt, out);
   return cudaGetLastError();
 }
 

@@ -732,7 +732,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           }
         }
       }
-      if (row < a.Tq) a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = lse2 / kLog2e;
+      if (row < a.Tq) a.lse[b * a.sl[0] + h * a.sl[1] + row * a.sl[2]] = stored_lse_log2(a.m.lse_fmt, lse2, m_run, l_run);
     }
   }
   tc_fence_before();

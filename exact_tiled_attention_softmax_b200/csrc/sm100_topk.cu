@@ -72,6 +72,7 @@ struct TopkArgs {
   int64_t so_t, so_h;
   float* lse;
   int64_t sl_t, sl_h;
+  uint32_t lse_fmt;
   uint32_t* status;
 };
 
@@ -333,7 +334,7 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
           oscale = exp2f(m_run - M) / tot;
           lse2 = M + log2f(tot);
         }
-        a.lse[(int64_t)t * a.sl_t + (int64_t)h * a.sl_h] = lse2 / kLog2e;
+        a.lse[(int64_t)t * a.sl_t + (int64_t)h * a.sl_h] = stored_lse_log2(a.lse_fmt, lse2, m_run, l_run);
       }
       oscale = __shfl_sync(0xffffffffu, oscale, (lane + 16) & 31);  // lower lane l <- upper lane l + 16
       __nv_bfloat16* orow = a.o + (int64_t)t * a.so_t + (int64_t)h * a.so_h;
@@ -1040,6 +1041,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   a.lse = lse;
   a.sl_t = sl_t;
   a.sl_h = sl_h;
+  a.lse_fmt = p.lse_fmt;
   a.status = status;
   cudaError_t e = raise_smem(reinterpret_cast<const void*>(topk_fwd_kernel), kTSmem, 0);
   if (e != cudaSuccess) return e;

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 103 /* major * 100 + minor */
+#define ATTN_VERSION 104 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -137,7 +137,20 @@ typedef struct attn_mask {
   const int32_t* lengths;
   const int32_t* starts;
   int64_t starts_stride_b;
+  /* Format of the LSE that attn_fwd writes and attn_bwd reads ("DeepSeek
+   * Sparse Attention Forward and Backward", section 7): 0 = natural log of
+   * the sink-inclusive denominator Z (section 7.1), or a combination of the
+   * ATTN_LSE_* bits below. attn_bwd must be given the format attn_fwd wrote. */
+  uint32_t lse_format;
 } attn_mask;
+
+/* ATTN_LSE_KV_ONLY: the denominator leaves the sink out, ln sum_j exp(s_j)
+ * (section 7.2; -inf for an empty allowed set even with a sink). The reverse
+ * pass combines it with the sink logit as logaddexp(LSE_kv, z) before use.
+ * ATTN_LSE_NEG_LOG2: the stored value is -log2 of the denominator, the
+ * base-2 form of section 7.3 (+inf for an empty row without a sink). */
+#define ATTN_LSE_KV_ONLY 0x1u
+#define ATTN_LSE_NEG_LOG2 0x2u
 
 /* Layouts
  *   Dense:  q [B,Hq,Tq,d], k [B,Hkv,Tk,d], v [B,Hkv,Tk,dv], o [B,Hq,Tq,dv],

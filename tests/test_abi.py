@@ -70,7 +70,7 @@ def test_invalid_arguments_rejected_on_host(lib):
     o, lse = _t([1, 4, 64, 128]), _t([1, 4, 64], dtype=0)
     # Hq not a multiple of Hkv
     assert _call_fwd(lib, q, _t([1, 3, 64, 128]), _t([1, 3, 64, 128]), o, lse) == eta.ATTN_ERR_INVALID_ARG
-    # key length differs from query length
+    # K and V lengths differ
     assert _call_fwd(lib, q, _t([1, 2, 65, 128]), v, o, lse) == eta.ATTN_ERR_INVALID_ARG
     # inner stride not 1
     assert _call_fwd(lib, _t([1, 4, 64, 128], stride=[64 * 256, 64 * 256, 256, 2]), k, v, o,
@@ -91,6 +91,24 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
     # unknown flag bits
     m.flags = 0x100
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # unknown LSE format bits
+    m = eta.AttnMaskC()
+    m.lse_format = 0x4
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # active lengths: a pointer is required, and Tq must equal Tk
+    m = eta.AttnMaskC()
+    m.flags = eta.ATTN_MASK_LENGTHS
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    m.lengths = 0x4000
+    k2, v2 = _t([1, 2, 96, 128]), _t([1, 2, 96, 128])
+    assert _call_fwd(lib, q, k2, v2, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # per-row starts: a pointer is required and the batch stride may not be negative
+    m = eta.AttnMaskC()
+    m.flags = eta.ATTN_MASK_STARTS
+    assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    m.starts = 0x4000
+    m.starts_stride_b = -1
     assert _call_fwd(lib, q, k, v, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
     # workspace missing or too small
     assert _call_fwd(lib, q, k, v, o, lse, ws=0) == eta.ATTN_ERR_WORKSPACE
@@ -120,6 +138,12 @@ def test_topk_arguments_rejected_on_host(lib):
     m.flags = eta.ATTN_MASK_TOPK
     m.topk_stride = 4
     assert _call_fwd(lib, q, kv, v_ok, o, lse, mask=m) == eta.ATTN_ERR_INVALID_ARG
+    # row-interval layouts are dense-only
+    m.topk_stride = 8
+    m.flags = eta.ATTN_MASK_TOPK | eta.ATTN_MASK_STARTS
+    m.starts = 0x4000
+    assert _call_fwd(lib, q, kv, v_ok, o, lse, mask=m) == eta.ATTN_ERR_UNSUPPORTED
+    m.flags = eta.ATTN_MASK_TOPK
     # Dv larger than Dqk
     assert _call_fwd(lib, q, kv, _t([32, 80], stride=[64, 1]), _t([16, 4, 80]), lse,
                      mask=m) == eta.ATTN_ERR_INVALID_ARG
