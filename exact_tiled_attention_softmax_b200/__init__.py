@@ -33,6 +33,7 @@ ATTN_DEVERR_TIMEOUT = 0x4
 
 ATTN_F32 = 0
 ATTN_BF16 = 1
+ATTN_F16 = 2
 
 ATTN_MASK_CAUSAL = 0x1
 ATTN_MASK_WINDOW = 0x2
@@ -117,7 +118,7 @@ def attn_version() -> int:
     return int(load_library().attn_version())
 
 
-_DTYPES = {torch.float32: ATTN_F32, torch.bfloat16: ATTN_BF16}
+_DTYPES = {torch.float32: ATTN_F32, torch.bfloat16: ATTN_BF16, torch.float16: ATTN_F16}
 
 
 def _tensor(t: torch.Tensor | None):

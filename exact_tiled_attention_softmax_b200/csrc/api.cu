@@ -19,7 +19,15 @@ struct Dense {
 
 bool inner_contiguous(const attn_tensor* t) { return t->ndim >= 1 && t->stride[t->ndim - 1] == 1; }
 
-bool valid_dtype(int32_t dt) { return dt == ATTN_F32 || dt == ATTN_BF16; }
+bool valid_dtype(int32_t dt) { return dt == ATTN_F32 || dt == ATTN_BF16 || dt == ATTN_F16; }
+
+// Calls f with a value of the storage type that dt names.
+template <class F>
+cudaError_t by_storage(int32_t dt, F&& f) {
+  if (dt == ATTN_F32) return f(float());
+  if (dt == ATTN_F16) return f(__half());
+  return f(__nv_bfloat16());
+}
 
 bool dims_fit_int(const attn_tensor* t) {
   for (int i = 0; i < t->ndim; ++i)
@@ -163,7 +171,7 @@ size_t bwd_topk_bytes(const Topk& s, const attn_tensor* q, const attn_mask* m) {
   size_t n = kStatusBytes;
   n += align_up((size_t)s.Tq * s.H * sizeof(float), 256);                       // delta
   n += align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);      // 32.32 dKV
-  if (q->dtype == ATTN_BF16)                                                    // G, P rows (tensor-core path)
+  if (q->dtype != ATTN_F32)                                                     // G, P rows (tensor-core path)
     n += align_up(attn::sm100_topk_bwd_scratch_bytes(s.Tq, s.H, s.Dqk, s.Dv, m->topk_max), 256);
   return n + lse_copy_bytes(m, (size_t)s.Tq * s.H);
 }
@@ -276,6 +284,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.H = s.H;
     p.Dqk = s.Dqk;
     p.Dv = s.Dv;
+    p.dtype = q->dtype;
     p.scale = scale;
     p.sink = mask->sink;
     p.lse_fmt = mask->lse_format;
@@ -283,12 +292,11 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       return cuda_status(sm100_topk_fwd(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
                                         lse->stride[0], lse->stride[1], status, cs));
     main_kernel_begin(cs);
-    cudaError_t e = q->dtype == ATTN_F32
-        ? launch_topk_fwd_rows<float>(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
-                                      lse->stride[0], lse->stride[1], status, cs)
-        : launch_topk_fwd_rows<__nv_bfloat16>(p, o->data, o->stride[0], o->stride[1],
-                                              static_cast<float*>(lse->data), lse->stride[0], lse->stride[1],
-                                              status, cs);
+    cudaError_t e = by_storage(q->dtype, [&](auto t) {
+      return launch_topk_fwd_rows<decltype(t)>(p, o->data, o->stride[0], o->stride[1],
+                                               static_cast<float*>(lse->data), lse->stride[0], lse->stride[1],
+                                               status, cs);
+    });
     main_kernel_end(cs);
     return cuda_status(e);
   }
@@ -320,6 +328,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.Tk = s.Tk;
   p.d = s.d;
   p.dv = s.dv;
+  p.dtype = q->dtype;
   p.scale = scale;
   p.m = mask_params(mask);
   p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
@@ -331,8 +340,9 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
                                        status, cs));
   }
   main_kernel_begin(cs);
-  cudaError_t e = q->dtype == ATTN_F32 ? launch_dense_fwd_rows<float>(p, o->data, so, lsep, sl, cs)
-                                       : launch_dense_fwd_rows<__nv_bfloat16>(p, o->data, so, lsep, sl, cs);
+  cudaError_t e = by_storage(q->dtype, [&](auto t) {
+    return launch_dense_fwd_rows<decltype(t)>(p, o->data, so, lsep, sl, cs);
+  });
   main_kernel_end(cs);
   return cuda_status(e);
 }
@@ -385,6 +395,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.H = s.H;
     p.Dqk = s.Dqk;
     p.Dv = s.Dv;
+    p.dtype = q->dtype;
     p.scale = scale;
     p.sink = mask->sink;
     p.lse_fmt = mask->lse_format;
@@ -402,35 +413,33 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       lst = s.H;
       lsh = 1;
     }
-    if (q->dtype == ATTN_F32) {
-      e = launch_rows_delta<float>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
-      main_kernel_begin(cs);
-      if (e == cudaSuccess)
-        e = launch_topk_bwd_rows<float>(p, do_->data, do_->stride[0], do_->stride[1],
-                                        lsep, lst, lsh,
-                                        delta, dq->data, dq->stride[0], dq->stride[1], acc, dk->data,
-                                        dk->stride[0], status, cs);
-      main_kernel_end(cs);
-    } else if (sm100_topk_bwd_supported(p, q, k, o, do_, dq)) {
+    if (sm100_topk_bwd_supported(p, q, k, o, do_, dq)) {
       // Tensor cores: dQ and the per-token dKV contributions; the fixed-point
       // accumulator starts at zero and is cast to dKV at the end.
       char* scratch = ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256) +
                       align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);
-      e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
-      if (e == cudaSuccess) e = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * (size_t)s.Tkv * s.Dqk, cs);
-      if (e == cudaSuccess)
-        e = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta, dq->data,
-                           dq->stride[0], dq->stride[1], acc,
-                           scratch, status, cs);
-      if (e == cudaSuccess) e = launch_fixed_to_out<__nv_bfloat16>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
+      e = by_storage(q->dtype, [&](auto t) {
+        using T = decltype(t);
+        cudaError_t r = launch_rows_delta<T>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
+        if (r == cudaSuccess) r = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * (size_t)s.Tkv * s.Dqk, cs);
+        if (r == cudaSuccess)
+          r = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta, dq->data,
+                             dq->stride[0], dq->stride[1], acc, scratch, status, cs);
+        if (r == cudaSuccess) r = launch_fixed_to_out<T>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
+        return r;
+      });
     } else {
-      e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
-      main_kernel_begin(cs);
-      if (e == cudaSuccess)
-        e = launch_topk_bwd_rows<__nv_bfloat16>(p, do_->data, do_->stride[0], do_->stride[1],
-                                                lsep, lst, lsh, delta, dq->data, dq->stride[0], dq->stride[1],
-                                                acc, dk->data, dk->stride[0], status, cs);
-      main_kernel_end(cs);
+      e = by_storage(q->dtype, [&](auto t) {
+        using T = decltype(t);
+        cudaError_t r = launch_rows_delta<T>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
+        main_kernel_begin(cs);
+        if (r == cudaSuccess)
+          r = launch_topk_bwd_rows<T>(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta,
+                                      dq->data, dq->stride[0], dq->stride[1], acc, dk->data, dk->stride[0],
+                                      status, cs);
+        main_kernel_end(cs);
+        return r;
+      });
     }
     if (e == cudaSuccess && want_dsink)
       e = launch_dsink(mask->sink, lsep, delta, s.Tq, s.H, 1, lst, lsh, 0, false, dsink, cs);
@@ -473,6 +482,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.Tk = s.Tk;
   p.d = s.d;
   p.dv = s.dv;
+  p.dtype = q->dtype;
   p.scale = scale;
   p.m = mask_params(mask);
   p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
@@ -496,20 +506,17 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   if (sm100_dense_supported(p, q, k, v, o) && sm100_dense_bwd_supported(p, do_, dq, dk, dv)) {
     e = sm100_dense_bwd(p, o->data, so, do_->data, sg, lsep, sl, delta, dq_acc, dq->data, sdq, dk->data, sdk,
                         dv->data, sdv, extra, status, cs);
-  } else if (q->dtype == ATTN_F32) {
-    e = launch_rows_delta<float>(o->data, do_->data, s.B, s.Hq, s.Tq, so, sg, s.dv, delta, cs);
-    main_kernel_begin(cs);
-    if (e == cudaSuccess)
-      e = launch_dense_bwd_rows<float>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk, dv->data,
-                                       sdv, cs);
-    main_kernel_end(cs);
   } else {
-    e = launch_rows_delta<__nv_bfloat16>(o->data, do_->data, s.B, s.Hq, s.Tq, so, sg, s.dv, delta, cs);
-    main_kernel_begin(cs);
-    if (e == cudaSuccess)
-      e = launch_dense_bwd_rows<__nv_bfloat16>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk,
-                                               dv->data, sdv, cs);
-    main_kernel_end(cs);
+    e = by_storage(q->dtype, [&](auto t) {
+      using T = decltype(t);
+      cudaError_t r = launch_rows_delta<T>(o->data, do_->data, s.B, s.Hq, s.Tq, so, sg, s.dv, delta, cs);
+      main_kernel_begin(cs);
+      if (r == cudaSuccess)
+        r = launch_dense_bwd_rows<T>(p, do_->data, sg, lsep, sl, delta, dq->data, sdq, dk->data, sdk, dv->data,
+                                     sdv, cs);
+      main_kernel_end(cs);
+      return r;
+    });
   }
   if (e == cudaSuccess && want_dsink)
     e = launch_dsink(mask->sink, lsep, delta, s.B, s.Hq, s.Tq, sl[0], sl[1], sl[2], true, dsink, cs);

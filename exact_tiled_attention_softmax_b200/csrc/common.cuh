@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -53,6 +54,7 @@ struct DenseP {
   const void* v;
   int64_t sq[3], sk[3], sv[3];
   int B, Hq, Hkv, Tq, Tk, d, dv;
+  int32_t dtype;  // attn_dtype of every tensor
   float scale;
   MaskP m;
 };
@@ -67,6 +69,7 @@ struct TopkP {
   int32_t topk_max;
   const int32_t* len;  // may be null
   int Tq, Tkv, H, Dqk, Dv;
+  int32_t dtype;  // attn_dtype of every tensor
   float scale;
   const float* sink;
   uint32_t lse_fmt;  // ATTN_LSE_* bits of the LSE output
@@ -94,8 +97,10 @@ __device__ __forceinline__ float stored_lse_ln(uint32_t fmt, float lse_total, fl
 
 __device__ __forceinline__ float ld(const float* p) { return *p; }
 __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float ld(const __half* p) { return __half2float(*p); }
 __device__ __forceinline__ void st(float* p, float x) { *p = x; }
 __device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void st(__half* p, float x) { *p = __float2half_rn(x); }
 
 // The allowed-set predicate A_i (flags intersect).
 __device__ __forceinline__ bool allowed(const MaskP& m, int b, int h, int64_t i, int64_t j) {

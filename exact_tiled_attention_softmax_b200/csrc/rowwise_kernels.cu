@@ -586,5 +586,6 @@ cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta
 
 ATTN_INSTANTIATE(float)
 ATTN_INSTANTIATE(__nv_bfloat16)
+ATTN_INSTANTIATE(__half)
 
 }  // namespace attn

@@ -1,4 +1,4 @@
-// Tensor-core path for dense bf16 attention with d = dv = 128 on sm_100a.
+// Tensor-core path for dense bf16 or fp16 attention with d = dv = 128 on sm_100a.
 //
 // Forward: one CTA per (128-row query tile, query head, batch row). A TMA
 // producer warp streams 128-key K/V tiles through a two-stage ring; one
@@ -181,7 +181,7 @@ struct FwdArgs {
   int B, Hq, Hkv, Tq, Tk;
   int block_aligned;  // block mask constant over every (64-row slice, 128-key tile)
   float scale_log2;   // c * log2(e)
-  __nv_bfloat16* o;
+  uint16_t* o;  // 16-bit storage: bf16 or fp16
   int64_t so[3];
   float* lse;
   int64_t sl[3];
@@ -357,6 +357,7 @@ __device__ __forceinline__ float move_max(float mx, float& m_run) {
 // the maximum and the exponentials (one TMEM wait); x = s c log2(e) - m is
 // formed on packed fp32 pairs and every kPolyEvery-th pair of exponentials
 // runs on the FMA pipe instead of MUFU. Returns alpha.
+template <bool kH>
 __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2, float& m_run, float& l_run) {
   uint32_t s0[32], s1[32], s2[32], s3[32];
   tmem_ld32(tS, s0);
@@ -406,7 +407,7 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
         acc0 = f2_add(acc0, pp);
       float p0, p1;
       f2_unpack(pp, p0, p1);
-      pk[e] = pack_bf16(p0, p1);
+      pk[e] = pack16<kH>(p0, p1);
     }
     tmem_st16(tS + q * 16, pk);
   };
@@ -426,6 +427,7 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
 // columns per pass for the exponentials. The sum and the maximum use
 // every allowed key (undropped); P carries only the kept ones (the 1/(1-rho)
 // factor is applied to O in fp32 at the end). Returns alpha.
+template <bool kH>
 __device__ __forceinline__ float softmax_masked_tile(uint32_t tS, float scale_log2, uint64_t mw0, uint64_t mw1,
                                                      uint64_t kb0, uint64_t kb1, float& m_run, float& l_run) {
   float mx = -INFINITY;
@@ -460,7 +462,7 @@ __device__ __forceinline__ float softmax_masked_tile(uint32_t tS, float scale_lo
       const float p0 = ((mw >> bit) & 1ull) ? ex2(__uint_as_float(r[2 * e]) * scale_log2 - msub) : 0.f;
       const float p1 = ((mw >> (bit + 1)) & 1ull) ? ex2(__uint_as_float(r[2 * e + 1]) * scale_log2 - msub) : 0.f;
       sum += p0 + p1;
-      pk[e] = pack_bf16(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+      pk[e] = pack16<kH>(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
     }
     tmem_st16(tS + q * 16, pk);
   }
@@ -474,6 +476,7 @@ __device__ __forceinline__ float softmax_masked_tile(uint32_t tS, float scale_lo
 // into the warpgroup's own S columns of TMEM and read from there by the PV
 // MMA; S of the next tile lands in the same columns only after that PV, in
 // issue order.
+template <bool kH>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
@@ -562,8 +565,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    constexpr uint32_t idS = idesc_bf16(128, 128, 0, 0);
-    constexpr uint32_t idPV = idesc_bf16(128, 128, 0, 1);
+    constexpr uint32_t idS = idesc16<kH>(128, 128, 0, 0);
+    constexpr uint32_t idPV = idesc16<kH>(128, 128, 0, 1);
     bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
     // Descriptors of every operand tile, formed once; a K step adds its byte
     // offset >> 4 to the start-address field.
@@ -668,9 +671,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tc_fence_after();
       float alpha;
       if (cls == kFull && !a.m.dropout)
-        alpha = softmax_full_tile(tS, a.scale_log2, m_run, l_run);
+        alpha = softmax_full_tile<kH>(tS, a.scale_log2, m_run, l_run);
       else
-        alpha = softmax_masked_tile(tS, a.scale_log2, mw0, mw1, kb0, kb1, m_run, l_run);
+        alpha = softmax_masked_tile<kH>(tS, a.scale_log2, mw0, mw1, kb0, kb1, m_run, l_run);
       // Every earlier P V of this warpgroup has completed (the S commit covers
       // them) and the next one waits for p_full: O can be rescaled in place.
       if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -711,7 +714,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (a.m.dropout) oscale *= a.m.inv_keep;
         lse2 = M + log2f(tot);
       }
-      __nv_bfloat16* orow = a.o + b * a.so[0] + h * a.so[1] + row * a.so[2];
+      uint16_t* orow = a.o + b * a.so[0] + h * a.so[1] + row * a.so[2];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
@@ -726,7 +729,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int idx = c8 * 8 + 2 * e;
-              pkd[e] = have_o ? pack_bf16(__uint_as_float(o[idx]) * oscale, __uint_as_float(o[idx + 1]) * oscale) : 0u;
+              pkd[e] = have_o ? pack16<kH>(__uint_as_float(o[idx]) * oscale, __uint_as_float(o[idx + 1]) * oscale) : 0u;
             }
             *reinterpret_cast<uint4*>(orow + c * 32 + c8 * 8) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
           }
@@ -754,9 +757,9 @@ struct BwdArgs {
   const float* lse2;    // [B*Hq, Tpad] minus the base-2 LSE (-inf on rows without keys)
   const float* dpad;    // [B*Hq, Tpad] minus delta, zero on padding rows
   float* dq_acc;        // [B, Hq, Tq, 128] fp32
-  __nv_bfloat16* dk;
+  uint16_t* dk;  // 16-bit storage: bf16 or fp16
   int64_t sdk[3];
-  __nv_bfloat16* dv;
+  uint16_t* dv;
   int64_t sdv[3];
   float scale;
   uint32_t* status;
@@ -921,6 +924,7 @@ __device__ __forceinline__ void bulk_wait_read0() {
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+template <bool kH>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
@@ -1028,9 +1032,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     // ---------------- MMA issuer: S^T/dP^T of step n+1 go ahead of the
     // dV, dK, dQ^T products of step n so the tensor core overlaps the
     // compute warpgroup.
-    constexpr uint32_t idST = idesc_bf16(128, 64, 0, 0);   // K Q^T, V dO^T
-    constexpr uint32_t idACC = idesc_bf16(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
-    constexpr uint32_t idDQ = idesc_bf16(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
+    constexpr uint32_t idST = idesc16<kH>(128, 64, 0, 0);   // K Q^T, V dO^T
+    constexpr uint32_t idACC = idesc16<kH>(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
+    constexpr uint32_t idDQ = idesc16<kH>(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
     bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
     // Descriptors formed once; a K step adds its byte offset >> 4.
     const uint64_t dK = smem_desc_sw128(sbase + kBwdK, 16, 1024), dV = smem_desc_sw128(sbase + kBwdV, 16, 1024);
@@ -1158,12 +1162,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0, x1);
             const float p0 = ex2(x0), p1 = ex2(x1);
-            ppk[c2] = pack_bf16(p0, p1);
+            ppk[c2] = pack16<kH>(p0, p1);
             const uint64_t g = f2_mul(f2_pack(p0, p1),
                                       f2_add(f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1])), dp[e]));
             float g0, g1;
             f2_unpack(g, g0, g1);
-            dpk[c2] = pack_bf16(g0, g1);
+            dpk[c2] = pack16<kH>(g0, g1);
           }
         }
       } else {
@@ -1181,8 +1185,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             const float dpv = kp ? __uint_as_float(rp[c]) * inv : 0.f;
             ds[e] = p * (dpv + nd[c]);
           }
-          ppk[c2] = pack_bf16(pt[0], pt[1]);
-          dpk[c2] = pack_bf16(ds[0], ds[1]);
+          ppk[c2] = pack16<kH>(pt[0], pt[1]);
+          dpk[c2] = pack16<kH>(ds[0], ds[1]);
         }
       }
       // P~^T as bf16 pairs over this warpgroup's own dP^T columns (already read).
@@ -1210,7 +1214,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     const float osc = hf == 0 ? a.scale : (a.m.dropout ? a.m.inv_keep : 1.f);
     if (ok || n == 0) {
-      __nv_bfloat16* orow = hf == 0 ? a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2]
+      uint16_t* orow = hf == 0 ? a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2]
                                     : a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
       const uint32_t tacc = (hf == 0 ? tDK : tDV) + lane_off;
 #pragma unroll
@@ -1227,7 +1231,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int idx = c8 * 8 + e * 2;
-              pk[e] = have ? pack_bf16(__uint_as_float(r[idx]) * osc, __uint_as_float(r[idx + 1]) * osc) : 0u;
+              pk[e] = have ? pack16<kH>(__uint_as_float(r[idx]) * osc, __uint_as_float(r[idx + 1]) * osc) : 0u;
             }
             *reinterpret_cast<uint4*>(orow + c * 32 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
@@ -1290,8 +1294,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 // Reverse-pass preparation, one warp per (b, h, row < Tpad): delta from the
 // stored O and dO (kept, and negated in the padded array), the negated base-2
 // LSE, and a zeroed dQ accumulator row.
+template <bool kH>
 __global__ void __launch_bounds__(256)
-bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2, const __nv_bfloat16* g,
+bwd_prepare_kernel(const uint16_t* o, int64_t so0, int64_t so1, int64_t so2, const uint16_t* g,
                    int64_t sg0, int64_t sg1, int64_t sg2, const float* lse, int64_t sl0, int64_t sl1, int64_t sl2,
                    int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta, float* dq_acc) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -1307,16 +1312,14 @@ bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2
     }
     return;
   }
-  const __nv_bfloat16* orow = o + b * so0 + h * so1 + (int64_t)i * so2;
-  const __nv_bfloat16* grow = g + b * sg0 + h * sg1 + (int64_t)i * sg2;
+  const uint16_t* orow = o + b * so0 + h * so1 + (int64_t)i * so2;
+  const uint16_t* grow = g + b * sg0 + h * sg1 + (int64_t)i * sg2;
   const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
   const uint2 gv = *reinterpret_cast<const uint2*>(grow + lane * 4);
-  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-  const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
   float s = 0.f;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    const float2 a2 = __bfloat1622float2(o2[e]), b2 = __bfloat1622float2(g2[e]);
+    const float2 a2 = unpack16<kH>(e ? ov.y : ov.x), b2 = unpack16<kH>(e ? gv.y : gv.x);
     s = fmaf(a2.x, b2.x, s);
     s = fmaf(a2.y, b2.y, s);
   }
@@ -1331,8 +1334,9 @@ bwd_prepare_kernel(const __nv_bfloat16* o, int64_t so0, int64_t so1, int64_t so2
   }
 }
 
+template <bool kH>
 __global__ void __launch_bounds__(256)
-dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, __nv_bfloat16* dq, int64_t s0, int64_t s1,
+dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, uint16_t* dq, int64_t s0, int64_t s1,
                  int64_t s2) {
   const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
   if (e >= (int64_t)B * Hq * T * kD) return;
@@ -1343,8 +1347,8 @@ dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, __nv_bf
   const int b = (int)(r / ((int64_t)T * Hq));
   const float4 v = *reinterpret_cast<const float4*>(dq_acc + e);
   uint2 out;
-  out.x = pack_bf16(v.x * scale, v.y * scale);
-  out.y = pack_bf16(v.z * scale, v.w * scale);
+  out.x = pack16<kH>(v.x * scale, v.y * scale);
+  out.y = pack16<kH>(v.z * scale, v.w * scale);
   *reinterpret_cast<uint2*>(dq + b * s0 + h * s1 + (int64_t)i * s2 + c) = out;
 }
 
@@ -1362,16 +1366,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D bf16 map over (d, T, H, B) with a (64, rows, 1, 1) box and 128-byte swizzle.
+// 4-D 16-bit (bf16 or fp16) map over (d, T, H, B) with a (64, rows, 1, 1) box
+// and 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, int T, int H, int B, int64_t st, int64_t sh, int64_t sb,
-              int box_rows) {
+              int box_rows, bool f16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)st * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+  return fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+            const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1398,7 +1404,7 @@ bool make_dq_map(CUtensorMap* map, float* base, int T, int BH) {
 }
 
 bool tma_ok(const attn_tensor* t) {
-  if (!t || t->dtype != ATTN_BF16 || t->ndim != 4 || t->stride[3] != 1) return false;
+  if (!t || (t->dtype != ATTN_BF16 && t->dtype != ATTN_F16) || t->ndim != 4 || t->stride[3] != 1) return false;
   if (reinterpret_cast<uintptr_t>(t->data) % 16) return false;
   for (int i = 0; i < 3; ++i) {
     if ((t->stride[i] * 2) % 16) return false;
@@ -1409,7 +1415,7 @@ bool tma_ok(const attn_tensor* t) {
 
 // Raise a kernel's dynamic shared-memory limit once per device.
 cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
-  static bool done[2][64] = {};
+  static bool done[4][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1489,10 +1495,11 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   cudaError_t err;
   ClassTable ct = build_class_table(p, ws, st, err);
   if (err != cudaSuccess) return err;
+  const bool f16 = p.dtype == ATTN_F16;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM) ||
-      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
-      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN))
+  if (!make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM, f16) ||
+      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN, f16) ||
+      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN, f16))
     return cudaErrorInvalidValue;
   FwdArgs a;
   a.m = p.m;
@@ -1504,17 +1511,18 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   a.Tq = p.Tq;
   a.Tk = p.Tk;
   a.scale_log2 = p.scale * kLog2e;
-  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o = static_cast<uint16_t*>(o);
   for (int i = 0; i < 3; ++i) {
     a.so[i] = so[i];
     a.sl[i] = sl[i];
   }
   a.lse = lse;
   a.status = status;
-  if ((err = set_smem_attr(reinterpret_cast<const void*>(fwd_kernel), kFwdSmem, 0)) != cudaSuccess) return err;
+  auto kern = f16 ? fwd_kernel<true> : fwd_kernel<false>;
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kFwdSmem, f16 ? 2 : 0)) != cudaSuccess) return err;
   const int nct = (p.Tq + kFwdRows - 1) / kFwdRows;
   main_kernel_begin(st);
-  fwd_kernel<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
+  kern<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
   main_kernel_end(st);
   return cudaGetLastError();
 }
@@ -1530,17 +1538,18 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   cudaError_t err;
   ClassTable ct = build_class_table(p, static_cast<char*>(ws_extra) + 2 * padb, st, err);
   if (err != cudaSuccess) return err;
+  const bool f16 = p.dtype == ATTN_F16;
   const int64_t rows = (int64_t)p.B * p.Hq * Tpad;
-  bwd_prepare_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(o), so[0], so[1], so[2], static_cast<const __nv_bfloat16*>(g), sg[0], sg[1],
-      sg[2], lse, sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta, dq_acc);
+  (f16 ? bwd_prepare_kernel<true> : bwd_prepare_kernel<false>)<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint16_t*>(o), so[0], so[1], so[2], static_cast<const uint16_t*>(g), sg[0], sg[1], sg[2], lse,
+      sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta, dq_acc);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   CUtensorMap mq, mk, mv, mg, mdq;
   if (!make_dq_map(&mdq, dq_acc, p.Tq, p.B * p.Hq) ||
-      !make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb) ||
-      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN) ||
-      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN) ||
-      !make_map(&mg, g, p.Tq, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb))
+      !make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb, f16) ||
+      !make_map(&mk, p.k, p.Tk, p.Hkv, p.B, p.sk[2], p.sk[1], p.sk[0], kBN, f16) ||
+      !make_map(&mv, p.v, p.Tk, p.Hkv, p.B, p.sv[2], p.sv[1], p.sv[0], kBN, f16) ||
+      !make_map(&mg, g, p.Tq, p.Hq, p.B, sg[2], sg[1], sg[0], kBMb, f16))
     return cudaErrorInvalidValue;
   BwdArgs a;
   a.m = p.m;
@@ -1556,24 +1565,24 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   a.lse2 = lse2;
   a.dpad = dpad;
   a.dq_acc = dq_acc;
-  a.dk = static_cast<__nv_bfloat16*>(dk);
-  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.dk = static_cast<uint16_t*>(dk);
+  a.dv = static_cast<uint16_t*>(dv);
   for (int i = 0; i < 3; ++i) {
     a.sdk[i] = sdk[i];
     a.sdv[i] = sdv[i];
   }
   a.scale = p.scale;
   a.status = status;
-  if ((err = set_smem_attr(reinterpret_cast<const void*>(bwd_kernel), kBwdSmem, 1)) != cudaSuccess) return err;
+  auto kern = f16 ? bwd_kernel<true> : bwd_kernel<false>;
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kBwdSmem, f16 ? 3 : 1)) != cudaSuccess) return err;
   const int nkt = (p.Tk + kBN - 1) / kBN;
   main_kernel_begin(st);
-  bwd_kernel<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
+  kern<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
   main_kernel_end(st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n4 = (int64_t)p.B * p.Hq * p.Tq * kD / 4;
-  dq_finish_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(dq_acc, p.B, p.Hq, p.Tq, p.scale,
-                                                                 static_cast<__nv_bfloat16*>(dq), sdq[0], sdq[1],
-                                                                 sdq[2]);
+  (f16 ? dq_finish_kernel<true> : dq_finish_kernel<false>)<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+      dq_acc, p.B, p.Hq, p.Tq, p.scale, static_cast<uint16_t*>(dq), sdq[0], sdq[1], sdq[2]);
   return cudaGetLastError();
 }
 

@@ -202,6 +202,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// The same descriptor with both operands fp16 (A and B format 0).
+__host__ __device__ constexpr uint32_t idesc_fp16(int M, int N, int a_mn, int b_mn) {
+  return idesc_bf16(M, N, a_mn, b_mn) & ~((7u << 7) | (7u << 10));
+}
+
+template <bool kH>
+__host__ __device__ constexpr uint32_t idesc16(int M, int N, int a_mn, int b_mn) {
+  return kH ? idesc_fp16(M, N, a_mn, b_mn) : idesc_bf16(M, N, a_mn, b_mn);
+}
+
 // Byte offset of element (r, c) inside a 128-byte-swizzled region whose rows
 // are 128 bytes (64 bf16) wide: 8-row atoms of 1024 bytes, 16-byte chunks
 // permuted by the row's position in its atom.
@@ -212,6 +222,30 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t byte_in_ro
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_fp16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two fp32 values rounded to the 16-bit storage type (kH: fp16, else bf16),
+// low half first.
+template <bool kH>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  if constexpr (kH)
+    return pack_fp16(lo, hi);
+  else
+    return pack_bf16(lo, hi);
+}
+
+// Both halves of a packed 16-bit pair as fp32.
+template <bool kH>
+__device__ __forceinline__ float2 unpack16(uint32_t v) {
+  if constexpr (kH)
+    return __half22float2(*reinterpret_cast<const __half2*>(&v));
+  else
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

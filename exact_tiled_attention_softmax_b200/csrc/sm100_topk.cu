@@ -10,7 +10,7 @@
 // "lower" half) or, addressed at lane 16, lanes 16-31 (the "upper" half).
 //   lower half, columns 0-511:   O, 64 heads x 512 fp32
 //   upper half, columns 0-127:   two S buffers, 64 heads x 64 keys fp32
-//   upper half, columns 128-415: Q as bf16 pairs, the A operand of S = Q K^T
+//   upper half, columns 128-415: Q as 16-bit pairs, the A operand of S = Q K^T
 // A warp reads its quarter with 32-lane loads: its upper 16 lanes own the
 // S rows (softmax), its lower 16 lanes the O rows of the same heads.
 //
@@ -40,7 +40,7 @@ constexpr uint32_t kTPlane = kTK * 128;        // 8 KB: 64 rows x 128 bytes
 constexpr uint32_t kTTile = kTPlanes * kTPlane;  // 72 KB per KV tile
 constexpr int kTStages = 3;
 constexpr uint32_t kTKV = 0;
-constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys bf16
+constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kTCtl = kTP + kTH * 128;
 constexpr uint32_t kTSmem = kTCtl + 512 + 1024;  // control block + alignment slack
 constexpr int kTThreads = 192;                   // producer, MMA issuer, 4 softmax warps
@@ -59,7 +59,7 @@ struct TopkCtl {
 };
 
 struct TopkArgs {
-  const __nv_bfloat16* q;
+  const uint16_t* q;  // 16-bit storage: bf16 or fp16
   int64_t sq_t, sq_h;
   const int32_t* idx;
   int64_t idx_stride;
@@ -68,7 +68,7 @@ struct TopkArgs {
   int Tq, Tkv;
   float scale_log2;
   const float* sink;
-  __nv_bfloat16* o;
+  uint16_t* o;
   int64_t so_t, so_h;
   float* lse;
   int64_t sl_t, sl_h;
@@ -87,6 +87,7 @@ __device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* map, ui
 
 __device__ __forceinline__ bool key_valid(const uint32_t (&vm)[2], int k) { return (vm[k & 1] >> (k >> 1)) & 1u; }
 
+template <bool kH>
 __global__ void __launch_bounds__(kTThreads, 1)
 topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -166,8 +167,8 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
         wait_bar(smem_u32(&ctl->kv_full[r % kTStages]), (r / kTStages) & 1, abort_flag, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S(n) = Q K(n)^T two tiles ahead of O += P(n) V(n).
-    constexpr uint32_t idS = idesc_bf16(64, kTK, 0, 0);
-    constexpr uint32_t idPV = idesc_bf16(64, 256, 0, 1);
+    constexpr uint32_t idS = idesc16<kH>(64, kTK, 0, 0);
+    constexpr uint32_t idPV = idesc16<kH>(64, 256, 0, 1);
     const uint64_t dKV0 = smem_desc_sw128(sbase + kTKV, 16, 1024);        // K-major rows of a plane
     const uint64_t dV0 = smem_desc_sw128(sbase + kTKV, kTPlane, 1024);    // MN-major: planes are 64-wide chunks
     const uint64_t dP0 = smem_desc_sw128(sbase + kTP, 16, 1024);
@@ -211,7 +212,7 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
     const bool upper = lane >= 16;
     const int h = 16 * qt + (lane & 15);
     const uint32_t tq = tmem + ((uint32_t)(32 * qt) << 16);  // this warp's lanes, column 0
-    // Q row h into TMEM (upper half, columns 128-415) as bf16 pairs. The lower
+    // Q row h into TMEM (upper half, columns 128-415) as 16-bit pairs. The lower
     // lanes store zeros into O's columns, which the first P V overwrites.
     {
       const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (int64_t)t * a.sq_t + (int64_t)h * a.sq_h);
@@ -274,8 +275,8 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
         const float p2 = key_valid(vm, 32 + k0) ? ex2(__uint_as_float(s1[k0]) * a.scale_log2 - msub) : 0.f;
         const float p3 = key_valid(vm, 32 + k1) ? ex2(__uint_as_float(s1[k1]) * a.scale_log2 - msub) : 0.f;
         sum += (p0 + p1) + (p2 + p3);
-        pk[e] = pack_bf16(p0, p1);
-        pk[16 + e] = pack_bf16(p2, p3);
+        pk[e] = pack16<kH>(p0, p1);
+        pk[16 + e] = pack16<kH>(p2, p3);
       }
       l_run = l_run * alpha + sum;
       // The single P buffer is free once P(n-1) V(n-1) has completed; O is
@@ -337,7 +338,7 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
         a.lse[(int64_t)t * a.sl_t + (int64_t)h * a.sl_h] = stored_lse_log2(a.lse_fmt, lse2, m_run, l_run);
       }
       oscale = __shfl_sync(0xffffffffu, oscale, (lane + 16) & 31);  // lower lane l <- upper lane l + 16
-      __nv_bfloat16* orow = a.o + (int64_t)t * a.so_t + (int64_t)h * a.so_h;
+      uint16_t* orow = a.o + (int64_t)t * a.so_t + (int64_t)h * a.so_h;
 #pragma unroll 1
       for (int c = 0; c < kTDV / 32; ++c) {
         uint32_t o[32];
@@ -352,7 +353,7 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int idx = c8 * 8 + 2 * e;
-              pkd[e] = have_o ? pack_bf16(__uint_as_float(o[idx]) * oscale, __uint_as_float(o[idx + 1]) * oscale) : 0u;
+              pkd[e] = have_o ? pack16<kH>(__uint_as_float(o[idx]) * oscale, __uint_as_float(o[idx + 1]) * oscale) : 0u;
             }
             *reinterpret_cast<uint4*>(orow + c * 32 + c8 * 8) = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
           }
@@ -373,14 +374,14 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
 // Reverse, first kernel (one CTA per query token): recompute S = Q K^T,
 // P = 2^(S c log2(e) - LSE2) on the listed keys, dP = dO V^T, and
 // G = c P (dP - delta) (DSA note, sections 3.3-3.4, 8); accumulate
-// dQ = G K_sel in TMEM over the tiles, and store G and P as bf16 rows
+// dQ = G K_sel in TMEM over the tiles, and store G and P as 16-bit rows
 // [token][head][listed position] for the dKV kernel.
 //   upper half: S cols 0-63, dP 64-127, Q 128-415, dQ[:, 512:576] 416-479
 //   lower half: dQ[:, 0:512] cols 0-511
 constexpr int kBStages = 2;
 constexpr uint32_t kBKV = 0;
 constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads x 64 columns
-constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys bf16
+constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kBCtl = kBG + kTH * 128;
 constexpr uint32_t kBSmem = kBCtl + 512 + 1024;
 constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
@@ -394,7 +395,7 @@ struct TopkBwdCtl {
 };
 
 struct TopkBwdArgs {
-  const __nv_bfloat16* q;
+  const uint16_t* q;  // 16-bit storage: bf16 or fp16
   int64_t sq_t, sq_h;
   const int32_t* idx;
   int64_t idx_stride;
@@ -405,13 +406,14 @@ struct TopkBwdArgs {
   const float* lse;
   int64_t sl_t, sl_h;
   const float* delta;  // [Tq, 64]
-  __nv_bfloat16* dq;
+  uint16_t* dq;
   int64_t sd_t, sd_h;
-  __nv_bfloat16* g_scr;  // [Tq, 64, topk_pad]
-  __nv_bfloat16* p_scr;
+  uint16_t* g_scr;  // [Tq, 64, topk_pad]
+  uint16_t* p_scr;
   uint32_t* status;
 };
 
+template <bool kH>
 __global__ void __launch_bounds__(kTThreads, 1)
 topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constant__ CUtensorMap tdo,
                    const TopkBwdArgs a) {
@@ -501,9 +503,9 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S(n), dP(n) as soon as the compute warps
     // have read S(n-1), dP(n-1); dQ += G(n) K(n) once G(n) is in shared memory.
-    constexpr uint32_t idS = idesc_bf16(64, kTK, 0, 0);
-    constexpr uint32_t idDQ = idesc_bf16(64, 256, 0, 1);
-    constexpr uint32_t idDQ64 = idesc_bf16(64, 64, 0, 1);
+    constexpr uint32_t idS = idesc16<kH>(64, kTK, 0, 0);
+    constexpr uint32_t idDQ = idesc16<kH>(64, 256, 0, 1);
+    constexpr uint32_t idDQ64 = idesc16<kH>(64, 64, 0, 1);
     const uint64_t dKV0 = smem_desc_sw128(sbase + kBKV, 16, 1024);
     const uint64_t dKmn0 = smem_desc_sw128(sbase + kBKV, kTPlane, 1024);
     const uint64_t dDO = smem_desc_sw128(sbase + kBDO, 16, 1024);
@@ -581,8 +583,8 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
     const float dl = a.delta[(int64_t)t * kTH + h];
     const bool live = L != -INFINITY;
     const uint32_t g_row = sbase + kBG + h * 128;
-    __nv_bfloat16* gs = a.g_scr + ((int64_t)t * kTH + h) * a.topk_pad;
-    __nv_bfloat16* ps = a.p_scr + ((int64_t)t * kTH + h) * a.topk_pad;
+    uint16_t* gs = a.g_scr + ((int64_t)t * kTH + h) * a.topk_pad;
+    uint16_t* ps = a.p_scr + ((int64_t)t * kTH + h) * a.topk_pad;
     bool ok = true;
     for (int n = 0; n < ntiles && ok; ++n) {
       const int s = n % kBStages;
@@ -615,10 +617,10 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
           pv[u] = p;
           gv[u] = a.scale * p * (__uint_as_float(dv) - dl);
         }
-        pp[e] = pack_bf16(pv[0], pv[1]);
-        pp[16 + e] = pack_bf16(pv[2], pv[3]);
-        gp[e] = pack_bf16(gv[0], gv[1]);
-        gp[16 + e] = pack_bf16(gv[2], gv[3]);
+        pp[e] = pack16<kH>(pv[0], pv[1]);
+        pp[16 + e] = pack16<kH>(pv[2], pv[3]);
+        gp[e] = pack16<kH>(gv[0], gv[1]);
+        gp[16 + e] = pack16<kH>(gv[2], gv[3]);
       }
       // G's shared-memory tile is free once dQ += G(n-1) K(n-1) has completed.
       if (n > 0)
@@ -648,7 +650,7 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
       if (have) tc_fence_after();
     }
     if (ok) {
-      __nv_bfloat16* drow = a.dq + (int64_t)t * a.sd_t + (int64_t)h * a.sd_h;
+      uint16_t* drow = a.dq + (int64_t)t * a.sd_t + (int64_t)h * a.sd_h;
       auto put = [&](const uint32_t (&r)[32], int col0) {
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
@@ -656,7 +658,7 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int idx = c8 * 8 + 2 * e;
-            pk[e] = have ? pack_bf16(__uint_as_float(r[idx]), __uint_as_float(r[idx + 1])) : 0u;
+            pk[e] = have ? pack16<kH>(__uint_as_float(r[idx]), __uint_as_float(r[idx + 1])) : 0u;
           }
           *reinterpret_cast<uint4*>(drow + col0 + c8 * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
@@ -721,6 +723,7 @@ struct TopkDkvArgs {
   uint32_t* status;
 };
 
+template <bool kH>
 __global__ void __launch_bounds__(kTThreads, 1)
 topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                     const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tp,
@@ -798,8 +801,8 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: C^T = Q^T G + dO^T P per tile.
-    constexpr uint32_t id128 = idesc_bf16(128, kTK, 1, 1);
-    constexpr uint32_t id64 = idesc_bf16(64, kTK, 1, 1);
+    constexpr uint32_t id128 = idesc16<kH>(128, kTK, 1, 1);
+    constexpr uint32_t id64 = idesc16<kH>(64, kTK, 1, 1);
     const uint64_t dQ0 = smem_desc_sw128(sbase + kCQ, kTPlane, 1024);    // [heads x d], d contiguous
     const uint64_t dDO0 = smem_desc_sw128(sbase + kCDO, kTPlane, 1024);
     const uint64_t dGP0 = smem_desc_sw128(sbase + kCGP, kTPlane, 1024);  // [heads x keys], keys contiguous
@@ -899,30 +902,31 @@ bool aligned16(const void* p, int64_t stride_elems) {
   return reinterpret_cast<uintptr_t>(p) % 16 == 0 && (stride_elems * 2) % 16 == 0;
 }
 
-// 3-D bf16 map (inner, 64, Tq) with (64, 64, 1) boxes and 128-byte swizzle:
+// 3-D 16-bit map (inner, 64, Tq) with (64, 64, 1) boxes and 128-byte swizzle:
 // one token's 64 rows of a 64-column plane per load.
-bool make_map3(CUtensorMap* map, const void* base, int64_t inner, int Tq, int64_t s_row, int64_t s_tok) {
+bool make_map3(CUtensorMap* map, const void* base, int64_t inner, int Tq, int64_t s_row, int64_t s_tok, bool f16) {
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)kTH, (cuuint64_t)Tq};
   cuuint64_t strides[2] = {(cuuint64_t)s_row * 2, (cuuint64_t)s_tok * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)kTH, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return topk_encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return topk_encode_fn()(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_kv_gather_map(CUtensorMap* map, const TopkP& p) {
+  const bool f16 = p.dtype == ATTN_F16;
   cuuint64_t dims[2] = {(cuuint64_t)p.Dqk, (cuuint64_t)p.Tkv};
   cuuint64_t strides[1] = {(cuuint64_t)p.skv * 2};
   cuuint32_t box[2] = {64, 1};
   cuuint32_t es[2] = {1, 1};
-  return topk_encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.kv), dims, strides, box, es,
+  return topk_encode_fn()(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.kv), dims, strides, box, es,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 cudaError_t raise_smem(const void* fn, uint32_t bytes, int which) {
-  static bool done[3][64] = {};
+  static bool done[6][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -938,13 +942,13 @@ int sm100_topk_pad(int topk_max) { return ((topk_max + kTK - 1) / kTK) * kTK; }
 
 size_t sm100_topk_bwd_scratch_bytes(int Tq, int H, int Dqk, int Dv, int topk_max) {
   if (H != kTH || Dqk != kTD || Dv != kTDV) return 0;
-  return 2 * (size_t)Tq * kTH * sm100_topk_pad(topk_max) * sizeof(__nv_bfloat16);
+  return 2 * (size_t)Tq * kTH * sm100_topk_pad(topk_max) * sizeof(uint16_t);
 }
 
 bool sm100_topk_bwd_supported(const TopkP& p, const attn_tensor* q, const attn_tensor* kv, const attn_tensor* o,
                               const attn_tensor* do_, const attn_tensor* dq) {
   if (!sm100_topk_supported(p, q, kv, o)) return false;
-  if (do_->dtype != ATTN_BF16 || dq->dtype != ATTN_BF16) return false;
+  if (do_->dtype != q->dtype || dq->dtype != q->dtype) return false;
   return aligned16(do_->data, do_->stride[0]) && aligned16(do_->data, do_->stride[1]) &&
          aligned16(dq->data, dq->stride[0]) && aligned16(dq->data, dq->stride[1]);
 }
@@ -953,15 +957,17 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
                            int64_t sl_t, int64_t sl_h, const float* delta, void* dq, int64_t sd_t, int64_t sd_h,
                            unsigned long long* acc, void* scratch, uint32_t* status, cudaStream_t st) {
   const int pad = sm100_topk_pad(p.topk_max);
-  __nv_bfloat16* g_scr = static_cast<__nv_bfloat16*>(scratch);
-  __nv_bfloat16* p_scr = g_scr + (size_t)p.Tq * kTH * pad;
+  const bool f16 = p.dtype == ATTN_F16;
+  uint16_t* g_scr = static_cast<uint16_t*>(scratch);
+  uint16_t* p_scr = g_scr + (size_t)p.Tq * kTH * pad;
   CUtensorMap mkv, mdo, mq, mg, mp;
-  if (!make_kv_gather_map(&mkv, p) || !make_map3(&mdo, g, kTDV, p.Tq, sg_h, sg_t) ||
-      !make_map3(&mq, p.q, kTD, p.Tq, p.sq_h, p.sq_t) || !make_map3(&mg, g_scr, pad, p.Tq, pad, (int64_t)kTH * pad) ||
-      !make_map3(&mp, p_scr, pad, p.Tq, pad, (int64_t)kTH * pad))
+  if (!make_kv_gather_map(&mkv, p) || !make_map3(&mdo, g, kTDV, p.Tq, sg_h, sg_t, f16) ||
+      !make_map3(&mq, p.q, kTD, p.Tq, p.sq_h, p.sq_t, f16) ||
+      !make_map3(&mg, g_scr, pad, p.Tq, pad, (int64_t)kTH * pad, f16) ||
+      !make_map3(&mp, p_scr, pad, p.Tq, pad, (int64_t)kTH * pad, f16))
     return cudaErrorInvalidValue;
   TopkBwdArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(p.q);
+  a.q = static_cast<const uint16_t*>(p.q);
   a.sq_t = p.sq_t;
   a.sq_h = p.sq_h;
   a.idx = p.idx;
@@ -977,7 +983,7 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   a.sl_t = sl_t;
   a.sl_h = sl_h;
   a.delta = delta;
-  a.dq = static_cast<__nv_bfloat16*>(dq);
+  a.dq = static_cast<uint16_t*>(dq);
   a.sd_t = sd_t;
   a.sd_h = sd_h;
   a.g_scr = g_scr;
@@ -994,18 +1000,21 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   c.acc = acc;
   c.status = status;
   cudaError_t e;
-  if ((e = raise_smem(reinterpret_cast<const void*>(topk_bwd_dq_kernel), kBSmem, 1)) != cudaSuccess) return e;
-  if ((e = raise_smem(reinterpret_cast<const void*>(topk_bwd_dkv_kernel), kCSmem, 2)) != cudaSuccess) return e;
+  auto kdq = f16 ? topk_bwd_dq_kernel<true> : topk_bwd_dq_kernel<false>;
+  auto kdkv = f16 ? topk_bwd_dkv_kernel<true> : topk_bwd_dkv_kernel<false>;
+  if ((e = raise_smem(reinterpret_cast<const void*>(kdq), kBSmem, f16 ? 4 : 1)) != cudaSuccess) return e;
+  if ((e = raise_smem(reinterpret_cast<const void*>(kdkv), kCSmem, f16 ? 5 : 2)) != cudaSuccess) return e;
   main_kernel_begin(st);
-  topk_bwd_dq_kernel<<<p.Tq, kTThreads, kBSmem, st>>>(mkv, mdo, a);
+  kdq<<<p.Tq, kTThreads, kBSmem, st>>>(mkv, mdo, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  topk_bwd_dkv_kernel<<<p.Tq, kTThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
+  kdkv<<<p.Tq, kTThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
   main_kernel_end(st);
   return cudaGetLastError();
 }
 
 bool sm100_topk_supported(const TopkP& p, const attn_tensor* q, const attn_tensor* kv, const attn_tensor* o) {
-  if (q->dtype != ATTN_BF16 || kv->dtype != ATTN_BF16 || o->dtype != ATTN_BF16) return false;
+  if (q->dtype != ATTN_BF16 && q->dtype != ATTN_F16) return false;
+  if (kv->dtype != q->dtype || o->dtype != q->dtype) return false;
   if (p.H != kTH || p.Dqk != kTD || p.Dv != kTDV || p.Tq < 1 || p.Tkv < 1) return false;
   if (!aligned16(p.q, p.sq_t) || !aligned16(p.q, p.sq_h) || !aligned16(p.kv, p.skv)) return false;
   if (!aligned16(o->data, o->stride[0]) || !aligned16(o->data, o->stride[1])) return false;
@@ -1024,7 +1033,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   CUtensorMap map;
   if (!make_kv_gather_map(&map, p)) return cudaErrorInvalidValue;
   TopkArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(p.q);
+  a.q = static_cast<const uint16_t*>(p.q);
   a.sq_t = p.sq_t;
   a.sq_h = p.sq_h;
   a.idx = p.idx;
@@ -1035,7 +1044,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   a.Tkv = p.Tkv;
   a.scale_log2 = p.scale * kLog2e;
   a.sink = p.sink;
-  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o = static_cast<uint16_t*>(o);
   a.so_t = so_t;
   a.so_h = so_h;
   a.lse = lse;
@@ -1043,10 +1052,12 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   a.sl_h = sl_h;
   a.lse_fmt = p.lse_fmt;
   a.status = status;
-  cudaError_t e = raise_smem(reinterpret_cast<const void*>(topk_fwd_kernel), kTSmem, 0);
+  const bool f16 = p.dtype == ATTN_F16;
+  auto kern = f16 ? topk_fwd_kernel<true> : topk_fwd_kernel<false>;
+  cudaError_t e = raise_smem(reinterpret_cast<const void*>(kern), kTSmem, f16 ? 3 : 0);
   if (e != cudaSuccess) return e;
   main_kernel_begin(st);
-  topk_fwd_kernel<<<p.Tq, kTThreads, kTSmem, st>>>(map, a);
+  kern<<<p.Tq, kTThreads, kTSmem, st>>>(map, a);
   main_kernel_end(st);
   return cudaGetLastError();
 }

@@ -27,6 +27,21 @@ from dataclasses import dataclass
 import numpy as np
 
 
+def round_to_fp16(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest IEEE half (ties to even), returned
+    as float32."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
+def round_to_storage(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Inputs as the library will store them: "bf16", "f16" or "f32"."""
+    if dtype == "bf16":
+        return round_to_bf16(x)
+    if dtype == "f16":
+        return round_to_fp16(x)
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even), returned
     as float32 so that both sides can read them."""

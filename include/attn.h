@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 104 /* major * 100 + minor */
+#define ATTN_VERSION 105 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -69,7 +69,7 @@ typedef enum attn_status {
 #define ATTN_DEVERR_OVERFLOW 0x2u    /* a fixed-point dKV contribution saturated */
 #define ATTN_DEVERR_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
 
-typedef enum attn_dtype { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype;
+typedef enum attn_dtype { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_F16 = 2 } attn_dtype;
 
 /* A strided tensor view. Strides count elements, not bytes; the innermost
  * dimension must have stride 1. Unused trailing entries are ignored. */
@@ -163,8 +163,10 @@ typedef struct attn_mask {
  *           o [Tq,H,Dv], lse fp32 [Tq,H]. dk receives dKV [Tkv,Dqk]; dv is NULL.
  *           Query token t sits at causal position Tkv - Tq + t; the lists
  *           must respect causality themselves.
- *   dtype: all of q, k, v, o (and do, dq, dk, dv) share one dtype, ATTN_F32
- *   or ATTN_BF16. Accumulation is fp32 in every path.
+ *   dtype: all of q, k, v, o (and do, dq, dk, dv) share one dtype, ATTN_F32,
+ *   ATTN_BF16 or ATTN_F16 (the DSA note's storage table: BF16 or FP16).
+ *   Accumulation is fp32 in every path; the probability and score-gradient
+ *   operands of the tensor-core MMAs take the storage type.
  */
 
 /* Workspace bytes attn_fwd needs for these shapes and mask (>= 256). */

@@ -19,6 +19,7 @@ from oracle import philox as P  # noqa: E402
 from tests.parity_util import check_close, to_dev, to_np  # noqa: E402
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -31,8 +32,7 @@ def _cuda():
 def _dense_case(B, Hq, Hkv, T, d, dv, dtype, seed, *, causal=True, window=0, block=0, p_keep=0.5,
                 dropout=0.0, sink=False, scale=None):
     rng = np.random.default_rng(seed)
-    f = (lambda s: W.round_to_bf16(rng.standard_normal(s, dtype=np.float32))) if dtype == "bf16" else \
-        (lambda s: rng.standard_normal(s, dtype=np.float32))
+    f = lambda s: W.round_to_storage(rng.standard_normal(s, dtype=np.float32), dtype)  # noqa: E731
     q, k, v, g = f((B, Hq, T, d)), f((B, Hkv, T, d)), f((B, Hkv, T, dv)), f((B, Hq, T, dv))
     bm = None
     if block:
@@ -47,7 +47,7 @@ def _dense_case(B, Hq, Hkv, T, d, dv, dtype, seed, *, causal=True, window=0, blo
 
 
 def _run_gpu(c):
-    tdt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float32
+    tdt = TORCH_DTYPE[c["dtype"]]
     q, k, v, g = (to_dev(c[n], tdt) for n in ("q", "k", "v", "g"))
     allowed = eta.AllowedSet(
         causal=c["causal"], window_left=c["window"],
@@ -104,7 +104,7 @@ def test_tiny_causal_fp32_full():
 
 
 @pytest.mark.parametrize("kind", ["causal", "window_block", "gqa_dropout", "sink", "noncausal_mqa"])
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "f16"])
 def test_small_dense_cases(kind, dtype):
     """Multi-tile shapes with a ragged tail (T=300) for every allowed-set kind."""
     if kind == "causal":
@@ -204,20 +204,19 @@ def test_dropout_replay_example_on_gpu():
 
 def _topk_small(dtype, seed, Tq=40, Tkv=300, H=8, Dqk=96, Dv=64, topk=128, lo=20, hi=128, sink=True):
     rng = np.random.default_rng(seed)
-    f = (lambda s: W.round_to_bf16(rng.standard_normal(s, dtype=np.float32))) if dtype == "bf16" else \
-        (lambda s: rng.standard_normal(s, dtype=np.float32))
+    f = lambda s: W.round_to_storage(rng.standard_normal(s, dtype=np.float32), dtype)  # noqa: E731
     q, kv, g = f((Tq, H, Dqk)), f((Tkv, Dqk)), f((Tq, H, Dv))
     idx, ln = W.topk_lists(Tq, Tkv, topk, lo, hi, seed + 1)
     sk = rng.standard_normal(H).astype(np.float32) if sink else None
     return q, kv, g, idx, ln, sk
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32", "f16"])
 def test_small_topk(dtype):
     q, kv, g, idx, ln, sk = _topk_small(dtype, 31)
     Dv = g.shape[-1]
     scale = 1 / math.sqrt(q.shape[-1])
-    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    tdt = TORCH_DTYPE[dtype]
     qd, kvd, gd = to_dev(q, tdt), to_dev(kv, tdt), to_dev(g, tdt)
     al = eta.AllowedSet(topk_idxs=to_dev(idx, torch.int32), topk_length=to_dev(ln, torch.int32),
                         sink=to_dev(sk, torch.float32))
@@ -252,8 +251,7 @@ def test_topk_bad_index_sets_status_and_returns():
 
 def _qk_case(B, Hq, Hkv, Tq, Tk, d, dv, dtype, seed, *, causal=True, window=0, block=0, dropout=0.0, sink=False):
     rng = np.random.default_rng(seed)
-    f = (lambda s: W.round_to_bf16(rng.standard_normal(s, dtype=np.float32))) if dtype == "bf16" else \
-        (lambda s: rng.standard_normal(s, dtype=np.float32))
+    f = lambda s: W.round_to_storage(rng.standard_normal(s, dtype=np.float32), dtype)  # noqa: E731
     q, g = f((B, Hq, Tq, d)), f((B, Hq, Tq, dv))
     k, v = f((B, Hkv, Tk, d)), f((B, Hkv, Tk, dv))
     bm = None
@@ -299,7 +297,7 @@ def _segment_starts(bounds_per_batch, T):
 
 
 def _run_layout_case(c, lengths=None, starts=None):
-    tdt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float32
+    tdt = TORCH_DTYPE[c["dtype"]]
     q, k, v, g = (to_dev(c[n], tdt) for n in ("q", "k", "v", "g"))
     allowed = eta.AllowedSet(
         causal=c["causal"], window_left=c["window"],

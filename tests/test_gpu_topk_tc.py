@@ -133,3 +133,37 @@ def test_topk_tc_backward_matches_oracle_and_is_reproducible():
     dq2, dkv2, _, ds2 = eta.attn_bwd(qd, kvd, kvd[:, :DV], o, gd, lse, al, scale, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(dkv2, dkv) and torch.equal(ds2, ds)
+
+
+def test_topk_tc_fp16_storage():
+    """fp16 storage (the DSA note's storage table allows BF16 or FP16): the
+    same kernels with fp16 operands, forward and reverse against the oracle
+    on the fp16-rounded inputs."""
+    from tests.parity_util import BF16_GRAD_REL, rel_fro
+    rng = np.random.default_rng(76)
+    Tq, Tkv = 24, 700
+    q = W.round_to_fp16(rng.standard_normal((Tq, H, DQK), dtype=np.float32))
+    kv = W.round_to_fp16(rng.standard_normal((Tkv, DQK), dtype=np.float32))
+    g = W.round_to_fp16(rng.standard_normal((Tq, H, DV), dtype=np.float32))
+    idx, ln = W.topk_lists(Tq, Tkv, 256, 128, 256, 77)   # every list holds >= 128 entries
+    ln[5] = 0
+    ln[6] = 64
+    ln[7] = 65
+    sk = rng.standard_normal(H).astype(np.float32)
+    scale = 1 / math.sqrt(DQK)
+    qd, kvd, gd = to_dev(q, torch.float16), to_dev(kv, torch.float16), to_dev(g, torch.float16)
+    al = eta.AllowedSet(topk_idxs=to_dev(idx, torch.int32), topk_length=to_dev(ln, torch.int32),
+                        sink=to_dev(sk, torch.float32))
+    wf = torch.empty(eta.attn_fwd_workspace_size(qd, kvd, kvd[:, :DV], al), dtype=torch.uint8, device="cuda")
+    o, lse = eta.attn_fwd(qd, kvd, kvd[:, :DV], al, scale, workspace=wf)
+    assert eta.attn_get_status(wf) == 0
+    ws = torch.empty(eta.attn_bwd_workspace_size(qd, kvd, kvd[:, :DV], al), dtype=torch.uint8, device="cuda")
+    dq, dkv, _, ds = eta.attn_bwd(qd, kvd, kvd[:, :DV], o, gd, lse, al, scale, workspace=ws)
+    assert eta.attn_get_status(ws) == 0
+    sink64 = sk.astype(np.float64)
+    o_ref, lse_ref, _ = oracle.topk_forward(q, kv, idx, ln, DV, scale, sink64)
+    _check(to_np(o), to_np(lse), o_ref, lse_ref)
+    dq_ref, dkv_ref, ds_ref = oracle.topk_backward(q, kv, idx, ln, DV, scale, g, sink64, o=o_ref)
+    assert rel_fro(to_np(dq), dq_ref) <= BF16_GRAD_REL
+    assert rel_fro(to_np(dkv), dkv_ref) <= BF16_GRAD_REL
+    assert np.abs(to_np(ds) - ds_ref).max() <= 2e-2 * max(1.0, np.abs(ds_ref).max())
