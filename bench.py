@@ -214,14 +214,15 @@ class Problem:
         self.config, self.bound, self.launches = config, bound, launches
 
 
-def dense_problem(case: W.DenseCase, dev, torch, eta) -> Problem:
+def dense_problem(case: W.DenseCase, dev, torch, eta, deterministic: bool = False) -> Problem:
     q, k, v, g = W.dense_inputs(case)
     tq, tk, tv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v, g))
     bm = W.block_mask(case)
     allowed = eta.AllowedSet(causal=case.causal, window_left=case.window_left,
                              block_mask=torch.from_numpy(bm).to(dev) if bm is not None else None,
                              block_q=case.block_size or 128, block_k=case.block_size or 128,
-                             dropout_p=case.dropout_p, dropout_seed=case.dropout_seed)
+                             dropout_p=case.dropout_p, dropout_seed=case.dropout_seed,
+                             deterministic=deterministic)
     o = torch.empty_like(tq)
     lse = torch.empty(tq.shape[:-1], dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
@@ -232,13 +233,16 @@ def dense_problem(case: W.DenseCase, dev, torch, eta) -> Problem:
         (f", dropout {case.dropout_p}" if case.dropout_p else "")
     config = {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "T": case.T, "d": case.d,
               "dv": case.dv, "mask": mask}
+    if deterministic:
+        config["reverse"] = "deterministic (dQ from the query-centric pass)"
     return Problem(case.name, allowed_pairs(case), 2 * case.d + 2 * case.dv, 6 * case.d + 4 * case.dv,
                    [tq, tk, tv, tg], [dq, dk, dv],
                    lambda: eta.attn_fwd(tq, tk, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
                    lambda: eta.attn_bwd(tq, tk, tv, o, tg, lse, allowed, case.scale, dq=dq, dk=dk, dv=dv,
                                         workspace=ws_b),
                    config, "tensor",
-                   # fwd_kernel; prepare, bwd_kernel, dq_finish; plus a tile-class pass per call
+                   # fwd_kernel; prepare, bwd_kernel, dq_finish (or the query-centric dQ kernel);
+                   # plus a tile-class pass per call
                    # when a block mask is present
                    4 + (2 if bm is not None else 0))
 
@@ -277,6 +281,8 @@ def main():
                     choices=["causal_8k", "causal_2k", "window_block_8k", "gqa_dropout_16k", "topk_shared_kv"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="bitwise reproducible reverse pass (dense workloads)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -303,7 +309,7 @@ def main():
     if args.workload in W.TOPK_WORKLOADS:
         prob = topk_problem(W.TOPK_WORKLOADS[args.workload], dev, torch, eta)
     else:
-        prob = dense_problem(W.WORKLOADS[args.workload], dev, torch, eta)
+        prob = dense_problem(W.WORKLOADS[args.workload], dev, torch, eta, args.deterministic)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 

@@ -43,6 +43,7 @@ ATTN_MASK_LENGTHS = 0x10
 ATTN_MASK_STARTS = 0x20
 ATTN_LSE_KV_ONLY = 0x1
 ATTN_LSE_NEG_LOG2 = 0x2
+ATTN_BWD_DETERMINISTIC = 0x1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -66,7 +67,7 @@ class AttnMaskC(ctypes.Structure):
                 ("sink", ctypes.c_void_p), ("dropout_p", ctypes.c_float),
                 ("dropout_seed", ctypes.c_uint64), ("lengths", ctypes.c_void_p),
                 ("starts", ctypes.c_void_p), ("starts_stride_b", ctypes.c_int64),
-                ("lse_format", ctypes.c_uint32)]
+                ("lse_format", ctypes.c_uint32), ("bwd_flags", ctypes.c_uint32)]
 
 
 _LIB = None
@@ -151,6 +152,7 @@ class AllowedSet:
     allowed key of each query row, e.g. its packed segment's first cell).
     lse_kv_only / lse_neg_log2 select the LSE format that attn_fwd writes
     and attn_bwd expects: the sink left out, and/or stored as -log2 Z.
+    deterministic makes every gradient of attn_bwd bitwise reproducible.
     """
     causal: bool = False
     window_left: int = 0
@@ -167,6 +169,7 @@ class AllowedSet:
     starts: torch.Tensor | None = None
     lse_kv_only: bool = False
     lse_neg_log2: bool = False
+    deterministic: bool = False
 
     def to_c(self) -> AttnMaskC:
         m = AttnMaskC()
@@ -208,6 +211,7 @@ class AllowedSet:
             m.sink = self.sink.data_ptr()
         m.lse_format = (ATTN_LSE_KV_ONLY if self.lse_kv_only else 0) | \
             (ATTN_LSE_NEG_LOG2 if self.lse_neg_log2 else 0)
+        m.bwd_flags = ATTN_BWD_DETERMINISTIC if self.deterministic else 0
         m.dropout_p = float(self.dropout_p)
         m.dropout_seed = int(self.dropout_seed) & 0xFFFFFFFFFFFFFFFF
         m.flags = flags

@@ -62,6 +62,7 @@ attn_status check_mask(const attn_mask* m) {
     if (m->dropout_p != 0.f) return ATTN_ERR_UNSUPPORTED;
   }
   if (m->lse_format & ~(ATTN_LSE_KV_ONLY | ATTN_LSE_NEG_LOG2)) return ATTN_ERR_INVALID_ARG;
+  if (m->bwd_flags & ~ATTN_BWD_DETERMINISTIC) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_LENGTHS) && !m->lengths) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_STARTS) && (!m->starts || m->starts_stride_b < 0)) return ATTN_ERR_INVALID_ARG;
   if (!(m->dropout_p >= 0.f && m->dropout_p < 1.f)) return ATTN_ERR_INVALID_ARG;
@@ -329,6 +330,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.d = s.d;
   p.dv = s.dv;
   p.dtype = q->dtype;
+  p.bwd_flags = mask ? mask->bwd_flags : 0u;
   p.scale = scale;
   p.m = mask_params(mask);
   p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows
@@ -483,6 +485,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   p.d = s.d;
   p.dv = s.dv;
   p.dtype = q->dtype;
+  p.bwd_flags = mask ? mask->bwd_flags : 0u;
   p.scale = scale;
   p.m = mask_params(mask);
   p.m.qoff = (int64_t)s.Tk - s.Tq;  // bottom-right alignment of the query rows

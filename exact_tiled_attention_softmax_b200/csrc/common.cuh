@@ -54,7 +54,8 @@ struct DenseP {
   const void* v;
   int64_t sq[3], sk[3], sv[3];
   int B, Hq, Hkv, Tq, Tk, d, dv;
-  int32_t dtype;  // attn_dtype of every tensor
+  int32_t dtype;       // attn_dtype of every tensor
+  uint32_t bwd_flags;  // ATTN_BWD_* bits
   float scale;
   MaskP m;
 };

@@ -1291,6 +1291,303 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   }
 }
 
+// ---------------------------------------------- deterministic dQ (query-centric)
+//
+// dQ_i = c sum_j gamma_ij K_j evaluated per query tile, key tiles in order,
+// with P and gamma recomputed from the saved statistics ("Tiled attention and
+// its recomputed reverse pass are exact", proof step 7.1: the reverse rebuilds
+// P from the scores and the stored normaliser). Every dQ element is summed by
+// one CTA in a fixed order, so the result is bitwise reproducible; the
+// key-centric kernel then leaves dQ alone.
+//
+// One CTA per (128-row query tile, query head, batch row). Warp 0: TMA
+// producer (Q and dO once, then K/V stages). Warp 1: MMA issuer. Warps 2-9:
+// two warpgroups that split each key tile's columns (warpgroup w: keys
+// 64 w .. 64 w + 63); thread t of a warpgroup owns query row t (TMEM lane t).
+// TMEM: S double-buffered at columns 0 and 128, dP at 256, dQ at 384. gamma
+// (16-bit pairs) is written over the warpgroup's own S columns and read from
+// there by the dQ MMA.
+
+struct DqArgs {
+  FwdArgs f;             // mask, class table, sizes (o, lse unused)
+  const float* lse2;     // [B*Hq, Tpad] minus the base-2 LSE
+  const float* dpad;     // [B*Hq, Tpad] minus delta
+  uint16_t* dq;          // 16-bit storage
+  int64_t sdq[3];
+  float scale;
+  int Tpad;
+};
+
+constexpr uint32_t kDqQ = 0;                              // Q tile
+constexpr uint32_t kDqG = kDqQ + kTileBytes;              // dO tile
+constexpr uint32_t kDqK = kDqG + kTileBytes;              // K stages
+constexpr uint32_t kDqV = kDqK + kStages * kTileBytes;    // V stages
+constexpr uint32_t kDqCtl = kDqV + kStages * kTileBytes;
+constexpr uint32_t kDqSmem = kDqCtl + 1024 + 1024;
+constexpr int kDqThreads = 320;
+
+struct DqCtl {
+  uint64_t q_full;
+  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], dp_full, g_full;
+  uint64_t dq_final;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+// Next key tile after `from` (up to kt_hi) with allowed keys for query tile
+// qt; kt_hi + 1 when none. Every role walks the same sequence.
+__device__ __forceinline__ int dq_next_tile(const FwdArgs& a, int b, int h, int qt, int kt_hi, int from) {
+  for (int kt = from + 1; kt <= kt_hi; ++kt)
+    if (wg_class(a, b, h, qt, kt) != kEmpty) return kt;
+  return kt_hi + 1;
+}
+
+template <bool kH>
+__global__ void __launch_bounds__(kDqThreads, 1)
+dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg, const DqArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  DqCtl* ctl = reinterpret_cast<DqCtl*>(smem + kDqCtl);
+  volatile uint32_t* abort_flag = &ctl->abort_flag;
+  const FwdArgs& f = a.f;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqt = (f.Tq + kBM - 1) / kBM;
+  const int bh = blockIdx.x % (f.B * f.Hq);
+  const int qt = nqt - 1 - (int)(blockIdx.x / (f.B * f.Hq));  // longest rows first
+  const int h = bh % f.Hq, b = bh / f.Hq;
+  const int kvh = h / (f.Hq / f.Hkv);
+  const int q0 = qt * kBM;
+  int kt_lo, kt_hi;
+  fwd_key_tiles(f.m, b, f.Tq, f.Tk, q0, kBM, kt_lo, kt_hi);
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&ctl->q_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl->k_full[s]), 1);
+      mbar_init(smem_u32(&ctl->v_full[s]), 1);
+      mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->s_full[0]), 1);
+    mbar_init(smem_u32(&ctl->s_full[1]), 1);
+    mbar_init(smem_u32(&ctl->dp_full), 1);
+    mbar_init(smem_u32(&ctl->g_full), 8);  // one arrival per compute warp
+    mbar_init(smem_u32(&ctl->dq_final), 1);
+    ctl->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const int first = dq_next_tile(f, b, h, qt, kt_hi, kt_lo - 1);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&tg);
+    const uint32_t qf = smem_u32(&ctl->q_full);
+    mbar_expect_tx(qf, 2 * kTileBytes);
+    tma_load_4d(sbase + kDqQ, &tq, qf, 0, q0, h, b);
+    tma_load_4d(sbase + kDqQ + kTileBytes / 2, &tq, qf, 64, q0, h, b);
+    tma_load_4d(sbase + kDqG, &tg, qf, 0, q0, h, b);
+    tma_load_4d(sbase + kDqG + kTileBytes / 2, &tg, qf, 64, q0, h, b);
+    int n = 0;
+    for (int kt = first; kt <= kt_hi; kt = dq_next_tile(f, b, h, qt, kt_hi, kt), ++n) {
+      const int s = n % kStages;
+      if (!wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kStages) & 1) ^ 1, abort_flag, f.status)) break;
+      const uint32_t kf = smem_u32(&ctl->k_full[s]), vf = smem_u32(&ctl->v_full[s]);
+      const uint32_t kd = sbase + kDqK + s * kTileBytes, vd = sbase + kDqV + s * kTileBytes;
+      mbar_expect_tx(kf, kTileBytes);
+      tma_load_4d(kd, &tk, kf, 0, kt * kBN, kvh, b);
+      tma_load_4d(kd + kTileBytes / 2, &tk, kf, 64, kt * kBN, kvh, b);
+      mbar_expect_tx(vf, kTileBytes);
+      tma_load_4d(vd, &tv, vf, 0, kt * kBN, kvh, b);
+      tma_load_4d(vd + kTileBytes / 2, &tv, vf, 64, kt * kBN, kvh, b);
+    }
+    for (int r = (n > kStages ? n - kStages : 0); r < n; ++r) {
+      const int s = r % kStages;
+      wait_bar(smem_u32(&ctl->k_full[s]), (r / kStages) & 1, abort_flag, nullptr);
+      wait_bar(smem_u32(&ctl->v_full[s]), (r / kStages) & 1, abort_flag, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idS = idesc16<kH>(128, 128, 0, 0);   // Q K^T and dO V^T
+    constexpr uint32_t idDQ = idesc16<kH>(128, 128, 0, 1);  // gamma K (B = K, d contiguous)
+    const uint64_t dQ0 = smem_desc_sw128(sbase + kDqQ, 16, 1024), dG0 = smem_desc_sw128(sbase + kDqG, 16, 1024);
+    const uint64_t dK0 = smem_desc_sw128(sbase + kDqK, 16, 1024), dV0 = smem_desc_sw128(sbase + kDqV, 16, 1024);
+    const uint64_t dKmn0 = smem_desc_sw128(sbase + kDqK, kTileBytes / 2, 1024);
+    constexpr uint64_t kTileStep = kTileBytes >> 4;
+    auto kstep = [](int kk) { return (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4); };
+    auto issue_s = [&](int stage, int buf) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tmem + buf * 128, dQ0 + kstep(kk), dK0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
+      mma_commit(smem_u32(&ctl->s_full[buf]));
+    };
+    auto issue_dp = [&](int stage) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tmem + 256, dG0 + kstep(kk), dV0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
+      mma_commit(smem_u32(&ctl->dp_full));
+    };
+    bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, f.status);
+    int n = 0;
+    if (ok && first <= kt_hi) {
+      ok = wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, f.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        ok = wait_bar(smem_u32(&ctl->v_full[0]), 0, abort_flag, f.status);
+        if (ok) {
+          tc_fence_after();
+          issue_dp(0);
+        }
+      }
+    }
+    for (int kt = first; ok && kt <= kt_hi; ++n) {
+      const int nk = dq_next_tile(f, b, h, qt, kt_hi, kt);
+      const int s = n % kStages, s1 = (n + 1) % kStages;
+      const bool more = nk <= kt_hi;
+      if (more) {  // S of the next tile into the other buffer while the warps work on this one
+        if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, f.status))) break;
+        tc_fence_after();
+        issue_s(s1, (n + 1) & 1);
+      }
+      if (!(ok = wait_bar(smem_u32(&ctl->g_full), n & 1, abort_flag, f.status))) break;
+      tc_fence_after();
+      // dQ += gamma K: keys 16 kk .. 16 kk + 15 of warpgroup kk >> 2, 8 packed columns per step.
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(tmem + 384, tmem + (n & 1) * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
+               dKmn0 + (uint64_t)s * kTileStep + (uint64_t)(kk * (2048 >> 4)), idDQ, (n > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(smem_u32(&ctl->kv_empty[s]));
+      if (more) {
+        if (!(ok = wait_bar(smem_u32(&ctl->v_full[s1]), ((n + 1) / kStages) & 1, abort_flag, f.status))) break;
+        tc_fence_after();
+        issue_dp(s1);
+      }
+      kt = nk;
+    }
+    mma_commit(smem_u32(&ctl->dq_final));
+  } else if (warp >= 2) {
+    // ---------------- compute warpgroups
+    const int w = (warp - 2) >> 2;               // key columns 64 w .. 64 w + 63
+    const int t = ((warp & 3) << 5) | lane;      // query row within the tile = TMEM lane
+    const int64_t row = (int64_t)q0 + t;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int64_t srow = ((int64_t)b * f.Hq + h) * a.Tpad + row;  // row < Tpad = 128 * nqt
+    const float nlse2 = row < f.Tq ? a.lse2[srow] : -INFINITY;  // -log2 Z (-inf: no keys)
+    const float ndelta = row < f.Tq ? a.dpad[srow] : 0.f;       // -delta
+    const float dscale = f.m.dropout ? f.m.inv_keep : 1.f;
+    const uint8_t slice_tile_shift = (uint8_t)(t >> 6);         // this row's 64-row slice in the tile
+    int n = 0;
+    bool ok = true;
+    for (int kt = first; ok && kt <= kt_hi; kt = dq_next_tile(f, b, h, qt, kt_hi, kt), ++n) {
+      const uint8_t cls = wg_class(f, b, h, qt, kt);
+      uint64_t mw = ~0ull, kw = ~0ull;
+      if (cls == kPartial) {
+        uint64_t w0 = 0ull, w1 = 0ull;
+        if (row < f.Tq) {
+          const uint8_t scls = lookup_class(f.ct, f.m, f.Tq, f.Tk, b, h, 2 * qt + slice_tile_shift, kt);
+          fwd_row_bits(f, b, h, row, (int64_t)kt * kBN, scls, w0, w1);
+        }
+        mw = w ? w1 : w0;
+      }
+      if (f.m.dropout) {
+        uint64_t k0, k1;
+        fwd_keep_bits(f.m, b, h, row, (int64_t)kt * kBN, k0, k1);
+        kw = w ? k1 : k0;
+      }
+      const uint32_t tS = tmem + lane_off + (n & 1) * 128 + 64 * w;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[n & 1]), (n >> 1) & 1, abort_flag, f.status));
+      if (!ok) break;
+      tc_fence_after();
+      float p[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tS, r0);
+        tmem_ld32(tS + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          p[e] = ((mw >> e) & 1ull) ? ex2(fmaf(__uint_as_float(r0[e]), f.scale_log2, nlse2)) : 0.f;
+          p[32 + e] = ((mw >> (32 + e)) & 1ull) ? ex2(fmaf(__uint_as_float(r1[e]), f.scale_log2, nlse2)) : 0.f;
+        }
+      }
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dp_full), n & 1, abort_flag, f.status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tP = tmem + lane_off + 256 + 64 * w;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r[32];
+        tmem_ld32(tP + 32 * hh, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * hh + 2 * e, c1 = c0 + 1;
+          const float d0 = ((kw >> c0) & 1ull) ? __uint_as_float(r[2 * e]) * dscale : 0.f;
+          const float d1 = ((kw >> c1) & 1ull) ? __uint_as_float(r[2 * e + 1]) * dscale : 0.f;
+          pk[e] = pack16<kH>(p[c0] * (d0 + ndelta), p[c1] * (d1 + ndelta));
+        }
+        // gamma over this warpgroup's own S columns (already read above).
+        tmem_st16(tS + 16 * hh, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->g_full));
+    }
+    // ---------------- epilogue: dQ = c * accumulator; warpgroup w writes d columns 64 w .. 64 w + 63
+    bool have = false;
+    if (ok && n > 0) {
+      have = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_final), 0, abort_flag, f.status));
+      if (have) tc_fence_after();
+    }
+    if (ok || n == 0) {
+      uint16_t* drow = a.dq + b * a.sdq[0] + h * a.sdq[1] + row * a.sdq[2] + 64 * w;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        if (have) {
+          tmem_ld32(tmem + lane_off + 384 + 64 * w + 32 * c, r);
+          tmem_wait_ld();
+        }
+        if (row < f.Tq) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int idx = c8 * 8 + 2 * e;
+              pk[e] = have ? pack16<kH>(__uint_as_float(r[idx]) * a.scale, __uint_as_float(r[idx + 1]) * a.scale)
+                           : 0u;
+            }
+            *reinterpret_cast<uint4*>(drow + 32 * c + 8 * c8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // Reverse-pass preparation, one warp per (b, h, row < Tpad): delta from the
 // stored O and dO (kept, and negated in the padded array), the negated base-2
 // LSE, and a zeroed dQ accumulator row.
@@ -1415,7 +1712,7 @@ bool tma_ok(const attn_tensor* t) {
 
 // Raise a kernel's dynamic shared-memory limit once per device.
 cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
-  static bool done[4][64] = {};
+  static bool done[6][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1580,6 +1877,38 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   kern<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
   main_kernel_end(st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (p.bwd_flags & ATTN_BWD_DETERMINISTIC) {
+    // dQ from the query-centric pass: one CTA sums each element in key order.
+    CUtensorMap dq_mq, dq_mg;
+    if (!make_map(&dq_mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBM, f16) ||
+        !make_map(&dq_mg, g, p.Tq, p.Hq, p.B, sg[2], sg[1], sg[0], kBM, f16))
+      return cudaErrorInvalidValue;
+    DqArgs d;
+    d.f.m = p.m;
+    d.f.ct = ct;
+    d.f.block_aligned = block_aligned(p.m);
+    d.f.B = p.B;
+    d.f.Hq = p.Hq;
+    d.f.Hkv = p.Hkv;
+    d.f.Tq = p.Tq;
+    d.f.Tk = p.Tk;
+    d.f.scale_log2 = p.scale * kLog2e;
+    d.f.o = nullptr;
+    d.f.lse = nullptr;
+    for (int i = 0; i < 3; ++i) d.f.so[i] = d.f.sl[i] = 0;
+    d.f.status = status;
+    d.lse2 = lse2;
+    d.dpad = dpad;
+    d.dq = static_cast<uint16_t*>(dq);
+    for (int i = 0; i < 3; ++i) d.sdq[i] = sdq[i];
+    d.scale = p.scale;
+    d.Tpad = Tpad;
+    auto kdq = f16 ? dq_kernel<true> : dq_kernel<false>;
+    if ((err = set_smem_attr(reinterpret_cast<const void*>(kdq), kDqSmem, f16 ? 5 : 4)) != cudaSuccess) return err;
+    const int nqt = (p.Tq + kBM - 1) / kBM;
+    kdq<<<nqt * p.B * p.Hq, kDqThreads, kDqSmem, st>>>(dq_mq, mk, mv, dq_mg, d);
+    return cudaGetLastError();
+  }
   const int64_t n4 = (int64_t)p.B * p.Hq * p.Tq * kD / 4;
   (f16 ? dq_finish_kernel<true> : dq_finish_kernel<false>)<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
       dq_acc, p.B, p.Hq, p.Tq, p.scale, static_cast<uint16_t*>(dq), sdq[0], sdq[1], sdq[2]);

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 105 /* major * 100 + minor */
+#define ATTN_VERSION 106 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -142,7 +142,17 @@ typedef struct attn_mask {
    * the sink-inclusive denominator Z (section 7.1), or a combination of the
    * ATTN_LSE_* bits below. attn_bwd must be given the format attn_fwd wrote. */
   uint32_t lse_format;
+  /* Options of attn_bwd: 0 or ATTN_BWD_DETERMINISTIC. */
+  uint32_t bwd_flags;
 } attn_mask;
+
+/* ATTN_BWD_DETERMINISTIC: every gradient is bitwise reproducible from run to
+ * run. dK, dV and the top-k dKV always are (one CTA per key tile, or a
+ * fixed-point accumulator); with this flag the dense tensor-core path also
+ * computes dQ in a query-centric pass (one CTA sums each dQ element over the
+ * key tiles in order, recomputing P and gamma) instead of reducing per-key-
+ * tile partials with floating-point atomics. Costs one extra pass. */
+#define ATTN_BWD_DETERMINISTIC 0x1u
 
 /* ATTN_LSE_KV_ONLY: the denominator leaves the sink out, ln sum_j exp(s_j)
  * (section 7.2; -inf for an empty allowed set even with a sink). The reverse
