@@ -924,7 +924,9 @@ __device__ __forceinline__ void bulk_wait_read0() {
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-template <bool kH>
+// kDQ = false (the deterministic mode) leaves dQ to the query-centric pass:
+// no dQ^T product, no dQ warpgroup work.
+template <bool kH, bool kDQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
@@ -1057,7 +1059,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint32_t par = (m >> 1) & 1;
       if (!wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)) return false;
       info = ctl->qinfo[sq][0];
-      if (!wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
+      if (kDQ && !wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
       tc_fence_after();
       const uint32_t dst = tmem + s * 128;
 #pragma unroll
@@ -1095,12 +1097,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       for (int kk = 0; kk < 4; ++kk)
         mma_ss(tDK, dDS(s) + (uint64_t)(kk * (32 >> 4)), dQmn(sq) + (uint64_t)(kk * (2048 >> 4)), idACC,
                (n > 0 || kk > 0) ? 1u : 0u);
+      if constexpr (kDQ) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
-        mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
-               kk > 0);
+        for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
+          mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
+                 kk > 0);
+      }
       mma_commit(smem_u32(&ctl->q_empty[sq]));
-      mma_commit(smem_u32(&ctl->dq_full[s]));
+      if constexpr (kDQ) mma_commit(smem_u32(&ctl->dq_full[s]));
       have = next;
       info = ninfo;
       ++n;
@@ -1238,7 +1242,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
       }
     }
-  } else if (warp >= 12) {
+  } else if (kDQ && warp >= 12) {
     // ---------------- dQ warpgroup: warp wq reads head-dimension indices
     // 32 wq .. 32 wq + 31 of the dQ^T tile (its TMEM lanes), stages them as a
     // [64 rows][32] fp32 box and adds the box into the fp32 accumulator with
@@ -1489,18 +1493,33 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
     const float nlse2 = row < f.Tq ? a.lse2[srow] : -INFINITY;  // -log2 Z (-inf: no keys)
     const float ndelta = row < f.Tq ? a.dpad[srow] : 0.f;       // -delta
     const float dscale = f.m.dropout ? f.m.inv_keep : 1.f;
-    const uint8_t slice_tile_shift = (uint8_t)(t >> 6);         // this row's 64-row slice in the tile
+    const int slice = 2 * qt + ((warp & 3) >> 1);               // this warp's 64-row slice
+    const uint64_t sc2 = f2_pack(f.scale_log2, f.scale_log2), nl2 = f2_pack(nlse2, nlse2);
+    const uint64_t nd2 = f2_pack(ndelta, ndelta);
     int n = 0;
     bool ok = true;
-    for (int kt = first; ok && kt <= kt_hi; kt = dq_next_tile(f, b, h, qt, kt_hi, kt), ++n) {
-      const uint8_t cls = wg_class(f, b, h, qt, kt);
+    // Tile classes, 32 key tiles per round: lane l holds tile cbase + l
+    // (bits 0-1: the query tile's class, bits 2-3: this warp's slice).
+    int cbase = kt_lo - 32;
+    uint32_t cword = 0;
+    for (int kt = kt_lo; ok && kt <= kt_hi; ++kt) {
+      if (kt - cbase >= 32) {
+        cbase = kt;
+        const int mk = kt + lane;
+        cword = 0;
+        if (mk <= kt_hi) {
+          cword = wg_class(f, b, h, qt, mk);
+          if (cword == kPartial) cword |= ((uint32_t)lookup_class(f.ct, f.m, f.Tq, f.Tk, b, h, slice, mk) & 3u) << 2;
+        }
+      }
+      const uint32_t cv = __shfl_sync(0xffffffffu, cword, kt - cbase);
+      const uint8_t cls = cv & 3u;
+      if (cls == kEmpty) continue;
+      const bool plain = cls == kFull && !f.m.dropout;
       uint64_t mw = ~0ull, kw = ~0ull;
       if (cls == kPartial) {
         uint64_t w0 = 0ull, w1 = 0ull;
-        if (row < f.Tq) {
-          const uint8_t scls = lookup_class(f.ct, f.m, f.Tq, f.Tk, b, h, 2 * qt + slice_tile_shift, kt);
-          fwd_row_bits(f, b, h, row, (int64_t)kt * kBN, scls, w0, w1);
-        }
+        if (row < f.Tq) fwd_row_bits(f, b, h, row, (int64_t)kt * kBN, (uint8_t)(cv >> 2), w0, w1);
         mw = w ? w1 : w0;
       }
       if (f.m.dropout) {
@@ -1518,10 +1537,23 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
         tmem_ld32(tS, r0);
         tmem_ld32(tS + 32, r1);
         tmem_wait_ld();
+        if (plain) {  // P = 2^(s c log2(e) - log2 Z) on packed pairs
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          p[e] = ((mw >> e) & 1ull) ? ex2(fmaf(__uint_as_float(r0[e]), f.scale_log2, nlse2)) : 0.f;
-          p[32 + e] = ((mw >> (32 + e)) & 1ull) ? ex2(fmaf(__uint_as_float(r1[e]), f.scale_log2, nlse2)) : 0.f;
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1, y0, y1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1])), sc2, nl2), x0, x1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1])), sc2, nl2), y0, y1);
+            p[2 * e] = ex2(x0);
+            p[2 * e + 1] = ex2(x1);
+            p[32 + 2 * e] = ex2(y0);
+            p[32 + 2 * e + 1] = ex2(y1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            p[e] = ((mw >> e) & 1ull) ? ex2(fmaf(__uint_as_float(r0[e]), f.scale_log2, nlse2)) : 0.f;
+            p[32 + e] = ((mw >> (32 + e)) & 1ull) ? ex2(fmaf(__uint_as_float(r1[e]), f.scale_log2, nlse2)) : 0.f;
+          }
         }
       }
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dp_full), n & 1, abort_flag, f.status));
@@ -1534,12 +1566,24 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
         tmem_ld32(tP + 32 * hh, r);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (!f.m.dropout) {  // gamma = P (dP - delta) on packed pairs
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * hh + 2 * e, c1 = c0 + 1;
-          const float d0 = ((kw >> c0) & 1ull) ? __uint_as_float(r[2 * e]) * dscale : 0.f;
-          const float d1 = ((kw >> c1) & 1ull) ? __uint_as_float(r[2 * e + 1]) * dscale : 0.f;
-          pk[e] = pack16<kH>(p[c0] * (d0 + ndelta), p[c1] * (d1 + ndelta));
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * hh + 2 * e;
+            const uint64_t g2 = f2_mul(f2_pack(p[c0], p[c0 + 1]),
+                                       f2_add(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), nd2));
+            float g0, g1;
+            f2_unpack(g2, g0, g1);
+            pk[e] = pack16<kH>(g0, g1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * hh + 2 * e, c1 = c0 + 1;
+            const float d0 = ((kw >> c0) & 1ull) ? __uint_as_float(r[2 * e]) * dscale : 0.f;
+            const float d1 = ((kw >> c1) & 1ull) ? __uint_as_float(r[2 * e + 1]) * dscale : 0.f;
+            pk[e] = pack16<kH>(p[c0] * (d0 + ndelta), p[c1] * (d1 + ndelta));
+          }
         }
         // gamma over this warpgroup's own S columns (already read above).
         tmem_st16(tS + 16 * hh, pk);
@@ -1548,6 +1592,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->g_full));
+      ++n;
     }
     // ---------------- epilogue: dQ = c * accumulator; warpgroup w writes d columns 64 w .. 64 w + 63
     bool have = false;
@@ -1710,9 +1755,11 @@ bool tma_ok(const attn_tensor* t) {
   return true;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device.
+// Raise a kernel's dynamic shared-memory limit once per device. which: 0/2
+// forward bf16/fp16, 1/3 reverse, 4/5 query-centric dQ, 6/7 reverse without dQ.
 cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
-  static bool done[6][64] = {};
+  static bool done[8][64] = {};
+  if (which < 0 || which >= 8) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1870,8 +1917,12 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   }
   a.scale = p.scale;
   a.status = status;
-  auto kern = f16 ? bwd_kernel<true> : bwd_kernel<false>;
-  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kBwdSmem, f16 ? 3 : 1)) != cudaSuccess) return err;
+  const bool det = p.bwd_flags & ATTN_BWD_DETERMINISTIC;
+  auto kern = f16 ? (det ? bwd_kernel<true, false> : bwd_kernel<true, true>)
+                  : (det ? bwd_kernel<false, false> : bwd_kernel<false, true>);
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kBwdSmem, det ? (f16 ? 7 : 6) : (f16 ? 3 : 1))) !=
+      cudaSuccess)
+    return err;
   const int nkt = (p.Tk + kBN - 1) / kBN;
   main_kernel_begin(st);
   kern<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
