@@ -357,8 +357,9 @@ __device__ __forceinline__ float move_max(float mx, float& m_run) {
 // the maximum and the exponentials (one TMEM wait); x = s c log2(e) - m is
 // formed on packed fp32 pairs and every kPolyEvery-th pair of exponentials
 // runs on the FMA pipe instead of MUFU. Returns alpha.
-template <bool kH>
-__device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2, float& m_run, float& l_run) {
+template <bool kH, bool kDrop>
+__device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2, float& m_run, float& l_run,
+                                                   uint64_t kb0, uint64_t kb1) {
   uint32_t s0[32], s1[32], s2[32], s3[32];
   tmem_ld32(tS, s0);
   tmem_ld32(tS + 32, s1);
@@ -407,6 +408,12 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
         acc0 = f2_add(acc0, pp);
       float p0, p1;
       f2_unpack(pp, p0, p1);
+      if constexpr (kDrop) {  // xi only in the P operand; the sum keeps every term
+        const uint64_t kw = q < 2 ? kb0 : kb1;
+        const int bit = (q & 1) * 32 + 2 * e;
+        p0 = ((kw >> bit) & 1ull) ? p0 : 0.f;
+        p1 = ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f;
+      }
       pk[e] = pack16<kH>(p0, p1);
     }
     tmem_st16(tS + q * 16, pk);
@@ -476,7 +483,7 @@ __device__ __forceinline__ float softmax_masked_tile(uint32_t tS, float scale_lo
 // into the warpgroup's own S columns of TMEM and read from there by the PV
 // MMA; S of the next tile lands in the same columns only after that PV, in
 // issue order.
-template <bool kH>
+template <bool kH, bool kDrop>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
@@ -665,13 +672,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (row < a.Tq) fwd_row_bits(a, b, h, row, (int64_t)kt * kBN, (uint8_t)(cv >> 2), mw0, mw1);
       }
       uint64_t kb0 = ~0ull, kb1 = ~0ull;
-      if (a.m.dropout) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
+      if constexpr (kDrop) fwd_keep_bits(a.m, b, h, row, (int64_t)kt * kBN, kb0, kb1);
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->s_full[w]), n & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
       float alpha;
-      if (cls == kFull && !a.m.dropout)
-        alpha = softmax_full_tile<kH>(tS, a.scale_log2, m_run, l_run);
+      if (cls == kFull)
+        alpha = softmax_full_tile<kH, kDrop>(tS, a.scale_log2, m_run, l_run, kb0, kb1);
       else
         alpha = softmax_masked_tile<kH>(tS, a.scale_log2, mw0, mw1, kb0, kb1, m_run, l_run);
       // Every earlier P V of this warpgroup has completed (the S commit covers
@@ -926,7 +933,7 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 // kDQ = false (the deterministic mode) leaves dQ to the query-centric pass:
 // no dQ^T product, no dQ warpgroup work.
-template <bool kH, bool kDQ>
+template <bool kH, bool kDQ, bool kDrop>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
@@ -1138,9 +1145,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint8_t cls = (uint8_t)((info >> 28) & 3u);
       more = info & (1u << 30);
       const int64_t i0 = (int64_t)qs * kBMb;
-      const bool general = cls == kPartial || a.m.dropout;
+      const bool general = cls == kPartial;
       const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
-      const uint32_t keep = a.m.dropout ? bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j) : ~0u;
+      uint32_t keep = ~0u;
+      if constexpr (kDrop) keep = bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j);
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
       tc_fence_after();
       uint32_t rs[32], rp[32];
@@ -1166,9 +1174,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0, x1);
             const float p0 = ex2(x0), p1 = ex2(x1);
-            ppk[c2] = pack16<kH>(p0, p1);
-            const uint64_t g = f2_mul(f2_pack(p0, p1),
-                                      f2_add(f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1])), dp[e]));
+            uint64_t dv2 = f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1]));
+            if constexpr (kDrop) {  // xi in the P~ operand and in dP; p itself stays undropped
+              const bool k0 = (keep >> (2 * c2)) & 1u, k1 = (keep >> (2 * c2 + 1)) & 1u;
+              ppk[c2] = pack16<kH>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
+              dv2 = f2_pack(k0 ? __uint_as_float(rp[2 * c2]) * a.m.inv_keep : 0.f,
+                            k1 ? __uint_as_float(rp[2 * c2 + 1]) * a.m.inv_keep : 0.f);
+            } else {
+              ppk[c2] = pack16<kH>(p0, p1);
+            }
+            const uint64_t g = f2_mul(f2_pack(p0, p1), f2_add(dv2, dp[e]));
             float g0, g1;
             f2_unpack(g, g0, g1);
             dpk[c2] = pack16<kH>(g0, g1);
@@ -1755,11 +1770,12 @@ bool tma_ok(const attn_tensor* t) {
   return true;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device. which: 0/2
-// forward bf16/fp16, 1/3 reverse, 4/5 query-centric dQ, 6/7 reverse without dQ.
+// Raise a kernel's dynamic shared-memory limit once per device. which names
+// the kernel instantiation, one slot each: forward 0-3, query-centric dQ 4-5,
+// reverse 8-15.
 cudaError_t set_smem_attr(const void* fn, uint32_t bytes, int which) {
-  static bool done[8][64] = {};
-  if (which < 0 || which >= 8) return cudaErrorInvalidValue;
+  static bool done[16][64] = {};
+  if (which < 0 || which >= 16) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1862,8 +1878,12 @@ cudaError_t sm100_dense_fwd(const DenseP& p, void* o, const int64_t so[3], float
   }
   a.lse = lse;
   a.status = status;
-  auto kern = f16 ? fwd_kernel<true> : fwd_kernel<false>;
-  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kFwdSmem, f16 ? 2 : 0)) != cudaSuccess) return err;
+  const bool drop = p.m.dropout != 0;
+  auto kern = f16 ? (drop ? fwd_kernel<true, true> : fwd_kernel<true, false>)
+                  : (drop ? fwd_kernel<false, true> : fwd_kernel<false, false>);
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kFwdSmem, (f16 ? 1 : 0) + (drop ? 2 : 0))) !=
+      cudaSuccess)
+    return err;
   const int nct = (p.Tq + kFwdRows - 1) / kFwdRows;
   main_kernel_begin(st);
   kern<<<nct * p.B * p.Hq, kFwdThreads, kFwdSmem, st>>>(mq, mk, mv, a);
@@ -1917,12 +1937,17 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   }
   a.scale = p.scale;
   a.status = status;
-  const bool det = p.bwd_flags & ATTN_BWD_DETERMINISTIC;
-  auto kern = f16 ? (det ? bwd_kernel<true, false> : bwd_kernel<true, true>)
-                  : (det ? bwd_kernel<false, false> : bwd_kernel<false, true>);
-  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kBwdSmem, det ? (f16 ? 7 : 6) : (f16 ? 3 : 1))) !=
-      cudaSuccess)
-    return err;
+  const bool det = p.bwd_flags & ATTN_BWD_DETERMINISTIC, drop = p.m.dropout != 0;
+  using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                         const CUtensorMap, const BwdArgs);
+  // [fp16][no dQ][dropout]
+  const BwdFn table[2][2][2] = {{{bwd_kernel<false, true, false>, bwd_kernel<false, true, true>},
+                                 {bwd_kernel<false, false, false>, bwd_kernel<false, false, true>}},
+                                {{bwd_kernel<true, true, false>, bwd_kernel<true, true, true>},
+                                 {bwd_kernel<true, false, false>, bwd_kernel<true, false, true>}}};
+  auto kern = table[f16][det][drop];
+  const int which = 8 + (f16 ? 4 : 0) + (det ? 2 : 0) + (drop ? 1 : 0);  // 8 .. 15
+  if ((err = set_smem_attr(reinterpret_cast<const void*>(kern), kBwdSmem, which)) != cudaSuccess) return err;
   const int nkt = (p.Tk + kBN - 1) / kBN;
   main_kernel_begin(st);
   kern<<<nkt * p.B * p.Hkv, kBwdThreads, kBwdSmem, st>>>(mq, mk, mv, mg, mdq, a);
