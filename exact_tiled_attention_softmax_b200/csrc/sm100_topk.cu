@@ -706,6 +706,8 @@ constexpr uint32_t kCGP = kCDO + 8 * kTPlane;        // 2 stages x (G, P) tiles 
 constexpr uint32_t kCRow = kCGP + 2 * 2 * kTPlane;   // 2 stages x 64 KV rows (-1: not listed / invalid)
 constexpr uint32_t kCCtl = kCRow + 2 * kTK * 4;
 constexpr uint32_t kCSmem = kCCtl + 256 + 1024;
+constexpr int kCDrain = 16;                 // draining warps: four per TMEM lane quarter
+constexpr int kCThreads = 64 + 32 * kCDrain;  // producer, MMA issuer, draining warps
 
 struct TopkDkvCtl {
   uint64_t qdo_full, gp_full[2], gp_empty[2], c_full, c_empty;
@@ -724,7 +726,7 @@ struct TopkDkvArgs {
 };
 
 template <bool kH>
-__global__ void __launch_bounds__(kTThreads, 1)
+__global__ void __launch_bounds__(kCThreads, 1)
 topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                     const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tp,
                     const TopkDkvArgs a) {
@@ -743,10 +745,10 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     mbar_init(smem_u32(&ctl->qdo_full), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->gp_full[s]), 1);
-      mbar_init(smem_u32(&ctl->gp_empty[s]), 4);  // released by the draining warps: krow is theirs too
+      mbar_init(smem_u32(&ctl->gp_empty[s]), kCDrain);  // released by the draining warps: krow is theirs too
     }
     mbar_init(smem_u32(&ctl->c_full), 1);
-    mbar_init(smem_u32(&ctl->c_empty), 4);  // one arrival per draining warp
+    mbar_init(smem_u32(&ctl->c_empty), kCDrain);  // one arrival per draining warp
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -833,7 +835,10 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   } else if (warp >= 2) {
     // ---------------- drain: lane l of quarter qt holds column 128 c + 32 qt + l
     // of chunk c (and 512 + 16 qt + l of chunk 4 when l < 16) for all 64 keys.
-    const int qt = warp & 3;
+    // The four warps of a quarter split the work: keys 32 kh .. 32 kh + 31 of
+    // the even (cp = 0) or odd (cp = 1) chunks, so that many reductions are in
+    // flight at once.
+    const int qt = warp & 3, kq = (warp - 2) >> 2, kh = kq & 1, cp = kq >> 1;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
     bool ok = true, sat = false;
     for (int n = 0; n < ntiles && ok; ++n) {
@@ -845,10 +850,9 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       tc_fence_after();
       const int32_t* rows = krow + s * kTK;
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tq4 + 64 * c, v0);
-        tmem_ld32(tq4 + 64 * c + 32, v1);
+      for (int c = cp; c < 5; c += 2) {
+        uint32_t v0[32];
+        tmem_ld32(tq4 + 64 * c + 32 * kh, v0);
         tmem_wait_ld();
         const int col = c < 4 ? 128 * c + 32 * qt + lane : 512 + 16 * qt + lane;
         if (c == 4 && lane >= 16) continue;
@@ -866,8 +870,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
             atomicAdd(a.acc + (int64_t)j * a.Dqk + col, (unsigned long long)__float2ll_rn(x * 4294967296.f));
           }
         };
-        add(v0, 0);
-        add(v1, 32);
+        add(v0, 32 * kh);
       }
       tc_fence_before();
       __syncwarp();
@@ -1007,7 +1010,7 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   main_kernel_begin(st);
   kdq<<<p.Tq, kTThreads, kBSmem, st>>>(mkv, mdo, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kdkv<<<p.Tq, kTThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
+  kdkv<<<p.Tq, kCThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
   main_kernel_end(st);
   return cudaGetLastError();
 }
