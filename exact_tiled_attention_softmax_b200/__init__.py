@@ -15,7 +15,7 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "AllowedSet", "AttnError", "attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_fwd_workspace_size",
+    "AllowedSet", "AttentionFunction", "AttnError", "attention", "attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_fwd_workspace_size",
     "attn_bwd_workspace_size", "attn_get_status", "attn_set_kernel_events", "attn_status_string",
     "attn_version", "library_path", "load_library",
 ]
@@ -341,3 +341,39 @@ def attn_set_kernel_events(begin: "torch.cuda.Event | None", end: "torch.cuda.Ev
         if not ev.cuda_event:
             ev.record()
     load_library().attn_set_kernel_events(ctypes.c_void_p(begin.cuda_event), ctypes.c_void_p(end.cuda_event))
+
+
+class AttentionFunction(torch.autograd.Function):
+    """attn_fwd / attn_bwd as one autograd node. Saves Q, K, V, O and the LSE
+    (never P); the reverse pass recomputes the scores tile by tile.
+
+    Inputs: q, k, v, sink (float32 [Hq] or None, so that its gradient is
+    routed), the allowed set and the scale. Outputs: O and the LSE; the LSE is
+    not differentiable through this node. Top-k (shared KV): pass k = KV and
+    v = KV[:, :Dv]; the whole dKV comes back as k's gradient and v's is None,
+    so a KV leaf that both were sliced from receives the tied gradient once.
+    """
+
+    @staticmethod
+    def forward(ctx, q, k, v, sink, allowed, scale):
+        import dataclasses
+        al = dataclasses.replace(allowed, sink=sink.detach() if sink is not None else None)
+        o, lse = attn_fwd(q, k, v, al, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.allowed, ctx.scale, ctx.has_sink = al, scale, sink is not None
+        ctx.mark_non_differentiable(lse)
+        return o, lse
+
+    @staticmethod
+    def backward(ctx, d_o, d_lse):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv, dsink = attn_bwd(q, k, v, o, d_o.contiguous(), lse, ctx.allowed, ctx.scale)
+        return dq, dk, dv, (dsink if ctx.has_sink else None), None, None
+
+
+def attention(q, k, v, allowed: AllowedSet | None = None, scale: float | None = None, sink=None):
+    """Differentiable exact masked attention: returns (O, LSE). The allowed
+    set's own sink field is ignored here; pass the sink tensor as `sink`."""
+    if scale is None:
+        scale = q.shape[-1] ** -0.5
+    return AttentionFunction.apply(q, k, v, sink, allowed if allowed is not None else AllowedSet(), scale)
