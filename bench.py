@@ -203,6 +203,25 @@ def run_reference(args, case, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank contributes its device-timed total
+    and all of them receive the maximum (one all-reduce, identical on every
+    rank). Replicas run independent problems, so the whole job ends when the
+    slowest one does."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the work every rank did over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (max_ms / 1e3) / 1e12
+
+
 class Problem:
     """One workload on the device: the fwd and bwd calls through the public
     binding, their inputs (for the end-to-end copies) and outputs, and the
@@ -357,15 +376,11 @@ def main():
     t_bwd = [b.elapsed_time(c) for _, b, c in ev]
     t_fwd_kernel = [k0.elapsed_time(k1) for k0, k1, _, _ in kev]
     t_bwd_kernel = [k2.elapsed_time(k3) for _, _, k2, k3 in kev]
-    total_ms = sum(f + b for f, b in zip(t_fwd, t_bwd))
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(f + b for f, b in zip(t_fwd, t_bwd)), world, dev)
     ms_step = total_ms / n_ev
     pairs = prob.pairs
     flops_step = pairs * (prob.fwd_fpp + prob.bwd_fpp)
-    value = world * flops_step * n_ev / (total_ms / 1e3) / 1e12
+    value = whole_job_tflops(world, flops_step, n_ev, total_ms)
 
     # End to end through the public API: pinned host inputs in, results out.
     hosts_in = [x.to("cpu").pin_memory() for x in prob.inputs]
@@ -386,12 +401,8 @@ def main():
         torch.cuda.synchronize()
         if s >= 2:
             e2e_ms.append(a0.elapsed_time(a1))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        tt = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_total = float(tt.item())
-    e2e_value = world * flops_step * len(e2e_ms) / (e2e_total / 1e3) / 1e12
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
+    e2e_value = whole_job_tflops(world, flops_step, len(e2e_ms), e2e_total)
 
     peaks, peak_src = load_peaks()
     bwd_flops, fwd_flops = pairs * prob.bwd_fpp, pairs * prob.fwd_fpp
