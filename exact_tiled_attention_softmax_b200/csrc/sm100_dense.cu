@@ -1648,54 +1648,60 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
   }
 }
 
-// Reverse-pass preparation, one warp per (b, h, row < Tpad): delta from the
-// stored O and dO (kept, and negated in the padded array), the negated base-2
-// LSE, and a zeroed dQ accumulator row.
+// Reverse-pass preparation: delta from the stored O and dO (kept, and negated
+// in the padded array) and the negated base-2 LSE. A half-warp reads one row
+// with 16-byte loads; a warp takes eight rows (B*Hq*Tpad is a multiple of 128,
+// so a warp's rows are all in range or all out).
 template <bool kH>
 __global__ void __launch_bounds__(256)
 bwd_prepare_kernel(const uint16_t* o, int64_t so0, int64_t so1, int64_t so2, const uint16_t* g,
                    int64_t sg0, int64_t sg1, int64_t sg2, const float* lse, int64_t sl0, int64_t sl1, int64_t sl2,
-                   int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta, float* dq_acc) {
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= (int64_t)B * Hq * Tpad) return;
-  const int i = (int)(w % Tpad);
-  const int64_t bh = w / Tpad;
-  const int h = (int)(bh % Hq), b = (int)(bh / Hq);
-  if (i >= T) {
-    if (lane == 0) {
-      lse2[w] = -INFINITY;
-      dpad[w] = 0.f;
-    }
-    return;
-  }
-  const uint16_t* orow = o + b * so0 + h * so1 + (int64_t)i * so2;
-  const uint16_t* grow = g + b * sg0 + h * sg1 + (int64_t)i * sg2;
-  const uint2 ov = *reinterpret_cast<const uint2*>(orow + lane * 4);
-  const uint2 gv = *reinterpret_cast<const uint2*>(grow + lane * 4);
-  float s = 0.f;
+                   int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta) {
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31, hl = lane & 15;
+  const int64_t nrows = (int64_t)B * Hq * Tpad;
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float2 a2 = unpack16<kH>(e ? ov.y : ov.x), b2 = unpack16<kH>(e ? gv.y : gv.x);
-    s = fmaf(a2.x, b2.x, s);
-    s = fmaf(a2.y, b2.y, s);
-  }
-  s = warp_sum(s);
-  float4* dqr = reinterpret_cast<float4*>(dq_acc + (bh * T + i) * kD);
-  dqr[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (lane == 0) {
-    const float L = lse[b * sl0 + h * sl1 + (int64_t)i * sl2];
-    lse2[w] = L == -INFINITY ? -INFINITY : -L * kLog2e;  // negated: the reverse adds them
-    dpad[w] = -s;
-    delta[bh * T + i] = s;
+  for (int it = 0; it < 4; ++it) {
+    const int64_t w = wid * 8 + 2 * it + (lane >> 4);
+    const bool valid = w < nrows;
+    const int i = valid ? (int)(w % Tpad) : 0;
+    const int64_t bh = valid ? w / Tpad : 0;
+    const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+    const bool live = valid && i < T;
+    float s = 0.f;
+    if (live) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + b * so0 + h * so1 + (int64_t)i * so2 + hl * 8);
+      const uint4 gv = *reinterpret_cast<const uint4*>(g + b * sg0 + h * sg1 + (int64_t)i * sg2 + hl * 8);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 a2 = unpack16<kH>(ow[e]), b2 = unpack16<kH>(gw[e]);
+        s = fmaf(a2.x, b2.x, s);
+        s = fmaf(a2.y, b2.y, s);
+      }
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);  // within the half-warp
+    if (valid && hl == 0) {
+      if (!live) {
+        lse2[w] = -INFINITY;
+        dpad[w] = 0.f;
+      } else {
+        const float L = lse[b * sl0 + h * sl1 + (int64_t)i * sl2];
+        lse2[w] = L == -INFINITY ? -INFINITY : -L * kLog2e;  // negated: the reverse adds them
+        dpad[w] = -s;
+        delta[bh * T + i] = s;
+      }
+    }
   }
 }
 
+// dQ = c * accumulator in the storage type, eight elements per thread.
 template <bool kH>
 __global__ void __launch_bounds__(256)
 dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, uint16_t* dq, int64_t s0, int64_t s1,
                  int64_t s2) {
-  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (e >= (int64_t)B * Hq * T * kD) return;
   const int c = (int)(e % kD);
   const int64_t r = e / kD;
@@ -1703,10 +1709,13 @@ dq_finish_kernel(const float* dq_acc, int B, int Hq, int T, float scale, uint16_
   const int h = (int)((r / T) % Hq);
   const int b = (int)(r / ((int64_t)T * Hq));
   const float4 v = *reinterpret_cast<const float4*>(dq_acc + e);
-  uint2 out;
+  const float4 u = *reinterpret_cast<const float4*>(dq_acc + e + 4);
+  uint4 out;
   out.x = pack16<kH>(v.x * scale, v.y * scale);
   out.y = pack16<kH>(v.z * scale, v.w * scale);
-  *reinterpret_cast<uint2*>(dq + b * s0 + h * s1 + (int64_t)i * s2 + c) = out;
+  out.z = pack16<kH>(u.x * scale, u.y * scale);
+  out.w = pack16<kH>(u.z * scale, u.w * scale);
+  *reinterpret_cast<uint4*>(dq + b * s0 + h * s1 + (int64_t)i * s2 + c) = out;
 }
 
 // ----------------------------------------------------------- host helpers
@@ -1903,11 +1912,16 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   ClassTable ct = build_class_table(p, static_cast<char*>(ws_extra) + 2 * padb, st, err);
   if (err != cudaSuccess) return err;
   const bool f16 = p.dtype == ATTN_F16;
-  const int64_t rows = (int64_t)p.B * p.Hq * Tpad;
-  (f16 ? bwd_prepare_kernel<true> : bwd_prepare_kernel<false>)<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
+  const bool det = p.bwd_flags & ATTN_BWD_DETERMINISTIC;
+  const int64_t rows = (int64_t)p.B * p.Hq * Tpad;  // a multiple of 128: eight rows per warp
+  (f16 ? bwd_prepare_kernel<true> : bwd_prepare_kernel<false>)<<<(unsigned)((rows * 4 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint16_t*>(o), so[0], so[1], so[2], static_cast<const uint16_t*>(g), sg[0], sg[1], sg[2], lse,
-      sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta, dq_acc);
+      sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  // The key-centric kernel adds its dQ partials into a zeroed accumulator
+  // (not used at all in the deterministic mode).
+  if (!det && (err = cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)p.B * p.Hq * p.Tq * kD, st)) != cudaSuccess)
+    return err;
   CUtensorMap mq, mk, mv, mg, mdq;
   if (!make_dq_map(&mdq, dq_acc, p.Tq, p.B * p.Hq) ||
       !make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb, f16) ||
@@ -1937,7 +1951,7 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   }
   a.scale = p.scale;
   a.status = status;
-  const bool det = p.bwd_flags & ATTN_BWD_DETERMINISTIC, drop = p.m.dropout != 0;
+  const bool drop = p.m.dropout != 0;
   using BwdFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
                          const CUtensorMap, const BwdArgs);
   // [fp16][no dQ][dropout]
@@ -1985,8 +1999,8 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
     kdq<<<nqt * p.B * p.Hq, kDqThreads, kDqSmem, st>>>(dq_mq, mk, mv, dq_mg, d);
     return cudaGetLastError();
   }
-  const int64_t n4 = (int64_t)p.B * p.Hq * p.Tq * kD / 4;
-  (f16 ? dq_finish_kernel<true> : dq_finish_kernel<false>)<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(
+  const int64_t n8 = (int64_t)p.B * p.Hq * p.Tq * kD / 8;
+  (f16 ? dq_finish_kernel<true> : dq_finish_kernel<false>)<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(
       dq_acc, p.B, p.Hq, p.Tq, p.scale, static_cast<uint16_t*>(dq), sdq[0], sdq[1], sdq[2]);
   return cudaGetLastError();
 }
