@@ -706,7 +706,7 @@ constexpr uint32_t kCGP = kCDO + 8 * kTPlane;        // 2 stages x (G, P) tiles 
 constexpr uint32_t kCRow = kCGP + 2 * 2 * kTPlane;   // 2 stages x 64 KV rows (-1: not listed / invalid)
 constexpr uint32_t kCCtl = kCRow + 2 * kTK * 4;
 constexpr uint32_t kCSmem = kCCtl + 256 + 1024;
-constexpr int kCDrain = 16;                 // draining warps: four per TMEM lane quarter
+constexpr int kCDrain = 24;                 // draining warps: six per TMEM lane quarter
 constexpr int kCThreads = 64 + 32 * kCDrain;  // producer, MMA issuer, draining warps
 
 struct TopkDkvCtl {
@@ -835,8 +835,8 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   } else if (warp >= 2) {
     // ---------------- drain: lane l of quarter qt holds column 128 c + 32 qt + l
     // of chunk c (and 512 + 16 qt + l of chunk 4 when l < 16) for all 64 keys.
-    // The four warps of a quarter split the work: keys 32 kh .. 32 kh + 31 of
-    // the even (cp = 0) or odd (cp = 1) chunks, so that many reductions are in
+    // The six warps of a quarter split the work: keys 32 kh .. 32 kh + 31 of
+    // chunks cg and cg + 3 (cg = 0, 1, 2), so that many reductions are in
     // flight at once.
     const int qt = warp & 3, kq = (warp - 2) >> 2, kh = kq & 1, cp = kq >> 1;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
@@ -850,7 +850,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       tc_fence_after();
       const int32_t* rows = krow + s * kTK;
 #pragma unroll 1
-      for (int c = cp; c < 5; c += 2) {
+      for (int c = cp; c < 5; c += 3) {
         uint32_t v0[32];
         tmem_ld32(tq4 + 64 * c + 32 * kh, v0);
         tmem_wait_ld();
