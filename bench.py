@@ -300,6 +300,8 @@ def main():
                     choices=["causal_8k", "causal_2k", "window_block_8k", "gqa_dropout_16k", "topk_shared_kv"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--topk-tokens", type=int, default=0,
+                    help="top-k workload with only this many query tokens (a smaller case for ncu)")
     ap.add_argument("--deterministic", action="store_true",
                     help="bitwise reproducible reverse pass (dense workloads)")
     args = ap.parse_args()
@@ -326,7 +328,11 @@ def main():
     eta.load_library()
 
     if args.workload in W.TOPK_WORKLOADS:
-        prob = topk_problem(W.TOPK_WORKLOADS[args.workload], dev, torch, eta)
+        case = W.TOPK_WORKLOADS[args.workload]
+        if args.topk_tokens:  # the same lists and shapes for fewer query tokens (profiling captures)
+            import dataclasses
+            case = dataclasses.replace(case, Tq=args.topk_tokens)
+        prob = topk_problem(case, dev, torch, eta)
     else:
         prob = dense_problem(W.WORKLOADS[args.workload], dev, torch, eta, args.deterministic)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)

@@ -128,18 +128,28 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
     // of all nine planes.
     if (lane == 0) tma_prefetch_desc(&tkv);
     const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
+    // The listed indices of tile n + 1 are read while tile n's gathers go
+    // out, so their latency is not on the producer's path.
+    auto read_idx = [&](int m, int e) {
+      const int pos = m * kTK + 2 * lane + e;
+      return (m < ntiles && pos < n_keys) ? list[pos] : -1;
+    };
+    int jn[2] = {read_idx(0, 0), read_idx(0, 1)};
     int n = 0;
     for (; n < ntiles; ++n) {
       const int s = n % kTStages;
       if (!__all_sync(0xffffffffu,
                       wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kTStages) & 1) ^ 1, abort_flag, a.status)))
         break;
+      const int jc[2] = {jn[0], jn[1]};
+      jn[0] = read_idx(n + 1, 0);
+      jn[1] = read_idx(n + 1, 1);
       int row[2];
       bool valid[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int pos = n * kTK + 2 * lane + e;
-        const int j = pos < n_keys ? list[pos] : -1;
+        const int j = jc[e];
         valid[e] = pos < n_keys && j >= 0 && j < a.Tkv;
         if (pos < n_keys && !valid[e]) set_status(a.status, ATTN_DEVERR_TOPK_INDEX);
         row[e] = valid[e] ? j : 0;  // unlisted and out-of-range keys read row 0 and are masked
@@ -462,18 +472,28 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
     }
     __syncwarp();
     const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
+    // The listed indices of tile n + 1 are read while tile n's gathers go
+    // out, so their latency is not on the producer's path.
+    auto read_idx = [&](int m, int e) {
+      const int pos = m * kTK + 2 * lane + e;
+      return (m < ntiles && pos < n_keys) ? list[pos] : -1;
+    };
+    int jn[2] = {read_idx(0, 0), read_idx(0, 1)};
     int n = 0;
     for (; n < ntiles; ++n) {
       const int s = n % kBStages;
       if (!__all_sync(0xffffffffu,
                       wait_bar(smem_u32(&ctl->kv_empty[s]), ((n / kBStages) & 1) ^ 1, abort_flag, a.status)))
         break;
+      const int jc[2] = {jn[0], jn[1]};
+      jn[0] = read_idx(n + 1, 0);
+      jn[1] = read_idx(n + 1, 1);
       int row[2];
       bool valid[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int pos = n * kTK + 2 * lane + e;
-        const int j = pos < n_keys ? list[pos] : -1;
+        const int j = jc[e];
         valid[e] = pos < n_keys && j >= 0 && j < a.Tkv;
         if (pos < n_keys && !valid[e]) set_status(a.status, ATTN_DEVERR_TOPK_INDEX);
         row[e] = valid[e] ? j : 0;
@@ -776,15 +796,23 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     }
     __syncwarp();
     const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
+    auto read_idx = [&](int m, int e) {  // tile m + 1's indices are read while tile m's rows go out
+      const int pos = m * kTK + 2 * lane + e;
+      return (m < ntiles && pos < n_keys) ? list[pos] : -1;
+    };
+    int jn[2] = {read_idx(0, 0), read_idx(0, 1)};
     int n = 0;
     for (; n < ntiles; ++n) {
       const int s = n & 1;
       if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)))
         break;
+      const int jc[2] = {jn[0], jn[1]};
+      jn[0] = read_idx(n + 1, 0);
+      jn[1] = read_idx(n + 1, 1);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int k = 2 * lane + e, pos = n * kTK + k;
-        const int j = pos < n_keys ? list[pos] : -1;
+        const int k = 2 * lane + e;
+        const int j = jc[e];
         krow[s * kTK + k] = (j >= 0 && j < a.Tkv) ? j : -1;  // the first kernel flagged invalid entries
       }
       __syncwarp();
