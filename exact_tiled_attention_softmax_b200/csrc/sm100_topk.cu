@@ -42,23 +42,27 @@ constexpr int kTStages = 3;
 constexpr uint32_t kTKV = 0;
 constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kTCtl = kTP + kTH * 128;
-constexpr uint32_t kTSmem = kTCtl + 512 + 1024;  // control block + alignment slack
-constexpr int kTThreads = 192;                   // producer, MMA issuer, 4 softmax warps
+constexpr uint32_t kTSmem = kTCtl + 1024 + 1024;  // control block + alignment slack
+constexpr int kTThreads = 192;                    // producer, MMA issuer, 4 softmax warps
+constexpr int kTFThreads = 320;                   // forward: the same plus 4 gather warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;                 // move the running max only past 2^8
 constexpr uint32_t kUpper = 16u << 16;           // TMEM lane offset of the upper half
 constexpr uint32_t kQCol = 128;                  // first TMEM column of Q (upper half)
 
 struct TopkCtl {
-  uint64_t kv_full[kTStages], kv_empty[kTStages];
+  uint64_t kv_full[kTStages], kv_empty[kTStages], rows_full[kTStages];
   uint64_t s_full[2];
   uint64_t p_full, pv_done, q_ready, o_final;
   uint32_t vmask[kTStages][2];  // valid listed keys of the stage: key 2i+e <-> bit i of word e
   uint32_t tmem_base;
   uint32_t abort_flag;
+  int32_t grow[kTStages][kTK];  // forward: the KV row each listed key of the stage reads
 };
 
 struct TopkArgs {
+  const uint8_t* kv;  // KV rows, skv_bytes apart (the forward's gather source)
+  int64_t skv_bytes;
   const uint16_t* q;  // 16-bit storage: bf16 or fp16
   int64_t sq_t, sq_h;
   const int32_t* idx;
@@ -88,7 +92,7 @@ __device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* map, ui
 __device__ __forceinline__ bool key_valid(const uint32_t (&vm)[2], int k) { return (vm[k & 1] >> (k >> 1)) & 1u; }
 
 template <bool kH>
-__global__ void __launch_bounds__(kTThreads, 1)
+__global__ void __launch_bounds__(kTFThreads, 1)
 topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,8 +106,9 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTStages; ++s) {
-      mbar_init(smem_u32(&ctl->kv_full[s]), 1);
+      mbar_init(smem_u32(&ctl->kv_full[s]), 4);  // one arrival per gather warp
       mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+      mbar_init(smem_u32(&ctl->rows_full[s]), 1);
     }
     for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&ctl->s_full[b]), 1);
     mbar_init(smem_u32(&ctl->p_full), 4);   // one arrival per softmax warp
@@ -123,10 +128,9 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0) {
-    // ---------------- gather producer (whole warp): lane l holds listed keys
-    // 2l and 2l+1 of the tile; lanes 0-15 then gather rows 4g..4g+3 (g = lane)
-    // of all nine planes.
-    if (lane == 0) tma_prefetch_desc(&tkv);
+    // ---------------- row producer (whole warp): lane l holds listed keys 2l
+    // and 2l+1 of the tile; it publishes the stage's KV rows and valid-key
+    // mask to the gather warps.
     const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
     // The listed indices of tile n + 1 are read while tile n's gathers go
     // out, so their latency is not on the producer's path.
@@ -155,26 +159,48 @@ topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
         row[e] = valid[e] ? j : 0;  // unlisted and out-of-range keys read row 0 and are masked
       }
       const uint32_t vm0 = __ballot_sync(0xffffffffu, valid[0]), vm1 = __ballot_sync(0xffffffffu, valid[1]);
-      const uint32_t kf = smem_u32(&ctl->kv_full[s]);
+      ctl->grow[s][2 * lane] = row[0];
+      ctl->grow[s][2 * lane + 1] = row[1];
       if (lane == 0) {
         ctl->vmask[s][0] = vm0;
         ctl->vmask[s][1] = vm1;
-        mbar_expect_tx(kf, kTTile);  // its release publishes vmask with the stage
       }
       __syncwarp();
-      const int g = lane & 15;
-      const int r0 = __shfl_sync(0xffffffffu, row[0], 2 * g), r1 = __shfl_sync(0xffffffffu, row[1], 2 * g);
-      const int r2 = __shfl_sync(0xffffffffu, row[0], 2 * g + 1), r3 = __shfl_sync(0xffffffffu, row[1], 2 * g + 1);
-      if (lane < 16) {
-        const uint32_t dst = sbase + kTKV + s * kTTile + g * 512;
-#pragma unroll 1
-        for (int c = 0; c < kTPlanes; ++c) gather4(dst + c * kTPlane, &tkv, kf, 64 * c, r0, r1, r2, r3);
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->rows_full[s]));  // publishes grow and vmask
+    }
+  } else if (warp >= 6) {
+    // ---------------- gather warps: 16-byte asynchronous copies of the 64
+    // listed rows (72 chunks of 16 bytes each) into the stage's nine 128-byte-
+    // swizzled planes; consecutive threads take consecutive chunks of a row.
+    // A stage is signalled when its copies have landed, one stage behind the
+    // copies being issued.
+    const int gt = threadIdx.x - 192;
+    auto signal = [&](int m) {
+      fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->kv_full[m % kTStages]));
+    };
+    int n = 0;
+    bool ok = true;
+    for (; n < ntiles; ++n) {
+      const int s = n % kTStages;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->rows_full[s]), (n / kTStages) & 1, abort_flag, a.status));
+      if (!ok) break;
+      const uint32_t dst = sbase + kTKV + s * kTTile;
+#pragma unroll 4
+      for (int it = 0; it < kTK * 72 / 128; ++it) {
+        const int q = it * 128 + gt, r = q / 72, c = q - r * 72;
+        cp_async_16(dst + (uint32_t)(c >> 3) * kTPlane + sw128_offset(r, (c & 7) * 16),
+                    a.kv + (int64_t)ctl->grow[s][r] * a.skv_bytes + c * 16);
+      }
+      cp_async_commit();
+      if (n > 0) {
+        cp_async_wait<1>();
+        signal(n - 1);
       }
     }
-    // Leave only after this warp's copies have landed.
-    if (lane == 0)
-      for (int r = (n > kTStages ? n - kTStages : 0); r < n; ++r)
-        wait_bar(smem_u32(&ctl->kv_full[r % kTStages]), (r / kTStages) & 1, abort_flag, nullptr);
+    cp_async_wait<0>();  // nothing stays in flight past the loop
+    if (ok && n > 0) signal(n - 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S(n) = Q K(n)^T two tiles ahead of O += P(n) V(n).
     constexpr uint32_t idS = idesc16<kH>(64, kTK, 0, 0);
@@ -1064,6 +1090,8 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   CUtensorMap map;
   if (!make_kv_gather_map(&map, p)) return cudaErrorInvalidValue;
   TopkArgs a;
+  a.kv = static_cast<const uint8_t*>(p.kv);
+  a.skv_bytes = p.skv * 2;
   a.q = static_cast<const uint16_t*>(p.q);
   a.sq_t = p.sq_t;
   a.sq_h = p.sq_h;
@@ -1088,7 +1116,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   cudaError_t e = raise_smem(reinterpret_cast<const void*>(kern), kTSmem, f16 ? 3 : 0);
   if (e != cudaSuccess) return e;
   main_kernel_begin(st);
-  kern<<<p.Tq, kTThreads, kTSmem, st>>>(map, a);
+  kern<<<p.Tq, kTFThreads, kTSmem, st>>>(map, a);
   main_kernel_end(st);
   return cudaGetLastError();
 }
