@@ -14,10 +14,10 @@
 // A warp reads its quarter with 32-lane loads: its upper 16 lanes own the
 // S rows (softmax), its lower 16 lanes the O rows of the same heads.
 //
-// Warp 0 gathers each tile's 64 listed KV rows with TMA gather4 into a
-// three-stage ring (9 planes of 64 columns, 128-byte swizzle); warp 1 issues
-// the MMAs (S, then O += P V with P staged in shared memory); warps 2-5 run
-// the softmax and the epilogue.
+// Warp 0 publishes each tile's 64 listed KV rows; four gather warps copy them
+// with 16-byte cp.async into a three-stage ring (9 planes of 64 columns,
+// 128-byte swizzle); warp 1 issues the MMAs (S, then O += P V with P staged
+// in shared memory); warps 2-5 run the softmax and the epilogue.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -43,8 +43,7 @@ constexpr uint32_t kTKV = 0;
 constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kTCtl = kTP + kTH * 128;
 constexpr uint32_t kTSmem = kTCtl + 1024 + 1024;  // control block + alignment slack
-constexpr int kTThreads = 192;                    // producer, MMA issuer, 4 softmax warps
-constexpr int kTFThreads = 320;                   // forward: the same plus 4 gather warps
+constexpr int kTFThreads = 320;  // forward: row producer, MMA issuer, 4 softmax warps, 4 gather warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;                 // move the running max only past 2^8
 constexpr uint32_t kUpper = 16u << 16;           // TMEM lane offset of the upper half
@@ -80,20 +79,11 @@ struct TopkArgs {
   uint32_t* status;
 };
 
-__device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int r0, int r1,
-                                        int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 __device__ __forceinline__ bool key_valid(const uint32_t (&vm)[2], int k) { return (vm[k & 1] >> (k >> 1)) & 1u; }
 
 template <bool kH>
 __global__ void __launch_bounds__(kTFThreads, 1)
-topk_fwd_kernel(const __grid_constant__ CUtensorMap tkv, const TopkArgs a) {
+topk_fwd_kernel(const TopkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -419,18 +409,22 @@ constexpr uint32_t kBKV = 0;
 constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads x 64 columns
 constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kBCtl = kBG + kTH * 128;
-constexpr uint32_t kBSmem = kBCtl + 512 + 1024;
+constexpr uint32_t kBSmem = kBCtl + 1024 + 1024;
+constexpr int kBThreads = 256;  // producer, MMA issuer, 4 softmax warps, 2 gather warps
 constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
 
 struct TopkBwdCtl {
-  uint64_t kv_full[kBStages], kv_empty[kBStages];
+  uint64_t kv_full[kBStages], kv_empty[kBStages], rows_full[kBStages];
   uint64_t do_full, q_ready, st_full, st_empty, g_full, g_free, dq_done;
   uint32_t vmask[kBStages][2];
   uint32_t tmem_base;
   uint32_t abort_flag;
+  int32_t grow[kBStages][kTK];  // the KV row each listed key of the stage reads
 };
 
 struct TopkBwdArgs {
+  const uint8_t* kv;  // KV rows, skv_bytes apart (the gather source)
+  int64_t skv_bytes;
   const uint16_t* q;  // 16-bit storage: bf16 or fp16
   int64_t sq_t, sq_h;
   const int32_t* idx;
@@ -450,8 +444,8 @@ struct TopkBwdArgs {
 };
 
 template <bool kH>
-__global__ void __launch_bounds__(kTThreads, 1)
-topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constant__ CUtensorMap tdo,
+__global__ void __launch_bounds__(kBThreads, 1)
+topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
                    const TopkBwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -465,8 +459,9 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBStages; ++s) {
-      mbar_init(smem_u32(&ctl->kv_full[s]), 1);
+      mbar_init(smem_u32(&ctl->kv_full[s]), 2);  // one arrival per gather warp
       mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
+      mbar_init(smem_u32(&ctl->rows_full[s]), 1);
     }
     mbar_init(smem_u32(&ctl->do_full), 1);
     mbar_init(smem_u32(&ctl->q_ready), 4);
@@ -490,7 +485,6 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
   if (warp == 0) {
     // ---------------- producer: dO once (8 planes), then the KV gathers.
     if (lane == 0) {
-      tma_prefetch_desc(&tkv);
       tma_prefetch_desc(&tdo);
       const uint32_t df = smem_u32(&ctl->do_full);
       mbar_expect_tx(df, 8 * kTPlane);
@@ -525,27 +519,45 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tkv, const __grid_constan
         row[e] = valid[e] ? j : 0;
       }
       const uint32_t vm0 = __ballot_sync(0xffffffffu, valid[0]), vm1 = __ballot_sync(0xffffffffu, valid[1]);
-      const uint32_t kf = smem_u32(&ctl->kv_full[s]);
+      ctl->grow[s][2 * lane] = row[0];
+      ctl->grow[s][2 * lane + 1] = row[1];
       if (lane == 0) {
         ctl->vmask[s][0] = vm0;
         ctl->vmask[s][1] = vm1;
-        mbar_expect_tx(kf, kTTile);
       }
       __syncwarp();
-      const int g = lane & 15;
-      const int r0 = __shfl_sync(0xffffffffu, row[0], 2 * g), r1 = __shfl_sync(0xffffffffu, row[1], 2 * g);
-      const int r2 = __shfl_sync(0xffffffffu, row[0], 2 * g + 1), r3 = __shfl_sync(0xffffffffu, row[1], 2 * g + 1);
-      if (lane < 16) {
-        const uint32_t dst = sbase + kBKV + s * kTTile + g * 512;
-#pragma unroll 1
-        for (int c = 0; c < kTPlanes; ++c) gather4(dst + c * kTPlane, &tkv, kf, 64 * c, r0, r1, r2, r3);
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->rows_full[s]));  // publishes grow and vmask
+    }
+    if (lane == 0) wait_bar(smem_u32(&ctl->do_full), 0, abort_flag, nullptr);
+  } else if (warp >= 6) {
+    // ---------------- gather warps: 16-byte asynchronous copies of the 64
+    // listed rows into the stage's nine 128-byte-swizzled planes (as in the
+    // forward); with two stages each one is signalled as soon as its own
+    // copies have landed.
+    const int gt = threadIdx.x - 192;
+    auto signal = [&](int m) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->kv_full[m % kBStages]));
+    };
+    int n = 0;
+    bool ok = true;
+    for (; n < ntiles; ++n) {
+      const int s = n % kBStages;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->rows_full[s]), (n / kBStages) & 1, abort_flag, a.status));
+      if (!ok) break;
+      const uint32_t dst = sbase + kBKV + s * kTTile;
+#pragma unroll 4
+      for (int it = 0; it < kTK * 72 / 64; ++it) {
+        const int q = it * 64 + gt, r = q / 72, c = q - r * 72;
+        cp_async_16(dst + (uint32_t)(c >> 3) * kTPlane + sw128_offset(r, (c & 7) * 16),
+                    a.kv + (int64_t)ctl->grow[s][r] * a.skv_bytes + c * 16);
       }
+      cp_async_commit();
+      cp_async_wait<0>();
+      signal(n);
     }
-    if (lane == 0) {
-      for (int r = (n > kBStages ? n - kBStages : 0); r < n; ++r)
-        wait_bar(smem_u32(&ctl->kv_full[r % kBStages]), (r / kBStages) & 1, abort_flag, nullptr);
-      wait_bar(smem_u32(&ctl->do_full), 0, abort_flag, nullptr);
-    }
+    cp_async_wait<0>();
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: S(n), dP(n) as soon as the compute warps
     // have read S(n-1), dP(n-1); dQ += G(n) K(n) once G(n) is in shared memory.
@@ -971,17 +983,6 @@ bool make_map3(CUtensorMap* map, const void* base, int64_t inner, int Tq, int64_
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_kv_gather_map(CUtensorMap* map, const TopkP& p) {
-  const bool f16 = p.dtype == ATTN_F16;
-  cuuint64_t dims[2] = {(cuuint64_t)p.Dqk, (cuuint64_t)p.Tkv};
-  cuuint64_t strides[1] = {(cuuint64_t)p.skv * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t es[2] = {1, 1};
-  return topk_encode_fn()(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.kv), dims, strides, box, es,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t raise_smem(const void* fn, uint32_t bytes, int which) {
   static bool done[6][64] = {};
   int dev = 0;
@@ -1017,13 +1018,15 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   const bool f16 = p.dtype == ATTN_F16;
   uint16_t* g_scr = static_cast<uint16_t*>(scratch);
   uint16_t* p_scr = g_scr + (size_t)p.Tq * kTH * pad;
-  CUtensorMap mkv, mdo, mq, mg, mp;
-  if (!make_kv_gather_map(&mkv, p) || !make_map3(&mdo, g, kTDV, p.Tq, sg_h, sg_t, f16) ||
+  CUtensorMap mdo, mq, mg, mp;
+  if (!make_map3(&mdo, g, kTDV, p.Tq, sg_h, sg_t, f16) ||
       !make_map3(&mq, p.q, kTD, p.Tq, p.sq_h, p.sq_t, f16) ||
       !make_map3(&mg, g_scr, pad, p.Tq, pad, (int64_t)kTH * pad, f16) ||
       !make_map3(&mp, p_scr, pad, p.Tq, pad, (int64_t)kTH * pad, f16))
     return cudaErrorInvalidValue;
   TopkBwdArgs a;
+  a.kv = static_cast<const uint8_t*>(p.kv);
+  a.skv_bytes = p.skv * 2;
   a.q = static_cast<const uint16_t*>(p.q);
   a.sq_t = p.sq_t;
   a.sq_h = p.sq_h;
@@ -1062,7 +1065,7 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   if ((e = raise_smem(reinterpret_cast<const void*>(kdq), kBSmem, f16 ? 4 : 1)) != cudaSuccess) return e;
   if ((e = raise_smem(reinterpret_cast<const void*>(kdkv), kCSmem, f16 ? 5 : 2)) != cudaSuccess) return e;
   main_kernel_begin(st);
-  kdq<<<p.Tq, kTThreads, kBSmem, st>>>(mkv, mdo, a);
+  kdq<<<p.Tq, kBThreads, kBSmem, st>>>(mdo, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kdkv<<<p.Tq, kCThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
   main_kernel_end(st);
@@ -1085,10 +1088,6 @@ bool sm100_topk_supported(const TopkP& p, const attn_tensor* q, const attn_tenso
 
 cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, float* lse, int64_t sl_t,
                            int64_t sl_h, uint32_t* status, cudaStream_t st) {
-  // 2-D map over the KV rows: 64-column boxes one row high (the gather4 form)
-  // with 128-byte swizzle, matching the planes the MMAs read.
-  CUtensorMap map;
-  if (!make_kv_gather_map(&map, p)) return cudaErrorInvalidValue;
   TopkArgs a;
   a.kv = static_cast<const uint8_t*>(p.kv);
   a.skv_bytes = p.skv * 2;
@@ -1116,7 +1115,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   cudaError_t e = raise_smem(reinterpret_cast<const void*>(kern), kTSmem, f16 ? 3 : 0);
   if (e != cudaSuccess) return e;
   main_kernel_begin(st);
-  kern<<<p.Tq, kTFThreads, kTSmem, st>>>(map, a);
+  kern<<<p.Tq, kTFThreads, kTSmem, st>>>(a);
   main_kernel_end(st);
   return cudaGetLastError();
 }

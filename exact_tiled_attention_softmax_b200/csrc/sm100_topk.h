@@ -1,4 +1,4 @@
-// Tensor-core (tcgen05 / TMEM / TMA gather4) path for the top-k forward and reverse with a
+// Tensor-core (tcgen05 / TMEM, cp.async row gathers) path for the top-k forward and reverse with a
 // shared KV: bf16, 64 heads, Dqk = 576, Dv = 512, on sm_100a (internal; not
 // part of the ABI).
 #pragma once
