@@ -43,7 +43,8 @@ constexpr uint32_t kTKV = 0;
 constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kTCtl = kTP + kTH * 128;
 constexpr uint32_t kTSmem = kTCtl + 1024 + 1024;  // control block + alignment slack
-constexpr int kTFThreads = 320;  // forward: row producer, MMA issuer, 4 softmax warps, 4 gather warps
+constexpr int kTFGather = 6;                         // forward gather warps
+constexpr int kTFThreads = 192 + 32 * kTFGather;    // row producer, MMA issuer, 4 softmax warps, gather warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;                 // move the running max only past 2^8
 constexpr uint32_t kUpper = 16u << 16;           // TMEM lane offset of the upper half
@@ -96,7 +97,7 @@ topk_fwd_kernel(const TopkArgs a) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTStages; ++s) {
-      mbar_init(smem_u32(&ctl->kv_full[s]), 4);  // one arrival per gather warp
+      mbar_init(smem_u32(&ctl->kv_full[s]), kTFGather);  // one arrival per gather warp
       mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
       mbar_init(smem_u32(&ctl->rows_full[s]), 1);
     }
@@ -178,8 +179,8 @@ topk_fwd_kernel(const TopkArgs a) {
       if (!ok) break;
       const uint32_t dst = sbase + kTKV + s * kTTile;
 #pragma unroll 4
-      for (int it = 0; it < kTK * 72 / 128; ++it) {
-        const int q = it * 128 + gt, r = q / 72, c = q - r * 72;
+      for (int it = 0; it < kTK * 72 / (32 * kTFGather); ++it) {
+        const int q = it * (32 * kTFGather) + gt, r = q / 72, c = q - r * 72;
         cp_async_16(dst + (uint32_t)(c >> 3) * kTPlane + sw128_offset(r, (c & 7) * 16),
                     a.kv + (int64_t)ctl->grow[s][r] * a.skv_bytes + c * 16);
       }
