@@ -192,3 +192,28 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_fp16_lse_formats_and_reverse_flags_on_host(lib):
+    """fp16 tensors pass the dtype checks (the call stops at the workspace
+    check, before any launch); a non-default LSE format adds room for the
+    reverse pass's natural-log copy; unknown reverse flags are rejected."""
+    import exact_tiled_attention_softmax_b200 as eta
+    q, k, v = _t([1, 4, 64, 128], dtype=2), _t([1, 2, 64, 128], dtype=2), _t([1, 2, 64, 128], dtype=2)
+    o, lse = _t([1, 4, 64, 128], dtype=2), _t([1, 4, 64], dtype=0)
+    assert _call_fwd(lib, q, k, v, o, lse, ws_bytes=16) == eta.ATTN_ERR_WORKSPACE
+    base = eta.AttnMaskC()
+    base.flags = eta.ATTN_MASK_CAUSAL
+    kv_only = eta.AttnMaskC()
+    kv_only.flags = eta.ATTN_MASK_CAUSAL
+    kv_only.lse_format = eta.ATTN_LSE_KV_ONLY
+    args = (ctypes.byref(q), ctypes.byref(k), ctypes.byref(v))
+    b0 = lib.attn_bwd_workspace_size(*args, ctypes.byref(base))
+    b1 = lib.attn_bwd_workspace_size(*args, ctypes.byref(kv_only))
+    assert b1 >= b0 + 4 * 64 * 4
+    bad = eta.AttnMaskC()
+    bad.bwd_flags = 0x2
+    assert _call_fwd(lib, q, k, v, o, lse, mask=bad) == eta.ATTN_ERR_INVALID_ARG
+    det = eta.AttnMaskC()
+    det.bwd_flags = eta.ATTN_BWD_DETERMINISTIC
+    assert _call_fwd(lib, q, k, v, o, lse, mask=det, ws_bytes=16) == eta.ATTN_ERR_WORKSPACE
