@@ -1,0 +1,66 @@
+"""bench.py's host-side accounting on CPU: the allowed-pair count that the
+TFLOP/s figures divide by (checked against the oracle's allowed sets on small
+shapes and against the causal closed form at the headline size), the
+whole-job throughput arithmetic, and the rule that a recorded DRAM traffic
+figure is reported only for the kernel source it was captured from."""
+import dataclasses
+import json
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import oracle  # noqa: E402
+from exact_tiled_attention_softmax_b200 import workloads as W  # noqa: E402
+
+
+@pytest.mark.parametrize("kind", ["causal", "window", "window_block", "noncausal"])
+def test_allowed_pairs_equal_the_oracle_sets(kind):
+    base = W.WORKLOADS["window_block_8k"]
+    case = dataclasses.replace(base, B=2, Hq=3, Hkv=3, T=300, block_size=0, window_left=0, causal=True)
+    if kind == "window":
+        case = dataclasses.replace(case, window_left=70)
+    elif kind == "window_block":
+        case = dataclasses.replace(case, window_left=90, block_size=64)
+    elif kind == "noncausal":
+        case = dataclasses.replace(case, causal=False)
+    bm = W.block_mask(case)
+    allow = oracle.allowed_dense(case.T, case.T, causal=case.causal, window_left=case.window_left,
+                                 block_mask=bm, block_q=case.block_size or 1, block_k=case.block_size or 1)
+    expect = int(np.broadcast_to(allow, (case.B, case.Hq, case.T, case.T)).sum())
+    assert bench.allowed_pairs(case) == expect
+
+
+def test_headline_pairs_and_throughput_arithmetic():
+    case = W.WORKLOADS["causal_8k"]
+    assert bench.allowed_pairs(case) == case.B * case.Hq * case.T * (case.T + 1) // 2
+    # 2 ranks x 10 steps x 1.5 TFLOP over a 30 ms slowest-rank time
+    assert abs(bench.whole_job_tflops(2, 1.5e12, 10, 30.0) - 1000.0) < 1e-9
+    assert bench.max_over_ranks(12.5, 1) == 12.5
+
+
+def test_recorded_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    entry = rec["bwd_kernel"]["causal_8k"]
+    got = bench.recorded_traffic("bwd_kernel", "causal_8k")
+    import hashlib
+    digest = hashlib.sha256(open(os.path.join(ROOT, entry["source"]), "rb").read()).hexdigest()
+    if digest == entry["source_sha256"]:
+        assert got == entry["dram_bytes_read"] + entry["dram_bytes_write"]
+    else:
+        assert got is None
+    # A copy of the tree whose kernel source differs reports no traffic.
+    (tmp_path / "profiles").mkdir()
+    bad = dict(rec)
+    bad["bwd_kernel"] = {"causal_8k": dict(entry, source_sha256="0" * 64)}
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps(bad))
+    src = tmp_path / entry["source"]
+    src.parent.mkdir(parents=True)
+    src.write_text("// not the captured kernel\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("bwd_kernel", "causal_8k") is None
