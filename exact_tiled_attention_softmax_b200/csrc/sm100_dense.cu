@@ -41,7 +41,7 @@ constexpr int kBMb = 64;         // reverse query rows per step
 constexpr int kStages = 2;       // K/V ring depth (forward), Q/dO ring depth (reverse)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // move the running max only past 2^8
-constexpr int kPolyEvery = 0;              // forward: every k-th pair of exponentials on the FMA pipe (0: none)
+constexpr int kPolyEvery = 4;              // forward: every k-th pair of exponentials on the FMA pipe (0: none)
 
 // Does pair e of a 16-pair chunk take its exponentials on the FMA pipe?
 __host__ __device__ constexpr bool poly_pair(int e) {
@@ -353,41 +353,43 @@ __device__ __forceinline__ float move_max(float mx, float& m_run) {
 
 // One S row (128 keys, all allowed, no dropout) of the calling thread's TMEM
 // lane -> P (bf16 pairs written over the row's first 64 columns), with the
-// running summary (m_run, l_run) updated. The row stays in registers between
-// the maximum and the exponentials (one TMEM wait); x = s c log2(e) - m is
-// formed on packed fp32 pairs and every kPolyEvery-th pair of exponentials
-// runs on the FMA pipe instead of MUFU. Returns alpha.
+// running summary (m_run, l_run) updated. The maximum takes two 64-column
+// TMEM loads and the exponentials four 32-column reloads, so that no more
+// than 64 scores are live at once (the forward then needs no spill slots);
+// x = s c log2(e) - m is formed on packed fp32 pairs and every kPolyEvery-th
+// pair of exponentials runs on the FMA pipe instead of MUFU. Returns alpha.
 template <bool kH, bool kDrop>
 __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2, float& m_run, float& l_run,
                                                    uint64_t kb0, uint64_t kb1) {
-  uint32_t s0[32], s1[32], s2[32], s3[32];
-  tmem_ld32(tS, s0);
-  tmem_ld32(tS + 32, s1);
-  tmem_ld32(tS + 64, s2);
-  tmem_ld32(tS + 96, s3);
-  tmem_wait_ld();
-  // Extremum of the raw scores, scaled once.
   float mx;
-  if (scale_log2 >= 0.f) {
-    float e0 = -INFINITY, e1 = -INFINITY, e2 = -INFINITY, e3 = -INFINITY;
+  {
+    const bool pos = scale_log2 >= 0.f;
+    float e0 = pos ? -INFINITY : INFINITY, e1 = e0, e2 = e0, e3 = e0;
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      e0 = max3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
-      e1 = max3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
-      e2 = max3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
-      e3 = max3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
-    }
-    mx = max3f(e0, e1, fmaxf(e2, e3)) * scale_log2;
-  } else {
-    float e0 = INFINITY, e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t s0[32], s1[32];
+      tmem_ld32(tS + 64 * hf, s0);
+      tmem_ld32(tS + 64 * hf + 32, s1);
+      tmem_wait_ld();
+      if (pos) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      e0 = min3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
-      e1 = min3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
-      e2 = min3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
-      e3 = min3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
+        for (int e = 0; e < 32; e += 4) {
+          e0 = max3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+          e1 = max3f(e1, __uint_as_float(s0[e + 2]), __uint_as_float(s0[e + 3]));
+          e2 = max3f(e2, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+          e3 = max3f(e3, __uint_as_float(s1[e + 2]), __uint_as_float(s1[e + 3]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          e0 = min3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+          e1 = min3f(e1, __uint_as_float(s0[e + 2]), __uint_as_float(s0[e + 3]));
+          e2 = min3f(e2, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+          e3 = min3f(e3, __uint_as_float(s1[e + 2]), __uint_as_float(s1[e + 3]));
+        }
+      }
     }
-    mx = min3f(e0, e1, fminf(e2, e3)) * scale_log2;
+    mx = (pos ? max3f(e0, e1, fmaxf(e2, e3)) : min3f(e0, e1, fminf(e2, e3))) * scale_log2;
   }
   const float alpha = move_max(mx, m_run);
   const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
@@ -418,10 +420,13 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
     }
     tmem_st16(tS + q * 16, pk);
   };
-  chunk(s0, 0);
-  chunk(s1, 1);
-  chunk(s2, 2);
-  chunk(s3, 3);
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    uint32_t r[32];
+    tmem_ld32(tS + 32 * q, r);
+    tmem_wait_ld();
+    chunk(r, q);
+  }
   float a0, a1, b0, b1;
   f2_unpack(acc0, a0, a1);
   f2_unpack(acc1, b0, b1);
