@@ -457,11 +457,16 @@ def main():
             peak = float(peaks["bf16_tflops"])
             kname = "bwd_kernel" if args.workload not in W.TOPK_WORKLOADS else \
                 "top-k reverse kernels (dQ + G/P, dKV contributions)"
+            if args.deterministic and args.workload not in W.TOPK_WORKLOADS:
+                kname = "bwd_kernel (key-centric, without dQ)"
             src = f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
         else:
             peak = fp32_alu_peak_tflops(clocks.get("sm_max_mhz") or 1965.0)
             kname = "row-wise reverse kernels (CUDA cores, fp32 FFMA)"
             src = "derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock"
+        # The deterministic reverse runs another bwd_kernel instantiation (no
+        # dQ product, no dQ accumulator traffic): its capture is keyed apart.
+        traffic_key = prob.name + ("_deterministic" if args.deterministic else "")
         config = dict(prob.config)
         config.update({"allowed_pairs": pairs, "flops_per_pair": prob.fwd_fpp + prob.bwd_fpp,
                        "l2": "flushed (256 MB write) before every step", "parallelism": f"replicas x{world}"})
@@ -478,7 +483,7 @@ def main():
                         "bwd_main": {"ms": bwd_kernel_ms, "tflops": achieved}},
             "roofline": {"bound": prob.bound, "kernel": kname,
                          "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                         "traffic": recorded_traffic("bwd_kernel", prob.name) if prob.bound == "tensor" else None,
+                         "traffic": recorded_traffic("bwd_kernel", traffic_key) if prob.bound == "tensor" else None,
                          "work_per_launch": f"{kernel_flops:.4e} flops = {pairs} allowed pairs x {kernel_fpp}",
                          "peak_source": src},
             "clocks": clocks,

@@ -64,3 +64,11 @@ def test_recorded_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
     src.write_text("// not the captured kernel\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.recorded_traffic("bwd_kernel", "causal_8k") is None
+
+
+def test_deterministic_reverse_has_no_borrowed_traffic():
+    # The deterministic reverse launches the key-centric bwd_kernel without its
+    # dQ product; the capture of the fused instantiation must not stand in for it.
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    if "causal_8k_deterministic" not in rec.get("bwd_kernel", {}):
+        assert bench.recorded_traffic("bwd_kernel", "causal_8k_deterministic") is None
