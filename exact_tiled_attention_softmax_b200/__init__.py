@@ -16,7 +16,8 @@ import torch
 
 __all__ = [
     "AllowedSet", "AttentionFunction", "AttnError", "attention", "attn_fwd", "attn_bwd", "attn_bwd_noalloc", "attn_fwd_workspace_size",
-    "attn_bwd_workspace_size", "attn_get_status", "attn_set_kernel_events", "attn_status_string",
+    "attn_bwd_workspace_size", "attn_get_status", "attn_selftest_wait_timeout", "attn_set_kernel_events",
+    "attn_status_string",
     "attn_version", "library_path", "load_library",
 ]
 
@@ -99,6 +100,8 @@ def load_library():
     lib.attn_bwd_noalloc.argtypes = [T, T, T, T, T, T, M, ctypes.c_float, T, T, T, vp, vp]
     lib.attn_get_status.restype = ctypes.c_int
     lib.attn_get_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.attn_selftest_wait_timeout.restype = ctypes.c_int
+    lib.attn_selftest_wait_timeout.argtypes = [vp, sz, vp]
     lib.attn_set_kernel_events.restype = ctypes.c_int
     lib.attn_set_kernel_events.argtypes = [vp, vp]
     _LIB = lib
@@ -327,6 +330,17 @@ def attn_get_status(workspace: torch.Tensor, stream=None) -> int:
     if rc not in (ATTN_OK, ATTN_ERR_DEVICE):
         raise AttnError(rc, "attn_get_status")
     return int(bits.value)
+
+
+def attn_selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> None:
+    """Enqueue the failure-detection self-test: a wait that nothing completes
+    runs out after its limit (2 s) and sets ATTN_DEVERR_TIMEOUT in the status
+    word of `workspace` (a device tensor of at least 256 bytes); read it with
+    attn_get_status."""
+    rc = load_library().attn_selftest_wait_timeout(workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                                   _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_selftest_wait_timeout")
 
 
 def attn_set_kernel_events(begin: "torch.cuda.Event | None", end: "torch.cuda.Event | None") -> None:

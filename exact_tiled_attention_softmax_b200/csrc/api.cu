@@ -526,6 +526,15 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
   return cuda_status(e);
 }
 
+attn_status attn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, void* stream) {
+  attn_status st;
+  if ((st = check_workspace(workspace, workspace_bytes, kStatusBytes)) != ATTN_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, kStatusBytes, cs) != cudaSuccess) return ATTN_ERR_CUDA;
+  return cuda_status(launch_wait_timeout_probe(status, cs));
+}
+
 attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits) {
   if (!workspace || !device_bits) return ATTN_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);

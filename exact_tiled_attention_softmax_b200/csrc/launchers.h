@@ -36,5 +36,8 @@ cudaError_t launch_lse_to_total(const float* in, int n0, int n1, int n2, const i
 cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta, int n_outer, int n_heads,
                          int n_inner, int64_t sl_outer, int64_t sl_head, int64_t sl_inner,
                          bool delta_head_major, float* dsink, cudaStream_t st);
+// One CTA that waits on an mbarrier phase nothing completes, until the bounded
+// wait gives up and sets the timeout bit in *status.
+cudaError_t launch_wait_timeout_probe(uint32_t* status, cudaStream_t st);
 
 }  // namespace attn

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ATTN_VERSION 106 /* major * 100 + minor */
+#define ATTN_VERSION 107 /* major * 100 + minor */
 
 typedef enum attn_status {
   ATTN_OK = 0,
@@ -246,6 +246,19 @@ attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits
  * finishing kernels around it (tile classes, delta, the dq cast) fall
  * outside the pair. NULL, NULL cancels a pending pair. Always ATTN_OK. */
 attn_status attn_set_kernel_events(void* begin, void* end);
+
+/* Failure-detection self-test; no attention arithmetic. Clears the status
+ * word at the start of `workspace`, then enqueues on `stream` one CTA whose
+ * threads wait, through the same bounded mbarrier wait that every stage of
+ * the tensor-core pipelines uses, on a barrier phase that nothing completes.
+ * When the wait's limit (2 s) runs out the kernel sets ATTN_DEVERR_TIMEOUT in
+ * the status word and returns: no trap, and the context stays usable.
+ * attn_get_status on the same workspace then returns ATTN_ERR_DEVICE with
+ * that bit. workspace: device memory owned by the caller, 256-byte aligned,
+ * at least 256 bytes. Returns ATTN_ERR_WORKSPACE for a missing, misaligned
+ * or smaller workspace, ATTN_ERR_CUDA when the clear or the launch fails,
+ * otherwise ATTN_OK once the work is enqueued. */
+attn_status attn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Static, human-readable text for a status code. */
 const char* attn_status_string(attn_status status);

@@ -217,3 +217,11 @@ def test_fp16_lse_formats_and_reverse_flags_on_host(lib):
     det = eta.AttnMaskC()
     det.bwd_flags = eta.ATTN_BWD_DETERMINISTIC
     assert _call_fwd(lib, q, k, v, o, lse, mask=det, ws_bytes=16) == eta.ATTN_ERR_WORKSPACE
+
+
+def test_selftest_rejects_bad_workspace_on_host(lib):
+    import exact_tiled_attention_softmax_b200 as eta
+    # Each is refused before any CUDA call is made.
+    assert lib.attn_selftest_wait_timeout(None, 256, None) == eta.ATTN_ERR_WORKSPACE
+    assert lib.attn_selftest_wait_timeout(0x100000, 128, None) == eta.ATTN_ERR_WORKSPACE
+    assert lib.attn_selftest_wait_timeout(0x100010, 256, None) == eta.ATTN_ERR_WORKSPACE
