@@ -67,6 +67,36 @@ def allowed_pairs(case: W.DenseCase) -> int:
     return int(case.B * case.Hq * total)
 
 
+def conventional_flops(case: W.DenseCase):
+    """The FlashAttention-style count for a purely causal dense workload: the
+    dense count B Hq T^2 (8d + 6dv) halved, i.e. T^2/2 pairs per head where
+    the algorithmic count has T(T+1)/2. None for other allowed sets, where
+    that convention has no agreed meaning."""
+    if not case.causal or case.window_left or case.block_size:
+        return None
+    return case.B * case.Hq * case.T * case.T * (8 * case.d + 6 * case.dv) // 2
+
+
+def conventional_rate(config: dict, value: float, flops_step: float):
+    """`value` (algorithmic TFLOP/s) restated under the conventional count
+    recorded in `config`, or None when the workload has none."""
+    conv = config.get("conventional_flops_per_step")
+    if not conv:
+        return None
+    return {"flops_per_step": conv, "tflops": value * conv / flops_step,
+            "rule": "dense count halved for causal (T^2/2 pairs per head, not T(T+1)/2)"}
+
+
+def topk_gather_rate(config: dict, fwd_kernel_ms: float):
+    """Bytes of listed KV rows the top-k forward gathers (every listed row of
+    Dqk 16-bit values, once per query token) and their rate over the forward
+    kernel's time; None for dense workloads."""
+    nbytes = config.get("gathered_bytes_per_pass")
+    if not nbytes:
+        return None
+    return {"bytes_per_pass": nbytes, "fwd_gbs": nbytes / (fwd_kernel_ms / 1e3) / 1e9}
+
+
 def fp32_alu_peak_tflops(sm_mhz: float) -> float:
     """Dense fp32 FFMA rate: 148 SMs x 128 lanes x 2 flops x clock."""
     return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -254,6 +284,8 @@ def dense_problem(case: W.DenseCase, dev, torch, eta, deterministic: bool = Fals
               "dv": case.dv, "mask": mask}
     if deterministic:
         config["reverse"] = "deterministic (dQ from the query-centric pass)"
+    if conventional_flops(case):
+        config["conventional_flops_per_step"] = conventional_flops(case)
     return Problem(case.name, allowed_pairs(case), 2 * case.d + 2 * case.dv, 6 * case.d + 4 * case.dv,
                    [tq, tk, tv, tg], [dq, dk, dv],
                    lambda: eta.attn_fwd(tq, tk, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
@@ -280,7 +312,8 @@ def topk_problem(case: W.TopkCase, dev, torch, eta) -> Problem:
     ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tkv, tv, allowed), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tkv, tv, allowed), dtype=torch.uint8, device=dev)
     config = {"workload": case.name, "Tq": case.Tq, "Tkv": case.Tkv, "H": case.H, "Dqk": case.Dqk, "Dv": case.Dv,
-              "mask": f"top-k lists, lengths U[{case.len_lo},{case.len_hi}], sink"}
+              "mask": f"top-k lists, lengths U[{case.len_lo},{case.len_hi}], sink",
+              "gathered_bytes_per_pass": int(ln.astype(np.int64).sum()) * case.Dqk * 2}
     return Problem(case.name, case.H * int(ln.astype(np.int64).sum()), 2 * case.Dqk + 2 * case.Dv,
                    6 * case.Dqk + 4 * case.Dv, [tq, tkv, tg], [dq, dkv],
                    lambda: eta.attn_fwd(tq, tkv, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
@@ -477,6 +510,8 @@ def main():
             "config": config,
             "pct_of_peak": {"measured_bf16_burst": 100 * value / world / float(peaks["bf16_tflops"]),
                             "nvidia_dense_bf16_spec_2250": 100 * value / world / 2250.0},
+            "conventional": conventional_rate(prob.config, value, flops_step),
+            "gather": topk_gather_rate(prob.config, fwd_kernel_ms),
             "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_flops / (fwd_ms / 1e3) / 1e12,
             "bwd_tflops": bwd_flops / (bwd_ms / 1e3) / 1e12,
             "kernels": {"fwd_main": {"ms": fwd_kernel_ms, "tflops": fwd_flops / (fwd_kernel_ms / 1e3) / 1e12},

@@ -72,3 +72,22 @@ def test_deterministic_reverse_has_no_borrowed_traffic():
     rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
     if "causal_8k_deterministic" not in rec.get("bwd_kernel", {}):
         assert bench.recorded_traffic("bwd_kernel", "causal_8k_deterministic") is None
+
+
+def test_conventional_count_is_the_dense_half_for_causal_only():
+    for name in ("causal_8k", "causal_2k", "gqa_dropout_16k"):
+        case = W.WORKLOADS[name]
+        conv = bench.conventional_flops(case)
+        alg = bench.allowed_pairs(case) * (8 * case.d + 6 * case.dv)
+        # T^2/2 pairs per head against the algorithmic T(T+1)/2
+        assert conv * (case.T + 1) == alg * case.T
+    assert bench.conventional_flops(W.WORKLOADS["window_block_8k"]) is None
+    r = bench.conventional_rate({"conventional_flops_per_step": 900}, 830.0, 1000.0)
+    assert abs(r["tflops"] - 747.0) < 1e-9 and r["flops_per_step"] == 900
+    assert bench.conventional_rate({}, 830.0, 1000.0) is None
+
+
+def test_topk_gather_rate():
+    got = bench.topk_gather_rate({"gathered_bytes_per_pass": 7_000_000_000}, 3.5)
+    assert abs(got["fwd_gbs"] - 2000.0) < 1e-9
+    assert bench.topk_gather_rate({}, 3.5) is None
