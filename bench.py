@@ -211,6 +211,11 @@ def cpu_baseline(case: W.DenseCase, budget_s: float = 12.0):
                       f"{el:.1f} s; oracle BLAS threads = all host cores"}
 
 
+def reference_ms_per_step(flops_step: float, tflops: float):
+    """Time one full step would take at the rate the sampled slices ran."""
+    return flops_step / (tflops * 1e12) * 1e3 if tflops > 0 else None
+
+
 def run_reference(args, case, rank, world):
     """--impl reference: the oracle is the reference arm (rank 0 only)."""
     if rank != 0:
@@ -223,11 +228,15 @@ def run_reference(args, case, rank, world):
     v = statistics.median(vals)
     cb = cpu_baseline(case, budget_s=1.0)
     cb["value"] = v
+    pairs = allowed_pairs(case)
+    config = dense_config(case)
+    config.update({"allowed_pairs": pairs, "flops_per_pair": case.flops_per_pair})
     line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": case.name, "B": case.B, "H": case.Hq, "T": case.T, "d": case.d,
-                       "mask": "causal"},
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": reference_ms_per_step(pairs * case.flops_per_pair, v),
+            "ms_per_step_basis": "the full workload's flops at the sampled slices' rate",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -263,6 +272,20 @@ class Problem:
         self.config, self.bound, self.launches = config, bound, launches
 
 
+def dense_config(case: W.DenseCase, deterministic: bool = False) -> dict:
+    """The `config` object both arms print for a dense workload."""
+    mask = "causal" + (f" & window {case.window_left}" if case.window_left else "") + \
+        (f" & {case.block_size}-blocks p={case.block_p_keep}" if case.block_size else "") + \
+        (f", dropout {case.dropout_p}" if case.dropout_p else "")
+    config = {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "T": case.T, "d": case.d,
+              "dv": case.dv, "mask": mask}
+    if deterministic:
+        config["reverse"] = "deterministic (dQ from the query-centric pass)"
+    if conventional_flops(case):
+        config["conventional_flops_per_step"] = conventional_flops(case)
+    return config
+
+
 def dense_problem(case: W.DenseCase, dev, torch, eta, deterministic: bool = False) -> Problem:
     q, k, v, g = W.dense_inputs(case)
     tq, tk, tv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v, g))
@@ -277,15 +300,7 @@ def dense_problem(case: W.DenseCase, dev, torch, eta, deterministic: bool = Fals
     dq, dk, dv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
     ws_f = torch.empty(eta.attn_fwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tk, tv, allowed), dtype=torch.uint8, device=dev)
-    mask = "causal" + (f" & window {case.window_left}" if case.window_left else "") + \
-        (f" & {case.block_size}-blocks p={case.block_p_keep}" if case.block_size else "") + \
-        (f", dropout {case.dropout_p}" if case.dropout_p else "")
-    config = {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "T": case.T, "d": case.d,
-              "dv": case.dv, "mask": mask}
-    if deterministic:
-        config["reverse"] = "deterministic (dQ from the query-centric pass)"
-    if conventional_flops(case):
-        config["conventional_flops_per_step"] = conventional_flops(case)
+    config = dense_config(case, deterministic)
     return Problem(case.name, allowed_pairs(case), 2 * case.d + 2 * case.dv, 6 * case.d + 4 * case.dv,
                    [tq, tk, tv, tg], [dq, dk, dv],
                    lambda: eta.attn_fwd(tq, tk, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),

@@ -91,3 +91,16 @@ def test_topk_gather_rate():
     got = bench.topk_gather_rate({"gathered_bytes_per_pass": 7_000_000_000}, 3.5)
     assert abs(got["fwd_gbs"] - 2000.0) < 1e-9
     assert bench.topk_gather_rate({}, 3.5) is None
+
+
+def test_both_arms_name_the_workload_alike():
+    case = W.WORKLOADS["causal_8k"]
+    cfg = bench.dense_config(case)
+    assert {"workload", "B", "Hq", "Hkv", "T", "d", "dv", "mask"} <= set(cfg)
+    assert cfg["workload"] == "causal_8k" and cfg["mask"] == "causal"
+    assert cfg["conventional_flops_per_step"] == bench.conventional_flops(case)
+    assert "reverse" in bench.dense_config(case, deterministic=True)
+    # 1.924 TFLOP at 0.0192 TFLOP/s is about 100 s per full step
+    flops = bench.allowed_pairs(case) * case.flops_per_pair
+    assert abs(bench.reference_ms_per_step(flops, flops / 1e14) - 1e5) < 1e-6
+    assert bench.reference_ms_per_step(flops, 0.0) is None
