@@ -144,6 +144,26 @@ def _ref(c):
     return ctypes.byref(c) if c is not None else None
 
 
+def _check_on(device: torch.device, *tensors) -> None:
+    """Every tensor a kernel reads or writes must sit on `device`, a CUDA
+    device: the library receives raw pointers and cannot tell a host
+    pointer, or another GPU's, from its own."""
+    if device.type != "cuda":
+        raise ValueError(f"attention tensors must be CUDA tensors (got {device})")
+    for t in tensors:
+        if t is not None and t.device != device:
+            raise ValueError(f"a tensor is on {t.device}, the query on {device}")
+
+
+def _check_mask_tensor(t: torch.Tensor, name: str, dtypes, dims) -> None:
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
+    if t.dim() not in dims:
+        raise ValueError(f"{name}: {t.dim()} dimensions, expected {' or '.join(map(str, dims))}")
+    if t.numel() > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name}: the innermost dimension must be contiguous")
+
+
 @dataclass
 class AllowedSet:
     """The allowed-set descriptor (attn_mask). Tensors must live on the GPU.
@@ -174,7 +194,23 @@ class AllowedSet:
     lse_neg_log2: bool = False
     deterministic: bool = False
 
+    def tensors(self) -> list:
+        """The device tensors the descriptor points at."""
+        return [t for t in (self.block_mask, self.topk_idxs, self.topk_length, self.sink, self.lengths,
+                            self.starts) if t is not None]
+
     def to_c(self) -> AttnMaskC:
+        """The C descriptor. Checks each tensor's dtype and rank first, since
+        the library sees only its pointer and strides."""
+        for t, name, dtypes, dims in (
+                (self.block_mask, "block_mask", (torch.uint8, torch.bool), (2, 4)),
+                (self.topk_idxs, "topk_idxs", (torch.int32,), (2,)),
+                (self.topk_length, "topk_length", (torch.int32,), (1,)),
+                (self.sink, "sink", (torch.float32,), (1,)),
+                (self.lengths, "lengths", (torch.int32,), (1,)),
+                (self.starts, "starts", (torch.int32,), (1, 2))):
+            if t is not None:
+                _check_mask_tensor(t, name, dtypes, dims)
         m = AttnMaskC()
         flags = 0
         if self.causal:
@@ -265,8 +301,9 @@ def attn_fwd(q, k, v, allowed: AllowedSet | None = None, scale: float | None = N
     need = lib.attn_fwd_workspace_size(_ref(cq), _ref(ck), _ref(cv), _ref(m))
     if workspace is None:
         workspace = _workspace(need, q.device)
+    _check_on(q.device, k, v, out, lse, workspace, *(allowed.tensors() if allowed else ()))
     rc = lib.attn_fwd(_ref(cq), _ref(ck), _ref(cv), _ref(m), ctypes.c_float(scale), _ref(co), _ref(cl),
-                      workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
     return out, lse
@@ -294,10 +331,12 @@ def attn_bwd(q, k, v, o, do, lse, allowed: AllowedSet | None = None, scale: floa
     need = lib.attn_bwd_workspace_size(_ref(cq), _ref(ck), _ref(cv), _ref(m))
     if workspace is None:
         workspace = _workspace(need, q.device)
+    _check_on(q.device, k, v, o, do, lse, dq, dk, dv, dsink, workspace,
+              *(allowed.tensors() if allowed else ()))
     rc = lib.attn_bwd(_ref(cq), _ref(ck), _ref(cv), _ref(co), _ref(cdo), _ref(cl), _ref(m),
                       ctypes.c_float(scale), _ref(cdq), _ref(cdk), _ref(cdv),
                       dsink.data_ptr() if dsink is not None else None,
-                      workspace.data_ptr(), workspace.numel(), _stream_handle(stream))
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_bwd")
     return dq, dk, (None if topk else dv), dsink
@@ -315,6 +354,7 @@ def attn_bwd_noalloc(q, k, v, o, do, lse, allowed: AllowedSet | None = None, sca
     m = allowed.to_c() if allowed else None
     cq, ck, cv, co, cdo, cl = (_tensor(x) for x in (q, k, v, o, do, lse))
     cdq, cdk, cdv = _tensor(dq), _tensor(dk), _tensor(dv)
+    _check_on(q.device, k, v, o, do, lse, dq, dk, dv, dsink, *(allowed.tensors() if allowed else ()))
     rc = lib.attn_bwd_noalloc(_ref(cq), _ref(ck), _ref(cv), _ref(co), _ref(cdo), _ref(cl), _ref(m),
                               ctypes.c_float(scale), _ref(cdq), _ref(cdk), _ref(cdv),
                               dsink.data_ptr() if dsink is not None else None, _stream_handle(stream))

@@ -225,3 +225,36 @@ def test_selftest_rejects_bad_workspace_on_host(lib):
     assert lib.attn_selftest_wait_timeout(None, 256, None) == eta.ATTN_ERR_WORKSPACE
     assert lib.attn_selftest_wait_timeout(0x100000, 128, None) == eta.ATTN_ERR_WORKSPACE
     assert lib.attn_selftest_wait_timeout(0x100010, 256, None) == eta.ATTN_ERR_WORKSPACE
+
+
+def test_binding_checks_mask_tensors_before_the_library_sees_them(lib):
+    import torch
+
+    import exact_tiled_attention_softmax_b200 as eta
+    ok_bm = torch.ones(4, 4, dtype=torch.uint8)
+    eta.AllowedSet(block_mask=ok_bm).to_c()
+    eta.AllowedSet(block_mask=ok_bm.bool()[None, None]).to_c()
+    bad = [
+        dict(block_mask=ok_bm[None]),                               # 3-D grid would be misread
+        dict(block_mask=ok_bm.to(torch.int32)),
+        dict(block_mask=ok_bm.t().contiguous().t()),                # columns not contiguous
+        dict(topk_idxs=torch.zeros(4, 8, dtype=torch.int64)),
+        dict(topk_idxs=torch.zeros(4, 8, dtype=torch.int32), topk_length=torch.zeros(4, dtype=torch.int64)),
+        dict(sink=torch.zeros(4, dtype=torch.float64)),
+        dict(lengths=torch.zeros(2, 1, dtype=torch.int32)),
+        dict(starts=torch.zeros(2, 3, 4, dtype=torch.int32)),
+    ]
+    for kw in bad:
+        with pytest.raises(ValueError):
+            eta.AllowedSet(**kw).to_c()
+
+
+def test_binding_refuses_host_tensors(lib):
+    import torch
+
+    import exact_tiled_attention_softmax_b200 as eta
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        eta.attn_fwd(q, q, q, eta.AllowedSet(causal=True), 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        eta.attn_bwd(q, q, q, q, q, torch.zeros(1, 2, 8), None, 0.1)
