@@ -104,3 +104,11 @@ def test_both_arms_name_the_workload_alike():
     flops = bench.allowed_pairs(case) * case.flops_per_pair
     assert abs(bench.reference_ms_per_step(flops, flops / 1e14) - 1e5) < 1e-6
     assert bench.reference_ms_per_step(flops, 0.0) is None
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    import argparse
+    args = argparse.Namespace(steps=1, warmup=0)
+    # Any rank but 0 leaves at once, with nothing printed and no oracle work.
+    assert bench.run_reference(args, W.WORKLOADS["causal_8k"], rank=1, world=2) is None
+    assert capsys.readouterr().out == ""
