@@ -258,3 +258,31 @@ def test_binding_refuses_host_tensors(lib):
         eta.attn_fwd(q, q, q, eta.AllowedSet(causal=True), 0.1)
     with pytest.raises(ValueError, match="CUDA"):
         eta.attn_bwd(q, q, q, q, q, torch.zeros(1, 2, 8), None, 0.1)
+
+
+def test_a_plain_c_program_links_and_calls_the_library(lib, tmp_path):
+    """tests/c_abi_caller.c links against libattn.so with no Python in
+    between; its workspace sizes equal the ctypes calls' and the library
+    refuses its bad call on the host."""
+    import shutil
+    import subprocess
+    import exact_tiled_attention_softmax_b200 as eta
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    libdir = os.path.dirname(eta.library_path())
+    cuda_lib = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
+    exe = tmp_path / "caller"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_caller.c"), "-o", str(exe),
+                    "-L", libdir, "-l:libattn.so", f"-Wl,-rpath,{libdir}", "-L", cuda_lib,
+                    f"-Wl,-rpath-link,{cuda_lib}"], check=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, run.stdout + run.stderr
+    words = run.stdout.split()
+    q, k, v = _t([1, 4, 300, 128]), _t([1, 2, 300, 128]), _t([1, 2, 300, 128])
+    m = eta.AllowedSet(causal=True).to_c()
+    refs = [ctypes.byref(x) for x in (q, k, v, m)]
+    assert int(words[1]) == lib.attn_fwd_workspace_size(*refs)
+    assert int(words[3]) == lib.attn_bwd_workspace_size(*refs)
+    assert int(words[5]) == eta.ATTN_ERR_INVALID_ARG
