@@ -31,6 +31,7 @@ ATTN_ERR_DEVICE = 5
 ATTN_DEVERR_TOPK_INDEX = 0x1
 ATTN_DEVERR_OVERFLOW = 0x2
 ATTN_DEVERR_TIMEOUT = 0x4
+ATTN_DEVERR_TOPK_CAUSAL = 0x8
 
 ATTN_F32 = 0
 ATTN_BF16 = 1
@@ -42,6 +43,7 @@ ATTN_MASK_BLOCK = 0x4
 ATTN_MASK_TOPK = 0x8
 ATTN_MASK_LENGTHS = 0x10
 ATTN_MASK_STARTS = 0x20
+ATTN_MASK_TOPK_CHECK_CAUSAL = 0x40
 ATTN_LSE_KV_ONLY = 0x1
 ATTN_LSE_NEG_LOG2 = 0x2
 ATTN_BWD_DETERMINISTIC = 0x1
@@ -176,6 +178,8 @@ class AllowedSet:
     lse_kv_only / lse_neg_log2 select the LSE format that attn_fwd writes
     and attn_bwd expects: the sink left out, and/or stored as -log2 Z.
     deterministic makes every gradient of attn_bwd bitwise reproducible.
+    topk_check_causal turns on the debug check of the top-k lists against
+    each token's causal position (ATTN_DEVERR_TOPK_CAUSAL in the status).
     """
     causal: bool = False
     window_left: int = 0
@@ -193,6 +197,7 @@ class AllowedSet:
     lse_kv_only: bool = False
     lse_neg_log2: bool = False
     deterministic: bool = False
+    topk_check_causal: bool = False
 
     def tensors(self) -> list:
         """The device tensors the descriptor points at."""
@@ -236,6 +241,8 @@ class AllowedSet:
             m.topk_stride = self.topk_idxs.stride(0)
             m.topk_max = int(self.topk_max if self.topk_max is not None else self.topk_idxs.shape[1])
             m.topk_length = self.topk_length.data_ptr() if self.topk_length is not None else 0
+            if self.topk_check_causal:
+                flags |= ATTN_MASK_TOPK_CHECK_CAUSAL
         if self.lengths is not None:
             flags |= ATTN_MASK_LENGTHS
             m.lengths = self.lengths.data_ptr()
@@ -363,10 +370,13 @@ def attn_bwd_noalloc(q, k, v, o, do, lse, allowed: AllowedSet | None = None, sca
     return dq, dk, dv, dsink
 
 
-def attn_get_status(workspace: torch.Tensor, stream=None) -> int:
-    """Synchronise and return (then clear) the device status bits."""
+def attn_get_status(workspace: torch.Tensor | None, stream=None) -> int:
+    """Synchronise and return (then clear) the device status bits of a
+    workspace, or with workspace=None those of attn_bwd_noalloc's fixed
+    scratch array on the current device."""
     bits = ctypes.c_uint32(0)
-    rc = load_library().attn_get_status(workspace.data_ptr(), _stream_handle(stream), ctypes.byref(bits))
+    ptr = workspace.data_ptr() if workspace is not None else None
+    rc = load_library().attn_get_status(ptr, _stream_handle(stream), ctypes.byref(bits))
     if rc not in (ATTN_OK, ATTN_ERR_DEVICE):
         raise AttnError(rc, "attn_get_status")
     return int(bits.value)

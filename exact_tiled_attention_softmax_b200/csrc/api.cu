@@ -48,8 +48,9 @@ uint32_t flags_of(const attn_mask* m) { return m ? m->flags : 0u; }
 attn_status check_mask(const attn_mask* m) {
   if (!m) return ATTN_OK;
   const uint32_t known = ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_BLOCK | ATTN_MASK_TOPK |
-                         ATTN_MASK_LENGTHS | ATTN_MASK_STARTS;
+                         ATTN_MASK_LENGTHS | ATTN_MASK_STARTS | ATTN_MASK_TOPK_CHECK_CAUSAL;
   if (m->flags & ~known) return ATTN_ERR_INVALID_ARG;
+  if ((m->flags & ATTN_MASK_TOPK_CHECK_CAUSAL) && !(m->flags & ATTN_MASK_TOPK)) return ATTN_ERR_INVALID_ARG;
   if ((m->flags & ATTN_MASK_WINDOW) && m->window_left < 1) return ATTN_ERR_INVALID_ARG;
   if (m->flags & ATTN_MASK_BLOCK) {
     if (!m->block_mask || m->block_q < 1 || m->block_k < 1) return ATTN_ERR_INVALID_ARG;
@@ -171,7 +172,7 @@ size_t lse_copy_bytes(const attn_mask* m, size_t rows) {
 size_t bwd_topk_bytes(const Topk& s, const attn_tensor* q, const attn_mask* m) {
   size_t n = kStatusBytes;
   n += align_up((size_t)s.Tq * s.H * sizeof(float), 256);                       // delta
-  n += align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);      // 32.32 dKV
+  n += topk_acc_total_bytes(s.Tkv, s.Dqk);                                      // 32.32 dKV, counts, bound
   if (q->dtype != ATTN_F32)                                                     // G, P rows (tensor-core path)
     n += align_up(attn::sm100_topk_bwd_scratch_bytes(s.Tq, s.H, s.Dqk, s.Dv, m->topk_max), 256);
   return n + lse_copy_bytes(m, (size_t)s.Tq * s.H);
@@ -289,6 +290,7 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.scale = scale;
     p.sink = mask->sink;
     p.lse_fmt = mask->lse_format;
+    p.check_causal = (mask->flags & ATTN_MASK_TOPK_CHECK_CAUSAL) ? 1 : 0;
     if (sm100_topk_supported(p, q, k, o))
       return cuda_status(sm100_topk_fwd(p, o->data, o->stride[0], o->stride[1], static_cast<float*>(lse->data),
                                         lse->stride[0], lse->stride[1], status, cs));
@@ -380,8 +382,8 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     if ((st = check_workspace(workspace, workspace_bytes, bwd_topk_bytes(s, q, mask))) != ATTN_OK) return st;
     if (cudaMemsetAsync(status, 0, kStatusBytes, cs) != cudaSuccess) return ATTN_ERR_CUDA;
     float* delta = reinterpret_cast<float*>(ws + kStatusBytes);
-    unsigned long long* acc = reinterpret_cast<unsigned long long*>(
-        ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256));
+    const FixedAcc acc = fixed_acc_at(ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256), s.Tkv,
+                                      s.Dqk);
     TopkP p;
     p.q = q->data;
     p.kv = k->data;
@@ -401,6 +403,7 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
     p.scale = scale;
     p.sink = mask->sink;
     p.lse_fmt = mask->lse_format;
+    p.check_causal = (mask->flags & ATTN_MASK_TOPK_CHECK_CAUSAL) ? 1 : 0;
     const int64_t so[3] = {0, o->stride[0], o->stride[1]}, sg[3] = {0, do_->stride[0], do_->stride[1]};
     cudaError_t e = cudaSuccess;
     const float* lsep = static_cast<const float*>(lse->data);
@@ -419,15 +422,15 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       // Tensor cores: dQ and the per-token dKV contributions; the fixed-point
       // accumulator starts at zero and is cast to dKV at the end.
       char* scratch = ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256) +
-                      align_up((size_t)s.Tkv * s.Dqk * sizeof(unsigned long long), 256);
+                      topk_acc_total_bytes(s.Tkv, s.Dqk);
       e = by_storage(q->dtype, [&](auto t) {
         using T = decltype(t);
         cudaError_t r = launch_rows_delta<T>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
-        if (r == cudaSuccess) r = cudaMemsetAsync(acc, 0, sizeof(unsigned long long) * (size_t)s.Tkv * s.Dqk, cs);
+        if (r == cudaSuccess) r = cudaMemsetAsync(acc.acc, 0, topk_acc_total_bytes(s.Tkv, s.Dqk), cs);
         if (r == cudaSuccess)
           r = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta, dq->data,
                              dq->stride[0], dq->stride[1], acc, scratch, status, cs);
-        if (r == cudaSuccess) r = launch_fixed_to_out<T>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
+        if (r == cudaSuccess) r = launch_fixed_to_out<T>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], status, cs);
         return r;
       });
     } else {
@@ -536,8 +539,12 @@ attn_status attn_selftest_wait_timeout(void* workspace, size_t workspace_bytes, 
 }
 
 attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits) {
-  if (!workspace || !device_bits) return ATTN_ERR_INVALID_ARG;
+  if (!device_bits) return ATTN_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (!workspace) {  // the status word of attn_bwd_noalloc's array on the current device
+    attn_status st;
+    if (!(workspace = attn::noalloc_status_word(cs, &st))) return st;
+  }
   if (cudaStreamSynchronize(cs) != cudaSuccess) return ATTN_ERR_CUDA;
   uint32_t bits = 0;
   if (cudaMemcpy(&bits, workspace, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;

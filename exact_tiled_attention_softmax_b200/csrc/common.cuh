@@ -74,6 +74,7 @@ struct TopkP {
   float scale;
   const float* sink;
   uint32_t lse_fmt;  // ATTN_LSE_* bits of the LSE output
+  int32_t check_causal;  // ATTN_MASK_TOPK_CHECK_CAUSAL: flag listed indices past Tkv - Tq + t
 };
 
 // The LSE value to store for a row, from base-2 quantities: lse2_total =
@@ -196,6 +197,56 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
+}
+
+// The debug check of a valid listed index j of token t against the token's
+// causal position Tkv - Tq + t (ATTN_MASK_TOPK_CHECK_CAUSAL).
+__device__ __forceinline__ void check_topk_causal(int check, int64_t j, int t, int Tq, int Tkv, uint32_t* status) {
+  if (check && j > (int64_t)Tkv - Tq + t) set_status(status, ATTN_DEVERR_TOPK_CAUSAL);
+}
+
+// The fixed-point dKV accumulator of the top-k reverse: [Tkv, Dqk] signed
+// 32.32 integers, then per KV row the number of contributions it received,
+// then one word holding the largest contribution magnitude of the call (the
+// bit pattern of a non-negative float, ordered like the value). The counts
+// and the magnitude bound every row's sum (|sum| <= count * largest), which
+// the conversion to the output checks against the accumulator's range.
+inline size_t topk_acc_bytes(int Tkv, int Dqk) { return align_up((size_t)Tkv * Dqk * sizeof(unsigned long long), 256); }
+inline size_t topk_acc_total_bytes(int Tkv, int Dqk) {
+  return topk_acc_bytes(Tkv, Dqk) + align_up(((size_t)Tkv + 1) * sizeof(uint32_t), 256);
+}
+struct FixedAcc {
+  unsigned long long* acc;  // [Tkv, Dqk]
+  uint32_t* count;          // [Tkv]
+  uint32_t* maxbits;        // one word
+};
+inline FixedAcc fixed_acc_at(void* base, int Tkv, int Dqk) {
+  FixedAcc f;
+  f.acc = static_cast<unsigned long long*>(base);
+  f.count = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + topk_acc_bytes(Tkv, Dqk));
+  f.maxbits = f.count + Tkv;
+  return f;
+}
+
+// One contribution x to a fixed-point dKV element: clamped to |x| < 2^30
+// (flagged), converted to 32.32 and added; *amax keeps the largest |x| seen.
+__device__ __forceinline__ void fixed_add(unsigned long long* dst, float x, bool& sat, float& amax) {
+  const float lim = 1073741824.f;  // 2^30: |x| 2^32 stays below 2^62
+  const float ax = fabsf(x);
+  if (!(ax < lim)) {
+    sat = true;
+    x = x != x ? 0.f : copysignf(lim, x);
+  }
+  amax = fmaxf(amax, fminf(ax, lim));
+  atomicAdd(dst, (unsigned long long)__float2ll_rn(x * 4294967296.f));
+}
+
+// The warp's largest contribution magnitude into the call's word (once per
+// warp; whole warp, converged).
+__device__ __forceinline__ void fixed_publish_max(uint32_t* maxbits, float amax) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0 && amax > 0.f) atomicMax(maxbits, __float_as_uint(amax));
 }
 
 // Caller-supplied timing events around the main kernel of the next call on

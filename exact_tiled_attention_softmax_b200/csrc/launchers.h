@@ -26,10 +26,12 @@ cudaError_t launch_dense_bwd_rows(const DenseP& p, const void* g, const int64_t 
 template <typename T>
 cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, int64_t sg_h,
                                  const float* lse, int64_t sl_t, int64_t sl_h, const float* delta,
-                                 void* dq, int64_t sd_t, int64_t sd_h, unsigned long long* acc_fixed,
+                                 void* dq, int64_t sd_t, int64_t sd_h, FixedAcc acc,
                                  void* dkv, int64_t sdkv, uint32_t* status, cudaStream_t st);
+// dKV from the fixed-point accumulator, with the per-row range check (sets
+// ATTN_DEVERR_OVERFLOW in *status when a row's sum may have wrapped).
 template <typename T>
-cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int cols, void* out, int64_t so,
+cudaError_t launch_fixed_to_out(FixedAcc acc, int rows, int cols, void* out, int64_t so, uint32_t* status,
                                 cudaStream_t st);
 cudaError_t launch_lse_to_total(const float* in, int n0, int n1, int n2, const int64_t s[3], int head_dim,
                                 const float* sink, uint32_t fmt, float* out, cudaStream_t st);
@@ -39,5 +41,8 @@ cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta
 // One CTA that waits on an mbarrier phase nothing completes, until the bounded
 // wait gives up and sets the timeout bit in *status.
 cudaError_t launch_wait_timeout_probe(uint32_t* status, cudaStream_t st);
+// Device address of attn_bwd_noalloc's status word on the current device
+// (the start of its fixed scratch array); null with *st set on failure.
+void* noalloc_status_word(cudaStream_t stream, attn_status* st);
 
 }  // namespace attn

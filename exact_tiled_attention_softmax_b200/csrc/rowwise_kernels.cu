@@ -128,6 +128,7 @@ topk_fwd_rows(TopkP p, T* o, int64_t so_t, int64_t so_h, float* lse, int64_t sl_
       if (lane == 0) set_status(status, ATTN_DEVERR_TOPK_INDEX);
       continue;
     }
+    if (lane == 0) check_topk_causal(p.check_causal, j, t, p.Tq, p.Tkv, status);
     const T* row = KV + (int64_t)j * p.skv;
     float kr[NQ];
     load_row(row, p.Dqk, lane, kr);
@@ -324,11 +325,12 @@ topk_dq_rows(TopkP p, const T* g, int64_t sg_t, int64_t sg_h, const float* lse, 
 // One warp per (token t, list position): the tied row contribution
 // C_j = sum_h (c gamma_thj Q_th + [p_thj G_th, 0]) added into a signed 32.32
 // fixed-point accumulator. Integer addition is associative, so the reduced
-// dKV does not depend on the order in which warps arrive.
+// dKV does not depend on the order in which warps arrive. The row's
+// contribution count and the largest magnitude feed the range check.
 template <typename T, int NQ, int NV>
 __global__ void __launch_bounds__(kWarps * 32)
 topk_dkv_pairs(TopkP p, const T* g, int64_t sg_t, int64_t sg_h, const float* lse, int64_t sl_t,
-               int64_t sl_h, const float* delta, unsigned long long* acc_fixed, uint32_t* status) {
+               int64_t sl_h, const float* delta, FixedAcc fa, uint32_t* status) {
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= (int64_t)p.Tq * p.topk_max) return;
@@ -340,6 +342,10 @@ topk_dkv_pairs(TopkP p, const T* g, int64_t sg_t, int64_t sg_h, const float* lse
   if (j < 0 || j >= p.Tkv) {
     if (lane == 0) set_status(status, ATTN_DEVERR_TOPK_INDEX);
     return;
+  }
+  if (lane == 0) {
+    check_topk_causal(p.check_causal, j, t, p.Tq, p.Tkv, status);
+    atomicAdd(fa.count + j, 1u);
   }
   const T* row = static_cast<const T*>(p.kv) + (int64_t)j * p.skv;
   float kr[NQ], vr[NV], ak[NQ], av[NV];
@@ -363,31 +369,31 @@ topk_dkv_pairs(TopkP p, const T* g, int64_t sg_t, int64_t sg_h, const float* lse
 #pragma unroll
     for (int c = 0; c < NV; ++c) av[c] = fmaf(pij, gr[c], av[c]);
   }
-  unsigned long long* dst = acc_fixed + (int64_t)j * p.Dqk;
+  unsigned long long* dst = fa.acc + (int64_t)j * p.Dqk;
   bool sat = false;
+  float amax = 0.f;
 #pragma unroll
   for (int c = 0; c < NQ; ++c) {
     const int idx = lane + 32 * c;
-    if (idx < p.Dqk) {
-      float x = ak[c] + (c < NV && idx < p.Dv ? av[c] : 0.f);
-      const float lim = 1073741824.f;  // 2^30: |x| 2^32 must stay below 2^62
-      if (!(fabsf(x) < lim)) {
-        sat = true;
-        x = x != x ? 0.f : copysignf(lim, x);
-      }
-      const long long fx = __float2ll_rn(x * 4294967296.f);
-      atomicAdd(dst + idx, (unsigned long long)fx);
-    }
+    if (idx < p.Dqk) fixed_add(dst + idx, ak[c] + (c < NV && idx < p.Dv ? av[c] : 0.f), sat, amax);
   }
+  fixed_publish_max(fa.maxbits, amax);
   if (__any_sync(0xffffffffu, sat) && lane == 0) set_status(status, ATTN_DEVERR_OVERFLOW);
 }
 
+// dKV = the fixed-point sums in the output type. The first element of each
+// row also checks the row's bound: count * largest contribution < 2^31 means
+// no partial order of additions can have left the 32.32 range, so the
+// integer sum is exact; otherwise the row may have wrapped and the overflow
+// bit is set.
 template <typename T>
-__global__ void fixed_to_out(const unsigned long long* acc, int rows, int cols, T* out, int64_t so) {
+__global__ void fixed_to_out(FixedAcc fa, int rows, int cols, T* out, int64_t so, uint32_t* status) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (int64_t)rows * cols) return;
   const int r = (int)(e / cols), c = (int)(e % cols);
-  const long long v = (long long)acc[e];
+  if (c == 0 && (double)fa.count[r] * (double)__uint_as_float(*fa.maxbits) >= 2147483648.0)
+    set_status(status, ATTN_DEVERR_OVERFLOW);
+  const long long v = (long long)fa.acc[e];
   st(out + (int64_t)r * so + c, (float)((double)v * (1.0 / 4294967296.0)));
 }
 
@@ -493,11 +499,11 @@ cudaError_t launch_dense_bwd_rows(const DenseP& p, const void* g, const int64_t 
 template <typename T>
 cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, int64_t sg_h,
                                  const float* lse, int64_t sl_t, int64_t sl_h, const float* delta,
-                                 void* dq, int64_t sd_t, int64_t sd_h, unsigned long long* acc_fixed,
+                                 void* dq, int64_t sd_t, int64_t sd_h, FixedAcc fa,
                                  void* dkv, int64_t sdkv, uint32_t* status, cudaStream_t st) {
   const int w = width_class(p.Dqk > p.Dv ? p.Dqk : p.Dv);
   const int64_t rows = (int64_t)p.Tq * p.H, pairs = (int64_t)p.Tq * p.topk_max;
-  cudaError_t e = cudaMemsetAsync(acc_fixed, 0, sizeof(unsigned long long) * (size_t)p.Tkv * p.Dqk, st);
+  cudaError_t e = cudaMemsetAsync(fa.acc, 0, topk_acc_total_bytes(p.Tkv, p.Dqk), st);
   if (e != cudaSuccess) return e;
   if (rows > 0) {
     ATTN_DISPATCH_WIDTH(w,
@@ -505,20 +511,21 @@ cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, in
             p, static_cast<const T*>(g), sg_t, sg_h, lse, sl_t, sl_h, delta, static_cast<T*>(dq), sd_t,
             sd_h);
         if (pairs > 0) topk_dkv_pairs<T, NQ, NV><<<blocks_for_warps(pairs), kWarps * 32, 0, st>>>(
-            p, static_cast<const T*>(g), sg_t, sg_h, lse, sl_t, sl_h, delta, acc_fixed, status);)
+            p, static_cast<const T*>(g), sg_t, sg_h, lse, sl_t, sl_h, delta, fa, status);)
   }
   const int64_t n = (int64_t)p.Tkv * p.Dqk;
   if (n > 0)
-    fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(acc_fixed, p.Tkv, p.Dqk,
-                                                                 static_cast<T*>(dkv), sdkv);
+    fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(fa, p.Tkv, p.Dqk, static_cast<T*>(dkv), sdkv,
+                                                                 status);
   return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_fixed_to_out(const unsigned long long* acc, int rows, int cols, void* out, int64_t so,
+cudaError_t launch_fixed_to_out(FixedAcc fa, int rows, int cols, void* out, int64_t so, uint32_t* status,
                                 cudaStream_t st) {
   const int64_t n = (int64_t)rows * cols;
-  if (n > 0) fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(acc, rows, cols, static_cast<T*>(out), so);
+  if (n > 0)
+    fixed_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(fa, rows, cols, static_cast<T*>(out), so, status);
   return cudaGetLastError();
 }
 
@@ -580,9 +587,9 @@ cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta
                                                 const int64_t[3], cudaStream_t);                        \
   template cudaError_t launch_topk_bwd_rows<T>(const TopkP&, const void*, int64_t, int64_t,             \
                                                const float*, int64_t, int64_t, const float*, void*,     \
-                                               int64_t, int64_t, unsigned long long*, void*, int64_t,   \
+                                               int64_t, int64_t, FixedAcc, void*, int64_t,              \
                                                uint32_t*, cudaStream_t);                               \
-  template cudaError_t launch_fixed_to_out<T>(const unsigned long long*, int, int, void*, int64_t, cudaStream_t);
+  template cudaError_t launch_fixed_to_out<T>(FixedAcc, int, int, void*, int64_t, uint32_t*, cudaStream_t);
 
 ATTN_INSTANTIATE(float)
 ATTN_INSTANTIATE(__nv_bfloat16)

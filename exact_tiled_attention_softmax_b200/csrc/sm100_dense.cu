@@ -1,10 +1,12 @@
 // Tensor-core path for dense bf16 or fp16 attention with d = dv = 128 on sm_100a.
 //
-// Forward: one CTA per (128-row query tile, query head, batch row). A TMA
-// producer warp streams 128-key K/V tiles through a two-stage ring; one
-// thread issues tcgen05 MMAs (S = Q K^T into a double-buffered TMEM tile,
-// O += P V into a TMEM accumulator); a 128-thread softmax warpgroup owns one
-// row per thread (TMEM lane = row) and applies the running-summary update of
+// Forward: one CTA per (256 query rows, query head, batch row), held as two
+// 128-row query tiles. A TMA producer warp streams 128-key K/V tiles through
+// a two-stage ring; one thread issues tcgen05 MMAs (per query tile, S = Q K^T
+// into that tile's TMEM columns and O += P V into its TMEM accumulator, the
+// two tiles alternating on the tensor core); two 128-thread softmax
+// warpgroups, one per query tile, own one row per thread (TMEM lane = row)
+// and apply the running-summary update of
 // "Accumulate attention without keeping the full grid", section "Rescale
 // earlier mass before adding a new tile": tile maximum, new maximum, the
 // rescale factor alpha, shifted exponentials and the running sum, with empty
@@ -43,9 +45,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // move the running max only past 2^8
 constexpr int kPolyEvery = 4;              // forward: every k-th pair of exponentials on the FMA pipe (0: none)
 
-// Does pair e of a 16-pair chunk take its exponentials on the FMA pipe?
+// Does pair e of a 16-pair chunk take its exponentials on the FMA pipe? Not
+// with dropout: there the softmax warps also run Philox4x32-10, whose
+// multiplies share the pipe the polynomial would use.
+template <bool kDrop>
 __host__ __device__ constexpr bool poly_pair(int e) {
-  return kPolyEvery > 0 && e % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
+  return !kDrop && kPolyEvery > 0 && e % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1;
 }
 
 enum : uint8_t { kEmpty = 0, kFull = 1, kPartial = 2 };
@@ -401,7 +406,7 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
       const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sc2, nm2);
       float x0, x1;
       f2_unpack(x, x0, x1);
-      const uint64_t pp = poly_pair(e)
+      const uint64_t pp = poly_pair<kDrop>(e)
                               ? exp2_fma2(f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f)))
                               : f2_pack(ex2(x0), ex2(x1));
       if (e & 1)
@@ -1654,14 +1659,16 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
 }
 
 // Reverse-pass preparation: delta from the stored O and dO (kept, and negated
-// in the padded array) and the negated base-2 LSE. A half-warp reads one row
-// with 16-byte loads; a warp takes eight rows (B*Hq*Tpad is a multiple of 128,
-// so a warp's rows are all in range or all out).
+// in the padded array) and the negated base-2 LSE; with dq_acc set, the row's
+// 128 fp32 dQ accumulator entries are zeroed too (the key-centric kernel adds
+// into them). A half-warp reads one row with 16-byte loads; a warp takes eight
+// rows (B*Hq*Tpad is a multiple of 128, so a warp's rows are all in range or
+// all out).
 template <bool kH>
 __global__ void __launch_bounds__(256)
 bwd_prepare_kernel(const uint16_t* o, int64_t so0, int64_t so1, int64_t so2, const uint16_t* g,
                    int64_t sg0, int64_t sg1, int64_t sg2, const float* lse, int64_t sl0, int64_t sl1, int64_t sl2,
-                   int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta) {
+                   int B, int Hq, int T, int Tpad, float* lse2, float* dpad, float* delta, float* dq_acc) {
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31, hl = lane & 15;
   const int64_t nrows = (int64_t)B * Hq * Tpad;
@@ -1674,6 +1681,11 @@ bwd_prepare_kernel(const uint16_t* o, int64_t so0, int64_t so1, int64_t so2, con
     const int h = (int)(bh % Hq), b = (int)(bh / Hq);
     const bool live = valid && i < T;
     float s = 0.f;
+    if (live && dq_acc) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + (bh * T + i) * kD + hl * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (live) {
       const uint4 ov = *reinterpret_cast<const uint4*>(o + b * so0 + h * so1 + (int64_t)i * so2 + hl * 8);
       const uint4 gv = *reinterpret_cast<const uint4*>(g + b * sg0 + h * sg1 + (int64_t)i * sg2 + hl * 8);
@@ -1921,12 +1933,8 @@ cudaError_t sm100_dense_bwd(const DenseP& p, const void* o, const int64_t so[3],
   const int64_t rows = (int64_t)p.B * p.Hq * Tpad;  // a multiple of 128: eight rows per warp
   (f16 ? bwd_prepare_kernel<true> : bwd_prepare_kernel<false>)<<<(unsigned)((rows * 4 + 255) / 256), 256, 0, st>>>(
       static_cast<const uint16_t*>(o), so[0], so[1], so[2], static_cast<const uint16_t*>(g), sg[0], sg[1], sg[2], lse,
-      sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta);
+      sl[0], sl[1], sl[2], p.B, p.Hq, p.Tq, Tpad, lse2, dpad, delta, det ? nullptr : dq_acc);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  // The key-centric kernel adds its dQ partials into a zeroed accumulator
-  // (not used at all in the deterministic mode).
-  if (!det && (err = cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)p.B * p.Hq * p.Tq * kD, st)) != cudaSuccess)
-    return err;
   CUtensorMap mq, mk, mv, mg, mdq;
   if (!make_dq_map(&mdq, dq_acc, p.Tq, p.B * p.Hq) ||
       !make_map(&mq, p.q, p.Tq, p.Hq, p.B, p.sq[2], p.sq[1], p.sq[0], kBMb, f16) ||

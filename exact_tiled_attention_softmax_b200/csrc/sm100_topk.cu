@@ -77,6 +77,7 @@ struct TopkArgs {
   float* lse;
   int64_t sl_t, sl_h;
   uint32_t lse_fmt;
+  int check_causal;  // ATTN_MASK_TOPK_CHECK_CAUSAL
   uint32_t* status;
 };
 
@@ -147,6 +148,7 @@ topk_fwd_kernel(const TopkArgs a) {
         const int j = jc[e];
         valid[e] = pos < n_keys && j >= 0 && j < a.Tkv;
         if (pos < n_keys && !valid[e]) set_status(a.status, ATTN_DEVERR_TOPK_INDEX);
+        if (valid[e]) check_topk_causal(a.check_causal, j, t, a.Tq, a.Tkv, a.status);
         row[e] = valid[e] ? j : 0;  // unlisted and out-of-range keys read row 0 and are masked
       }
       const uint32_t vm0 = __ballot_sync(0xffffffffu, valid[0]), vm1 = __ballot_sync(0xffffffffu, valid[1]);
@@ -441,6 +443,7 @@ struct TopkBwdArgs {
   int64_t sd_t, sd_h;
   uint16_t* g_scr;  // [Tq, 64, topk_pad]
   uint16_t* p_scr;
+  int check_causal;  // ATTN_MASK_TOPK_CHECK_CAUSAL
   uint32_t* status;
 };
 
@@ -517,6 +520,7 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
         const int j = jc[e];
         valid[e] = pos < n_keys && j >= 0 && j < a.Tkv;
         if (pos < n_keys && !valid[e]) set_status(a.status, ATTN_DEVERR_TOPK_INDEX);
+        if (valid[e]) check_topk_causal(a.check_causal, j, t, a.Tq, a.Tkv, a.status);
         row[e] = valid[e] ? j : 0;
       }
       const uint32_t vm0 = __ballot_sync(0xffffffffu, valid[0]), vm1 = __ballot_sync(0xffffffffu, valid[1]);
@@ -780,7 +784,7 @@ struct TopkDkvArgs {
   int32_t topk_max;
   const int32_t* len;
   int Tq, Tkv, Dqk;
-  unsigned long long* acc;  // [Tkv, Dqk] signed 32.32 fixed point
+  FixedAcc fa;  // [Tkv, Dqk] signed 32.32 fixed point, per-row counts, largest magnitude
   uint32_t* status;
 };
 
@@ -852,7 +856,9 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       for (int e = 0; e < 2; ++e) {
         const int k = 2 * lane + e;
         const int j = jc[e];
-        krow[s * kTK + k] = (j >= 0 && j < a.Tkv) ? j : -1;  // the first kernel flagged invalid entries
+        const bool ok_j = j >= 0 && j < a.Tkv;
+        krow[s * kTK + k] = ok_j ? j : -1;  // the first kernel flagged invalid entries
+        if (ok_j) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
       }
       __syncwarp();
       if (lane == 0) {
@@ -908,6 +914,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const int qt = warp & 3, kq = (warp - 2) >> 2, kh = kq & 1, cp = kq >> 1;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
     bool ok = true, sat = false;
+    float amax = 0.f;
     for (int n = 0; n < ntiles && ok; ++n) {
       const int s = n & 1;
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full), n & 1, abort_flag, a.status));
@@ -928,13 +935,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
           for (int k = 0; k < 32; ++k) {
             const int j = rows[k0 + k];
             if (j < 0) continue;
-            float x = __uint_as_float(v[k]);
-            const float lim = 1073741824.f;  // 2^30: |x| 2^32 stays below 2^62
-            if (!(fabsf(x) < lim)) {
-              sat = true;
-              x = x != x ? 0.f : copysignf(lim, x);
-            }
-            atomicAdd(a.acc + (int64_t)j * a.Dqk + col, (unsigned long long)__float2ll_rn(x * 4294967296.f));
+            fixed_add(a.fa.acc + (int64_t)j * a.Dqk + col, __uint_as_float(v[k]), sat, amax);
           }
         };
         add(v0, 32 * kh);
@@ -946,6 +947,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         mbar_arrive(smem_u32(&ctl->gp_empty[s]));  // c_full(n) implies the MMAs are done with G and P
       }
     }
+    fixed_publish_max(a.fa.maxbits, amax);
     if (__any_sync(0xffffffffu, sat) && lane == 0) set_status(a.status, ATTN_DEVERR_OVERFLOW);
   }
   tc_fence_before();
@@ -1014,7 +1016,7 @@ bool sm100_topk_bwd_supported(const TopkP& p, const attn_tensor* q, const attn_t
 
 cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t sg_h, const float* lse,
                            int64_t sl_t, int64_t sl_h, const float* delta, void* dq, int64_t sd_t, int64_t sd_h,
-                           unsigned long long* acc, void* scratch, uint32_t* status, cudaStream_t st) {
+                           FixedAcc acc, void* scratch, uint32_t* status, cudaStream_t st) {
   const int pad = sm100_topk_pad(p.topk_max);
   const bool f16 = p.dtype == ATTN_F16;
   uint16_t* g_scr = static_cast<uint16_t*>(scratch);
@@ -1049,6 +1051,7 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   a.sd_h = sd_h;
   a.g_scr = g_scr;
   a.p_scr = p_scr;
+  a.check_causal = p.check_causal;
   a.status = status;
   TopkDkvArgs c;
   c.idx = p.idx;
@@ -1058,7 +1061,7 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   c.Tq = p.Tq;
   c.Tkv = p.Tkv;
   c.Dqk = p.Dqk;
-  c.acc = acc;
+  c.fa = acc;
   c.status = status;
   cudaError_t e;
   auto kdq = f16 ? topk_bwd_dq_kernel<true> : topk_bwd_dq_kernel<false>;
@@ -1110,6 +1113,7 @@ cudaError_t sm100_topk_fwd(const TopkP& p, void* o, int64_t so_t, int64_t so_h, 
   a.sl_t = sl_t;
   a.sl_h = sl_h;
   a.lse_fmt = p.lse_fmt;
+  a.check_causal = p.check_causal;
   a.status = status;
   const bool f16 = p.dtype == ATTN_F16;
   auto kern = f16 ? topk_fwd_kernel<true> : topk_fwd_kernel<false>;

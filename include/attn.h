@@ -66,8 +66,17 @@ typedef enum attn_status {
 
 /* Device-side error bits reported through attn_get_status. */
 #define ATTN_DEVERR_TOPK_INDEX 0x1u  /* a listed index outside [0, Tkv) was skipped */
-#define ATTN_DEVERR_OVERFLOW 0x2u    /* a fixed-point dKV contribution saturated */
+#define ATTN_DEVERR_OVERFLOW 0x2u    /* the fixed-point dKV sum of a row may not fit (see below) */
 #define ATTN_DEVERR_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
+#define ATTN_DEVERR_TOPK_CAUSAL 0x8u /* ATTN_MASK_TOPK_CHECK_CAUSAL: a listed index lies
+                                        beyond its token's causal position */
+/* ATTN_DEVERR_OVERFLOW: the top-k reverse pass sums each dKV element in a
+ * signed 32.32 fixed-point integer (range +-2^31). The bit is set when a
+ * single contribution was at least 2^30 in magnitude (it is then clamped),
+ * and whenever some KV row's number of contributions times the largest
+ * contribution magnitude of the call reaches 2^31: a bound on |sum| that
+ * every overflow exceeds, so a sum that wrapped always sets the bit (the
+ * bound can also set it for sums that did fit). */
 
 typedef enum attn_dtype { ATTN_F32 = 0, ATTN_BF16 = 1, ATTN_F16 = 2 } attn_dtype;
 
@@ -91,6 +100,13 @@ typedef struct attn_tensor {
 #define ATTN_MASK_TOPK 0x8u   /* j listed in topk_idxs[t][0 : topk_length[t]] */
 #define ATTN_MASK_LENGTHS 0x10u /* i < lengths[b] and j < lengths[b] (needs Tq = Tk) */
 #define ATTN_MASK_STARTS 0x20u  /* j >= starts[b][i] */
+/* Debug check for ATTN_MASK_TOPK (no set of its own): every listed entry
+ * inside the token's length is also compared with the token's causal
+ * position Tkv - Tq + t; an entry beyond it sets ATTN_DEVERR_TOPK_CAUSAL in
+ * the status word. The entry is still used: the lists' causality is the
+ * caller's contract, and the check reports a broken one without changing the
+ * result. Costs one compare per listed entry. */
+#define ATTN_MASK_TOPK_CHECK_CAUSAL 0x40u
 
 /* The allowed-set descriptor ("Tiled attention and its recomputed reverse
  * pass are exact": the fixed allowed sets A_i; causal, windowed and packed
@@ -219,12 +235,16 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k,
  * GPU that loads the library, held until the process exits). A problem whose
  * attn_bwd_workspace_size exceeds 64 MiB is rejected with
  * ATTN_ERR_WORKSPACE before anything is enqueued. The first call on each
- * device looks up the array's device address with that device current; make
- * that first call before any stream capture. Every call shares the one array
- * and it keeps the previous call's contents (the pass clears what must start
- * at zero itself), so calls whose GPU work overlaps in time, on different
- * streams or from different threads, race on it: serialise them. The status
- * word lives in that array too and cannot be read with attn_get_status. */
+ * device looks up the array's device address with that device current (and
+ * again after the device's context has been destroyed and re-created, e.g. by
+ * cudaDeviceReset); make that first call before any stream capture: made
+ * while `stream` is being captured it returns ATTN_ERR_UNSUPPORTED. Every call
+ * shares the one array and it keeps the previous call's contents (the pass
+ * clears what must start at zero itself), so calls whose GPU work overlaps in
+ * time, on different streams or from different threads, race on it:
+ * serialise them. The device status word is the first word of that array:
+ * read and clear it with attn_get_status(NULL, stream, &bits) with the same
+ * device current. */
 attn_status attn_bwd_noalloc(const attn_tensor* q, const attn_tensor* k,
                              const attn_tensor* v, const attn_tensor* o,
                              const attn_tensor* do_, const attn_tensor* lse,
@@ -233,8 +253,10 @@ attn_status attn_bwd_noalloc(const attn_tensor* q, const attn_tensor* k,
                              void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word at the
- * start of `workspace`. *device_bits receives the ATTN_DEVERR_* bits (0 when
- * clean). Returns ATTN_ERR_DEVICE when any bit was set. */
+ * start of `workspace` (workspace NULL: the status word of attn_bwd_noalloc's
+ * scratch array on the current device). *device_bits receives the
+ * ATTN_DEVERR_* bits (0 when clean). Returns ATTN_ERR_DEVICE when any bit was
+ * set. */
 attn_status attn_get_status(void* workspace, void* stream, uint32_t* device_bits);
 
 /* Kernel timing without a profiler. `begin` and `end` are cudaEvent_t

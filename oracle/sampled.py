@@ -52,6 +52,26 @@ def keep_at(seed: int, rho: float, b: int, h: int, rows, cols) -> np.ndarray:
     return w >= thr
 
 
+def keep_range(seed: int, rho: float, b: int, h: int, rows, c0: int, c1: int) -> np.ndarray:
+    """xi for rows x the contiguous key range [c0, c1) of (b, h), c0 a
+    multiple of 4: the same values as keep_at, but each generator call's four
+    words serve the four keys j = 4 (j >> 2) + 0..3 that share its counter,
+    so every call is made once instead of once per key."""
+    if c0 % 4:
+        raise ValueError("c0 must be a multiple of 4")
+    rows = np.asarray(rows, np.uint64)
+    nblk = (c1 - c0 + 3) // 4
+    thr = np.uint32(keep_threshold(rho))
+    key = np.array([seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF], dtype=np.uint64)
+    ctr = np.empty((rows.size, nblk, 4), dtype=np.uint64)
+    ctr[..., 0] = np.arange(c0 // 4, c0 // 4 + nblk, dtype=np.uint64)[None, :]
+    ctr[..., 1] = rows[:, None]
+    ctr[..., 2] = h
+    ctr[..., 3] = b
+    words = philox4x32(ctr, key)  # [rows, nblk, 4]: word w is key 4 * block + w
+    return (words >= thr).reshape(rows.size, nblk * 4)[:, :c1 - c0]
+
+
 def row_softmax(s: np.ndarray, allow: np.ndarray, z: float):
     """p, p_sink, LSE of each row (sink-inclusive LSE; empty rows: p = 0,
     LSE = -inf or z)."""

@@ -3,9 +3,10 @@ benchmark times, against the float64 oracle.
 
 causal_2k            every head, every element.
 window_block_8k      4 sampled heads (0, 9, 18, 31), every element of those heads.
-gqa_dropout_16k      2 K/V groups ((b=0, kv=0) and (b=1, kv=7), 8 query heads):
-                     Y/LSE/dQ on 128 sampled rows, dK/dV on the last 256 keys
-                     (whose allowed query rows are the last 256 rows).
+gqa_dropout_16k      K/V group (b=0, kv=0): every row of its 4 query heads
+                     (Y, LSE, dQ) and dK/dV on keys 0-255 (every row sees them),
+                     8064-8319 and the last 256; group (b=1, kv=7): Y/LSE/dQ on
+                     128 sampled rows, dK/dV on the last 256 keys.
 topk_shared_kv       O/LSE/dQ on 256 sampled tokens; dKV on the last 256 KV
                      rows (selectable only by the last 256 tokens); dSink over
                      all tokens.
@@ -26,7 +27,7 @@ import exact_tiled_attention_softmax_b200 as eta  # noqa: E402
 from exact_tiled_attention_softmax_b200 import workloads as W  # noqa: E402
 import oracle  # noqa: E402
 from oracle import sampled as S  # noqa: E402
-from tests.parity_util import BF16_GRAD_REL, BF16_O_ABS, rel_fro  # noqa: E402
+from tests.parity_util import BF16_GRAD_REL, BF16_O_ABS, o_excess, rel_fro  # noqa: E402
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -122,43 +123,91 @@ def test_window_block_8k_sampled_heads():
     _identities(tensors, outs)
 
 
-def test_gqa_dropout_16k_sampled():
+def _dropout_head_rows(q, k, v, g, case, b, h, kvh, chunk=256, threads=16):
+    """Y, LSE, delta and dQ of every row of one causal dropout head, from the
+    oracle's row evaluator over chunks of rows (each chunk against the keys
+    it can see). NumPy releases the GIL in its array kernels, so chunks run
+    on a thread pool."""
+    from concurrent.futures import ThreadPoolExecutor
+    T, rho, seed = case.T, case.dropout_p, case.dropout_seed
+    kk = k[b, kvh].astype(np.float64)
+    vv = v[b, kvh].astype(np.float64)
+
+    def one(r0):
+        r1 = min(r0 + chunk, T)
+        rows = np.arange(r0, r1)
+        ar = S.allowed_at(rows, np.arange(r1), causal=True)
+        kr = S.keep_range(seed, rho, b, h, rows, 0, r1)
+        return S.rows_forward_backward(q[b, h], kk[:r1], vv[:r1], g[b, h], rows, ar, case.scale,
+                                       keep_rows=kr, rho=rho)
+
+    with ThreadPoolExecutor(threads) as ex:
+        parts = list(ex.map(one, range(0, T, chunk)))
+    return tuple(np.concatenate([p[i] for p in parts]) for i in range(4))
+
+
+def test_gqa_dropout_16k_whole_group_and_first_key_tiles():
+    """One K/V group (b=0, kv=0: 4 query heads) in full: Y, LSE and dQ of every
+    row of every head, and dK/dV on the first two key tiles (keys 0-255, the
+    longest accumulation of the key-centric reverse: every one of the
+    16384 rows of the 4 heads sees them, with dropout replayed throughout), on
+    a middle band across a tile edge (keys 8064-8319) and on the last 256
+    keys, from the oracle's own LSE and delta of every row."""
     case = W.WORKLOADS["gqa_dropout_16k"]
     (q, k, v, g, _), outs, tensors = _run_dense(case)
     o, lse, dq, dk, dv = outs
     T, group, rho, seed = case.T, case.Hq // case.Hkv, case.dropout_p, case.dropout_seed
+    b, kvh = 0, 0
+    heads = [kvh * group + hh for hh in range(group)]
+    lse_g, delta_g = [], []
+    for h in heads:
+        y_r, lse_r, delta_r, dq_r = _dropout_head_rows(q, k, v, g, case, b, h, kvh)
+        assert o_excess(_np(o[b, h]), y_r) <= BF16_O_ABS, h
+        assert np.abs(_np(lse[b, h]) - lse_r).max() <= 1e-3, h
+        assert rel_fro(_np(dq[b, h]), dq_r) <= BF16_GRAD_REL, h
+        lse_g.append(lse_r)
+        delta_g.append(delta_r)
+    for c0, c1 in ((0, 256), (8064, 8320), (T - 256, T)):
+        cols = np.arange(c0, c1)
+        dk_r, dv_r = S.cols_backward(
+            [q[b, h] for h in heads], [g[b, h] for h in heads], k[b, kvh], v[b, kvh], cols,
+            lambda hh, r, c: S.allowed_at(r, c, causal=True), lse_g, delta_g, case.scale,
+            keep_fn=lambda hh, r, c: S.keep_range(seed, rho, b, heads[hh], r, int(c[0]), int(c[-1]) + 1), rho=rho)
+        assert rel_fro(_np(dk[b, kvh])[cols], dk_r) <= BF16_GRAD_REL, (c0, c1)
+        assert rel_fro(_np(dv[b, kvh])[cols], dv_r) <= BF16_GRAD_REL, (c0, c1)
+    _identities(tensors, outs)
+    # A second group on sampled rows and its last 256 keys (whose allowed
+    # query rows are the last 256 rows).
     rng = np.random.default_rng(5)
     rows = np.unique(np.concatenate([[0, 1, 127, 128, T - 1], rng.integers(0, T, 123)]))
     tail = np.arange(T - 256, T)
     cols = np.arange(T)
-    for b, kvh in ((0, 0), (1, 7)):
-        heads = [kvh * group + hh for hh in range(group)]
-        lse_g, delta_g = [], []
-        for h in heads:
-            ar = S.allowed_at(rows, cols, causal=True)
-            kr = S.keep_at(seed, rho, b, h, rows, cols)
-            y_r, lse_r, _, dq_r = S.rows_forward_backward(q[b, h], k[b, kvh], v[b, kvh], g[b, h], rows, ar,
-                                                          case.scale, keep_rows=kr, rho=rho)
-            assert np.abs(_np(o[b, h])[rows] - y_r).max() <= BF16_O_ABS, h
-            assert np.abs(_np(lse[b, h])[rows] - lse_r).max() <= 1e-3, h
-            assert rel_fro(_np(dq[b, h])[rows], dq_r) <= BF16_GRAD_REL, h
-            # LSE and delta of the rows that can see the last 256 keys.
-            at = S.allowed_at(tail, cols, causal=True)
-            kt = S.keep_at(seed, rho, b, h, tail, cols)
-            _, l_t, d_t, _ = S.rows_forward_backward(q[b, h], k[b, kvh], v[b, kvh], g[b, h], tail, at, case.scale,
-                                                     keep_rows=kt, rho=rho)
-            lf = np.full(T, np.nan)
-            df = np.full(T, np.nan)
-            lf[tail], df[tail] = l_t, d_t
-            lse_g.append(lf)
-            delta_g.append(df)
-        dk_r, dv_r = S.cols_backward(
-            [q[b, h] for h in heads], [g[b, h] for h in heads], k[b, kvh], v[b, kvh], tail,
-            lambda hh, r, c: S.allowed_at(r, c, causal=True), lse_g, delta_g, case.scale,
-            keep_fn=lambda hh, r, c, hs=heads, bb=b: S.keep_at(seed, rho, bb, hs[hh], r, c), rho=rho)
-        assert rel_fro(_np(dk[b, kvh])[tail], dk_r) <= BF16_GRAD_REL
-        assert rel_fro(_np(dv[b, kvh])[tail], dv_r) <= BF16_GRAD_REL
-    _identities(tensors, outs)
+    b, kvh = 1, 7
+    heads = [kvh * group + hh for hh in range(group)]
+    lse_g, delta_g = [], []
+    for h in heads:
+        ar = S.allowed_at(rows, cols, causal=True)
+        kr = S.keep_range(seed, rho, b, h, rows, 0, T)
+        y_r, lse_r, _, dq_r = S.rows_forward_backward(q[b, h], k[b, kvh], v[b, kvh], g[b, h], rows, ar,
+                                                      case.scale, keep_rows=kr, rho=rho)
+        assert o_excess(_np(o[b, h])[rows], y_r) <= BF16_O_ABS, h
+        assert np.abs(_np(lse[b, h])[rows] - lse_r).max() <= 1e-3, h
+        assert rel_fro(_np(dq[b, h])[rows], dq_r) <= BF16_GRAD_REL, h
+        at = S.allowed_at(tail, cols, causal=True)
+        kt = S.keep_range(seed, rho, b, h, tail, 0, T)
+        _, l_t, d_t, _ = S.rows_forward_backward(q[b, h], k[b, kvh], v[b, kvh], g[b, h], tail, at, case.scale,
+                                                 keep_rows=kt, rho=rho)
+        lf = np.full(T, np.nan)
+        df = np.full(T, np.nan)
+        lf[tail], df[tail] = l_t, d_t
+        lse_g.append(lf)
+        delta_g.append(df)
+    dk_r, dv_r = S.cols_backward(
+        [q[b, h] for h in heads], [g[b, h] for h in heads], k[b, kvh], v[b, kvh], tail,
+        lambda hh, r, c: S.allowed_at(r, c, causal=True), lse_g, delta_g, case.scale,
+        keep_fn=lambda hh, r, c: S.keep_range(seed, rho, b, heads[hh], r, int(c[0]), int(c[-1]) + 1), rho=rho)
+    assert rel_fro(_np(dk[b, kvh])[tail], dk_r) <= BF16_GRAD_REL
+    assert rel_fro(_np(dv[b, kvh])[tail], dv_r) <= BF16_GRAD_REL
 
 
 def test_topk_shared_kv_sampled():

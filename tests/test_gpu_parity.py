@@ -77,9 +77,9 @@ def _run_oracle(c):
     return fw, bw
 
 
-def _compare(c, gpu, fw, bw, row_scale=False):
+def _compare(c, gpu, fw, bw):
     fp32 = c["dtype"] == "f32"
-    check_close("O", to_np(gpu["o"]), fw.y, fp32=fp32, grad=False, row_scale=row_scale)
+    check_close("O", to_np(gpu["o"]), fw.y, fp32=fp32, grad=False, storage=c["dtype"])
     lse_g, lse_o = to_np(gpu["lse"]), fw.lse
     fin = np.isfinite(lse_o)
     assert np.array_equal(np.isfinite(lse_g), fin)
@@ -227,7 +227,7 @@ def test_small_topk(dtype):
     dq_ref, dkv_ref, ds_ref = oracle.topk_backward(q, kv, idx, ln, Dv, scale, g, sk.astype(np.float64),
                                                    o=o_ref)
     fp32 = dtype == "f32"
-    check_close("O", to_np(o), o_ref, fp32=fp32, grad=False)
+    check_close("O", to_np(o), o_ref, fp32=fp32, grad=False, storage=dtype)
     check_close("dQ", to_np(dq), dq_ref, fp32=fp32, grad=True)
     check_close("dKV", to_np(dkv), dkv_ref, fp32=fp32, grad=True)
     assert np.abs(to_np(lse) - lse_ref).max() <= (1e-5 if fp32 else 1e-3)
@@ -325,7 +325,7 @@ def _run_layout_case(c, lengths=None, starts=None):
     sink = c["sink"].astype(np.float64) if c["sink"] is not None else None
     fw = oracle.forward(qq, kk, vv, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"])
     bw = oracle.backward(qq, kk, vv, gg, allow, c["scale"], sink=sink, keep=keep, rho=c["dropout"], y=fw.y)
-    _compare(c, gpu, fw, bw, row_scale=True)
+    _compare(c, gpu, fw, bw)
     return gpu
 
 

@@ -469,6 +469,22 @@ def test_sampled_rows_and_columns_match_full_oracle():
         assert np.allclose(dvv, bw.dv[0, kvh][cols], atol=1e-12)
 
 
+def test_keep_range_equals_the_full_mask():
+    """The block-wise keep evaluator gives the full mask's values on every
+    row and contiguous key range it is asked for (ranges starting on a
+    4-key block, ending anywhere)."""
+    from oracle import sampled as S
+    seed, rho, B, Hq, T = (1 << 40) + 123, 0.3, 2, 3, 45
+    keep = P.dropout_keep(seed, rho, B, Hq, T, T)
+    rows = np.array([0, 5, 44])
+    for b, h, c0, c1 in ((0, 0, 0, 45), (1, 2, 8, 9), (1, 1, 4, 43), (0, 2, 40, 45)):
+        got = S.keep_range(seed, rho, b, h, rows, c0, c1)
+        assert np.array_equal(got, keep[b, h][rows][:, c0:c1])
+        assert np.array_equal(got, S.keep_at(seed, rho, b, h, rows, np.arange(c0, c1)))
+    with pytest.raises(ValueError):
+        S.keep_range(seed, rho, 0, 0, rows, 2, 10)
+
+
 def test_topk_empty_list_gives_zero_output_and_sink_lse():
     """An empty selection is an empty allowed set: Y = 0 and LSE = z with a
     sink, -inf without one; the other tokens are unaffected."""
