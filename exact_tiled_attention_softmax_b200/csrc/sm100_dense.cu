@@ -202,6 +202,7 @@ constexpr uint32_t kFwdV = kFwdK + kStages * kTileBytes;
 constexpr uint32_t kFwdCtl = kFwdV + kStages * kTileBytes;
 constexpr uint32_t kFwdSmem = kFwdCtl + 1024 + 1024;  // control block + alignment slack
 constexpr int kFwdThreads = 320;  // producer, MMA issuer, softmax warpgroups (warps 2-5, 6-9)
+constexpr int kFwdBand = 8;       // (batch row, query head) pairs per scheduling band
 
 struct FwdCtl {
   uint64_t q_full;
@@ -504,11 +505,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   volatile uint32_t* abort_flag = &ctl->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Longest query tiles (most keys under a causal mask) first over the whole
-  // grid: the tail of the launch is made of the shortest tiles.
+  // Bands of kFwdBand (batch row, query head) pairs; within a band the
+  // longest query tiles (most keys under a causal mask) go first. The CTAs
+  // resident at any time then read the K/V tiles of a few heads (adjacent
+  // query heads share their K/V head), which stay in L2 for every query tile
+  // that reuses them, and the tail of the launch is made of short tiles.
   const int nct = (a.Tq + kFwdRows - 1) / kFwdRows;
-  const int bh = blockIdx.x % (a.B * a.Hq);
-  const int ct = nct - 1 - (int)(blockIdx.x / (a.B * a.Hq));
+  const int nbh = a.B * a.Hq;
+  const int band0 = (int)(blockIdx.x / ((int64_t)kFwdBand * nct)) * kFwdBand;
+  const int bw = nbh - band0 < kFwdBand ? nbh - band0 : kFwdBand;
+  const int within = (int)(blockIdx.x - (int64_t)band0 * nct);
+  const int bh = band0 + within % bw;
+  const int ct = nct - 1 - within / bw;
   const int h = bh % a.Hq, b = bh / a.Hq;
   const int kvh = h / (a.Hq / a.Hkv);
   const int q0 = ct * kFwdRows;
@@ -789,6 +797,7 @@ constexpr uint32_t kBwdK = 0;
 constexpr uint32_t kBwdV = kBwdK + kTileBytes;
 constexpr int kQStages = 3;                             // Q / dO / LSE / delta ring depth
 constexpr int kBwdBand = 8;                             // (b, K/V head) pairs per scheduling band
+constexpr bool kBwdDqFirst = true;                      // issue a step's dQ^T product before its dV, dK
 constexpr uint32_t kBwdQ = kBwdV + kTileBytes;          // kQStages x 16 KB
 constexpr uint32_t kBwdG = kBwdQ + kQStages * kQTile;   // kQStages x 16 KB
 constexpr uint32_t kBwdDS = kBwdG + kQStages * kQTile;  // 2 buffers of gamma^T (P^T lives in TMEM)
@@ -981,7 +990,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&ctl->st_full[s]), 1);
-      mbar_init(smem_u32(&ctl->ds_full[s]), 8);
+      mbar_init(smem_u32(&ctl->ds_full[s]), kDrop ? 4 : 8);  // one arrival per warp working on the step
       mbar_init(smem_u32(&ctl->dq_full[s]), 1);
       mbar_init(smem_u32(&ctl->dq_empty[s]), 4);  // one arrival per dQ warp
     }
@@ -1017,16 +1026,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     // The step walk (query head, query slice, class) runs here, ahead of the
     // MMA issuer and the compute warpgroups, which read it from qinfo.
     int n = 0, hh = 0, qs = qs_lo - 1;
-    uint8_t cls;
+    uint8_t cls, ncls = 0;
     bool have = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh, qs, cls);
+    int nh = hh, nq = qs;
+    bool next = have && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
     while (have) {
-      int nh = hh, nq = qs;
-      uint8_t ncls;
-      const bool next = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, nh, nq, ncls);
+      int mh = nh, mq = nq;
+      uint8_t mcls = 0;
+      const bool next2 = next && bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, mh, mq, mcls);
       const int h = kvh * group + hh;
       const int s = n % kQStages;
       if (!wait_bar(smem_u32(&ctl->q_empty[s]), ((n / kQStages) & 1) ^ 1, abort_flag, a.status)) break;
-      ctl->qinfo[s][0] = (uint32_t)qs | ((uint32_t)cls << 28) | (next ? 1u << 30 : 0u);
+      ctl->qinfo[s][0] =
+          (uint32_t)qs | ((uint32_t)cls << 28) | (next ? 1u << 30 : 0u) | (next2 ? 1u << 31 : 0u);
       ctl->qinfo[s][1] = (uint32_t)hh;  // both published by the release of the arrive below
       const uint32_t qf = smem_u32(&ctl->q_full[s]);
       mbar_expect_tx(qf, 2 * kQTile + 512);
@@ -1043,6 +1055,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       qs = nq;
       cls = ncls;
       have = next;
+      nh = mh;
+      nq = mq;
+      ncls = mcls;
+      next = next2;
     }
     for (int r = (n > kQStages ? n - kQStages : 0); r < n; ++r)
       wait_bar(smem_u32(&ctl->q_full[r % kQStages]), (r / kQStages) & 1, abort_flag, nullptr);
@@ -1106,6 +1122,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const int s = n & 1, sq = n % kQStages;
       if (!(ok = wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
       tc_fence_after();
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
+          mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
+                 kk > 0);
+      };
+      // dQ^T first: the dQ warps drain it while dV and dK run, so its TMEM
+      // columns are free again before S^T of step n + 2 is issued.
+      if constexpr (kDQ && kBwdDqFirst) {
+        issue_dq();
+        mma_commit(smem_u32(&ctl->dq_full[s]));
+      }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows; A = P~^T from TMEM (16 rows = 8 columns)
         mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8, dGmn(sq) + (uint64_t)(kk * (2048 >> 4)),
@@ -1114,37 +1142,39 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       for (int kk = 0; kk < 4; ++kk)
         mma_ss(tDK, dDS(s) + (uint64_t)(kk * (32 >> 4)), dQmn(sq) + (uint64_t)(kk * (2048 >> 4)), idACC,
                (n > 0 || kk > 0) ? 1u : 0u);
-      if constexpr (kDQ) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // K = 128 keys
-          mma_ss(tmem + s * 128, dKmn + (uint64_t)(kk * (2048 >> 4)), dDSmn(s) + (uint64_t)(kk * (2048 >> 4)), idDQ,
-                 kk > 0);
-      }
+      if constexpr (kDQ && !kBwdDqFirst) issue_dq();
       mma_commit(smem_u32(&ctl->q_empty[sq]));
-      if constexpr (kDQ) mma_commit(smem_u32(&ctl->dq_full[s]));
+      if constexpr (kDQ && !kBwdDqFirst) mma_commit(smem_u32(&ctl->dq_full[s]));
       have = next;
       info = ninfo;
       ++n;
     }
     mma_commit(smem_u32(&ctl->acc_done));
   } else if (warp >= 4 && warp < 12) {
-    // ---------------- compute warpgroups: thread t owns key row k0 + t; warpgroup
-    // hf handles query columns 32 hf .. 32 hf + 31 of each step.
-    const int hf = (warp - 4) >> 2;
+    // ---------------- compute warpgroups: thread t owns key row k0 + t. Step
+    // n lives in S^T | dP^T buffer n & 1. Without dropout the two warpgroups
+    // split every step's 64 query columns (warpgroup w: columns 32 w ..
+    // 32 w + 31). With dropout (kAlt) each step carries Philox work as well,
+    // and the warpgroups take alternate steps instead (warpgroup w: steps w,
+    // w + 2, ..., all 64 columns as two passes of 32), so one warpgroup's
+    // element math overlaps the other's waits for the tensor core.
+    constexpr bool kAlt = kDrop;
+    const int w = (warp - 4) >> 2;
     const int t = ((warp & 3) << 5) | lane;
     const int64_t j = (int64_t)k0 + t;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    int n = 0;
     bool ok = true;
-    bool more;
+    bool any, mine;  // the CTA has a step; this warpgroup's next step exists
     {
       int hh0 = 0, qs0 = qs_lo - 1;
       uint8_t cls0;
-      more = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh0, qs0, cls0);
+      any = bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh0, qs0, cls0);
+      mine = any && (!kAlt || w == 0 || bwd_next_step(a, b, kvh, kt, group, qs_lo, qs_hi, hh0, qs0, cls0));
     }
-    while (ok && more) {
+    for (int n = kAlt ? w : 0; ok && mine; n += kAlt ? 2 : 1) {
       const int s = n & 1, sq = n % kQStages;
       const uint32_t par = (n >> 1) & 1;
+      const uint32_t tbuf = tmem + lane_off + s * 128;  // the step's S^T | dP^T buffer
       // The stage's step info arrives with its Q/dO tiles, long before S^T.
       if (!(ok = __all_sync(0xffffffffu,
                             wait_bar(smem_u32(&ctl->q_full[sq]), (n / kQStages) & 1, abort_flag, a.status))))
@@ -1153,99 +1183,108 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const int h = kvh * group + (int)ctl->qinfo[sq][1];
       const int qs = (int)(info & 0x0fffffffu);
       const uint8_t cls = (uint8_t)((info >> 28) & 3u);
-      more = info & (1u << 30);
+      mine = kAlt ? (info >> 31) : ((info >> 30) & 1u);  // step n + 2 (n + 1) follows
       const int64_t i0 = (int64_t)qs * kBMb;
       const bool general = cls == kPartial;
-      const uint32_t allow = cls == kPartial ? (uint32_t)(bwd_col_bits(a, b, h, i0, j) >> (32 * hf)) : ~0u;
-      uint32_t keep = ~0u;
-      if constexpr (kDrop) keep = bwd_keep_bits(a.m, b, h, i0 + 32 * hf, j);
+      const uint64_t allow64 = general ? bwd_col_bits(a, b, h, i0, j) : ~0ull;
+      // Keep bits of query columns 0-31 and 32-63, computed while S^T is on its way.
+      uint32_t keep_lo = ~0u, keep_hi = ~0u;
+      if constexpr (kDrop) {
+        keep_lo = bwd_keep_bits(a.m, b, h, i0, j);
+        keep_hi = bwd_keep_bits(a.m, b, h, i0 + 32, j);
+      }
       if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->st_full[s]), par, abort_flag, a.status)))) break;
       tc_fence_after();
-      uint32_t rs[32], rp[32];
-      tmem_ld32(tmem + lane_off + s * 128 + hf * 32, rs);
-      tmem_ld32(tmem + lane_off + s * 128 + 64 + hf * 32, rp);
-      const float* nl = stat + sq * 128 + hf * 32;       // -LSE (base 2) of the 32 columns
-      const float* nd = stat + sq * 128 + 64 + hf * 32;  // -delta
-      tmem_wait_ld();
-      uint32_t ppk[16], dpk[16];
-      if (!general) {
-        // Pairs of columns on packed fp32: x = s c log2(e) - LSE, p = 2^x,
-        // gamma = p (dP - delta); -LSE and -delta come as broadcast 16-byte loads.
-        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(nl + 4 * c4);
-          const float4 d4 = *reinterpret_cast<const float4*>(nd + 4 * c4);
-          const uint64_t lp[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
-          const uint64_t dp[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c2 = 2 * c4 + e;
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            uint64_t dv2 = f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1]));
-            if constexpr (kDrop) {  // xi in the P~ operand and in dP; p itself stays undropped
-              const bool k0 = (keep >> (2 * c2)) & 1u, k1 = (keep >> (2 * c2 + 1)) & 1u;
-              ppk[c2] = pack16<kH>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
-              dv2 = f2_pack(k0 ? __uint_as_float(rp[2 * c2]) * a.m.inv_keep : 0.f,
-                            k1 ? __uint_as_float(rp[2 * c2 + 1]) * a.m.inv_keep : 0.f);
-            } else {
-              ppk[c2] = pack16<kH>(p0, p1);
-            }
-            const uint64_t g = f2_mul(f2_pack(p0, p1), f2_add(dv2, dp[e]));
-            float g0, g1;
-            f2_unpack(g, g0, g1);
-            dpk[c2] = pack16<kH>(g0, g1);
-          }
-        }
-      } else {
-        const float inv = a.m.dropout ? a.m.inv_keep : 1.f;
-#pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          float pt[2], ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * c2 + e;
-            const float p = ((allow >> c) & 1u) ? ex2(fmaf(__uint_as_float(rs[c]), a.scale_log2, nl[c])) : 0.f;
-            const bool kp = (keep >> c) & 1u;
-            // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
-            pt[e] = kp ? p : 0.f;
-            const float dpv = kp ? __uint_as_float(rp[c]) * inv : 0.f;
-            ds[e] = p * (dpv + nd[c]);
-          }
-          ppk[c2] = pack16<kH>(pt[0], pt[1]);
-          dpk[c2] = pack16<kH>(ds[0], ds[1]);
-        }
-      }
-      // P~^T as bf16 pairs over this warpgroup's own dP^T columns (already read).
-      tmem_st16(tmem + lane_off + s * 128 + 64 + hf * 32, ppk);
       const uint32_t ds_base = sbase + kBwdDS + s * kPTile;
+#pragma unroll 1
+      for (int c = kAlt ? 0 : w; c < (kAlt ? 2 : w + 1); ++c) {
+        const uint32_t allow = (uint32_t)(allow64 >> (32 * c));
+        const uint32_t keep = c ? keep_hi : keep_lo;
+        uint32_t rs[32], rp[32];
+        tmem_ld32(tbuf + 32 * c, rs);
+        tmem_ld32(tbuf + 64 + 32 * c, rp);
+        const float* nl = stat + sq * 128 + 32 * c;       // -LSE (base 2) of the 32 columns
+        const float* nd = stat + sq * 128 + 64 + 32 * c;  // -delta
+        tmem_wait_ld();
+        uint32_t ppk[16], dpk[16];
+        if (!general) {
+          // Pairs of columns on packed fp32: x = s c log2(e) - LSE, p = 2^x,
+          // gamma = p (dP - delta); -LSE and -delta come as broadcast 16-byte loads.
+          const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const uint32_t off = sw128_offset(t, (hf * 4 + cc) * 16);
-        st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(nl + 4 * c4);
+            const float4 d4 = *reinterpret_cast<const float4*>(nd + 4 * c4);
+            const uint64_t lp[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+            const uint64_t dp[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c2 = 2 * c4 + e;
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0,
+                        x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              uint64_t dv2 = f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1]));
+              if constexpr (kDrop) {  // xi in the P~ operand and in dP; p itself stays undropped
+                const bool k0 = (keep >> (2 * c2)) & 1u, k1 = (keep >> (2 * c2 + 1)) & 1u;
+                ppk[c2] = pack16<kH>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
+                dv2 = f2_pack(k0 ? __uint_as_float(rp[2 * c2]) * a.m.inv_keep : 0.f,
+                              k1 ? __uint_as_float(rp[2 * c2 + 1]) * a.m.inv_keep : 0.f);
+              } else {
+                ppk[c2] = pack16<kH>(p0, p1);
+              }
+              const uint64_t g = f2_mul(f2_pack(p0, p1), f2_add(dv2, dp[e]));
+              float g0, g1;
+              f2_unpack(g, g0, g1);
+              dpk[c2] = pack16<kH>(g0, g1);
+            }
+          }
+        } else {
+          const float inv = a.m.dropout ? a.m.inv_keep : 1.f;
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) {
+            float pt[2], ds[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int cc = 2 * c2 + e;
+              const float p = ((allow >> cc) & 1u) ? ex2(fmaf(__uint_as_float(rs[cc]), a.scale_log2, nl[cc])) : 0.f;
+              const bool kp = (keep >> cc) & 1u;
+              // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
+              pt[e] = kp ? p : 0.f;
+              const float dpv = kp ? __uint_as_float(rp[cc]) * inv : 0.f;
+              ds[e] = p * (dpv + nd[cc]);
+            }
+            ppk[c2] = pack16<kH>(pt[0], pt[1]);
+            dpk[c2] = pack16<kH>(ds[0], ds[1]);
+          }
+        }
+        // P~^T as bf16 pairs over this pass's own dP^T columns (already read).
+        tmem_st16(tbuf + 64 + 32 * c, ppk);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t off = sw128_offset(t, (c * 4 + cc) * 16);
+          st_shared_v4(ds_base + off, dpk[cc * 4], dpk[cc * 4 + 1], dpk[cc * 4 + 2], dpk[cc * 4 + 3]);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctl->ds_full[s]));
-      ++n;
     }
     // ---------------- epilogue: warpgroup 0 writes dK = c * sum gamma^T Q,
-    // warpgroup 1 writes dV = sum P~^T dO.
+    // warpgroup 1 writes dV = sum P~^T dO (zeros when the CTA had no step).
     bool have = false;
-    if (ok && n > 0) {
+    if (ok && any) {
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->acc_done), 0, abort_flag, a.status));
       if (ok) tc_fence_after();
       have = ok;
     }
-    const float osc = hf == 0 ? a.scale : (a.m.dropout ? a.m.inv_keep : 1.f);
-    if (ok || n == 0) {
-      uint16_t* orow = hf == 0 ? a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2]
-                                    : a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
-      const uint32_t tacc = (hf == 0 ? tDK : tDV) + lane_off;
+    const float osc = w == 0 ? a.scale : (a.m.dropout ? a.m.inv_keep : 1.f);
+    if (ok) {
+      uint16_t* orow = w == 0 ? a.dk + b * a.sdk[0] + kvh * a.sdk[1] + j * a.sdk[2]
+                              : a.dv + b * a.sdv[0] + kvh * a.sdv[1] + j * a.sdv[2];
+      const uint32_t tacc = (w == 0 ? tDK : tDV) + lane_off;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];

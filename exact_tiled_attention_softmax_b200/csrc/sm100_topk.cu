@@ -413,7 +413,8 @@ constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads
 constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kBCtl = kBG + kTH * 128;
 constexpr uint32_t kBSmem = kBCtl + 1024 + 1024;
-constexpr int kBThreads = 256;  // producer, MMA issuer, 4 softmax warps, 2 gather warps
+constexpr int kBGather = 4;                       // reverse gather warps
+constexpr int kBThreads = 192 + 32 * kBGather;    // producer, MMA issuer, 4 compute warps, gather warps
 constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
 
 struct TopkBwdCtl {
@@ -463,7 +464,7 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBStages; ++s) {
-      mbar_init(smem_u32(&ctl->kv_full[s]), 2);  // one arrival per gather warp
+      mbar_init(smem_u32(&ctl->kv_full[s]), kBGather);  // one arrival per gather warp
       mbar_init(smem_u32(&ctl->kv_empty[s]), 1);
       mbar_init(smem_u32(&ctl->rows_full[s]), 1);
     }
@@ -553,8 +554,8 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
       if (!ok) break;
       const uint32_t dst = sbase + kBKV + s * kTTile;
 #pragma unroll 4
-      for (int it = 0; it < kTK * 72 / 64; ++it) {
-        const int q = it * 64 + gt, r = q / 72, c = q - r * 72;
+      for (int it = 0; it < kTK * 72 / (32 * kBGather); ++it) {
+        const int q = it * (32 * kBGather) + gt, r = q / 72, c = q - r * 72;
         cp_async_16(dst + (uint32_t)(c >> 3) * kTPlane + sw128_offset(r, (c & 7) * 16),
                     a.kv + (int64_t)ctl->grow[s][r] * a.skv_bytes + c * 16);
       }

@@ -33,3 +33,7 @@ def test_o_excess():
     # bf16 half ulps: 2^-9, 2^-6, 2^-7
     assert abs(o_excess(got, want) - (0.025 - 2.0 ** -6)) < 1e-12
     assert o_excess(np.zeros(0), np.zeros(0)) == 0.0
+    # with the P-operand term: 2^-8 * p_abs more is allowed
+    p_abs = np.array([0.0, 1.28, 0.0])
+    assert abs(o_excess(got, want, p_abs=p_abs) - max(0.009 - 2.0 ** -9, 0.025 - 2.0 ** -6 - 0.005,
+                                                      0.017 - 2.0 ** -7)) < 1e-12
