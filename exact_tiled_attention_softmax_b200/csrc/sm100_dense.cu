@@ -588,11 +588,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       wait_bar(smem_u32(&ctl->k_full[s]), (r / kStages) & 1, abort_flag, nullptr);
       wait_bar(smem_u32(&ctl->v_full[s]), (r / kStages) & 1, abort_flag, nullptr);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+  } else if (warp == 1) {
+    // ---------------- MMA issuer: the whole warp runs the loop (warp-uniform
+    // waits and descriptor arithmetic), one elected lane issues the MMAs.
+    const bool leader = elect_one();
     constexpr uint32_t idS = idesc16<kH>(128, 128, 0, 0);
     constexpr uint32_t idPV = idesc16<kH>(128, 128, 0, 1);
-    bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status);
+    bool ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, a.status));
     // Descriptors of every operand tile, formed once; a K step adds its byte
     // offset >> 4 to the start-address field.
     const uint64_t dQ0 = smem_desc_sw128(sbase + kFwdQ, 16, 1024), dK0 = smem_desc_sw128(sbase + kFwdK, 16, 1024);
@@ -602,12 +604,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto dK = [&](int i) { return dK0 + (uint64_t)i * kTileStep; };
     auto dV = [&](int i) { return dV0 + (uint64_t)i * kTileStep; };
     auto issue_s = [&](int w, int stage) {
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-        mma_ss(tmem + w * 128, dQ(w) + off, dK(stage) + off, idS, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + w * 128, dQ(w) + off, dK(stage) + off, idS, kk > 0);
+        }
+        mma_commit(smem_u32(&ctl->s_full[w]));
       }
-      mma_commit(smem_u32(&ctl->s_full[w]));
+      __syncwarp();
     };
     uint32_t fl0;
     const bool any = fwd_next_tile(a, b, h, qt0, kt_hi, kt_lo - 1, fl0) <= kt_hi;
@@ -615,7 +620,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     int npv[2] = {0, 0};
     int n = 0;
     if (ok && any) {
-      ok = wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, a.status));
       if (ok) {
         tc_fence_after();
         info = ctl->tinfo[0];
@@ -629,18 +634,26 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint32_t ninfo = 0;
       for (int w = 0; w < 2 && ok; ++w) {
         if ((info >> w) & 1u) {
-          if (!(ok = wait_bar(smem_u32(&ctl->p_full[w]), npv[w] & 1, abort_flag, a.status))) break;
-          if (!(ok = wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status))) break;
+          if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->p_full[w]), npv[w] & 1, abort_flag, a.status))))
+            break;
+          if (!(ok = __all_sync(0xffffffffu,
+                                wait_bar(smem_u32(&ctl->v_full[s]), (n / kStages) & 1, abort_flag, a.status))))
+            break;
           tc_fence_after();
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // A = P in TMEM: 16 keys = 8 packed columns per step
-            mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dV(s) + (uint64_t)(kk * (2048 >> 4)), idPV,
-                   (npv[w] > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)  // A = P in TMEM: 16 keys = 8 packed columns per step
+              mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dV(s) + (uint64_t)(kk * (2048 >> 4)), idPV,
+                     (npv[w] > 0 || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
           ++npv[w];
         }
         if (more) {
           if (w == 0) {
-            if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, a.status))) break;
+            if (!(ok = __all_sync(0xffffffffu,
+                                  wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, a.status))))
+              break;
             tc_fence_after();
             ninfo = ctl->tinfo[s1];
           }
@@ -648,12 +661,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
       }
       if (!ok) break;
-      mma_commit(smem_u32(&ctl->kv_empty[s]));
+      if (leader) mma_commit(smem_u32(&ctl->kv_empty[s]));
+      __syncwarp();
       if (!more) break;
       info = ninfo;
       ++n;
     }
-    mma_commit(smem_u32(&ctl->o_final));
+    if (leader) mma_commit(smem_u32(&ctl->o_final));
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- softmax warpgroups: thread t of warpgroup w owns query row
     // q0 + 128 w + t (TMEM lane t of that warpgroup's S/P and O columns).
@@ -950,6 +965,68 @@ __device__ __forceinline__ void bulk_wait_read0() {
 }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// The element math of one 32-column pass of a reverse step, for the
+// calling thread's key row: from S^T and dP^T (rs, rp) and the columns'
+// -LSE (base 2) and -delta (nl, nd), P~^T and gamma^T as 16-bit pairs.
+// Full tiles: x = s c log2(e) - LSE, p = 2^x, gamma = p (dP - delta) on
+// packed fp32 pairs, -LSE and -delta as broadcast 16-byte loads. Partial
+// tiles: per column, with the allowed-row bits. With dropout, xi enters the
+// P~ operand and dP (p itself stays undropped; dV is scaled by 1/(1-rho) at
+// the end).
+template <bool kH, bool kDrop>
+__device__ __forceinline__ void bwd_chunk_math(const uint32_t (&rs)[32], const uint32_t (&rp)[32], const float* nl,
+                                               const float* nd, bool general, uint32_t allow, uint32_t keep,
+                                               float scale_log2, float inv_keep, int dropout, uint32_t (&ppk)[16],
+                                               uint32_t (&dpk)[16]) {
+  if (!general) {
+    const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+#pragma unroll
+    for (int c4 = 0; c4 < 8; ++c4) {
+      const float4 l4 = *reinterpret_cast<const float4*>(nl + 4 * c4);
+      const float4 d4 = *reinterpret_cast<const float4*>(nd + 4 * c4);
+      const uint64_t lp[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+      const uint64_t dp[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c2 = 2 * c4 + e;
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        uint64_t dv2 = f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1]));
+        if constexpr (kDrop) {
+          const bool k0 = (keep >> (2 * c2)) & 1u, k1 = (keep >> (2 * c2 + 1)) & 1u;
+          ppk[c2] = pack16<kH>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
+          dv2 = f2_pack(k0 ? __uint_as_float(rp[2 * c2]) * inv_keep : 0.f,
+                        k1 ? __uint_as_float(rp[2 * c2 + 1]) * inv_keep : 0.f);
+        } else {
+          ppk[c2] = pack16<kH>(p0, p1);
+        }
+        const uint64_t g = f2_mul(f2_pack(p0, p1), f2_add(dv2, dp[e]));
+        float g0, g1;
+        f2_unpack(g, g0, g1);
+        dpk[c2] = pack16<kH>(g0, g1);
+      }
+    }
+  } else {
+    const float inv = dropout ? inv_keep : 1.f;
+#pragma unroll
+    for (int c2 = 0; c2 < 16; ++c2) {
+      float pt[2], ds[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int cc = 2 * c2 + e;
+        const float p = ((allow >> cc) & 1u) ? ex2(fmaf(__uint_as_float(rs[cc]), scale_log2, nl[cc])) : 0.f;
+        const bool kp = (keep >> cc) & 1u;
+        pt[e] = kp ? p : 0.f;
+        const float dpv = kp ? __uint_as_float(rp[cc]) * inv : 0.f;
+        ds[e] = p * (dpv + nd[cc]);
+      }
+      ppk[c2] = pack16<kH>(pt[0], pt[1]);
+      dpk[c2] = pack16<kH>(ds[0], ds[1]);
+    }
+  }
+}
+
 // kDQ = false (the deterministic mode) leaves dQ to the query-centric pass:
 // no dQ^T product, no dQ warpgroup work.
 template <bool kH, bool kDQ, bool kDrop>
@@ -1063,14 +1140,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     for (int r = (n > kQStages ? n - kQStages : 0); r < n; ++r)
       wait_bar(smem_u32(&ctl->q_full[r % kQStages]), (r / kQStages) & 1, abort_flag, nullptr);
     wait_bar(kvf, 0, abort_flag, nullptr);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer: S^T/dP^T of step n+1 go ahead of the
     // dV, dK, dQ^T products of step n so the tensor core overlaps the
-    // compute warpgroup.
+    // compute warpgroup. The whole warp runs the loop (waits, step info,
+    // descriptor arithmetic: warp-uniform values) and one elected lane
+    // issues the MMAs and commits; issued from a lone thread, the same
+    // loop spent about half again the tensor pipe's time issuing each group.
+    const bool leader = elect_one();
     constexpr uint32_t idST = idesc16<kH>(128, 64, 0, 0);   // K Q^T, V dO^T
     constexpr uint32_t idACC = idesc16<kH>(128, 128, 0, 1); // P^T dO, dS^T Q  (B MN-major)
     constexpr uint32_t idDQ = idesc16<kH>(128, 64, 1, 1);   // K^T dS^T (A and B MN-major)
-    bool ok = wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status);
+    bool ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->kv_full), 0, abort_flag, a.status));
     // Descriptors formed once; a K step adds its byte offset >> 4.
     const uint64_t dK = smem_desc_sw128(sbase + kBwdK, 16, 1024), dV = smem_desc_sw128(sbase + kBwdV, 16, 1024);
     const uint64_t dKmn = smem_desc_sw128(sbase + kBwdK, kTileBytes / 2, 1024);
@@ -1090,24 +1171,29 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto issue_st = [&](int m, uint32_t& info) -> bool {
       const int s = m & 1, sq = m % kQStages;
       const uint32_t par = (m >> 1) & 1;
-      if (!wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)) return false;
+      if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->q_full[sq]), (m / kQStages) & 1, abort_flag, a.status)))
+        return false;
       info = ctl->qinfo[sq][0];
-      if (kDQ && !wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)) return false;
+      if (kDQ && !__all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->dq_empty[s]), par ^ 1, abort_flag, a.status)))
+        return false;
       tc_fence_after();
       const uint32_t dst = tmem + s * 128;
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-        const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-        mma_ss(dst, dK + koff, dQk(sq) + qoff, idST, kk > 0);
-      }
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+          const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+          mma_ss(dst, dK + koff, dQk(sq) + qoff, idST, kk > 0);
+        }
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
-        const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
-        mma_ss(dst + 64, dV + koff, dGk(sq) + qoff, idST, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = ((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4;
+          const uint32_t qoff = ((kk >> 2) * kHalfQ + (kk & 3) * 32) >> 4;
+          mma_ss(dst + 64, dV + koff, dGk(sq) + qoff, idST, kk > 0);
+        }
+        mma_commit(smem_u32(&ctl->st_full[s]));
       }
-      mma_commit(smem_u32(&ctl->st_full[s]));
+      __syncwarp();
       return true;
     };
     int hh0 = 0, qs0 = qs_lo - 1, n = 0;
@@ -1120,7 +1206,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint32_t ninfo = 0;
       if (next && !(ok = issue_st(n + 1, ninfo))) break;
       const int s = n & 1, sq = n % kQStages;
-      if (!(ok = wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
+      if (!(ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->ds_full[s]), (n >> 1) & 1, abort_flag, a.status))))
+        break;
       tc_fence_after();
       auto issue_dq = [&]() {
 #pragma unroll
@@ -1130,26 +1217,30 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       };
       // dQ^T first: the dQ warps drain it while dV and dK run, so its TMEM
       // columns are free again before S^T of step n + 2 is issued.
-      if constexpr (kDQ && kBwdDqFirst) {
-        issue_dq();
-        mma_commit(smem_u32(&ctl->dq_full[s]));
+      if (leader) {
+        if constexpr (kDQ && kBwdDqFirst) {
+          issue_dq();
+          mma_commit(smem_u32(&ctl->dq_full[s]));
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows; A = P~^T from TMEM (16 rows = 8 columns)
+          mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8, dGmn(sq) + (uint64_t)(kk * (2048 >> 4)),
+                 idACC, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tDK, dDS(s) + (uint64_t)(kk * (32 >> 4)), dQmn(sq) + (uint64_t)(kk * (2048 >> 4)), idACC,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        if constexpr (kDQ && !kBwdDqFirst) issue_dq();
+        mma_commit(smem_u32(&ctl->q_empty[sq]));
+        if constexpr (kDQ && !kBwdDqFirst) mma_commit(smem_u32(&ctl->dq_full[s]));
       }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)  // K = 64 query rows; A = P~^T from TMEM (16 rows = 8 columns)
-        mma_ts(tDV, tmem + s * 128 + 64 + (kk >> 1) * 32 + (kk & 1) * 8, dGmn(sq) + (uint64_t)(kk * (2048 >> 4)),
-               idACC, (n > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tDK, dDS(s) + (uint64_t)(kk * (32 >> 4)), dQmn(sq) + (uint64_t)(kk * (2048 >> 4)), idACC,
-               (n > 0 || kk > 0) ? 1u : 0u);
-      if constexpr (kDQ && !kBwdDqFirst) issue_dq();
-      mma_commit(smem_u32(&ctl->q_empty[sq]));
-      if constexpr (kDQ && !kBwdDqFirst) mma_commit(smem_u32(&ctl->dq_full[s]));
+      __syncwarp();
       have = next;
       info = ninfo;
       ++n;
     }
-    mma_commit(smem_u32(&ctl->acc_done));
+    if (leader) mma_commit(smem_u32(&ctl->acc_done));
+    __syncwarp();
   } else if (warp >= 4 && warp < 12) {
     // ---------------- compute warpgroups: thread t owns key row k0 + t. Step
     // n lives in S^T | dP^T buffer n & 1. Without dropout the two warpgroups
@@ -1207,57 +1298,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const float* nd = stat + sq * 128 + 64 + 32 * c;  // -delta
         tmem_wait_ld();
         uint32_t ppk[16], dpk[16];
-        if (!general) {
-          // Pairs of columns on packed fp32: x = s c log2(e) - LSE, p = 2^x,
-          // gamma = p (dP - delta); -LSE and -delta come as broadcast 16-byte loads.
-          const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
-#pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(nl + 4 * c4);
-            const float4 d4 = *reinterpret_cast<const float4*>(nd + 4 * c4);
-            const uint64_t lp[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
-            const uint64_t dp[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c2 = 2 * c4 + e;
-              float x0, x1;
-              f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[2 * c2]), __uint_as_float(rs[2 * c2 + 1])), sc2, lp[e]), x0,
-                        x1);
-              const float p0 = ex2(x0), p1 = ex2(x1);
-              uint64_t dv2 = f2_pack(__uint_as_float(rp[2 * c2]), __uint_as_float(rp[2 * c2 + 1]));
-              if constexpr (kDrop) {  // xi in the P~ operand and in dP; p itself stays undropped
-                const bool k0 = (keep >> (2 * c2)) & 1u, k1 = (keep >> (2 * c2 + 1)) & 1u;
-                ppk[c2] = pack16<kH>(k0 ? p0 : 0.f, k1 ? p1 : 0.f);
-                dv2 = f2_pack(k0 ? __uint_as_float(rp[2 * c2]) * a.m.inv_keep : 0.f,
-                              k1 ? __uint_as_float(rp[2 * c2 + 1]) * a.m.inv_keep : 0.f);
-              } else {
-                ppk[c2] = pack16<kH>(p0, p1);
-              }
-              const uint64_t g = f2_mul(f2_pack(p0, p1), f2_add(dv2, dp[e]));
-              float g0, g1;
-              f2_unpack(g, g0, g1);
-              dpk[c2] = pack16<kH>(g0, g1);
-            }
-          }
-        } else {
-          const float inv = a.m.dropout ? a.m.inv_keep : 1.f;
-#pragma unroll
-          for (int c2 = 0; c2 < 16; ++c2) {
-            float pt[2], ds[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int cc = 2 * c2 + e;
-              const float p = ((allow >> cc) & 1u) ? ex2(fmaf(__uint_as_float(rs[cc]), a.scale_log2, nl[cc])) : 0.f;
-              const bool kp = (keep >> cc) & 1u;
-              // xi only in the bf16 operand; dV is scaled by 1/(1-rho) at the end.
-              pt[e] = kp ? p : 0.f;
-              const float dpv = kp ? __uint_as_float(rp[cc]) * inv : 0.f;
-              ds[e] = p * (dpv + nd[cc]);
-            }
-            ppk[c2] = pack16<kH>(pt[0], pt[1]);
-            dpk[c2] = pack16<kH>(ds[0], ds[1]);
-          }
-        }
+        bwd_chunk_math<kH, kDrop>(rs, rp, nl, nd, general, allow, keep, a.scale_log2, a.m.inv_keep, a.m.dropout, ppk,
+                                  dpk);
         // P~^T as bf16 pairs over this pass's own dP^T columns (already read).
         tmem_st16(tbuf + 64 + 32 * c, ppk);
 #pragma unroll
@@ -1487,8 +1529,12 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
       wait_bar(smem_u32(&ctl->k_full[s]), (r / kStages) & 1, abort_flag, nullptr);
       wait_bar(smem_u32(&ctl->v_full[s]), (r / kStages) & 1, abort_flag, nullptr);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (whole warp; one elected lane issues)
+    const bool leader = elect_one();
+    auto wait_all = [&](uint32_t bar, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bar(bar, par, abort_flag, f.status));
+    };
     constexpr uint32_t idS = idesc16<kH>(128, 128, 0, 0);   // Q K^T and dO V^T
     constexpr uint32_t idDQ = idesc16<kH>(128, 128, 0, 1);  // gamma K (B = K, d contiguous)
     const uint64_t dQ0 = smem_desc_sw128(sbase + kDqQ, 16, 1024), dG0 = smem_desc_sw128(sbase + kDqG, 16, 1024);
@@ -1497,25 +1543,31 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
     constexpr uint64_t kTileStep = kTileBytes >> 4;
     auto kstep = [](int kk) { return (uint64_t)(((kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32) >> 4); };
     auto issue_s = [&](int stage, int buf) {
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ss(tmem + buf * 128, dQ0 + kstep(kk), dK0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
-      mma_commit(smem_u32(&ctl->s_full[buf]));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + buf * 128, dQ0 + kstep(kk), dK0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
+        mma_commit(smem_u32(&ctl->s_full[buf]));
+      }
+      __syncwarp();
     };
     auto issue_dp = [&](int stage) {
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ss(tmem + 256, dG0 + kstep(kk), dV0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
-      mma_commit(smem_u32(&ctl->dp_full));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + 256, dG0 + kstep(kk), dV0 + (uint64_t)stage * kTileStep + kstep(kk), idS, kk > 0);
+        mma_commit(smem_u32(&ctl->dp_full));
+      }
+      __syncwarp();
     };
-    bool ok = wait_bar(smem_u32(&ctl->q_full), 0, abort_flag, f.status);
+    bool ok = wait_all(smem_u32(&ctl->q_full), 0);
     int n = 0;
     if (ok && first <= kt_hi) {
-      ok = wait_bar(smem_u32(&ctl->k_full[0]), 0, abort_flag, f.status);
+      ok = wait_all(smem_u32(&ctl->k_full[0]), 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
-        ok = wait_bar(smem_u32(&ctl->v_full[0]), 0, abort_flag, f.status);
+        ok = wait_all(smem_u32(&ctl->v_full[0]), 0);
         if (ok) {
           tc_fence_after();
           issue_dp(0);
@@ -1527,26 +1579,30 @@ dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtens
       const int s = n % kStages, s1 = (n + 1) % kStages;
       const bool more = nk <= kt_hi;
       if (more) {  // S of the next tile into the other buffer while the warps work on this one
-        if (!(ok = wait_bar(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1, abort_flag, f.status))) break;
+        if (!(ok = wait_all(smem_u32(&ctl->k_full[s1]), ((n + 1) / kStages) & 1))) break;
         tc_fence_after();
         issue_s(s1, (n + 1) & 1);
       }
-      if (!(ok = wait_bar(smem_u32(&ctl->g_full), n & 1, abort_flag, f.status))) break;
+      if (!(ok = wait_all(smem_u32(&ctl->g_full), n & 1))) break;
       tc_fence_after();
       // dQ += gamma K: keys 16 kk .. 16 kk + 15 of warpgroup kk >> 2, 8 packed columns per step.
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_ts(tmem + 384, tmem + (n & 1) * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
-               dKmn0 + (uint64_t)s * kTileStep + (uint64_t)(kk * (2048 >> 4)), idDQ, (n > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&ctl->kv_empty[s]));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + 384, tmem + (n & 1) * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
+                 dKmn0 + (uint64_t)s * kTileStep + (uint64_t)(kk * (2048 >> 4)), idDQ, (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&ctl->kv_empty[s]));
+      }
+      __syncwarp();
       if (more) {
-        if (!(ok = wait_bar(smem_u32(&ctl->v_full[s1]), ((n + 1) / kStages) & 1, abort_flag, f.status))) break;
+        if (!(ok = wait_all(smem_u32(&ctl->v_full[s1]), ((n + 1) / kStages) & 1))) break;
         tc_fence_after();
         issue_dp(s1);
       }
       kt = nk;
     }
-    mma_commit(smem_u32(&ctl->dq_final));
+    if (leader) mma_commit(smem_u32(&ctl->dq_final));
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- compute warpgroups
     const int w = (warp - 2) >> 2;               // key columns 64 w .. 64 w + 63

@@ -194,25 +194,33 @@ topk_fwd_kernel(const TopkArgs a) {
     }
     cp_async_wait<0>();  // nothing stays in flight past the loop
     if (ok && n > 0) signal(n - 1);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer: S(n) = Q K(n)^T two tiles ahead of O += P(n) V(n).
+    // The whole warp runs the loop; one elected lane issues the MMAs.
+    const bool leader = elect_one();
+    auto wait_all = [&](uint32_t bar, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bar(bar, par, abort_flag, a.status));
+    };
     constexpr uint32_t idS = idesc16<kH>(64, kTK, 0, 0);
     constexpr uint32_t idPV = idesc16<kH>(64, 256, 0, 1);
     const uint64_t dKV0 = smem_desc_sw128(sbase + kTKV, 16, 1024);        // K-major rows of a plane
     const uint64_t dV0 = smem_desc_sw128(sbase + kTKV, kTPlane, 1024);    // MN-major: planes are 64-wide chunks
     const uint64_t dP0 = smem_desc_sw128(sbase + kTP, 16, 1024);
     constexpr uint64_t kStageStep = kTTile >> 4;
-    bool ok = wait_bar(smem_u32(&ctl->q_ready), 0, abort_flag, a.status);
+    bool ok = wait_all(smem_u32(&ctl->q_ready), 0);
     auto issue_s = [&](int m) -> bool {
       const int s = m % kTStages, b = m & 1;
-      if (!wait_bar(smem_u32(&ctl->kv_full[s]), (m / kTStages) & 1, abort_flag, a.status)) return false;
+      if (!wait_all(smem_u32(&ctl->kv_full[s]), (m / kTStages) & 1)) return false;
       tc_fence_after();
       const uint64_t dk = dKV0 + (uint64_t)s * kStageStep;
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < kTD / 16; ++kk)  // A = Q from TMEM: 16 columns of Q = 8 packed columns per step
-        mma_ts(tmem + kUpper + b * kTK, tmem + kUpper + kQCol + kk * 8,
-               dk + (uint64_t)(((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
-      mma_commit(smem_u32(&ctl->s_full[b]));
+        for (int kk = 0; kk < kTD / 16; ++kk)  // A = Q from TMEM: 16 columns of Q = 8 packed columns per step
+          mma_ts(tmem + kUpper + b * kTK, tmem + kUpper + kQCol + kk * 8,
+                 dk + (uint64_t)(((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
+        mma_commit(smem_u32(&ctl->s_full[b]));
+      }
+      __syncwarp();
       return true;
     };
     if (ok) tc_fence_after();
@@ -220,20 +228,24 @@ topk_fwd_kernel(const TopkArgs a) {
     if (ok && ntiles > 1) ok = issue_s(1);
     for (int n = 0; ok && n < ntiles; ++n) {
       const int s = n % kTStages;
-      if (!(ok = wait_bar(smem_u32(&ctl->p_full), n & 1, abort_flag, a.status))) break;
+      if (!(ok = wait_all(smem_u32(&ctl->p_full), n & 1))) break;
       tc_fence_after();
       const uint64_t dv = dV0 + (uint64_t)s * kStageStep;
+      if (leader) {
 #pragma unroll
-      for (int nh = 0; nh < 2; ++nh)
+        for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
-        for (int kk = 0; kk < kTK / 16; ++kk)  // B = V: planes 4nh..4nh+3, 16 keys (rows) per step
-          mma_ss(tmem + nh * 256, dP0 + (uint64_t)(kk * 2),
-                 dv + (uint64_t)((4 * nh * kTPlane + kk * 2048) >> 4), idPV, (n > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(smem_u32(&ctl->pv_done));
-      mma_commit(smem_u32(&ctl->kv_empty[s]));
+          for (int kk = 0; kk < kTK / 16; ++kk)  // B = V: planes 4nh..4nh+3, 16 keys (rows) per step
+            mma_ss(tmem + nh * 256, dP0 + (uint64_t)(kk * 2),
+                   dv + (uint64_t)((4 * nh * kTPlane + kk * 2048) >> 4), idPV, (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&ctl->pv_done));
+        mma_commit(smem_u32(&ctl->kv_empty[s]));
+      }
+      __syncwarp();
       if (n + 2 < ntiles) ok = issue_s(n + 2);
     }
-    mma_commit(smem_u32(&ctl->o_final));
+    if (leader) mma_commit(smem_u32(&ctl->o_final));
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- softmax warps: quarter qt = warp & 3 of TMEM; lane l
     // works on head h = 16 qt + (l & 15): its S row if l >= 16, its O row if l < 16.
@@ -564,9 +576,14 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
       signal(n);
     }
     cp_async_wait<0>();
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer: S(n), dP(n) as soon as the compute warps
     // have read S(n-1), dP(n-1); dQ += G(n) K(n) once G(n) is in shared memory.
+    // The whole warp runs the loop; one elected lane issues the MMAs.
+    const bool leader = elect_one();
+    auto wait_all = [&](uint32_t bar, uint32_t par) {
+      return __all_sync(0xffffffffu, wait_bar(bar, par, abort_flag, a.status));
+    };
     constexpr uint32_t idS = idesc16<kH>(64, kTK, 0, 0);
     constexpr uint32_t idDQ = idesc16<kH>(64, 256, 0, 1);
     constexpr uint32_t idDQ64 = idesc16<kH>(64, 64, 0, 1);
@@ -575,45 +592,51 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
     const uint64_t dDO = smem_desc_sw128(sbase + kBDO, 16, 1024);
     const uint64_t dG = smem_desc_sw128(sbase + kBG, 16, 1024);
     constexpr uint64_t kStageStep = kTTile >> 4;
-    bool ok = wait_bar(smem_u32(&ctl->q_ready), 0, abort_flag, a.status) &&
-              wait_bar(smem_u32(&ctl->do_full), 0, abort_flag, a.status);
+    bool ok = wait_all(smem_u32(&ctl->q_ready), 0) && wait_all(smem_u32(&ctl->do_full), 0);
     auto issue_sdp = [&](int m) -> bool {
       const int s = m % kBStages;
-      if (!wait_bar(smem_u32(&ctl->kv_full[s]), (m / kBStages) & 1, abort_flag, a.status)) return false;
-      if (m > 0 && !wait_bar(smem_u32(&ctl->st_empty), (m - 1) & 1, abort_flag, a.status)) return false;
+      if (!wait_all(smem_u32(&ctl->kv_full[s]), (m / kBStages) & 1)) return false;
+      if (m > 0 && !wait_all(smem_u32(&ctl->st_empty), (m - 1) & 1)) return false;
       tc_fence_after();
       const uint64_t dk = dKV0 + (uint64_t)s * kStageStep;
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < kTD / 16; ++kk)  // S = Q K^T, A = Q from TMEM
-        mma_ts(tmem + kUpper, tmem + kUpper + kQCol + kk * 8,
-               dk + (uint64_t)(((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kTD / 16; ++kk)  // S = Q K^T, A = Q from TMEM
+          mma_ts(tmem + kUpper, tmem + kUpper + kQCol + kk * 8,
+                 dk + (uint64_t)(((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4), idS, kk > 0 ? 1u : 0u);
 #pragma unroll
-      for (int kk = 0; kk < kTDV / 16; ++kk) {  // dP = dO V^T, both K-major over the first 8 planes
-        const uint32_t off = ((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4;
-        mma_ss(tmem + kUpper + kDPCol, dDO + (uint64_t)off, dk + (uint64_t)off, idS, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kTDV / 16; ++kk) {  // dP = dO V^T, both K-major over the first 8 planes
+          const uint32_t off = ((kk >> 2) * kTPlane + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + kUpper + kDPCol, dDO + (uint64_t)off, dk + (uint64_t)off, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&ctl->st_full));
       }
-      mma_commit(smem_u32(&ctl->st_full));
+      __syncwarp();
       return true;
     };
     if (ok && ntiles > 0) ok = issue_sdp(0);
     for (int n = 0; ok && n < ntiles; ++n) {
       const int s = n % kBStages;
       if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
-      if (!(ok = wait_bar(smem_u32(&ctl->g_full), n & 1, abort_flag, a.status))) break;
+      if (!(ok = wait_all(smem_u32(&ctl->g_full), n & 1))) break;
       tc_fence_after();
       const uint64_t dk = dKmn0 + (uint64_t)s * kStageStep;
+      if (leader) {
 #pragma unroll
-      for (int kk = 0; kk < kTK / 16; ++kk) {  // dQ += G K: B = K rows as [keys x d], d contiguous
-        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-        mma_ss(tmem, dG + (uint64_t)(kk * 2), dk + (uint64_t)((kk * 2048) >> 4), idDQ, acc);
-        mma_ss(tmem + 256, dG + (uint64_t)(kk * 2), dk + (uint64_t)((4 * kTPlane + kk * 2048) >> 4), idDQ, acc);
-        mma_ss(tmem + kUpper + kDQHiCol, dG + (uint64_t)(kk * 2), dk + (uint64_t)((8 * kTPlane + kk * 2048) >> 4),
-               idDQ64, acc);
+        for (int kk = 0; kk < kTK / 16; ++kk) {  // dQ += G K: B = K rows as [keys x d], d contiguous
+          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          mma_ss(tmem, dG + (uint64_t)(kk * 2), dk + (uint64_t)((kk * 2048) >> 4), idDQ, acc);
+          mma_ss(tmem + 256, dG + (uint64_t)(kk * 2), dk + (uint64_t)((4 * kTPlane + kk * 2048) >> 4), idDQ, acc);
+          mma_ss(tmem + kUpper + kDQHiCol, dG + (uint64_t)(kk * 2), dk + (uint64_t)((8 * kTPlane + kk * 2048) >> 4),
+                 idDQ64, acc);
+        }
+        mma_commit(smem_u32(&ctl->g_free));
+        mma_commit(smem_u32(&ctl->kv_empty[s]));
       }
-      mma_commit(smem_u32(&ctl->g_free));
-      mma_commit(smem_u32(&ctl->kv_empty[s]));
+      __syncwarp();
     }
-    mma_commit(smem_u32(&ctl->dq_done));
+    if (leader) mma_commit(smem_u32(&ctl->dq_done));
+    __syncwarp();
   } else if (warp >= 2) {
     // ---------------- compute warps: lane l >= 16 of quarter qt owns row
     // h = 16 qt + l - 16 of S, dP and dQ[:, 512:576]; lane l < 16 the same
