@@ -440,6 +440,75 @@ __device__ __forceinline__ float softmax_full_tile(uint32_t tS, float scale_log2
   return alpha;
 }
 
+// The full row (128 keys, all allowed) with dropout: the row's 128 scores
+// loaded from TMEM at once (one wait), the maximum taken over them, then the
+// exponentials, every one on MUFU (the softmax warps' FMA pipe also runs
+// Philox4x32-10 here). With the keep bits' work in the same warps, the one
+// load per row beats re-reading the row in passes.
+template <bool kH>
+__device__ __forceinline__ float softmax_full_tile_drop(uint32_t tS, float scale_log2, float& m_run, float& l_run,
+                                                        uint64_t kb0, uint64_t kb1) {
+  uint32_t s0[32], s1[32], s2[32], s3[32];
+  tmem_ld32(tS, s0);
+  tmem_ld32(tS + 32, s1);
+  tmem_ld32(tS + 64, s2);
+  tmem_ld32(tS + 96, s3);
+  tmem_wait_ld();
+  float mx;
+  if (scale_log2 >= 0.f) {
+    float e0 = -INFINITY, e1 = -INFINITY, e2 = -INFINITY, e3 = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      e0 = max3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+      e1 = max3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+      e2 = max3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
+      e3 = max3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
+    }
+    mx = max3f(e0, e1, fmaxf(e2, e3)) * scale_log2;
+  } else {
+    float e0 = INFINITY, e1 = INFINITY, e2 = INFINITY, e3 = INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      e0 = min3f(e0, __uint_as_float(s0[e]), __uint_as_float(s0[e + 1]));
+      e1 = min3f(e1, __uint_as_float(s1[e]), __uint_as_float(s1[e + 1]));
+      e2 = min3f(e2, __uint_as_float(s2[e]), __uint_as_float(s2[e + 1]));
+      e3 = min3f(e3, __uint_as_float(s3[e]), __uint_as_float(s3[e + 1]));
+    }
+    mx = min3f(e0, e1, fminf(e2, e3)) * scale_log2;
+  }
+  const float alpha = move_max(mx, m_run);
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-m_run, -m_run);
+  uint64_t acc0 = 0ull, acc1 = 0ull;
+  auto chunk = [&](const uint32_t (&r)[32], int q) {
+    uint32_t pk[16];
+    const uint64_t kw = q < 2 ? kb0 : kb1;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sc2, nm2), x0, x1);
+      const uint64_t pp = f2_pack(ex2(x0), ex2(x1));
+      if (e & 1)
+        acc1 = f2_add(acc1, pp);
+      else
+        acc0 = f2_add(acc0, pp);
+      float p0, p1;
+      f2_unpack(pp, p0, p1);
+      const int bit = (q & 1) * 32 + 2 * e;  // xi only in the P operand; the sum keeps every term
+      pk[e] = pack16<kH>(((kw >> bit) & 1ull) ? p0 : 0.f, ((kw >> (bit + 1)) & 1ull) ? p1 : 0.f);
+    }
+    tmem_st16(tS + q * 16, pk);
+  };
+  chunk(s0, 0);
+  chunk(s1, 1);
+  chunk(s2, 2);
+  chunk(s3, 3);
+  float a0, a1, b0, b1;
+  f2_unpack(acc0, a0, a1);
+  f2_unpack(acc1, b0, b1);
+  l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
+  return alpha;
+}
+
 // The general row: allowed-key bits (mw0, mw1) and dropout keep bits
 // (kb0, kb1) per key; two TMEM passes of 64 columns for the maximum, then 32
 // columns per pass for the exponentials. The sum and the maximum use
@@ -711,7 +780,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       tc_fence_after();
       float alpha;
       if (cls == kFull)
-        alpha = softmax_full_tile<kH, kDrop>(tS, a.scale_log2, m_run, l_run, kb0, kb1);
+        alpha = kDrop ? softmax_full_tile_drop<kH>(tS, a.scale_log2, m_run, l_run, kb0, kb1)
+                      : softmax_full_tile<kH, kDrop>(tS, a.scale_log2, m_run, l_run, kb0, kb1);
       else
         alpha = softmax_masked_tile<kH>(tS, a.scale_log2, mw0, mw1, kb0, kb1, m_run, l_run);
       // Every earlier P V of this warpgroup has completed (the S commit covers

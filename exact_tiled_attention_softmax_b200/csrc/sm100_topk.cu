@@ -425,7 +425,7 @@ constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads
 constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kBCtl = kBG + kTH * 128;
 constexpr uint32_t kBSmem = kBCtl + 1024 + 1024;
-constexpr int kBGather = 4;                       // reverse gather warps
+constexpr int kBGather = 6;                       // reverse gather warps
 constexpr int kBThreads = 192 + 32 * kBGather;    // producer, MMA issuer, 4 compute warps, gather warps
 constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
 
