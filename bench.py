@@ -313,11 +313,11 @@ def dense_problem(case: W.DenseCase, dev, torch, eta, deterministic: bool = Fals
                    4 + (2 if bm is not None else 0))
 
 
-def topk_problem(case: W.TopkCase, dev, torch, eta) -> Problem:
+def topk_problem(case: W.TopkCase, dev, torch, eta, deterministic: bool = False) -> Problem:
     q, kv, g, idx, ln, sink = W.topk_inputs(case)
     tq, tkv, tg = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, kv, g))
     allowed = eta.AllowedSet(topk_idxs=torch.from_numpy(idx).to(dev), topk_length=torch.from_numpy(ln).to(dev),
-                             sink=torch.from_numpy(sink).to(dev))
+                             sink=torch.from_numpy(sink).to(dev), deterministic=deterministic)
     tv = tkv[:, :case.Dv]
     o = torch.empty((case.Tq, case.H, case.Dv), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((case.Tq, case.H), dtype=torch.float32, device=dev)
@@ -328,14 +328,16 @@ def topk_problem(case: W.TopkCase, dev, torch, eta) -> Problem:
     ws_b = torch.empty(eta.attn_bwd_workspace_size(tq, tkv, tv, allowed), dtype=torch.uint8, device=dev)
     config = {"workload": case.name, "Tq": case.Tq, "Tkv": case.Tkv, "H": case.H, "Dqk": case.Dqk, "Dv": case.Dv,
               "mask": f"top-k lists, lengths U[{case.len_lo},{case.len_hi}], sink",
-              "gathered_bytes_per_pass": int(ln.astype(np.int64).sum()) * case.Dqk * 2}
+              "gathered_bytes_per_pass": int(ln.astype(np.int64).sum()) * case.Dqk * 2,
+              "reverse": ("deterministic (dKV summed in 32.32 fixed point)" if deterministic
+                          else "dKV summed with fp32 atomics")}
     return Problem(case.name, case.H * int(ln.astype(np.int64).sum()), 2 * case.Dqk + 2 * case.Dv,
                    6 * case.Dqk + 4 * case.Dv, [tq, tkv, tg], [dq, dkv],
                    lambda: eta.attn_fwd(tq, tkv, tv, allowed, case.scale, out=o, lse=lse, workspace=ws_f),
                    lambda: eta.attn_bwd(tq, tkv, tv, o, tg, lse, allowed, case.scale, dq=dq, dk=dkv, dv=None,
                                         dsink=dsink, workspace=ws_b),
                    config, "tensor",
-                   # forward; delta, dQ + G/P, dKV contributions, fixed-point cast, dSink
+                   # forward; delta, dQ + G/P, dKV contributions, dKV cast, dSink
                    6)
 
 
@@ -351,7 +353,7 @@ def main():
     ap.add_argument("--topk-tokens", type=int, default=0,
                     help="top-k workload with only this many query tokens (a smaller case for ncu)")
     ap.add_argument("--deterministic", action="store_true",
-                    help="bitwise reproducible reverse pass (dense workloads)")
+                    help="bitwise reproducible reverse pass (dense dQ from a query-centric pass; top-k dKV in fixed point)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -381,7 +383,7 @@ def main():
             if args.topk_tokens:  # the same lists and shapes for fewer query tokens (profiling captures)
                 import dataclasses
                 case = dataclasses.replace(case, Tq=args.topk_tokens)
-            return topk_problem(case, dev, torch, eta)
+            return topk_problem(case, dev, torch, eta, args.deterministic)
         return dense_problem(W.WORKLOADS[args.workload], dev, torch, eta, args.deterministic)
 
     prob = make_problem()

@@ -172,7 +172,7 @@ size_t lse_copy_bytes(const attn_mask* m, size_t rows) {
 size_t bwd_topk_bytes(const Topk& s, const attn_tensor* q, const attn_mask* m) {
   size_t n = kStatusBytes;
   n += align_up((size_t)s.Tq * s.H * sizeof(float), 256);                       // delta
-  n += topk_acc_total_bytes(s.Tkv, s.Dqk);                                      // 32.32 dKV, counts, bound
+  n += topk_acc_total_bytes(s.Tkv, s.Dqk);  // 32.32 dKV, counts, bound (or, in its first half, an fp32 dKV)
   if (q->dtype != ATTN_F32)                                                     // G, P rows (tensor-core path)
     n += align_up(attn::sm100_topk_bwd_scratch_bytes(s.Tq, s.H, s.Dqk, s.Dv, m->topk_max), 256);
   return n + lse_copy_bytes(m, (size_t)s.Tq * s.H);
@@ -419,18 +419,25 @@ attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k, const attn_tens
       lsh = 1;
     }
     if (sm100_topk_bwd_supported(p, q, k, o, do_, dq)) {
-      // Tensor cores: dQ and the per-token dKV contributions; the fixed-point
-      // accumulator starts at zero and is cast to dKV at the end.
+      // Tensor cores: dQ and the per-token dKV contributions. The accumulator
+      // (fp32, or 32.32 fixed point for a bitwise reproducible dKV) starts at
+      // zero and is cast to dKV at the end.
       char* scratch = ws + kStatusBytes + align_up((size_t)s.Tq * s.H * sizeof(float), 256) +
                       topk_acc_total_bytes(s.Tkv, s.Dqk);
+      const bool fixed = (mask->bwd_flags & ATTN_BWD_DETERMINISTIC) != 0;
+      float* acc32 = fixed ? nullptr : reinterpret_cast<float*>(acc.acc);
       e = by_storage(q->dtype, [&](auto t) {
         using T = decltype(t);
         cudaError_t r = launch_rows_delta<T>(o->data, do_->data, 1, s.Tq, s.H, so, sg, s.Dv, delta, cs);
-        if (r == cudaSuccess) r = cudaMemsetAsync(acc.acc, 0, topk_acc_total_bytes(s.Tkv, s.Dqk), cs);
+        if (r == cudaSuccess)
+          r = cudaMemsetAsync(acc.acc, 0,
+                              fixed ? topk_acc_total_bytes(s.Tkv, s.Dqk) : (size_t)s.Tkv * s.Dqk * sizeof(float), cs);
         if (r == cudaSuccess)
           r = sm100_topk_bwd(p, do_->data, do_->stride[0], do_->stride[1], lsep, lst, lsh, delta, dq->data,
-                             dq->stride[0], dq->stride[1], acc, scratch, status, cs);
-        if (r == cudaSuccess) r = launch_fixed_to_out<T>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], status, cs);
+                             dq->stride[0], dq->stride[1], acc, acc32, scratch, status, cs);
+        if (r == cudaSuccess)
+          r = fixed ? launch_fixed_to_out<T>(acc, s.Tkv, s.Dqk, dk->data, dk->stride[0], status, cs)
+                    : launch_f32_to_out<T>(acc32, s.Tkv, s.Dqk, dk->data, dk->stride[0], cs);
         return r;
       });
     } else {

@@ -33,6 +33,9 @@ cudaError_t launch_topk_bwd_rows(const TopkP& p, const void* g, int64_t sg_t, in
 template <typename T>
 cudaError_t launch_fixed_to_out(FixedAcc acc, int rows, int cols, void* out, int64_t so, uint32_t* status,
                                 cudaStream_t st);
+// dKV from an fp32 accumulator [rows, cols].
+template <typename T>
+cudaError_t launch_f32_to_out(const float* acc, int rows, int cols, void* out, int64_t so, cudaStream_t st);
 cudaError_t launch_lse_to_total(const float* in, int n0, int n1, int n2, const int64_t s[3], int head_dim,
                                 const float* sink, uint32_t fmt, float* out, cudaStream_t st);
 cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta, int n_outer, int n_heads,

@@ -397,6 +397,14 @@ __global__ void fixed_to_out(FixedAcc fa, int rows, int cols, T* out, int64_t so
   st(out + (int64_t)r * so + c, (float)((double)v * (1.0 / 4294967296.0)));
 }
 
+template <typename T>
+__global__ void __launch_bounds__(256) f32_to_out(const float* acc, int rows, int cols, T* out, int64_t so) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)rows * cols) return;
+  const int r = (int)(e / cols), c = (int)(e % cols);
+  st(out + (int64_t)r * so + c, acc[e]);
+}
+
 // dz_h = -sum over rows of head h of exp(z_h - LSE_row) delta_row, summed in a
 // fixed order by one block per head (deterministic).
 __global__ void __launch_bounds__(256)
@@ -529,6 +537,13 @@ cudaError_t launch_fixed_to_out(FixedAcc fa, int rows, int cols, void* out, int6
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_f32_to_out(const float* acc, int rows, int cols, void* out, int64_t so, cudaStream_t st) {
+  const int64_t n = (int64_t)rows * cols;
+  if (n > 0) f32_to_out<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(acc, rows, cols, static_cast<T*>(out), so);
+  return cudaGetLastError();
+}
+
 // An LSE in the caller's format -> the natural-log, sink-inclusive LSE that
 // the reverse kernels read ("DeepSeek Sparse Attention Forward and
 // Backward", sections 7.2-7.3): undo the -log2 scaling, then fold the sink
@@ -589,7 +604,8 @@ cudaError_t launch_dsink(const float* sink, const float* lse, const float* delta
                                                const float*, int64_t, int64_t, const float*, void*,     \
                                                int64_t, int64_t, FixedAcc, void*, int64_t,              \
                                                uint32_t*, cudaStream_t);                               \
-  template cudaError_t launch_fixed_to_out<T>(FixedAcc, int, int, void*, int64_t, uint32_t*, cudaStream_t);
+  template cudaError_t launch_fixed_to_out<T>(FixedAcc, int, int, void*, int64_t, uint32_t*, cudaStream_t); \
+  template cudaError_t launch_f32_to_out<T>(const float*, int, int, void*, int64_t, cudaStream_t);
 
 ATTN_INSTANTIATE(float)
 ATTN_INSTANTIATE(__nv_bfloat16)

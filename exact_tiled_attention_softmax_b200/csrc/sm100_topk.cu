@@ -782,25 +782,34 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
 // contribution to dKV for each listed row j (DSA note, sections 8-9),
 // C_j = sum_h G[h, j] Q[h, :] + [sum_h P[h, j] dO[h, :], 0], as
 // C^T = Q^T G + dO^T P on the tensor cores (M = 128 columns of Dqk per
-// chunk, N = 64 listed keys, K = 64 heads), then added into the signed
-// 32.32 fixed-point dKV accumulator with 64-bit integer atomics: integer
-// addition is associative, so dKV is bitwise reproducible.
-//   TMEM: chunk c = 0..3 (columns 128c..128c+127 of Dqk) at columns 64c,
-//   chunk 4 (columns 512-575, M = 64, lower half) at 256.
-constexpr uint32_t kCQ = 0;                        // Q: 9 planes of 64 heads x 64 columns
-constexpr uint32_t kCDO = kCQ + kTPlanes * kTPlane;  // dO: 8 planes
-constexpr uint32_t kCGP = kCDO + 8 * kTPlane;        // 2 stages x (G, P) tiles of 64 heads x 64 keys
-constexpr uint32_t kCRow = kCGP + 2 * 2 * kTPlane;   // 2 stages x 64 KV rows (-1: not listed / invalid)
-constexpr uint32_t kCCtl = kCRow + 2 * kTK * 4;
+// chunk, N = 64 listed keys, K = 64 heads), then added into the dKV
+// accumulator with global reductions: fp32 atomics as in the note (kFixed
+// false; the order of the additions varies from run to run), or 64-bit
+// integer atomics into a signed 32.32 fixed-point accumulator (kFixed true:
+// integer addition is associative, so dKV is bitwise reproducible).
+//   Chunk c = 0..3 covers columns 128c..128c+127 of Dqk, chunk 4 columns
+//   512-575 (M = 64, Q part only). The CTA's chunks form one sequence
+//   (chunk q = 5 n + c for tile n) whose accumulators take eight 64-column
+//   TMEM slots in turn (slot q mod 8): the MMAs of the next chunks run while
+//   the draining warps reduce the previous ones, so the reductions stream.
+constexpr int kCStages = 4;  // G/P tiles with their listed rows
+constexpr int kCSlots = 8;   // 64-column accumulator slots
+constexpr uint32_t kCQ = 0;                                // Q: 9 planes of 64 heads x 64 columns
+constexpr uint32_t kCDO = kCQ + kTPlanes * kTPlane;        // dO: 8 planes
+constexpr uint32_t kCGP = kCDO + 8 * kTPlane;              // stages x (G, P) tiles of 64 heads x 64 keys
+constexpr uint32_t kCRow = kCGP + kCStages * 2 * kTPlane;  // stages x 64 KV rows (-1: not listed / invalid)
+constexpr uint32_t kCCtl = kCRow + kCStages * kTK * 4;
 constexpr uint32_t kCSmem = kCCtl + 256 + 1024;
-constexpr int kCDrain = 24;                 // draining warps: six per TMEM lane quarter
+constexpr int kCPerQ = 6;                     // draining warps per TMEM lane quarter
+constexpr int kCDrain = 4 * kCPerQ;
 constexpr int kCThreads = 64 + 32 * kCDrain;  // producer, MMA issuer, draining warps
 
 struct TopkDkvCtl {
-  uint64_t qdo_full, gp_full[2], gp_empty[2], c_full, c_empty;
+  uint64_t qdo_full, gp_full[kCStages], gp_empty[kCStages], c_full[kCSlots], c_empty[kCSlots];
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
+static_assert(sizeof(TopkDkvCtl) <= 256, "dKV control block");
 
 struct TopkDkvArgs {
   const int32_t* idx;
@@ -808,11 +817,12 @@ struct TopkDkvArgs {
   int32_t topk_max;
   const int32_t* len;
   int Tq, Tkv, Dqk;
-  FixedAcc fa;  // [Tkv, Dqk] signed 32.32 fixed point, per-row counts, largest magnitude
+  FixedAcc fa;  // kFixed: [Tkv, Dqk] signed 32.32 fixed point, per-row counts, largest magnitude
+  float* acc32;  // otherwise: [Tkv, Dqk] fp32
   uint32_t* status;
 };
 
-template <bool kH>
+template <bool kH, bool kFixed>
 __global__ void __launch_bounds__(kCThreads, 1)
 topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tdo,
                     const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tp,
@@ -830,12 +840,14 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->qdo_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kCStages; ++s) {
       mbar_init(smem_u32(&ctl->gp_full[s]), 1);
       mbar_init(smem_u32(&ctl->gp_empty[s]), kCDrain);  // released by the draining warps: krow is theirs too
     }
-    mbar_init(smem_u32(&ctl->c_full), 1);
-    mbar_init(smem_u32(&ctl->c_empty), kCDrain);  // one arrival per draining warp
+    for (int i = 0; i < kCSlots; ++i) {
+      mbar_init(smem_u32(&ctl->c_full[i]), 1);
+      mbar_init(smem_u32(&ctl->c_empty[i]), kCDrain);  // one arrival per draining warp
+    }
     ctl->abort_flag = 0;
     fence_barrier_init();
   }
@@ -870,8 +882,9 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     int jn[2] = {read_idx(0, 0), read_idx(0, 1)};
     int n = 0;
     for (; n < ntiles; ++n) {
-      const int s = n & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_empty[s]), ((n >> 1) & 1) ^ 1, abort_flag, a.status)))
+      const int s = n % kCStages;
+      if (!__all_sync(0xffffffffu,
+                      wait_bar(smem_u32(&ctl->gp_empty[s]), ((n / kCStages) & 1) ^ 1, abort_flag, a.status)))
         break;
       const int jc[2] = {jn[0], jn[1]};
       jn[0] = read_idx(n + 1, 0);
@@ -882,7 +895,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int j = jc[e];
         const bool ok_j = j >= 0 && j < a.Tkv;
         krow[s * kTK + k] = ok_j ? j : -1;  // the first kernel flagged invalid entries
-        if (ok_j) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
+        if (kFixed && ok_j) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
       }
       __syncwarp();
       if (lane == 0) {
@@ -893,86 +906,120 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       }
       __syncwarp();
     }
-    if (lane == 0) {
-      for (int r = (n > 2 ? n - 2 : 0); r < n; ++r)
-        wait_bar(smem_u32(&ctl->gp_full[r & 1]), (r >> 1) & 1, abort_flag, nullptr);
+    if (lane == 0) {  // copies still in flight land before the CTA exits
+      for (int r = (n > kCStages ? n - kCStages : 0); r < n; ++r)
+        wait_bar(smem_u32(&ctl->gp_full[r % kCStages]), (r / kCStages) & 1, abort_flag, nullptr);
       if (ntiles > 0) wait_bar(smem_u32(&ctl->qdo_full), 0, abort_flag, nullptr);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer: C^T = Q^T G + dO^T P per tile.
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (the warp waits, one elected lane issues):
+    // C^T = Q^T G + dO^T P, chunk by chunk into the slot ring.
     constexpr uint32_t id128 = idesc16<kH>(128, kTK, 1, 1);
     constexpr uint32_t id64 = idesc16<kH>(64, kTK, 1, 1);
     const uint64_t dQ0 = smem_desc_sw128(sbase + kCQ, kTPlane, 1024);    // [heads x d], d contiguous
     const uint64_t dDO0 = smem_desc_sw128(sbase + kCDO, kTPlane, 1024);
     const uint64_t dGP0 = smem_desc_sw128(sbase + kCGP, kTPlane, 1024);  // [heads x keys], keys contiguous
-    bool ok = ntiles == 0 || wait_bar(smem_u32(&ctl->qdo_full), 0, abort_flag, a.status);
+    const bool leader = elect_one();
+    int issued = 0;  // chunks committed
+    bool ok = ntiles == 0 || __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->qdo_full), 0, abort_flag, a.status));
     for (int n = 0; ok && n < ntiles; ++n) {
-      const int s = n & 1;
-      if (!(ok = wait_bar(smem_u32(&ctl->gp_full[s]), (n >> 1) & 1, abort_flag, a.status))) break;
-      if (n > 0 && !(ok = wait_bar(smem_u32(&ctl->c_empty), (n - 1) & 1, abort_flag, a.status))) break;
+      const int s = n % kCStages;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_full[s]), (n / kCStages) & 1, abort_flag, a.status));
+      if (!ok) break;
       tc_fence_after();
       const uint64_t dG = dGP0 + (uint64_t)((2 * s) * (kTPlane >> 4)), dP = dG + (uint64_t)(kTPlane >> 4);
+#pragma unroll 1
+      for (int c = 0; c < 5; ++c) {
+        const int q = 5 * n + c, slot = q % kCSlots;
+        if (q >= kCSlots) {
+          ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_empty[slot]), ((q / kCSlots) - 1) & 1,
+                                                abort_flag, a.status));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (leader) {
+          const uint32_t d = tmem + 64 * slot;
+          if (c < 4) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+            for (int kk = 0; kk < kTH / 16; ++kk)  // K = 16 heads = 16 rows of every plane per step
+              mma_ss(d, dQ0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128), id128,
+                     kk > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTH / 16; ++kk)  // K = 16 heads = 16 rows of every plane per step
-          mma_ss(tmem + 64 * c, dQ0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128),
-                 id128, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kTH / 16; ++kk)
+              mma_ss(d, dDO0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dP + (uint64_t)(kk * 128), id128,
+                     1u);
+          } else {
 #pragma unroll
-        for (int kk = 0; kk < kTH / 16; ++kk)
-          mma_ss(tmem + 64 * c, dDO0 + (uint64_t)((2 * c * kTPlane + kk * 2048) >> 4), dP + (uint64_t)(kk * 128),
-                 id128, 1u);
+            for (int kk = 0; kk < kTH / 16; ++kk)  // columns 512-575: Q part only, M = 64
+              mma_ss(d, dQ0 + (uint64_t)((8 * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128), id64,
+                     kk > 0 ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&ctl->c_full[slot]));
+        }
+        __syncwarp();
+        issued = q + 1;
       }
-#pragma unroll
-      for (int kk = 0; kk < kTH / 16; ++kk)  // columns 512-575: Q part only, M = 64
-        mma_ss(tmem + 256, dQ0 + (uint64_t)((8 * kTPlane + kk * 2048) >> 4), dG + (uint64_t)(kk * 128), id64,
-               kk > 0 ? 1u : 0u);
-      mma_commit(smem_u32(&ctl->c_full));
     }
-  } else if (warp >= 2) {
+    if (issued > 0 && lane == 0)  // the last chunk's MMAs complete before TMEM is released
+      wait_bar(smem_u32(&ctl->c_full[(issued - 1) % kCSlots]), ((issued - 1) / kCSlots) & 1, abort_flag, nullptr);
+  } else {
     // ---------------- drain: lane l of quarter qt holds column 128 c + 32 qt + l
-    // of chunk c (and 512 + 16 qt + l of chunk 4 when l < 16) for all 64 keys.
-    // The six warps of a quarter split the work: keys 32 kh .. 32 kh + 31 of
-    // chunks cg and cg + 3 (cg = 0, 1, 2), so that many reductions are in
-    // flight at once.
-    const int qt = warp & 3, kq = (warp - 2) >> 2, kh = kq & 1, cp = kq >> 1;
+    // of chunk c (512 + 16 qt + l of chunk 4 when l < 16) for the chunk's 64
+    // keys. A quarter's six warps take its 16-key units of the chunk sequence
+    // in turn (unit 4 q + g to warp (4 q + g) mod 6), so that the load stays
+    // even and many reductions are in flight at once.
+    const int qt = warp & 3, kq = (warp - 2) >> 2;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
     bool ok = true, sat = false;
     float amax = 0.f;
     for (int n = 0; n < ntiles && ok; ++n) {
-      const int s = n & 1;
-      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full), n & 1, abort_flag, a.status));
-      if (ok)  // the listed rows come with the stage's tiles
-        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_full[s]), (n >> 1) & 1, abort_flag, a.status));
+      const int s = n % kCStages;
+      // the listed rows come with the stage's tiles
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->gp_full[s]), (n / kCStages) & 1, abort_flag, a.status));
       if (!ok) break;
-      tc_fence_after();
       const int32_t* rows = krow + s * kTK;
 #pragma unroll 1
-      for (int c = cp; c < 5; c += 3) {
-        uint32_t v0[32];
-        tmem_ld32(tq4 + 64 * c + 32 * kh, v0);
-        tmem_wait_ld();
+      for (int c = 0; c < 5; ++c) {
+        const int q = 5 * n + c, slot = q % kCSlots;
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full[slot]), (q / kCSlots) & 1, abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
         const int col = c < 4 ? 128 * c + 32 * qt + lane : 512 + 16 * qt + lane;
-        if (c == 4 && lane >= 16) continue;
-        auto add = [&](const uint32_t (&v)[32], int k0) {
+        const bool live = c < 4 || lane < 16;
+#pragma unroll 1
+        for (int g = (kq + kCPerQ - (4 * q) % kCPerQ) % kCPerQ; g < 4; g += kCPerQ) {
+          uint32_t v[16];
+          tmem_ld16(tq4 + 64 * slot + 16 * g, v);
+          tmem_wait_ld();
+          if (!live) continue;
+          const int4* r4 = reinterpret_cast<const int4*>(rows + 16 * g);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int j = rows[k0 + k];
-            if (j < 0) continue;
-            fixed_add(a.fa.acc + (int64_t)j * a.Dqk + col, __uint_as_float(v[k]), sat, amax);
+          for (int i = 0; i < 4; ++i) {
+            const int4 jj = r4[i];
+            const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (js[e] < 0) continue;
+              const float x = __uint_as_float(v[4 * i + e]);
+              if constexpr (kFixed)
+                fixed_add(a.fa.acc + (int64_t)js[e] * a.Dqk + col, x, sat, amax);
+              else
+                atomicAdd(a.acc32 + (int64_t)js[e] * a.Dqk + col, x);
+            }
           }
-        };
-        add(v0, 32 * kh);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->c_empty[slot]));
       }
-      tc_fence_before();
+      if (!ok) break;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&ctl->c_empty));
-        mbar_arrive(smem_u32(&ctl->gp_empty[s]));  // c_full(n) implies the MMAs are done with G and P
-      }
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->gp_empty[s]));  // c_full of its chunks: the MMAs are done with G and P
     }
-    fixed_publish_max(a.fa.maxbits, amax);
-    if (__any_sync(0xffffffffu, sat) && lane == 0) set_status(a.status, ATTN_DEVERR_OVERFLOW);
+    if constexpr (kFixed) {
+      fixed_publish_max(a.fa.maxbits, amax);
+      if (__any_sync(0xffffffffu, sat) && lane == 0) set_status(a.status, ATTN_DEVERR_OVERFLOW);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1011,7 +1058,7 @@ bool make_map3(CUtensorMap* map, const void* base, int64_t inner, int Tq, int64_
 }
 
 cudaError_t raise_smem(const void* fn, uint32_t bytes, int which) {
-  static bool done[6][64] = {};
+  static bool done[8][64] = {};  // [kernel instantiation][device]
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1040,7 +1087,7 @@ bool sm100_topk_bwd_supported(const TopkP& p, const attn_tensor* q, const attn_t
 
 cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t sg_h, const float* lse,
                            int64_t sl_t, int64_t sl_h, const float* delta, void* dq, int64_t sd_t, int64_t sd_h,
-                           FixedAcc acc, void* scratch, uint32_t* status, cudaStream_t st) {
+                           FixedAcc acc, float* acc32, void* scratch, uint32_t* status, cudaStream_t st) {
   const int pad = sm100_topk_pad(p.topk_max);
   const bool f16 = p.dtype == ATTN_F16;
   uint16_t* g_scr = static_cast<uint16_t*>(scratch);
@@ -1086,12 +1133,15 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   c.Tkv = p.Tkv;
   c.Dqk = p.Dqk;
   c.fa = acc;
+  c.acc32 = acc32;
   c.status = status;
   cudaError_t e;
   auto kdq = f16 ? topk_bwd_dq_kernel<true> : topk_bwd_dq_kernel<false>;
-  auto kdkv = f16 ? topk_bwd_dkv_kernel<true> : topk_bwd_dkv_kernel<false>;
+  auto kdkv = acc32 ? (f16 ? topk_bwd_dkv_kernel<true, false> : topk_bwd_dkv_kernel<false, false>)
+                    : (f16 ? topk_bwd_dkv_kernel<true, true> : topk_bwd_dkv_kernel<false, true>);
   if ((e = raise_smem(reinterpret_cast<const void*>(kdq), kBSmem, f16 ? 4 : 1)) != cudaSuccess) return e;
-  if ((e = raise_smem(reinterpret_cast<const void*>(kdkv), kCSmem, f16 ? 5 : 2)) != cudaSuccess) return e;
+  if ((e = raise_smem(reinterpret_cast<const void*>(kdkv), kCSmem, acc32 ? (f16 ? 7 : 6) : (f16 ? 5 : 2))) != cudaSuccess)
+    return e;
   main_kernel_begin(st);
   kdq<<<p.Tq, kBThreads, kBSmem, st>>>(mdo, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

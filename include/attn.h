@@ -70,8 +70,9 @@ typedef enum attn_status {
 #define ATTN_DEVERR_TIMEOUT 0x4u     /* a bounded pipeline wait gave up */
 #define ATTN_DEVERR_TOPK_CAUSAL 0x8u /* ATTN_MASK_TOPK_CHECK_CAUSAL: a listed index lies
                                         beyond its token's causal position */
-/* ATTN_DEVERR_OVERFLOW: the top-k reverse pass sums each dKV element in a
- * signed 32.32 fixed-point integer (range +-2^31). The bit is set when a
+/* ATTN_DEVERR_OVERFLOW: when the top-k reverse pass sums each dKV element in
+ * a signed 32.32 fixed-point integer (range +-2^31: the row kernels, and the
+ * tensor-core path under ATTN_BWD_DETERMINISTIC), the bit is set when a
  * single contribution was at least 2^30 in magnitude (it is then clamped),
  * and whenever some KV row's number of contributions times the largest
  * contribution magnitude of the call reaches 2^31: a bound on |sum| that
@@ -163,11 +164,17 @@ typedef struct attn_mask {
 } attn_mask;
 
 /* ATTN_BWD_DETERMINISTIC: every gradient is bitwise reproducible from run to
- * run. dK, dV and the top-k dKV always are (one CTA per key tile, or a
- * fixed-point accumulator); with this flag the dense tensor-core path also
- * computes dQ in a query-centric pass (one CTA sums each dQ element over the
- * key tiles in order, recomputing P and gamma) instead of reducing per-key-
- * tile partials with floating-point atomics. Costs one extra pass. */
+ * run. Dense dK and dV always are (one CTA per key tile), and so is the
+ * top-k dQ (one CTA per query token). With this flag the dense tensor-core
+ * path also computes dQ in a query-centric pass (one CTA sums each dQ
+ * element over the key tiles in order, recomputing P and gamma) instead of
+ * reducing per-key-tile partials with floating-point atomics, at the cost of
+ * one extra pass; and the top-k tensor-core path adds the per-token dKV
+ * contributions into a signed 32.32 fixed-point accumulator with integer
+ * atomics (range check below) instead of fp32 atomics (the DSA note's
+ * choice, section 9), at about 1.5 times the reduction traffic. The top-k
+ * row kernels (other shapes, fp32 storage) always use the fixed-point
+ * accumulator. */
 #define ATTN_BWD_DETERMINISTIC 0x1u
 
 /* ATTN_LSE_KV_ONLY: the denominator leaves the sink out, ln sum_j exp(s_j)

@@ -13,7 +13,8 @@ checks of the top-k path.
    index past that position sets ATTN_DEVERR_TOPK_CAUSAL and is still used
    (the result equals the oracle on the given lists); without it nothing is
    reported.
-3. The fixed-point dKV sum. Planted contributions below the per-addend clamp
+3. The fixed-point dKV sum (the row kernels, and the tensor-core path with
+   ATTN_BWD_DETERMINISTIC). Planted contributions below the per-addend clamp
    (2^30) whose sum over the tokens that list one KV row exceeds the 32.32
    range (2^31) set ATTN_DEVERR_OVERFLOW; nothing faults.
 """
@@ -225,7 +226,8 @@ def test_fixed_point_sum_overflow_is_flagged(path):
     idx = np.full((Tq, 4), -1, np.int32)
     idx[:, 0] = 0
     ln = np.ones(Tq, np.int32)
-    al = eta.AllowedSet(topk_idxs=torch.from_numpy(idx).cuda(), topk_length=torch.from_numpy(ln).cuda())
+    al = eta.AllowedSet(topk_idxs=torch.from_numpy(idx).cuda(), topk_length=torch.from_numpy(ln).cuda(),
+                        deterministic=True)
     v = kv[:, :Dv]
     o, lse = eta.attn_fwd(q, kv, v, al, 1 / 24)
     for big, expect in ((2.0 ** 23, eta.ATTN_DEVERR_OVERFLOW), (1.0, 0)):
