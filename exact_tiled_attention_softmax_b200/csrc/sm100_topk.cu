@@ -788,10 +788,11 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
 // integer atomics into a signed 32.32 fixed-point accumulator (kFixed true:
 // integer addition is associative, so dKV is bitwise reproducible).
 //   Chunk c = 0..3 covers columns 128c..128c+127 of Dqk, chunk 4 columns
-//   512-575 (M = 64, Q part only). The CTA's chunks form one sequence
-//   (chunk q = 5 n + c for tile n) whose accumulators take eight 64-column
-//   TMEM slots in turn (slot q mod 8): the MMAs of the next chunks run while
-//   the draining warps reduce the previous ones, so the reductions stream.
+//   512-575 (M = 64, Q part only); a launch takes the chunks [c_lo, c_hi).
+//   The CTA's chunks form one sequence (chunk q = nch n + c - c_lo for tile
+//   n, nch = c_hi - c_lo) whose accumulators take eight 64-column TMEM slots
+//   in turn (slot q mod 8): the MMAs of the next chunks run while the
+//   draining warps reduce the previous ones, so the reductions stream.
 constexpr int kCStages = 4;  // G/P tiles with their listed rows
 constexpr int kCSlots = 8;   // 64-column accumulator slots
 constexpr uint32_t kCQ = 0;                                // Q: 9 planes of 64 heads x 64 columns
@@ -820,6 +821,7 @@ struct TopkDkvArgs {
   FixedAcc fa;  // kFixed: [Tkv, Dqk] signed 32.32 fixed point, per-row counts, largest magnitude
   float* acc32;  // otherwise: [Tkv, Dqk] fp32
   uint32_t* status;
+  int c_lo, c_hi;  // the launch's column chunks [c_lo, c_hi) of 0..4
 };
 
 template <bool kH, bool kFixed>
@@ -869,9 +871,10 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       tma_prefetch_desc(&tg);
       tma_prefetch_desc(&tp);
       const uint32_t f = smem_u32(&ctl->qdo_full);
-      mbar_expect_tx(f, (kTPlanes + 8) * kTPlane);
-      for (int c = 0; c < kTPlanes; ++c) tma_load_3d(sbase + kCQ + c * kTPlane, &tq, f, 64 * c, 0, t);
-      for (int c = 0; c < 8; ++c) tma_load_3d(sbase + kCDO + c * kTPlane, &tdo, f, 64 * c, 0, t);
+      const int p0 = 2 * a.c_lo, q1 = min(2 * a.c_hi, kTPlanes), d1 = min(2 * a.c_hi, 8);
+      mbar_expect_tx(f, (q1 - p0 + max(d1 - p0, 0)) * kTPlane);
+      for (int c = p0; c < q1; ++c) tma_load_3d(sbase + kCQ + c * kTPlane, &tq, f, 64 * c, 0, t);
+      for (int c = p0; c < d1; ++c) tma_load_3d(sbase + kCDO + c * kTPlane, &tdo, f, 64 * c, 0, t);
     }
     __syncwarp();
     const int32_t* list = a.idx + (int64_t)t * a.idx_stride;
@@ -895,7 +898,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int j = jc[e];
         const bool ok_j = j >= 0 && j < a.Tkv;
         krow[s * kTK + k] = ok_j ? j : -1;  // the first kernel flagged invalid entries
-        if (kFixed && ok_j) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
+        if (kFixed && ok_j && a.c_lo == 0) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
       }
       __syncwarp();
       if (lane == 0) {
@@ -928,9 +931,10 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       if (!ok) break;
       tc_fence_after();
       const uint64_t dG = dGP0 + (uint64_t)((2 * s) * (kTPlane >> 4)), dP = dG + (uint64_t)(kTPlane >> 4);
+      const int nch = a.c_hi - a.c_lo;
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
-        const int q = 5 * n + c, slot = q % kCSlots;
+      for (int c = a.c_lo; c < a.c_hi; ++c) {
+        const int q = nch * n + c - a.c_lo, slot = q % kCSlots;
         if (q >= kCSlots) {
           ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_empty[slot]), ((q / kCSlots) - 1) & 1,
                                                 abort_flag, a.status));
@@ -968,7 +972,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     // keys. A quarter's six warps take its 16-key units of the chunk sequence
     // in turn (unit 4 q + g to warp (4 q + g) mod 6), so that the load stays
     // even and many reductions are in flight at once.
-    const int qt = warp & 3, kq = (warp - 2) >> 2;
+    const int qt = warp & 3, kq = (warp - 2) >> 2, nch = a.c_hi - a.c_lo;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
     bool ok = true, sat = false;
     float amax = 0.f;
@@ -979,8 +983,8 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       if (!ok) break;
       const int32_t* rows = krow + s * kTK;
 #pragma unroll 1
-      for (int c = 0; c < 5; ++c) {
-        const int q = 5 * n + c, slot = q % kCSlots;
+      for (int c = a.c_lo; c < a.c_hi; ++c) {
+        const int q = nch * n + c - a.c_lo, slot = q % kCSlots;
         ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full[slot]), (q / kCSlots) & 1, abort_flag, a.status));
         if (!ok) break;
         tc_fence_after();
@@ -1145,7 +1149,17 @@ cudaError_t sm100_topk_bwd(const TopkP& p, const void* g, int64_t sg_t, int64_t 
   main_kernel_begin(st);
   kdq<<<p.Tq, kBThreads, kBSmem, st>>>(mdo, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kdkv<<<p.Tq, kCThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
+  // fp32: one launch over the five column chunks (the 75 MB accumulator fits
+  // L2). Fixed point: chunks 0-1, then 2-4, so that each launch's slice of
+  // the int64 accumulator (67 and 84 MB of 151 MB) stays in L2 while it is
+  // reduced into; the second launch re-reads the G/P rows.
+  const int split[3] = {0, acc32 ? 5 : 2, 5};
+  for (int i = 0; i < (acc32 ? 1 : 2) && e == cudaSuccess; ++i) {
+    c.c_lo = split[i];
+    c.c_hi = split[i + 1];
+    kdkv<<<p.Tq, kCThreads, kCSmem, st>>>(mq, mdo, mg, mp, c);
+    e = cudaGetLastError();
+  }
   main_kernel_end(st);
   return cudaGetLastError();
 }
