@@ -839,6 +839,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   const int t = blockIdx.x;
   const int n_keys = a.len ? min(max(a.len[t], 0), a.topk_max) : a.topk_max;
   const int ntiles = (n_keys + kTK - 1) / kTK;
+  const int c_lo = kFixed ? a.c_lo : 0, c_hi = kFixed ? a.c_hi : 5;  // the fp32 launch takes every chunk
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&ctl->qdo_full), 1);
@@ -871,7 +872,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       tma_prefetch_desc(&tg);
       tma_prefetch_desc(&tp);
       const uint32_t f = smem_u32(&ctl->qdo_full);
-      const int p0 = 2 * a.c_lo, q1 = min(2 * a.c_hi, kTPlanes), d1 = min(2 * a.c_hi, 8);
+      const int p0 = 2 * c_lo, q1 = min(2 * c_hi, kTPlanes), d1 = min(2 * c_hi, 8);
       mbar_expect_tx(f, (q1 - p0 + max(d1 - p0, 0)) * kTPlane);
       for (int c = p0; c < q1; ++c) tma_load_3d(sbase + kCQ + c * kTPlane, &tq, f, 64 * c, 0, t);
       for (int c = p0; c < d1; ++c) tma_load_3d(sbase + kCDO + c * kTPlane, &tdo, f, 64 * c, 0, t);
@@ -898,7 +899,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
         const int j = jc[e];
         const bool ok_j = j >= 0 && j < a.Tkv;
         krow[s * kTK + k] = ok_j ? j : -1;  // the first kernel flagged invalid entries
-        if (kFixed && ok_j && a.c_lo == 0) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
+        if (kFixed && ok_j && c_lo == 0) atomicAdd(a.fa.count + j, 1u);  // one contribution of this token to row j
       }
       __syncwarp();
       if (lane == 0) {
@@ -931,10 +932,10 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       if (!ok) break;
       tc_fence_after();
       const uint64_t dG = dGP0 + (uint64_t)((2 * s) * (kTPlane >> 4)), dP = dG + (uint64_t)(kTPlane >> 4);
-      const int nch = a.c_hi - a.c_lo;
+      const int nch = c_hi - c_lo;
 #pragma unroll 1
-      for (int c = a.c_lo; c < a.c_hi; ++c) {
-        const int q = nch * n + c - a.c_lo, slot = q % kCSlots;
+      for (int c = c_lo; c < c_hi; ++c) {
+        const int q = nch * n + c - c_lo, slot = q % kCSlots;
         if (q >= kCSlots) {
           ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_empty[slot]), ((q / kCSlots) - 1) & 1,
                                                 abort_flag, a.status));
@@ -972,7 +973,7 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     // keys. A quarter's six warps take its 16-key units of the chunk sequence
     // in turn (unit 4 q + g to warp (4 q + g) mod 6), so that the load stays
     // even and many reductions are in flight at once.
-    const int qt = warp & 3, kq = (warp - 2) >> 2, nch = a.c_hi - a.c_lo;
+    const int qt = warp & 3, kq = (warp - 2) >> 2, nch = c_hi - c_lo;
     const uint32_t tq4 = tmem + ((uint32_t)(32 * qt) << 16);
     bool ok = true, sat = false;
     float amax = 0.f;
@@ -983,8 +984,8 @@ topk_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
       if (!ok) break;
       const int32_t* rows = krow + s * kTK;
 #pragma unroll 1
-      for (int c = a.c_lo; c < a.c_hi; ++c) {
-        const int q = nch * n + c - a.c_lo, slot = q % kCSlots;
+      for (int c = c_lo; c < c_hi; ++c) {
+        const int q = nch * n + c - c_lo, slot = q % kCSlots;
         ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&ctl->c_full[slot]), (q / kCSlots) & 1, abort_flag, a.status));
         if (!ok) break;
         tc_fence_after();
