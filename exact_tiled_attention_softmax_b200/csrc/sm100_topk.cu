@@ -14,7 +14,7 @@
 // A warp reads its quarter with 32-lane loads: its upper 16 lanes own the
 // S rows (softmax), its lower 16 lanes the O rows of the same heads.
 //
-// Warp 0 publishes each tile's 64 listed KV rows; four gather warps copy them
+// Warp 0 publishes each tile's 64 listed KV rows; eight gather warps copy them
 // with 16-byte cp.async into a three-stage ring (9 planes of 64 columns,
 // 128-byte swizzle); warp 1 issues the MMAs (S, then O += P V with P staged
 // in shared memory); warps 2-5 run the softmax and the epilogue.
@@ -43,8 +43,9 @@ constexpr uint32_t kTKV = 0;
 constexpr uint32_t kTP = kTKV + kTStages * kTTile;  // P: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kTCtl = kTP + kTH * 128;
 constexpr uint32_t kTSmem = kTCtl + 1024 + 1024;  // control block + alignment slack
-constexpr int kTFGather = 6;                         // forward gather warps
+constexpr int kTFGather = 8;                         // forward gather warps
 constexpr int kTFThreads = 192 + 32 * kTFGather;    // row producer, MMA issuer, 4 softmax warps, gather warps
+static_assert(kTK * 72 % (32 * kTFGather) == 0, "a tile's 16-byte copies split evenly over the gather warps");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.0f;                 // move the running max only past 2^8
 constexpr uint32_t kUpper = 16u << 16;           // TMEM lane offset of the upper half
@@ -425,8 +426,9 @@ constexpr uint32_t kBDO = kBKV + kBStages * kTTile;  // dO: 8 planes of 64 heads
 constexpr uint32_t kBG = kBDO + 8 * kTPlane;         // G: 64 heads x 64 keys, 16-bit
 constexpr uint32_t kBCtl = kBG + kTH * 128;
 constexpr uint32_t kBSmem = kBCtl + 1024 + 1024;
-constexpr int kBGather = 6;                       // reverse gather warps
+constexpr int kBGather = 8;                       // reverse gather warps
 constexpr int kBThreads = 192 + 32 * kBGather;    // producer, MMA issuer, 4 compute warps, gather warps
+static_assert(kTK * 72 % (32 * kBGather) == 0, "a tile's 16-byte copies split evenly over the gather warps");
 constexpr uint32_t kDPCol = 64, kDQHiCol = 416;
 
 struct TopkBwdCtl {
