@@ -228,11 +228,28 @@ def test_topk_shared_kv_sampled():
     assert np.abs(_np(o)[tok] - o_r).max() <= BF16_O_ABS
     assert np.abs(_np(lse)[tok] - lse_r).max() <= 1e-3
     assert rel_fro(_np(dq)[tok], dq_r) <= BF16_GRAD_REL
+    # The deterministic reverse (fixed-point dKV in two column passes) on the
+    # same inputs.
+    al_det = eta.AllowedSet(topk_idxs=_dev(idx, torch.int32), topk_length=_dev(ln, torch.int32),
+                            sink=_dev(sink, torch.float32), deterministic=True)
+    dq_d, dkv_d, _, _ = eta.attn_bwd(tq, tkv, tkv[:, :Dv], o, tg, lse, al_det, case.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(dq_d, dq)  # dQ is summed by one CTA per token in both modes
     # KV rows >= Tkv - 256 can only be listed by the last 256 tokens.
     last = np.arange(case.Tq - 256, case.Tq)
     _, dkv_r, _ = oracle.topk_backward(q[last], kv, idx[last], ln[last], Dv, case.scale, g[last], sink64)
     rows = np.arange(case.Tkv - 256, case.Tkv)
     assert rel_fro(_np(dkv)[rows], dkv_r[rows]) <= BF16_GRAD_REL
+    assert rel_fro(_np(dkv_d)[rows], dkv_r[rows]) <= BF16_GRAD_REL
+    # Rows listed by about 200 tokens each (the longest sums, spread over
+    # both column passes of the fixed-point form): every token that lists
+    # one of them enters the oracle, so these rows of its dKV are exact.
+    rows2 = np.array([0, 1, 12345, 28000])
+    lists = np.array([np.isin(idx[t, :ln[t]], rows2).any() for t in range(case.Tq)])
+    tk = np.nonzero(lists)[0]
+    _, dkv_r2, _ = oracle.topk_backward(q[tk], kv, idx[tk], ln[tk], Dv, case.scale, g[tk], sink64)
+    assert rel_fro(_np(dkv)[rows2], dkv_r2[rows2]) <= BF16_GRAD_REL
+    assert rel_fro(_np(dkv_d)[rows2], dkv_r2[rows2]) <= BF16_GRAD_REL
     # dSink needs every token.
     ds_r = oracle.topk_dsink(q, kv, idx, ln, Dv, case.scale, g, sink64)
     assert np.abs(ds.cpu().numpy() - ds_r).max() <= 2e-2 * max(1.0, np.abs(ds_r).max())

@@ -150,10 +150,11 @@ def test_topk_tc_backward_matches_oracle_and_is_reproducible(deterministic):
         assert rel_fro(to_np(dkv2), to_np(dkv).astype(np.float64)) <= 1e-2
 
 
-def test_topk_tc_fp16_storage():
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_topk_tc_fp16_storage(deterministic):
     """fp16 storage (the DSA note's storage table allows BF16 or FP16): the
     same kernels with fp16 operands, forward and reverse against the oracle
-    on the fp16-rounded inputs."""
+    on the fp16-rounded inputs, with either dKV reduction."""
     from tests.parity_util import BF16_GRAD_REL, rel_fro
     rng = np.random.default_rng(76)
     Tq, Tkv = 24, 700
@@ -168,7 +169,7 @@ def test_topk_tc_fp16_storage():
     scale = 1 / math.sqrt(DQK)
     qd, kvd, gd = to_dev(q, torch.float16), to_dev(kv, torch.float16), to_dev(g, torch.float16)
     al = eta.AllowedSet(topk_idxs=to_dev(idx, torch.int32), topk_length=to_dev(ln, torch.int32),
-                        sink=to_dev(sk, torch.float32))
+                        sink=to_dev(sk, torch.float32), deterministic=deterministic)
     wf = torch.empty(eta.attn_fwd_workspace_size(qd, kvd, kvd[:, :DV], al), dtype=torch.uint8, device="cuda")
     o, lse = eta.attn_fwd(qd, kvd, kvd[:, :DV], al, scale, workspace=wf)
     assert eta.attn_get_status(wf) == 0
