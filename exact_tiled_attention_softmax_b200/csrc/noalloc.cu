@@ -109,7 +109,7 @@ extern "C" attn_status attn_bwd_noalloc(const attn_tensor* q, const attn_tensor*
   const attn_status st = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
   if (st != ATTN_OK) return st;
   // attn_bwd itself zeroes every part of the scratch that must start at zero
-  // (status word, dQ accumulator, fixed-point dKV accumulator) on `stream`.
+  // (status word, dQ accumulator, top-k dKV accumulator) on `stream`.
   return attn_bwd(q, k, v, o, do_, lse, mask, scale, dq, dk, dv, dsink, scratch, kNoAllocScratchBytes, stream);
 }
 #pragma GCC visibility pop

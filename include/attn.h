@@ -221,8 +221,11 @@ attn_status attn_fwd(const attn_tensor* q, const attn_tensor* k,
 /* Reverse pass for upstream gradient do_ (= G): recomputes the scores from
  * q, k and the saved lse, forms delta from o and do_, and writes dq, dk, dv
  * (top-k: dk = dKV, dv = NULL) and, when mask->sink is set and dsink is not
- * NULL, dsink fp32 [Hq]. dk, dv, dKV and dsink are deterministic (bitwise
- * identical across runs); dq is not guaranteed to be. */
+ * NULL, dsink fp32 [Hq]. Dense dk and dv, the top-k dq and dsink are
+ * deterministic (bitwise identical across runs); the dense dq and the
+ * tensor-core top-k dKV are summed with floating-point atomics and are
+ * not, unless mask->bwd_flags holds ATTN_BWD_DETERMINISTIC (then every
+ * output is). */
 attn_status attn_bwd(const attn_tensor* q, const attn_tensor* k,
                      const attn_tensor* v, const attn_tensor* o,
                      const attn_tensor* do_, const attn_tensor* lse,
