@@ -580,7 +580,9 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
     cp_async_wait<0>();
   } else if (warp == 1) {
     // ---------------- MMA issuer: S(n), dP(n) as soon as the compute warps
-    // have read S(n-1), dP(n-1); dQ += G(n) K(n) once G(n) is in shared memory.
+    // have read S(n-1), dP(n-1) and tile n is gathered; dQ += G(n) K(n) once
+    // G(n) is in shared memory, ahead of S(n+1), dP(n+1) when it is ready
+    // first.
     // The whole warp runs the loop; one elected lane issues the MMAs.
     const bool leader = elect_one();
     auto wait_all = [&](uint32_t bar, uint32_t par) {
@@ -617,9 +619,37 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
       return true;
     };
     if (ok && ntiles > 0) ok = issue_sdp(0);
+    auto ready = [&](uint32_t bar, uint32_t par) { return __all_sync(0xffffffffu, mbar_try_wait(bar, par)); };
     for (int n = 0; ok && n < ntiles; ++n) {
       const int s = n % kBStages;
-      if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
+      // dQ(n) needs G(n); S/dP(n + 1) needs tile n + 1 gathered and S/dP(n)
+      // read. Whichever is ready first is issued first (they touch different
+      // TMEM columns; a slow gather then no longer holds dQ(n) back, and with
+      // it the release of the stage the next gather fills).
+      bool sdp = n + 1 >= ntiles;
+      const uint64_t w0 = globaltimer();
+      while (!sdp) {
+        if (ready(smem_u32(&ctl->g_full), n & 1)) break;
+        if (ready(smem_u32(&ctl->kv_full[(n + 1) % kBStages]), ((n + 1) / kBStages) & 1) &&
+            ready(smem_u32(&ctl->st_empty), n & 1)) {
+          if (!(ok = issue_sdp(n + 1))) break;
+          sdp = true;
+          break;
+        }
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        if (globaltimer() - w0 > kTimeoutNs) {  // as wait_bar: raise the abort flag and the timeout bit
+          if (lane == 0) {
+            *abort_flag = 1u;
+            atomicOr(a.status, 0x4u);
+          }
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) break;
       if (!(ok = wait_all(smem_u32(&ctl->g_full), n & 1))) break;
       tc_fence_after();
       const uint64_t dk = dKmn0 + (uint64_t)s * kStageStep;
@@ -636,6 +666,7 @@ topk_bwd_dq_kernel(const __grid_constant__ CUtensorMap tdo,
         mma_commit(smem_u32(&ctl->kv_empty[s]));
       }
       __syncwarp();
+      if (!sdp && !(ok = issue_sdp(n + 1))) break;
     }
     if (leader) mma_commit(smem_u32(&ctl->dq_done));
     __syncwarp();
